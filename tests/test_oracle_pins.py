@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle against what the method description and mathematics
+fix, independently of the oracle's own code (no GPU needed).
+
+Each test names the fact it checks.  The method is the MicroQonv summary
+(onedev.kr/papers/182); formats follow OCP MX v1.0 / OFP8.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mqv_oracle as O
+
+
+# ---------------------------------------------------------------- P1 formats
+
+def test_e2m1_table_matches_ocp(golden):
+    for code, val in golden("e2m1_values.txt"):
+        c = int(code, 16)
+        v = O.decode_e2m1(c)
+        assert v == float(val) and math.copysign(1, v) == math.copysign(1, float(val))
+
+
+def test_e2m3_table_matches_ocp(golden):
+    for code, val in golden("e2m3_values.txt"):
+        c = int(code, 16)
+        assert O.decode_e2m3(c) == float(val)
+        assert O.decode_e2m3(c | 0x20) == -float(val)
+
+
+def test_e4m3_points_match_ofp8(golden):
+    for code, val in golden("e4m3_points.txt"):
+        v = O.decode_e4m3(int(code, 16))
+        if val == "nan":
+            assert math.isnan(v)
+        else:
+            assert v == float(val)
+
+
+def test_format_maxima():
+    assert O.element_max(O.FP4) == 6.0
+    assert O.element_max(O.FP6) == 7.5
+    assert O.E4M3_MAX == 448.0
+    assert len(O.E4M3_GRID) == 127 and np.all(np.diff(O.E4M3_GRID) > 0)
+
+
+def test_encode_decode_roundtrip():
+    for fmt, n in ((O.FP4, 8), (O.FP6, 32)):
+        grid = O.element_grid(fmt)
+        assert np.array_equal(O.round_rne(grid.astype(np.float32), fmt), np.arange(n))
+        u = np.random.default_rng(0).random(n)
+        assert np.array_equal(O.round_sr(grid.astype(np.float32), u, fmt), np.arange(n))
+    assert np.array_equal(O.cast_e4m3(O.E4M3_GRID.astype(np.float32)), np.arange(127))
+
+
+def test_e4m3_cast_matches_torch_float8():
+    """Within the finite range, CastE4M3 with RNE is what torch's
+    float8_e4m3fn conversion computes (a library routine for the same
+    definition)."""
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.uniform(0, 460, 20000), 2.0 ** rng.uniform(-14, 8.8, 20000),
+        (O.E4M3_GRID[:-1] + O.E4M3_GRID[1:]) / 2,        # every midpoint
+    ]).astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.cast_e4m3(vals), ref)
+
+
+# --------------------------------------------------------- P2 rounding ties
+
+def test_hand_derived_rounding_points(golden):
+    for fmt, x, code in golden("rounding_ties.txt"):
+        a = np.array([float(x)], np.float32)
+        if fmt == "e4m3":
+            got = int(O.cast_e4m3(a)[0])
+        else:
+            got = int(O.round_rne(a, O.FP4 if fmt == "e2m1" else O.FP6)[0])
+        assert got == int(code), (fmt, x, got, code)
+
+
+# ------------------------------------------------------------ P11 Philox
+
+def test_philox_known_answers(golden):
+    for row in golden("philox4x32_10_kat.txt"):
+        w = [int(t, 16) for t in row]
+        out = O.philox4x32_10(np.array([w[:4]], np.uint32), (w[4], w[5]))[0]
+        assert [int(v) for v in out] == w[6:]
+
+
+def test_sr_uniforms_use_counter_i_div_4_and_word_i_mod_4():
+    seed = 0x123456789
+    idx = np.arange(12, dtype=np.uint64)
+    u = O.sr_uniforms(seed, idx)
+    for g in range(3):
+        words = O.philox4x32_10(np.array([[g, 0, 0, 0]], np.uint32),
+                                (seed & 0xFFFFFFFF, seed >> 32))[0]
+        assert np.array_equal(u[4 * g:4 * g + 4], (words >> 8).astype(np.float64) * 2.0 ** -24)
+    assert np.all((u >= 0) & (u < 1))
+
+
+# ------------------------------------------------ tensor/block scale formula
+
+def test_tensor_scale_formula():
+    x = np.zeros((4, 4), np.float32)
+    x[1, 2] = -2688.0
+    assert O.tensor_scale(x, O.FP4) == np.float32(1.0)
+    x[1, 2] = 3360.0
+    assert O.tensor_scale(x, O.FP6) == np.float32(1.0)
+
+
+def test_zero_tensor_and_zero_block():
+    z = np.zeros((8, 8), np.float32)
+    z[0, 0] = -0.0
+    q = O.quantize(z, O.FP4, O.RNE)
+    assert q.T == 0 and not q.scales.any()
+    assert q.codes[0, 0] == 0x8 and not q.codes.flatten()[1:].any()   # sign kept
+    x = np.zeros((8, 8), np.float32)
+    x[0, 0] = 1.0
+    x[5, 5] = -0.0
+    q = O.quantize(x, O.FP4, O.RNE)
+    assert q.scales[1, 1] == 0 and q.codes[5, 5] == 0x8 and q.codes[4, 4] == 0
+
+
+# ------------------------------------- P3 exactness of representable blocks
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+@pytest.mark.parametrize("rounding", [O.RNE, O.SR])
+def test_representable_blocks_are_recovered_exactly(fmt, rounding):
+    """x = c·s·T with T a power of two, s an E4M3 scale and every block
+    holding one element of the top code: quantization must return (c, s)."""
+    rng = np.random.default_rng(7)
+    rows, cols = 16, 24
+    mb = O.element_bits(fmt) - 1
+    ntop = (1 << mb) - 1
+    grid = O.element_grid(fmt)
+    T = np.float32(2.0 ** -5)
+    s_codes = rng.integers(8, 127, size=(rows // 4, cols // 4))   # normal scales
+    s_codes[0, 0] = 126                                           # the 448 block
+    mags = rng.integers(0, ntop + 1, size=(rows, cols))
+    signs = rng.integers(0, 2, size=(rows, cols))
+    for bi in range(rows // 4):
+        for bj in range(cols // 4):
+            mags[4 * bi + rng.integers(4), 4 * bj + rng.integers(4)] = ntop
+    s = np.repeat(np.repeat(O.E4M3_GRID[s_codes], 4, 0), 4, 1)
+    x = (np.where(signs == 1, -1.0, 1.0) * grid[mags] * s * float(T)).astype(np.float32)
+    assert O.tensor_scale(x, fmt) == T
+    q = O.quantize(x, fmt, rounding, seed=3)
+    assert np.array_equal(q.scales, s_codes.astype(np.uint8))
+    assert np.array_equal(q.codes & ((1 << mb) - 1), mags)
+    nz = mags != 0
+    assert np.array_equal((q.codes >> mb)[nz], signs[nz])
+    assert np.array_equal(O.dequantize(q), x.astype(np.float64))
+
+
+# ------------------------------------------------------ P4 the global max
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+def test_global_max_gets_top_scale_and_top_code(fmt):
+    rng = np.random.default_rng(11)
+    mb = O.element_bits(fmt) - 1
+    for trial in range(20):
+        x = (rng.standard_normal((32, 48)) * 10.0 ** rng.uniform(-6, 6)).astype(np.float32)
+        if trial % 2:
+            x.flat[rng.integers(x.size)] *= 100
+        q = O.quantize(x, fmt, O.RNE)
+        i = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+        assert q.scales[i[0] // 4, i[1] // 4] == 126
+        assert q.codes[i] & ((1 << mb) - 1) == (1 << mb) - 1
+        assert (q.codes[i] >> mb) == int(np.signbit(x[i]))
+
+
+# --------------------------------------------------- P10 RNE error bound
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+def test_rne_error_within_half_spacing(fmt):
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((64, 64)).astype(np.float32)
+    q = O.quantize(x, fmt, O.RNE)
+    grid = O.element_grid(fmt)
+    d = np.repeat(np.repeat(O.E4M3_GRID[q.scales], 4, 0), 4, 1) * np.float64(q.T)
+    v = np.abs(x) / d
+    lo = np.clip(np.searchsorted(grid, v, side="right") - 1, 0, len(grid) - 2)
+    spacing = grid[lo + 1] - grid[lo]
+    err = np.abs(x - O.dequantize(q))
+    inside = v <= grid[-1]
+    # fp32 rounding of v adds at most a few ulps of v
+    assert np.all(err[inside] <= (0.5 * spacing[inside] + 4e-7 * v[inside]) * d[inside])
+
+
+# --------------------------------------------- P6 stochastic rounding
+
+def test_sr_is_unbiased_and_brackets():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((8, 8)) * 1e-3).astype(np.float32)
+    x[0, 0] = 5e-3                                                  # fixes T
+    q0 = O.quantize(x, O.FP4, O.RNE)
+    lo = O.quantize(x, O.FP4, O.SR, seed=0)
+    n = 2000
+    acc = np.zeros(x.shape)
+    acc2 = np.zeros(x.shape)
+    grid = O.element_grid(O.FP4)
+    d = np.repeat(np.repeat(O.E4M3_GRID[q0.scales], 4, 0), 4, 1) * np.float64(q0.T)
+    v = np.abs(x).astype(np.float64) / d
+    below = grid[np.clip(np.searchsorted(grid, v, side="right") - 1, 0, 7)]
+    above = grid[np.clip(np.searchsorted(grid, v, side="left"), 0, 7)]
+    for seed in range(n):
+        q = O.quantize(x, O.FP4, O.SR, seed=seed)
+        assert np.array_equal(q.scales, q0.scales) and q.T == q0.T
+        mag = grid[q.codes & 7]
+        assert np.all((mag == below) | (mag == above))
+        xh = O.dequantize(q)
+        acc += xh
+        acc2 += xh * xh
+    mean = acc / n
+    var = np.maximum(acc2 / n - mean ** 2, 0)
+    tol = 5 * np.sqrt(var / n) + 1e-6 * np.abs(x)   # + fp32 rounding of T
+    sat = v > grid[-1]            # block scale rounded down: clamps (reading R5)
+    assert np.all(np.abs(mean - x)[~sat] <= tol[~sat])
+    assert np.all(np.abs(mean[sat]) == grid[-1] * d[sat])
+    assert lo.codes.shape == x.shape
+
+
+def test_sr_depends_on_seed_only_through_codes():
+    x = np.random.default_rng(3).standard_normal((16, 16)).astype(np.float32)
+    a = O.quantize(x, O.FP6, O.SR, seed=1)
+    b = O.quantize(x, O.FP6, O.SR, seed=2)
+    assert np.array_equal(a.scales, b.scales) and a.T == b.T
+    assert not np.array_equal(a.codes, b.codes)
+
+
+# ------------------------------------------------------- packing (R16)
+
+def test_packing_bit_layout():
+    assert list(O.pack_codes(np.array([[1, 2, 15, 0]]), O.FP4)) == [0x21, 0x0F]
+    # codes 1, 2, 3, 4 -> 1 | 2<<6 | 3<<12 | 4<<18 = 0x103081, little-endian
+    assert list(O.pack_codes(np.array([[1, 2, 3, 4]]), O.FP6)) == [0x81, 0x30, 0x10]
+    rng = np.random.default_rng(0)
+    for fmt, hi in ((O.FP4, 16), (O.FP6, 64)):
+        c = rng.integers(0, hi, size=(8, 12))
+        p = O.pack_codes(c, fmt)
+        assert p.size == 8 * O.packed_row_bytes(12, fmt)
+        assert np.array_equal(O.unpack_codes(p, 8, 12, fmt), c)
+
+
+# --------------------------------- P9 dequantized products fit f16 / bf16
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+def test_code_times_scale_is_exact_in_half_precision(fmt):
+    grid = O.element_grid(fmt)
+    prods = np.outer(grid, O.E4M3_GRID).ravel()
+    assert np.array_equal(prods.astype(np.float16).astype(np.float64), prods)
+    t = torch.from_numpy(prods)
+    assert torch.equal(t.to(torch.bfloat16).double(), t)
+
+
+# ------------------------- P7 im2col GEMM == direct conv == library conv
+
+SHAPES = [O.ConvShape(2, 4, 8, 5, 6, 3, 3, 1, 0), O.ConvShape(2, 8, 4, 7, 7, 3, 3, 2, 1),
+          O.ConvShape(1, 4, 4, 4, 5, 1, 1, 1, 0), O.ConvShape(3, 4, 8, 6, 5, 3, 2, 2, 2)]
+
+
+def _dyadic(rng, shape):
+    return rng.integers(-8, 9, size=shape).astype(np.float64) / 8.0
+
+
+@pytest.mark.parametrize("s", SHAPES)
+def test_im2col_gemm_equals_seven_loop_conv(s):
+    rng = np.random.default_rng(0)
+    X = _dyadic(rng, (s.H, s.W, s.Cin, s.N))
+    Wt = _dyadic(rng, (s.Cout, s.Kh, s.Kw, s.Cin))
+    Y, _ = O.conv_fwd(Wt, X, s)
+    assert np.array_equal(Y, O.direct_conv_fwd(Wt, X, s))
+
+
+@pytest.mark.parametrize("s", SHAPES)
+def test_three_gemms_match_torch_conv_fp64(s):
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N))
+    Wt = rng.standard_normal((s.Cout, s.Kh, s.Kw, s.Cin))
+    G = rng.standard_normal((s.Ho, s.Wo, s.Cout, s.N))
+    Xt = torch.from_numpy(X).permute(3, 2, 0, 1)          # NCHW
+    Wtt = torch.from_numpy(Wt).permute(0, 3, 1, 2)        # OIHW
+    Gt = torch.from_numpy(G).permute(3, 2, 0, 1)
+    Y, _ = O.conv_fwd(Wt, X, s)
+    ref = torch.nn.functional.conv2d(Xt, Wtt, stride=s.stride, padding=s.pad)
+    assert np.allclose(Y, ref.permute(2, 3, 1, 0).numpy(), rtol=1e-12, atol=1e-12)
+    GW, _ = O.conv_wgrad(G, X, s)
+    ref = torch.nn.grad.conv2d_weight(Xt, Wtt.shape, Gt, stride=s.stride, padding=s.pad)
+    assert np.allclose(GW, ref.permute(0, 2, 3, 1).numpy(), rtol=1e-12, atol=1e-12)
+    GX, _ = O.conv_dgrad(Wt, G, s)
+    ref = torch.nn.grad.conv2d_input(Xt.shape, Wtt, Gt, stride=s.stride, padding=s.pad)
+    assert np.allclose(GX, ref.permute(2, 3, 1, 0).numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("s", SHAPES)
+def test_single_output_functions_match_full_passes(s):
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N))
+    Wt = rng.standard_normal((s.Cout, s.Kh, s.Kw, s.Cin))
+    G = rng.standard_normal((s.Ho, s.Wo, s.Cout, s.N))
+    Y, SY = O.conv_fwd(Wt, X, s)
+    GW, SW = O.conv_wgrad(G, X, s)
+    GX, SX = O.conv_dgrad(Wt, G, s)
+    for _ in range(20):
+        i = tuple(int(rng.integers(d)) for d in Y.shape)
+        v, S = O.fwd_at(Wt, X, s, *i)
+        assert np.isclose(v, Y[i], rtol=1e-12, atol=1e-12) and np.isclose(S, SY[i])
+        i = tuple(int(rng.integers(d)) for d in GW.shape)
+        v, S = O.wgrad_at(G, X, s, *i)
+        assert np.isclose(v, GW[i], rtol=1e-12, atol=1e-12) and np.isclose(S, SW[i])
+        i = tuple(int(rng.integers(d)) for d in GX.shape)
+        v, S = O.dgrad_at(Wt, G, s, *i)
+        assert np.isclose(v, GX[i], rtol=1e-12, atol=1e-12) and np.isclose(S, SX[i])
+
+
+# ------------------------------------------------------ P8 adjoint identity
+
+@pytest.mark.parametrize("s", SHAPES)
+def test_adjoint_identity_ties_the_three_gemms(s):
+    """<conv(X, W), G> = <X, dgrad(G, W)> = <W, wgrad(G, X)>."""
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N))
+    Wt = rng.standard_normal((s.Cout, s.Kh, s.Kw, s.Cin))
+    G = rng.standard_normal((s.Ho, s.Wo, s.Cout, s.N))
+    a = np.sum(O.conv_fwd(Wt, X, s)[0] * G)
+    b = np.sum(X * O.conv_dgrad(Wt, G, s)[0])
+    c = np.sum(Wt * O.conv_wgrad(G, X, s)[0])
+    assert np.isclose(a, b, rtol=1e-12) and np.isclose(a, c, rtol=1e-12)
+
+
+# ----------------------------------- P5 one quantized value per pixel
+
+def _values_per_pixel(mat, pix):
+    groups = {}
+    for k in range(pix.shape[0]):
+        for p in range(pix.shape[1]):
+            groups.setdefault(pix[k, p], set()).add(mat[k, p])
+    return groups
+
+
+@pytest.mark.parametrize("cin,along", [(16, "p"), (4, "k"), (8, "k")])
+def test_quantize_once_gives_one_value_per_pixel_naive_does_not(cin, along):
+    """Section "무엇인가": quantizing after im2col groups one pixel with
+    different neighbours in different blocks, so its copies get different
+    values; quantizing before im2col (the method) gives every copy one value."""
+    s = O.ConvShape(4, cin, 16, 6, 6, 3, 3, 1, 0)
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N)).astype(np.float32)
+    X[rng.random(X.shape) < 0.05] *= 30
+    pix = O.im2col(np.arange(X.size, dtype=np.float64).reshape(X.shape), s)
+    xq = O.dequantize(O.quantize(X.reshape(s.x_view()), O.FP4, O.RNE)).reshape(X.shape)
+    ours = _values_per_pixel(O.im2col(xq, s), pix)
+    assert all(len(v) == 1 for v in ours.values())
+    naive = _values_per_pixel(O.naive_quantize_after_im2col(X, s, O.FP4, along), pix)
+    assert sum(len(v) > 1 for v in naive.values()) > 0
+
+
+def test_naive_needs_two_copies():
+    """The two GEMM directions quantize the same X' differently."""
+    s = O.ConvShape(4, 16, 16, 6, 6, 3, 3, 1, 0)
+    X = np.random.default_rng(5).standard_normal((s.H, s.W, s.Cin, s.N)).astype(np.float32)
+    a = O.naive_quantize_after_im2col(X, s, O.FP4, "k")
+    b = O.naive_quantize_after_im2col(X, s, O.FP4, "p")
+    assert a.shape == b.shape and not np.array_equal(a, b)
+
+
+def test_quantize_work_ratio_naive_vs_once():
+    """Quantization work in elements: the naive scheme quantizes the
+    Kh·Kw-inflated activation matrix (and W, G twice, once per GEMM
+    direction); quantizing once touches each element once."""
+    s = O.ConvShape(64, 128, 128, 28, 28, 3, 3, 1, 1)
+    x_once = s.H * s.W * s.Cin * s.N
+    x_naive = s.Kh * s.Kw * s.Cin * s.Ho * s.Wo * s.N
+    assert x_naive / x_once == 9.0
+    assert O.bits_per_element(O.FP4) == 4.5 and O.bits_per_element(O.FP6) == 6.5
+
+
+# ------------------------ layer-level: T factors and rounding roles
+
+def test_layer_outputs_apply_tensor_scales_and_roles():
+    s = O.ConvShape(4, 8, 8, 5, 5, 3, 3, 1, 1)
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N)).astype(np.float32)
+    Wt = rng.standard_normal((s.Cout, s.Kh, s.Kw, s.Cin)).astype(np.float32)
+    G = (rng.standard_normal((s.Ho, s.Wo, s.Cout, s.N)) * 1e-3).astype(np.float32)
+    qx, qw, qg = O.quantize_layer(X, Wt, G, s, O.FP4, seed=5)
+    out = O.layer_outputs(qx, qw, qg, s)
+    Xh = O.dequantize(qx).reshape(X.shape)
+    Wh = O.dequantize(qw).reshape(Wt.shape)
+    Gh = O.dequantize(qg).reshape(G.shape)
+    assert np.allclose(out["y"][0], O.conv_fwd(Wh, Xh, s)[0], rtol=1e-12, atol=0)
+    assert np.allclose(out["gw"][0], O.conv_wgrad(Gh, Xh, s)[0], rtol=1e-12, atol=0)
+    assert np.allclose(out["gx"][0], O.conv_dgrad(Wh, Gh, s)[0], rtol=1e-12, atol=0)
+    # G_Y is stochastically rounded: another seed changes some codes
+    qg2 = O.quantize(G.reshape(s.gy_view()), O.FP4, O.SR, seed=6)
+    assert not np.array_equal(qg.codes, qg2.codes)
+    assert np.array_equal(qx.codes, O.quantize(X.reshape(s.x_view()), O.FP4, O.RNE).codes)
