@@ -1,0 +1,168 @@
+/*
+ * mqv.h -- C ABI of the MicroQonv hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method (MicroQonv summary, onedev.kr/papers/182):
+ *   section "어떻게 동작하나" (how it works): activations are quantized once,
+ *     before im2col, and kept in the channel-batch-first layout
+ *     X_{Cin,N} in R^{Cin·(Hin·Win·N)}: for every pixel (h, w) the Cin x N
+ *     values are one contiguous block, batch index n fastest;
+ *   section "무엇과 다른가" (how it differs): W is Cout x (Kh·Kw·Cin), G_Y is
+ *     Cout x (Hout·Wout·N); 4 x 4 square blocks (B = 16) so each block side
+ *     lies along the contraction of every one of the three GEMMs
+ *     Y = W·X', G_W = G_Y·X'^T, G_X' = W^T·G_Y; NVFP4 two-level scales
+ *     T = max|X| / (448·emax), B = CastE4M3(blockmax / (T·emax)),
+ *     code = Round(x / (B·T)); round-to-nearest for X and W, stochastic
+ *     rounding for G_Y;
+ *   section "어떻게 쓰나" (how it is used): the NVFP6 variant, E2M3 elements.
+ *
+ * Conventions for every entry point
+ *   - All pointers named src/dst/codes/scales/tscale/y/gw/gx/ws are DEVICE
+ *     pointers owned by the caller; the library never allocates, frees or
+ *     keeps them.  Descriptor structs are host memory, read during the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     Every call only enqueues work on it and returns; nothing synchronizes.
+ *   - Arguments are validated before anything is enqueued; on any error the
+ *     call returns a non-zero mqv_status, enqueues nothing, and
+ *     mqv_last_error() (per host thread) describes the problem.
+ *   - fp32 tensors use these layouts (row-major, last index fastest):
+ *       X   [H][W][Cin][N]     2D view rows = H·W·Cin,     cols = N
+ *       W   [Cout][Kh][Kw][Cin] 2D view rows = Cout,       cols = Kh·Kw·Cin
+ *       G_Y [Ho][Wo][Cout][N]  2D view rows = Ho·Wo·Cout,  cols = N
+ *       Y   [Ho][Wo][Cout][N], G_X [H][W][Cin][N], G_W [Cout][Kh][Kw][Cin]
+ *     with Ho = (H + 2·pad - Kh)/stride + 1 (floor), same for Wo.
+ *   - A quantized tensor (mqv_qtensor) of a rows x cols view holds
+ *       codes : packed element codes, row-major.  NVFP4: two 4-bit codes per
+ *               byte, even column in the low nibble (cols/2 bytes per row).
+ *               NVFP6: four 6-bit codes per 3 bytes, code j of a group at
+ *               bits [6j, 6j+6) of the little-endian 24-bit word
+ *               (3·cols/4 bytes per row).  Code = sign bit | magnitude bits
+ *               (E2M1 or E2M3 as in OCP MX v1.0).
+ *       scales: one E4M3 byte per 4 x 4 block, [rows/4][cols/4] row-major.
+ *       tscale: one fp32 tensor scale T.
+ *     A 4 x 4 block of X or G_Y is 4 channels x 4 batch items at one pixel;
+ *     of W, 4 output channels x 4 input channels at one tap.
+ */
+#ifndef MQV_H
+#define MQV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MQV_OK = 0,
+  MQV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer    */
+  MQV_ERR_UNSUPPORTED = 2,  /* shape/format outside what the kernels handle  */
+  MQV_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required    */
+  MQV_ERR_CUDA = 4,         /* a CUDA launch or query failed                 */
+  MQV_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up            */
+} mqv_status;
+
+typedef enum { MQV_NVFP4 = 0 /* E2M1 elements */, MQV_NVFP6 = 1 /* E2M3 */ } mqv_format;
+typedef enum { MQV_RNE = 0, MQV_SR = 1 } mqv_rounding;
+typedef enum { MQV_OP_FWD = 1, MQV_OP_WGRAD = 2, MQV_OP_DGRAD = 3 } mqv_op;
+
+/* Shape of one convolution layer (the pages' N, Cin, Cout, H, W, Kh, Kw,
+ * stride, pad, format).  Requirements: all > 0 (pad >= 0), Cin, Cout and N
+ * multiples of 4, pad < Kh and pad < Kw, Ho and Wo >= 1, fmt a mqv_format. */
+typedef struct {
+  int64_t N, Cin, Cout, H, W, Kh, Kw, stride, pad;
+  int32_t fmt;
+  int32_t reserved; /* must be 0 */
+} mqv_conv_desc;
+
+/* A quantized rows x cols view (see the layout notes above).  codes and
+ * scales must be 16-byte aligned device pointers. */
+typedef struct {
+  void* codes;
+  uint8_t* scales;
+  float* tscale;
+  int64_t rows, cols;
+  int32_t fmt;
+  int32_t reserved; /* must be 0 */
+} mqv_qtensor;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t mqv_version(void);
+
+/* Message of the last error returned on this host thread ("" if none). */
+const char* mqv_last_error(void);
+
+/* Bytes of the packed codes and of the scale plane of a rows x cols view.
+ * rows and cols must be positive multiples of 4. Host-only, no CUDA calls. */
+mqv_status mqv_qtensor_bytes(int64_t rows, int64_t cols, int32_t fmt,
+                             size_t* code_bytes, size_t* scale_bytes);
+
+/* Workspace bytes that mqv_quantize_cbf needs for a rows x cols view
+ * (per-CTA partial maxima of |x|).  Host-only. */
+mqv_status mqv_quantize_workspace_size(int64_t rows, int64_t cols, size_t* bytes);
+
+/* Quantize once, section "무엇과 다른가": amax = max|src| over the whole
+ * view, T = amax / (448·emax) (emax = 6 for NVFP4, 7.5 for NVFP6), per 4 x 4
+ * block B = CastE4M3(blockmax / (T·emax)), code = Round(x / (B·T)) with
+ * round-to-nearest-even (MQV_RNE) or Philox4x32-10 stochastic rounding
+ * (MQV_SR: element i of the row-major view uses word i&3 of counter
+ * (i>>2 as two 32-bit words, 0, 0) and key (seed as two 32-bit words);
+ * round up iff (word>>8)·2^-24 < fractional position).  Two launches: a
+ * |x| max reduction into `ws`, then the block quantizer (which finishes the
+ * reduction itself).  src: rows x cols fp32, 16-byte aligned.  out: codes,
+ * scales and tscale written; out->rows/cols/fmt must match. */
+mqv_status mqv_quantize_cbf(const float* src, int64_t rows, int64_t cols, int32_t fmt,
+                            int32_t rounding, uint64_t seed, const mqv_qtensor* out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* The reduction step alone: *amax (device fp32) = max|src| of the view.
+ * ws: at least mqv_quantize_workspace_size bytes.  Used when the amax of a
+ * tensor sharded across processes must be combined (a MAX all-reduce of one
+ * float) before quantizing. */
+mqv_status mqv_amax(const float* src, int64_t rows, int64_t cols, float* amax,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* The quantize step alone, given a device fp32 amax (from mqv_amax, possibly
+ * combined across processes).  Same arithmetic as mqv_quantize_cbf. */
+mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols,
+                                  int32_t fmt, int32_t rounding, uint64_t seed,
+                                  const float* amax, const mqv_qtensor* out, void* stream);
+
+/* dst[r][c] = code·B·T of a quantized view, fp32 (code·B is exact in fp16;
+ * the product with T is one fp32 rounding).  Reads a stored (for example
+ * latent-replay) tensor back.  dst: rows x cols fp32, 16-byte aligned. */
+mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream);
+
+/* Workspace bytes for a conv pass (op = mqv_op).  Host-only. */
+mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* bytes);
+
+/* Forward GEMM Y = W·X' (section "무엇과 다른가"), implicit: im2col rows of
+ * X' are gathered from the quantized X on chip, never stored.
+ * y[ho][wo][co][n] = T_w·T_x·sum_{kh,kw,ci} Wq[co][kh][kw][ci]·Xq[hi][wi][ci][n]
+ * with hi = ho·stride + kh - pad, wi = wo·stride + kw - pad, zero outside.
+ * w: view Cout x Kh·Kw·Cin; x: view H·W·Cin x N; y fp32 [Ho][Wo][Cout][N]. */
+mqv_status mqv_conv_fwd(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
+                        float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Weight-gradient GEMM G_W = G_Y·X'^T: contraction over (ho, wo, n), split
+ * across CTAs and summed in a fixed order (deterministic) through `ws`.
+ * gy: view Ho·Wo·Cout x N; x: view H·W·Cin x N; gw fp32 [Cout][Kh][Kw][Cin]. */
+mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const mqv_qtensor* x,
+                          float* gw, void* ws, size_t ws_bytes, void* stream);
+
+/* Input-gradient G_X = col2im(W^T·G_Y), computed directly as an implicit
+ * transposed convolution: gx[hi][wi][ci][n] = T_w·T_g·sum over (kh, kw, co)
+ * and every (ho, wo) with ho·stride + kh - pad = hi, wo·stride + kw - pad = wi.
+ * w: view Cout x Kh·Kw·Cin; gy: view Ho·Wo·Cout x N; gx fp32 [H][W][Cin][N]. */
+mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
+                          float* gx, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, then reports and clears the device error word that
+ * bounded waits inside the conv kernels set when they give up
+ * (*flags = 0: none).  Returns MQV_ERR_TIMEOUT if a flag was set. */
+mqv_status mqv_device_errors(uint32_t* flags, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MQV_H */

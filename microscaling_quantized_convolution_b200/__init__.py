@@ -1,0 +1,271 @@
+"""Python binding of libmqv.so, the C ABI declared in include/mqv.h.
+
+Argument marshalling only: every step of the quantize-once convolution path
+runs in the library's CUDA kernels.  PyTorch supplies device memory and the
+current stream.  There is no CPU fallback: if the library or a CUDA device is
+missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmqv.so")
+
+NVFP4, NVFP6 = 0, 1
+RNE, SR = 0, 1
+OP_FWD, OP_WGRAD, OP_DGRAD = 1, 2, 3
+FORMATS = {"nvfp4": NVFP4, "nvfp6": NVFP6, NVFP4: NVFP4, NVFP6: NVFP6}
+
+
+def _fmt(f) -> int:
+    """Format code; unknown integers pass through for the library to reject."""
+    return FORMATS[f] if f in FORMATS else int(f)
+
+MQV_OK = 0
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
+
+
+class MqvError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"mqv {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class ConvDesc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("Cin", ctypes.c_int64), ("Cout", ctypes.c_int64),
+                ("H", ctypes.c_int64), ("W", ctypes.c_int64), ("Kh", ctypes.c_int64),
+                ("Kw", ctypes.c_int64), ("stride", ctypes.c_int64), ("pad", ctypes.c_int64),
+                ("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class QTensorC(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tscale", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+_SIGS = {
+    "mqv_version": (ctypes.c_int32, []),
+    "mqv_last_error": (ctypes.c_char_p, []),
+    "mqv_qtensor_bytes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                         ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_quantize_workspace_size": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64,
+                                                   ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_quantize_cbf": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_uint64, ctypes.POINTER(QTensorC),
+                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_amax": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_quantize_with_amax": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_uint64,
+                                              ctypes.c_void_p, ctypes.POINTER(QTensorC), ctypes.c_void_p]),
+    "mqv_dequantize": (ctypes.c_int, [ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_conv_workspace_size": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_int32,
+                                               ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_conv_fwd": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                    ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_wgrad": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                      ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_dgrad": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                      ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_device_errors": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_void_p]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmqv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m microscaling_quantized_convolution_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _check(status: int):
+    if status != MQV_OK:
+        raise MqvError(status, lib().mqv_last_error().decode())
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _require_cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ---------------------------------------------------------------- tensors
+
+def qtensor_bytes(rows: int, cols: int, fmt) -> tuple[int, int]:
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().mqv_qtensor_bytes(rows, cols, _fmt(fmt), ctypes.byref(cb), ctypes.byref(sb)))
+    return cb.value, sb.value
+
+
+@dataclass
+class QTensor:
+    """A quantized rows x cols view: packed codes, E4M3 scale plane, fp32 T."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tscale: torch.Tensor
+    rows: int
+    cols: int
+    fmt: int
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, fmt, device="cuda") -> "QTensor":
+        fmt = _fmt(fmt)
+        cb, sb = qtensor_bytes(rows, cols, fmt)
+        return cls(torch.empty(cb, dtype=torch.uint8, device=device),
+                   torch.empty(sb, dtype=torch.uint8, device=device),
+                   torch.empty(1, dtype=torch.float32, device=device), rows, cols, fmt)
+
+    def c(self) -> QTensorC:
+        return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(), self.tscale.data_ptr(),
+                        self.rows, self.cols, self.fmt, 0)
+
+
+def quantize_workspace_bytes(rows: int, cols: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().mqv_quantize_workspace_size(rows, cols, ctypes.byref(b)))
+    return b.value
+
+
+def quantize(src: torch.Tensor, rows: int, cols: int, fmt, rounding: int = RNE, seed: int = 0,
+             out: QTensor | None = None, ws: torch.Tensor | None = None, stream=None) -> QTensor:
+    """Quantize the rows x cols fp32 view of `src` (see mqv_quantize_cbf)."""
+    _require_cuda(src, "src", torch.float32)
+    if src.numel() != rows * cols:
+        raise ValueError("src size does not match rows x cols")
+    out = out or QTensor.empty(rows, cols, fmt, src.device)
+    if ws is None:
+        ws = torch.empty(quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device=src.device)
+    qc = out.c()
+    _check(lib().mqv_quantize_cbf(src.data_ptr(), rows, cols, _fmt(fmt), rounding, seed,
+                                  ctypes.byref(qc), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return out
+
+
+def amax(src: torch.Tensor, rows: int, cols: int, out: torch.Tensor | None = None,
+         ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Device fp32 max|src| of the view (see mqv_amax)."""
+    _require_cuda(src, "src", torch.float32)
+    out = out if out is not None else torch.empty(1, dtype=torch.float32, device=src.device)
+    if ws is None:
+        ws = torch.empty(quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device=src.device)
+    _check(lib().mqv_amax(src.data_ptr(), rows, cols, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                          _stream(stream)))
+    return out
+
+
+def quantize_with_amax(src: torch.Tensor, rows: int, cols: int, fmt, rounding: int, seed: int,
+                       amax_dev: torch.Tensor, out: QTensor | None = None, stream=None) -> QTensor:
+    _require_cuda(src, "src", torch.float32)
+    _require_cuda(amax_dev, "amax", torch.float32)
+    out = out or QTensor.empty(rows, cols, fmt, src.device)
+    qc = out.c()
+    _check(lib().mqv_quantize_with_amax(src.data_ptr(), rows, cols, _fmt(fmt), rounding, seed,
+                                        amax_dev.data_ptr(), ctypes.byref(qc), _stream(stream)))
+    return out
+
+
+def dequantize(q: QTensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = out if out is not None else torch.empty(q.rows * q.cols, dtype=torch.float32,
+                                                  device=q.codes.device)
+    qc = q.c()
+    _check(lib().mqv_dequantize(ctypes.byref(qc), out.data_ptr(), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ conv
+
+def conv_desc(N, Cin, Cout, H, W, Kh, Kw, stride=1, pad=0, fmt=NVFP4) -> ConvDesc:
+    return ConvDesc(N, Cin, Cout, H, W, Kh, Kw, stride, pad, _fmt(fmt), 0)
+
+
+def out_hw(d: ConvDesc) -> tuple[int, int]:
+    return ((d.H + 2 * d.pad - d.Kh) // d.stride + 1, (d.W + 2 * d.pad - d.Kw) // d.stride + 1)
+
+
+def conv_workspace_bytes(d: ConvDesc, op: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().mqv_conv_workspace_size(ctypes.byref(d), op, ctypes.byref(b)))
+    return b.value
+
+
+def _ws(d, op, ws, device):
+    need = conv_workspace_bytes(d, op)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def conv_fwd(d: ConvDesc, w: QTensor, x: QTensor, y: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y [Ho][Wo][Cout][N] fp32 = T_w·T_x·(W·X'), implicit im2col."""
+    Ho, Wo = out_hw(d)
+    y = y if y is not None else torch.empty((Ho, Wo, d.Cout, d.N), dtype=torch.float32, device=x.codes.device)
+    ws = _ws(d, OP_FWD, ws, x.codes.device)
+    wc, xc = w.c(), x.c()
+    _check(lib().mqv_conv_fwd(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), y.data_ptr(),
+                              _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return y
+
+
+def conv_wgrad(d: ConvDesc, gy: QTensor, x: QTensor, gw: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """G_W [Cout][Kh][Kw][Cin] fp32 = T_g·T_x·(G_Y·X'^T)."""
+    gw = gw if gw is not None else torch.empty((d.Cout, d.Kh, d.Kw, d.Cin), dtype=torch.float32,
+                                               device=x.codes.device)
+    ws = _ws(d, OP_WGRAD, ws, x.codes.device)
+    gc, xc = gy.c(), x.c()
+    _check(lib().mqv_conv_wgrad(ctypes.byref(d), ctypes.byref(gc), ctypes.byref(xc), gw.data_ptr(),
+                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return gw
+
+
+def conv_dgrad(d: ConvDesc, w: QTensor, gy: QTensor, gx: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """G_X [H][W][Cin][N] fp32 = T_w·T_g·col2im(W^T·G_Y), implicit."""
+    gx = gx if gx is not None else torch.empty((d.H, d.W, d.Cin, d.N), dtype=torch.float32,
+                                               device=gy.codes.device)
+    ws = _ws(d, OP_DGRAD, ws, gy.codes.device)
+    wc, gc = w.c(), gy.c()
+    _check(lib().mqv_conv_dgrad(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(gc), gx.data_ptr(),
+                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return gx
+
+
+def device_errors(stream=None) -> int:
+    f = ctypes.c_uint32()
+    st = lib().mqv_device_errors(ctypes.byref(f), _stream(stream))
+    if st not in (MQV_OK, 5):
+        _check(st)
+    return f.value

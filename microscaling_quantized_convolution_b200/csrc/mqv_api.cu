@@ -1,0 +1,443 @@
+// C ABI of the MicroQonv hot path (declared in include/mqv.h): argument
+// validation, launch geometry and error reporting.  Every compute step runs
+// in the kernels of mqv_quantize.cuh and mqv_conv.cuh; this file only checks
+// arguments and enqueues launches on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mqv.h"
+#include "mqv_conv.cuh"
+#include "mqv_quantize.cuh"
+
+namespace {
+
+using namespace mqv;
+
+thread_local char g_msg[512] = "";
+
+mqv_status fail(mqv_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+mqv_status ok() {
+  g_msg[0] = '\0';
+  return MQV_OK;
+}
+
+mqv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MQV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device word that bounded waits set on timeout (see mqv_ptx.cuh).
+__device__ uint32_t g_device_error;
+
+constexpr int kMaxDevices = 64;
+uint32_t* g_err_ptr[kMaxDevices] = {};
+std::mutex g_err_mu;
+
+mqv_status device_error_word(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MQV_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return MQV_OK;
+}
+
+// ------------------------------------------------------------ quantize geometry
+
+constexpr int64_t kMaxAmaxCtas = 148 * 8;
+constexpr int64_t kMaxQuantCtas = 148 * 16;
+
+int64_t amax_ctas(int64_t rows, int64_t cols) {
+  const int64_t n4 = rows * cols / 4;
+  int64_t g = (n4 + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4);
+  if (g < 1) g = 1;
+  return g < kMaxAmaxCtas ? g : kMaxAmaxCtas;
+}
+
+int64_t quant_ctas(int64_t rows, int64_t cols) {
+  const int64_t nb = rows * cols / 16;
+  int64_t g = (nb + kQuantThreads - 1) / kQuantThreads;
+  if (g < 1) g = 1;
+  return g < kMaxQuantCtas ? g : kMaxQuantCtas;
+}
+
+mqv_status check_view(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0 || rows % 4 || cols % 4)
+    return fail(MQV_ERR_INVALID_ARG, "view %lld x %lld: rows and cols must be positive multiples of 4",
+                (long long)rows, (long long)cols);
+  if (rows > (int64_t(1) << 40) / cols)
+    return fail(MQV_ERR_UNSUPPORTED, "view %lld x %lld too large", (long long)rows, (long long)cols);
+  return MQV_OK;
+}
+
+mqv_status check_fmt(int32_t fmt) {
+  if (fmt != MQV_NVFP4 && fmt != MQV_NVFP6) return fail(MQV_ERR_INVALID_ARG, "unknown format %d", fmt);
+  return MQV_OK;
+}
+
+mqv_status check_qtensor(const mqv_qtensor* q, const char* name) {
+  if (!q) return fail(MQV_ERR_INVALID_ARG, "%s: null descriptor", name);
+  mqv_status st = check_view(q->rows, q->cols);
+  if (st) return st;
+  if ((st = check_fmt(q->fmt))) return st;
+  if (q->reserved) return fail(MQV_ERR_INVALID_ARG, "%s: reserved field must be 0", name);
+  if (!q->codes || !q->scales || !q->tscale) return fail(MQV_ERR_INVALID_ARG, "%s: null pointer", name);
+  if (!aligned16(q->codes) || !aligned16(q->scales))
+    return fail(MQV_ERR_INVALID_ARG, "%s: codes and scales must be 16-byte aligned", name);
+  if (reinterpret_cast<uintptr_t>(q->tscale) & 3u)
+    return fail(MQV_ERR_INVALID_ARG, "%s: tscale must be 4-byte aligned", name);
+  return MQV_OK;
+}
+
+template <int FMT, int RND>
+void launch_quantize(const float* src, int64_t rows, int64_t cols, const float* amax_src,
+                     int amax_count, uint64_t seed, const mqv_qtensor* out, cudaStream_t st) {
+  quantize_kernel<FMT, RND><<<(unsigned)quant_ctas(rows, cols), kQuantThreads, 0, st>>>(
+      src, rows, cols, amax_src, amax_count, seed, static_cast<uint8_t*>(out->codes), out->scales,
+      out->tscale);
+}
+
+mqv_status enqueue_quantize(const float* src, int64_t rows, int64_t cols, int32_t fmt,
+                            int32_t rounding, uint64_t seed, const float* amax_src,
+                            int amax_count, const mqv_qtensor* out, cudaStream_t st) {
+  if (fmt == MQV_NVFP4)
+    rounding == MQV_RNE ? launch_quantize<0, 0>(src, rows, cols, amax_src, amax_count, seed, out, st)
+                        : launch_quantize<0, 1>(src, rows, cols, amax_src, amax_count, seed, out, st);
+  else
+    rounding == MQV_RNE ? launch_quantize<1, 0>(src, rows, cols, amax_src, amax_count, seed, out, st)
+                        : launch_quantize<1, 1>(src, rows, cols, amax_src, amax_count, seed, out, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
+}
+
+mqv_status check_quantize_args(const float* src, int64_t rows, int64_t cols, int32_t fmt,
+                               int32_t rounding, const mqv_qtensor* out) {
+  mqv_status st = check_view(rows, cols);
+  if (st) return st;
+  if ((st = check_fmt(fmt))) return st;
+  if (rounding != MQV_RNE && rounding != MQV_SR)
+    return fail(MQV_ERR_INVALID_ARG, "unknown rounding %d", rounding);
+  if (!src || !aligned16(src)) return fail(MQV_ERR_INVALID_ARG, "src must be a 16-byte aligned pointer");
+  if ((st = check_qtensor(out, "out"))) return st;
+  if (out->rows != rows || out->cols != cols || out->fmt != fmt)
+    return fail(MQV_ERR_INVALID_ARG, "out describes a %lld x %lld fmt %d view, expected %lld x %lld fmt %d",
+                (long long)out->rows, (long long)out->cols, out->fmt, (long long)rows,
+                (long long)cols, fmt);
+  return MQV_OK;
+}
+
+// ------------------------------------------------------------- conv geometry
+
+struct ConvPlan {
+  ConvArgs a;
+  dim3 grid;
+  int splits;
+  size_t ws_bytes;
+};
+
+constexpr int kBN = 128;
+constexpr int kStages = 3;
+
+mqv_status check_desc(const mqv_conv_desc* d) {
+  if (!d) return fail(MQV_ERR_INVALID_ARG, "null conv descriptor");
+  if (d->reserved) return fail(MQV_ERR_INVALID_ARG, "conv descriptor reserved field must be 0");
+  if (d->N <= 0 || d->Cin <= 0 || d->Cout <= 0 || d->H <= 0 || d->W <= 0 || d->Kh <= 0 ||
+      d->Kw <= 0 || d->stride <= 0 || d->pad < 0)
+    return fail(MQV_ERR_INVALID_ARG, "conv shape fields must be positive (pad >= 0)");
+  if (d->N % 4 || d->Cin % 4 || d->Cout % 4)
+    return fail(MQV_ERR_INVALID_ARG, "N, Cin and Cout must be multiples of 4 (4 x 4 square blocks)");
+  if (d->pad >= d->Kh || d->pad >= d->Kw)
+    return fail(MQV_ERR_INVALID_ARG, "pad must be smaller than the kernel size");
+  mqv_status st = check_fmt(d->fmt);
+  if (st) return st;
+  const int64_t Ho = (d->H + 2 * d->pad - d->Kh) / d->stride + 1;
+  const int64_t Wo = (d->W + 2 * d->pad - d->Kw) / d->stride + 1;
+  if (d->H + 2 * d->pad < d->Kh || d->W + 2 * d->pad < d->Kw || Ho <= 0 || Wo <= 0)
+    return fail(MQV_ERR_INVALID_ARG, "kernel larger than the padded input");
+  const int64_t lim = int64_t(1) << 30;
+  if (d->H * d->W > lim || d->Cin > 65536 || d->Cout > 65536 || d->N > 65536 || d->Kh > 64 ||
+      d->Kw > 64 || d->H * d->W * d->Cin * d->N > (int64_t(1) << 36) ||
+      Ho * Wo * d->Cout * d->N > (int64_t(1) << 36))
+    return fail(MQV_ERR_UNSUPPORTED, "conv shape exceeds the supported range");
+  return MQV_OK;
+}
+
+QView make_view(const mqv_qtensor* q) {
+  QView v;
+  v.codes = static_cast<const uint8_t*>(q->codes);
+  v.scales = q->scales;
+  v.tscale = q->tscale;
+  v.row_bytes = q->fmt == MQV_NVFP4 ? q->cols / 2 : q->cols * 3 / 4;
+  v.scale_cols = q->cols / 4;
+  return v;
+}
+
+// Geometry of one pass (no pointers needed for sizing).
+void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
+  ConvArgs& a = pl->a;
+  std::memset(&a, 0, sizeof(a));
+  a.N = (int)d->N; a.Cin = (int)d->Cin; a.Cout = (int)d->Cout; a.H = (int)d->H; a.W = (int)d->W;
+  a.Kh = (int)d->Kh; a.Kw = (int)d->Kw; a.stride = (int)d->stride; a.pad = (int)d->pad;
+  a.Ho = (int)((d->H + 2 * d->pad - d->Kh) / d->stride + 1);
+  a.Wo = (int)((d->W + 2 * d->pad - d->Kw) / d->stride + 1);
+  const int64_t taps = d->Kh * d->Kw;
+  if (op == MQV_OP_FWD) {
+    a.M = a.Cout;
+    a.Ncols = (int64_t)a.Ho * a.Wo * a.N;
+    a.Kdim = taps * a.Cin;
+  } else if (op == MQV_OP_WGRAD) {
+    a.M = a.Cout;
+    a.Ncols = taps * a.Cin;
+    a.Kdim = (int64_t)a.Ho * a.Wo * a.N;
+  } else {
+    a.M = a.Cin;
+    a.Ncols = (int64_t)a.H * a.W * a.N;
+    a.Kdim = taps * a.Cout;
+  }
+  a.ktiles = (int)((a.Kdim + kBK - 1) / kBK);
+  const int64_t tiles_n = (a.Ncols + kBN - 1) / kBN;
+  const int64_t tiles_m = (a.M + kBM - 1) / kBM;
+  int splits = 1;
+  if (op == MQV_OP_WGRAD) {
+    const int64_t target = 2 * 148;
+    int64_t s = (target + tiles_n * tiles_m - 1) / (tiles_n * tiles_m);
+    if (s > a.ktiles) s = a.ktiles;
+    if (s < 1) s = 1;
+    const int64_t per = (a.ktiles + s - 1) / s;
+    splits = (int)((a.ktiles + per - 1) / per);
+    a.kt_per_split = (int)per;
+  } else {
+    a.kt_per_split = a.ktiles;
+  }
+  pl->splits = splits;
+  a.scale_out = splits == 1;
+  pl->grid = dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits);
+  pl->ws_bytes = splits > 1 ? (size_t)splits * a.M * a.Ncols * sizeof(float) : 0;
+}
+
+template <int PASS, int FMT>
+cudaError_t launch_conv(const ConvPlan& pl, cudaStream_t st) {
+  using L = ConvSmem<kBN, kStages>;
+  auto kern = conv_gemm_kernel<PASS, FMT, kBN, kStages>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  kern<<<pl.grid, kConvThreads, L::kBytes, st>>>(pl.a);
+  return cudaGetLastError();
+}
+
+template <int PASS>
+cudaError_t launch_conv_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
+  return fmt == MQV_NVFP4 ? launch_conv<PASS, 0>(pl, st) : launch_conv<PASS, 1>(pl, st);
+}
+
+mqv_status check_operand(const mqv_qtensor* q, const char* name, int64_t rows, int64_t cols, int32_t fmt) {
+  mqv_status st = check_qtensor(q, name);
+  if (st) return st;
+  if (q->rows != rows || q->cols != cols || q->fmt != fmt)
+    return fail(MQV_ERR_INVALID_ARG, "%s: view %lld x %lld fmt %d, expected %lld x %lld fmt %d", name,
+                (long long)q->rows, (long long)q->cols, q->fmt, (long long)rows, (long long)cols, fmt);
+  return MQV_OK;
+}
+
+mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const char* na,
+                    const mqv_qtensor* qb, const char* nb, float* out, void* ws, size_t ws_bytes,
+                    void* stream) {
+  mqv_status st = check_desc(d);
+  if (st) return st;
+  const int64_t Ho = (d->H + 2 * d->pad - d->Kh) / d->stride + 1;
+  const int64_t Wo = (d->W + 2 * d->pad - d->Kw) / d->stride + 1;
+  const int64_t xr = d->H * d->W * d->Cin, wr = d->Cout, wc = d->Kh * d->Kw * d->Cin;
+  const int64_t gr = Ho * Wo * d->Cout;
+  if (op == MQV_OP_FWD) {
+    if ((st = check_operand(qa, na, wr, wc, d->fmt)) || (st = check_operand(qb, nb, xr, d->N, d->fmt))) return st;
+  } else if (op == MQV_OP_WGRAD) {
+    if ((st = check_operand(qa, na, gr, d->N, d->fmt)) || (st = check_operand(qb, nb, xr, d->N, d->fmt))) return st;
+  } else {
+    if ((st = check_operand(qa, na, wr, wc, d->fmt)) || (st = check_operand(qb, nb, gr, d->N, d->fmt))) return st;
+  }
+  if (!out || !aligned16(out)) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
+  ConvPlan pl;
+  plan_conv(d, op, &pl);
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+                pl.ws_bytes, ws ? ws_bytes : (size_t)0);
+  uint32_t* err = nullptr;
+  if ((st = device_error_word(&err))) return st;
+  pl.a.a = make_view(qa);
+  pl.a.b = make_view(qb);
+  pl.a.err = err;
+  pl.a.out = pl.splits > 1 ? static_cast<float*>(ws) : out;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (op == MQV_OP_FWD) e = launch_conv_fmt<kFwd>(d->fmt, pl, s);
+  else if (op == MQV_OP_WGRAD) e = launch_conv_fmt<kWgrad>(d->fmt, pl, s);
+  else e = launch_conv_fmt<kDgrad>(d->fmt, pl, s);
+  if (e != cudaSuccess) return cuda_fail(e, "conv launch");
+  if (pl.splits > 1) {
+    const int64_t n4 = (int64_t)pl.a.M * pl.a.Ncols / 4;
+    int64_t g = (n4 + 255) / 256;
+    if (g > 148 * 8) g = 148 * 8;
+    wgrad_reduce_kernel<<<(unsigned)g, 256, 0, s>>>(reinterpret_cast<const float4*>(ws), pl.splits, n4,
+                                                     qa->tscale, qb->tscale, reinterpret_cast<float4*>(out));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "wgrad reduce launch");
+  }
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mqv_version(void) { return 100; }
+
+const char* mqv_last_error(void) { return g_msg; }
+
+mqv_status mqv_qtensor_bytes(int64_t rows, int64_t cols, int32_t fmt, size_t* code_bytes,
+                             size_t* scale_bytes) {
+  mqv_status st = check_view(rows, cols);
+  if (st) return st;
+  if ((st = check_fmt(fmt))) return st;
+  if (!code_bytes || !scale_bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  *code_bytes = (size_t)(fmt == MQV_NVFP4 ? rows * cols / 2 : rows * cols * 3 / 4);
+  *scale_bytes = (size_t)(rows * cols / 16);
+  return ok();
+}
+
+mqv_status mqv_quantize_workspace_size(int64_t rows, int64_t cols, size_t* bytes) {
+  mqv_status st = check_view(rows, cols);
+  if (st) return st;
+  if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  *bytes = (size_t)((amax_ctas(rows, cols) * sizeof(float) + 255) / 256 * 256);
+  return ok();
+}
+
+mqv_status mqv_amax(const float* src, int64_t rows, int64_t cols, float* amax, void* ws,
+                    size_t ws_bytes, void* stream) {
+  mqv_status st = check_view(rows, cols);
+  if (st) return st;
+  if (!src || !aligned16(src)) return fail(MQV_ERR_INVALID_ARG, "src must be a 16-byte aligned pointer");
+  if (!amax || (reinterpret_cast<uintptr_t>(amax) & 3u)) return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
+  const int64_t g = amax_ctas(rows, cols);
+  if (!ws || ws_bytes < (size_t)g * sizeof(float) || !aligned16(ws))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes required", (size_t)g * sizeof(float));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  amax_partial_kernel<<<(unsigned)g, kAmaxThreads, 0, s>>>(reinterpret_cast<const float4*>(src), rows * cols / 4, part);
+  amax_finish_kernel<<<1, kAmaxThreads, 0, s>>>(part, (int)g, amax);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  return ok();
+}
+
+mqv_status mqv_quantize_cbf(const float* src, int64_t rows, int64_t cols, int32_t fmt,
+                            int32_t rounding, uint64_t seed, const mqv_qtensor* out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  mqv_status st = check_quantize_args(src, rows, cols, fmt, rounding, out);
+  if (st) return st;
+  const int64_t g = amax_ctas(rows, cols);
+  if (!ws || ws_bytes < (size_t)g * sizeof(float) || !aligned16(ws))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes required", (size_t)g * sizeof(float));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  amax_partial_kernel<<<(unsigned)g, kAmaxThreads, 0, s>>>(reinterpret_cast<const float4*>(src), rows * cols / 4, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, part, (int)g, out, s);
+}
+
+mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols, int32_t fmt,
+                                  int32_t rounding, uint64_t seed, const float* amax,
+                                  const mqv_qtensor* out, void* stream) {
+  mqv_status st = check_quantize_args(src, rows, cols, fmt, rounding, out);
+  if (st) return st;
+  if (!amax || (reinterpret_cast<uintptr_t>(amax) & 3u)) return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
+  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, amax, 1, out,
+                          static_cast<cudaStream_t>(stream));
+}
+
+mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream) {
+  mqv_status st = check_qtensor(q, "q");
+  if (st) return st;
+  if (!dst || !aligned16(dst)) return fail(MQV_ERR_INVALID_ARG, "dst must be a 16-byte aligned pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned g = (unsigned)quant_ctas(q->rows, q->cols);
+  const uint8_t* c = static_cast<const uint8_t*>(q->codes);
+  if (q->fmt == MQV_NVFP4)
+    dequantize_kernel<0><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, dst);
+  else
+    dequantize_kernel<1><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, dst);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return ok();
+}
+
+mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* bytes) {
+  mqv_status st = check_desc(d);
+  if (st) return st;
+  if (op != MQV_OP_FWD && op != MQV_OP_WGRAD && op != MQV_OP_DGRAD)
+    return fail(MQV_ERR_INVALID_ARG, "unknown op %d", op);
+  if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  ConvPlan pl;
+  plan_conv(d, op, &pl);
+  *bytes = pl.ws_bytes;
+  return ok();
+}
+
+mqv_status mqv_conv_fwd(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
+                        float* y, void* ws, size_t ws_bytes, void* stream) {
+  return run_conv(MQV_OP_FWD, d, w, "w", x, "x", y, ws, ws_bytes, stream);
+}
+
+mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const mqv_qtensor* x,
+                          float* gw, void* ws, size_t ws_bytes, void* stream) {
+  return run_conv(MQV_OP_WGRAD, d, gy, "gy", x, "x", gw, ws, ws_bytes, stream);
+}
+
+mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
+                          float* gx, void* ws, size_t ws_bytes, void* stream) {
+  return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", gx, ws, ws_bytes, stream);
+}
+
+mqv_status mqv_device_errors(uint32_t* flags, void* stream) {
+  if (!flags) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  const uint32_t zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  *flags = v;
+  if (v) return fail(MQV_ERR_TIMEOUT, "device wait timed out (flags 0x%x)", v);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,270 @@
+// Quantize-once kernel pair: a global max|x| reduction, then the per-4x4
+// square-block two-level quantizer (MicroQonv summary, onedev.kr/papers/182,
+// section "무엇과 다른가": T_scale = max|X| / (max B_sf × max B_ef),
+// B_scale = CastE4M3(max|X_i| / (T_scale × max B_ef)),
+// X_i^q = Round(X_i / (B_scale × T_scale)); RNE for activations and weights,
+// stochastic rounding for gradients; NVFP6 = E2M3 elements, section
+// "어떻게 쓰나").  Every scale step is one IEEE fp32 operation in the order
+// the formula is written; divisions are correctly rounded (__fdiv_rn).
+#pragma once
+
+#include <cstdint>
+
+#include "mqv_ptx.cuh"
+
+namespace mqv {
+
+constexpr int kAmaxThreads = 256;
+constexpr int kQuantThreads = 256;
+
+// ---------------------------------------------------------------- Philox
+// Philox4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64-bit
+// multiplies with the round keys bumped by the Weyl constants.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// ------------------------------------------------- element rounding (a >= 0)
+// Each element grid is piecewise uniform: E2M1 steps 0.5 on [0,2), 1 on
+// [2,4), 2 on [4,6]; E2M3 steps 1/8 on [0,2), 1/4 on [2,4), 1/2 on [4,7.5].
+// Within a piece, magnitude code = piece base + (a - start)/step, and the
+// scaling by a power of two and the subtraction are exact, so rintf's
+// ties-to-even gives ties to the even code.
+template <int FMT>
+__device__ __forceinline__ uint32_t round_rne_mag(float a) {
+  if (FMT == 0) {
+    if (!(a <= 6.0f)) return 7u;
+    if (a < 2.0f) return static_cast<uint32_t>(rintf(a * 2.0f));
+    if (a < 4.0f) return 4u + static_cast<uint32_t>(rintf(a - 2.0f));
+    return 6u + static_cast<uint32_t>(rintf((a - 4.0f) * 0.5f));
+  } else {
+    if (!(a <= 7.5f)) return 31u;
+    if (a < 2.0f) return static_cast<uint32_t>(rintf(a * 8.0f));
+    if (a < 4.0f) return 16u + static_cast<uint32_t>(rintf((a - 2.0f) * 4.0f));
+    return 24u + static_cast<uint32_t>(rintf((a - 4.0f) * 2.0f));
+  }
+}
+
+// Stochastic rounding: q = position in units of the local step, round up
+// iff u < frac(q) (frac is exact: q is an exact rescaling of a).
+template <int FMT>
+__device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
+  float q;
+  uint32_t base;
+  if (FMT == 0) {
+    if (!(a < 6.0f)) return 7u;
+    if (a < 2.0f) { q = a * 2.0f; base = 0u; }
+    else if (a < 4.0f) { q = a - 2.0f; base = 4u; }
+    else { q = (a - 4.0f) * 0.5f; base = 6u; }
+  } else {
+    if (!(a < 7.5f)) return 31u;
+    if (a < 2.0f) { q = a * 8.0f; base = 0u; }
+    else if (a < 4.0f) { q = (a - 2.0f) * 4.0f; base = 16u; }
+    else { q = (a - 4.0f) * 2.0f; base = 24u; }
+  }
+  const float fl = floorf(q);
+  const float f = q - fl;
+  return base + static_cast<uint32_t>(fl) + (u < f ? 1u : 0u);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  return f16_lo_to_f32(e4m3x2_to_f16x2(code));
+}
+
+// ------------------------------------------------------------- amax
+// Pass 1: each CTA writes max|x| over its grid-stride share to partial[cta].
+__global__ void __launch_bounds__(kAmaxThreads)
+amax_partial_kernel(const float4* __restrict__ src, int64_t n4, float* __restrict__ partial) {
+  float m = 0.0f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kAmaxThreads;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * kAmaxThreads + threadIdx.x;
+  for (; i + 3 * stride < n4; i += 4 * stride) {
+    const float4 a = __ldg(src + i), b = __ldg(src + i + stride);
+    const float4 c = __ldg(src + i + 2 * stride), d = __ldg(src + i + 3 * stride);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(c.x), fabsf(c.y)), fmaxf(fabsf(c.z), fabsf(c.w))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(d.x), fabsf(d.y)), fmaxf(fabsf(d.z), fabsf(d.w))));
+  }
+  for (; i < n4; i += stride) {
+    const float4 a = __ldg(src + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float warp_max[kAmaxThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < kAmaxThreads / 32 ? warp_max[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) partial[blockIdx.x] = m;
+  }
+}
+
+// Block-wide max over `count` floats (every thread gets the result).
+__device__ __forceinline__ float block_max_of(const float* __restrict__ v, int count,
+                                              float* red /* >= 32 floats smem */) {
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < count; i += blockDim.x) m = fmaxf(m, v[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) red[0] = m;
+  }
+  __syncthreads();
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// Pass 1b (only for the split amax entry point): partials -> one float.
+__global__ void __launch_bounds__(kAmaxThreads)
+amax_finish_kernel(const float* __restrict__ partial, int count, float* __restrict__ amax) {
+  __shared__ float red[32];
+  const float m = block_max_of(partial, count, red);
+  if (threadIdx.x == 0) *amax = m;
+}
+
+// ----------------------------------------------------------- quantize
+// One thread per 4 x 4 block of the rows x cols view, consecutive threads on
+// consecutive column blocks (coalesced float4 reads of each of the 4 rows).
+// `amax_src` holds `amax_count` partial maxima; every CTA reduces them.
+template <int FMT, int RND>
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
+                const float* __restrict__ amax_src, int amax_count, uint64_t seed,
+                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                float* __restrict__ tscale) {
+  __shared__ float red[32];
+  const float amax = block_max_of(amax_src, amax_count, red);
+  const float emax = FMT == 0 ? 6.0f : 7.5f;
+  const float T = __fdiv_rn(amax, 448.0f * emax);         // 2688 or 3360, exact
+  const float Temax = __fmul_rn(T, emax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = T;
+
+  const int64_t cb = cols >> 2;
+  const int64_t nblocks = (rows >> 2) * cb;
+  const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
+  const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
+
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; b < nblocks;
+       b += stride) {
+    const int64_t br = b / cb, bc = b - br * cb;
+    const float* p = src + (br * 4) * cols + bc * 4;
+    float4 x[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) x[r] = __ldg(reinterpret_cast<const float4*>(p + r * cols));
+    float bmax = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[r].x), fabsf(x[r].y)),
+                               fmaxf(fabsf(x[r].z), fabsf(x[r].w))));
+    uint32_t scode = 0;
+    float d = 0.0f;
+    if (T > 0.0f) {
+      scode = f32_to_e4m3_satfinite(__fdiv_rn(bmax, Temax));
+      d = __fmul_rn(e4m3_to_f32(scode), T);
+    }
+    scales[b] = static_cast<uint8_t>(scode);
+
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float xv[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
+      float u[4] = {0.f, 0.f, 0.f, 0.f};
+      if (RND == 1) {
+        const uint64_t g = static_cast<uint64_t>((br * 4 + r) * cols + bc * 4) >> 2;
+        const uint4 w = philox4x32_10(
+            make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), k0, k1);
+        const float s24 = 5.9604644775390625e-08f;   // 2^-24
+        u[0] = __uint2float_rn(w.x >> 8) * s24;
+        u[1] = __uint2float_rn(w.y >> 8) * s24;
+        u[2] = __uint2float_rn(w.z >> 8) * s24;
+        u[3] = __uint2float_rn(w.w >> 8) * s24;
+      }
+      uint32_t packed = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t mag = 0;
+        if (d > 0.0f) {
+          const float v = __fdiv_rn(fabsf(xv[j]), d);
+          mag = RND == 0 ? round_rne_mag<FMT>(v) : round_sr_mag<FMT>(v, u[j]);
+        }
+        const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
+        const uint32_t code = FMT == 0 ? (mag | (sgn << 3)) : (mag | (sgn << 5));
+        packed |= code << (j * (FMT == 0 ? 4 : 6));
+      }
+      uint8_t* out = codes + (br * 4 + r) * row_bytes;
+      if (FMT == 0) {
+        *reinterpret_cast<uint16_t*>(out + bc * 2) = static_cast<uint16_t>(packed);
+      } else {
+        out += bc * 3;
+        out[0] = static_cast<uint8_t>(packed);
+        out[1] = static_cast<uint8_t>(packed >> 8);
+        out[2] = static_cast<uint8_t>(packed >> 16);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------- dequantize
+// dst = (code·B in fp16, exact) · T, one thread per 4 x 4 block.
+template <int FMT>
+__global__ void __launch_bounds__(kQuantThreads)
+dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                  const float* __restrict__ tscale, int64_t rows, int64_t cols,
+                  float* __restrict__ dst) {
+  const float T = *tscale;
+  const int64_t cb = cols >> 2;
+  const int64_t nblocks = (rows >> 2) * cb;
+  const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; b < nblocks;
+       b += stride) {
+    const int64_t br = b / cb, bc = b - br * cb;
+    const uint32_t s = scales[b];
+    const uint32_t s2 = e4m3x2_to_f16x2(s | (s << 8));
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint8_t* in = codes + (br * 4 + r) * row_bytes;
+      uint32_t h01, h23;
+      if (FMT == 0) {
+        const uint32_t q = *reinterpret_cast<const uint16_t*>(in + bc * 2);
+        h01 = e2m1x2_to_f16x2(q & 0xFF);
+        h23 = e2m1x2_to_f16x2(q >> 8);
+      } else {
+        in += bc * 3;
+        const uint32_t q = in[0] | (in[1] << 8) | (in[2] << 16);
+        h01 = e2m3x2_to_f16x2((q & 0x3F) | ((q << 2) & 0x3F00));
+        h23 = e2m3x2_to_f16x2(((q >> 12) & 0x3F) | ((q >> 10) & 0x3F00));
+      }
+      h01 = hmul2_u32(h01, s2);
+      h23 = hmul2_u32(h23, s2);
+      float4 o;
+      o.x = __fmul_rn(f16_lo_to_f32(h01), T);
+      o.y = __fmul_rn(f16_hi_to_f32(h01), T);
+      o.z = __fmul_rn(f16_lo_to_f32(h23), T);
+      o.w = __fmul_rn(f16_hi_to_f32(h23), T);
+      *reinterpret_cast<float4*>(dst + (br * 4 + r) * cols + bc * 4) = o;
+    }
+  }
+}
+
+}  // namespace mqv

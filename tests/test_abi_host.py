@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/mqv.h declares, sizes workspaces and codes, and
+rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import microscaling_quantized_convolution_b200 as mqv
+from microscaling_quantized_convolution_b200 import build as mqv_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mqv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mqv_build.build()
+    return mqv.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mqv_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ["mqv_quantize_cbf", "mqv_conv_fwd", "mqv_conv_wgrad", "mqv_conv_dgrad",
+                 "mqv_last_error", "mqv_qtensor_bytes", "mqv_conv_workspace_size"]:
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in mqv._SIGS, f"binding lacks {name}"
+
+
+def test_version_and_empty_error(lib):
+    assert lib.mqv_version() >= 100
+    assert isinstance(lib.mqv_last_error(), bytes)
+
+
+@pytest.mark.parametrize("rows,cols,fmt,codes,scales", [
+    (4, 4, mqv.NVFP4, 8, 1), (8, 16, mqv.NVFP4, 64, 8), (4, 4, mqv.NVFP6, 12, 1),
+    (28 * 28 * 128, 64, mqv.NVFP4, 28 * 28 * 128 * 32, 28 * 28 * 128 * 4),
+    (12, 84, mqv.NVFP6, 12 * 63, 3 * 21)])
+def test_qtensor_bytes(lib, rows, cols, fmt, codes, scales):
+    assert mqv.qtensor_bytes(rows, cols, fmt) == (codes, scales)
+
+
+@pytest.mark.parametrize("rows,cols", [(0, 4), (4, 0), (3, 4), (4, 6), (-4, 4)])
+def test_bad_views_rejected(lib, rows, cols):
+    with pytest.raises(mqv.MqvError) as e:
+        mqv.qtensor_bytes(rows, cols, mqv.NVFP4)
+    assert e.value.status == 1
+
+
+def test_bad_format_rejected(lib):
+    with pytest.raises(mqv.MqvError):
+        mqv.qtensor_bytes(4, 4, 7)
+
+
+def test_quantize_workspace_is_partial_maxima(lib):
+    assert mqv.quantize_workspace_bytes(4, 4) == 256
+    big = mqv.quantize_workspace_bytes(512 * 14 * 14, 10240)
+    assert big >= 4 * 148 and big % 256 == 0
+
+
+def _desc(**kw):
+    base = dict(N=64, Cin=128, Cout=128, H=28, W=28, Kh=3, Kw=3, stride=1, pad=1, fmt=mqv.NVFP4)
+    base.update(kw)
+    return mqv.conv_desc(**base)
+
+
+def test_conv_workspace_sizes(lib):
+    d = _desc()
+    assert mqv.conv_workspace_bytes(d, mqv.OP_FWD) == 0
+    assert mqv.conv_workspace_bytes(d, mqv.OP_DGRAD) == 0
+    ws = mqv.conv_workspace_bytes(d, mqv.OP_WGRAD)
+    assert ws > 0 and ws % (128 * 1152 * 4) == 0          # whole split partial tiles
+
+
+@pytest.mark.parametrize("kw", [dict(N=6), dict(Cin=3), dict(Cout=10), dict(stride=0),
+                                dict(pad=3), dict(H=1, pad=0), dict(fmt=5), dict(Kh=0)])
+def test_bad_conv_desc_rejected(lib, kw):
+    with pytest.raises(mqv.MqvError) as e:
+        mqv.conv_workspace_bytes(_desc(**kw), mqv.OP_FWD)
+    assert e.value.status in (1, 2)
+
+
+def test_conv_rejects_null_and_mismatched_operands(lib):
+    d = _desc()
+    w = mqv.QTensorC(16, 16, 16, 128, 1152, 0, 0)
+    x = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, 0)
+    bad = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 32, 0, 0)     # wrong N
+    st = lib.mqv_conv_fwd(ctypes.byref(d), ctypes.byref(w), ctypes.byref(bad), 16, None, 0, None)
+    assert st == 1 and b"x" in lib.mqv_last_error()
+    st = lib.mqv_conv_fwd(ctypes.byref(d), None, ctypes.byref(x), 16, None, 0, None)
+    assert st == 1
+    st = lib.mqv_conv_fwd(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 8, None, 0, None)
+    assert st == 1                                              # misaligned output
+    gy = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, 0)
+    st = lib.mqv_conv_wgrad(ctypes.byref(d), ctypes.byref(gy), ctypes.byref(x), 16, None, 0, None)
+    assert st == 3                                              # needs split workspace
+    wfp6 = mqv.QTensorC(16, 16, 16, 128, 1152, 1, 0)
+    st = lib.mqv_conv_dgrad(ctypes.byref(d), ctypes.byref(wfp6), ctypes.byref(gy), 16, None, 0, None)
+    assert st == 1                                              # format mismatch
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    q = mqv.QTensorC(16, 16, 16, 8, 8, 0, 0)
+    st = lib.mqv_quantize_cbf(None, 8, 8, 0, 0, 0, ctypes.byref(q), 16, 256, None)
+    assert st == 1
+    st = lib.mqv_quantize_cbf(16, 8, 8, 0, 2, 0, ctypes.byref(q), 16, 256, None)
+    assert st == 1                                              # rounding mode
+    st = lib.mqv_quantize_cbf(16, 8, 8, 1, 0, 0, ctypes.byref(q), 16, 256, None)
+    assert st == 1                                              # out fmt differs
+    st = lib.mqv_quantize_cbf(16, 8, 8, 0, 0, 0, ctypes.byref(q), None, 0, None)
+    assert st == 3                                              # workspace
+    st = lib.mqv_quantize_cbf(4, 8, 8, 0, 0, 0, ctypes.byref(q), 16, 256, None)
+    assert st == 1                                              # misaligned src
+
+
+def test_cuda_path_has_no_cpu_fallback():
+    import torch
+    x = torch.zeros(16)
+    with pytest.raises(ValueError):
+        mqv.quantize(x, 4, 4, "nvfp4")

@@ -1,0 +1,185 @@
+"""GPU parity of the three implicit-GEMM conv passes against the oracle.
+
+Small shapes (several tiles, ragged in every GEMM dimension) are compared
+element by element; full-size layers of the benchmarked workloads are
+compared on sampled outputs that the oracle computes one by one.  Both sides
+quantize the same seeded fp32 inputs themselves.  Tolerance per output:
+|y - y_ref| <= 1e-5·S + 1e-7 with S = T_a·T_b·sum_k |a_k·b_k|."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import microscaling_quantized_convolution_b200 as mqv
+import workloads
+from oracle import mqv_oracle as O
+from tests.parity_utils import FMT, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu_layer(X, Wt, G, s: O.ConvShape, fmt, seed):
+    d = mqv.conv_desc(s.N, s.Cin, s.Cout, s.H, s.W, s.Kh, s.Kw, s.stride, s.pad, fmt)
+    qx = mqv.quantize(X.cuda().view(-1), *s.x_view(), fmt, mqv.RNE)
+    qw = mqv.quantize(Wt.cuda().view(-1), *s.w_view(), fmt, mqv.RNE)
+    qg = mqv.quantize(G.cuda().view(-1), *s.gy_view(), fmt, mqv.SR, seed)
+    y = mqv.conv_fwd(d, qw, qx)
+    gw = mqv.conv_wgrad(d, qg, qx)
+    gx = mqv.conv_dgrad(d, qw, qg)
+    assert mqv.device_errors() == 0
+    return (qx, qw, qg), y.cpu().numpy(), gw.cpu().numpy(), gx.cpu().numpy()
+
+
+def make_inputs(s: O.ConvShape, seed):
+    g = torch.Generator().manual_seed(seed)
+    X = torch.relu(torch.randn((s.H, s.W, s.Cin, s.N), generator=g))
+    Wt = torch.randn((s.Cout, s.Kh, s.Kw, s.Cin), generator=g) * (2.0 / (s.Cin * s.Kh * s.Kw)) ** 0.5
+    G = torch.randn((s.Ho, s.Wo, s.Cout, s.N), generator=g) * 1e-3
+    return X, Wt, G
+
+
+SMALL = [
+    ("tiny_3x3_s1_p0", O.ConvShape(4, 16, 16, 8, 8, 3, 3, 1, 0), "nvfp4"),
+    ("ragged_3x3_s1_p1", O.ConvShape(8, 24, 40, 9, 9, 3, 3, 1, 1), "nvfp4"),
+    ("ragged_3x3_s2_p1", O.ConvShape(8, 24, 40, 9, 9, 3, 3, 2, 1), "nvfp4"),
+    ("pointwise_fp6", O.ConvShape(16, 32, 48, 10, 10, 1, 1, 1, 0), "nvfp6"),
+    ("cin4_3x3_s2_fp6", O.ConvShape(4, 4, 16, 12, 12, 3, 3, 2, 1), "nvfp6"),
+    ("rect_3x2_p1", O.ConvShape(4, 8, 12, 7, 6, 3, 2, 1, 1), "nvfp4"),
+    ("two_m_tiles", O.ConvShape(4, 16, 136, 6, 6, 3, 3, 1, 1), "nvfp4"),
+    ("n12_c8", O.ConvShape(12, 8, 8, 5, 5, 3, 3, 1, 1), "nvfp6"),
+    ("wide_k_s2_p2", O.ConvShape(4, 72, 68, 11, 11, 5, 5, 2, 2), "nvfp4"),
+    ("deep_cin", O.ConvShape(8, 256, 32, 4, 4, 3, 3, 1, 1), "nvfp4"),
+]
+
+
+@pytest.mark.parametrize("name,s,fmt", SMALL, ids=[c[0] for c in SMALL])
+def test_small_layers_elementwise(name, s, fmt):
+    X, Wt, G = make_inputs(s, zlib.crc32(name.encode()) % 1000)
+    seed = 77
+    _, y, gw, gx = run_gpu_layer(X, Wt, G, s, fmt, seed)
+    qx, qw, qg = O.quantize_layer(X.numpy(), Wt.numpy(), G.numpy(), s, FMT[fmt], seed)
+    ref = O.layer_outputs(qx, qw, qg, s)
+    assert_close(y, *ref["y"], f"{name} fwd")
+    assert_close(gw, *ref["gw"], f"{name} wgrad")
+    assert_close(gx, *ref["gx"], f"{name} dgrad")
+
+
+def test_outputs_not_trivially_zero():
+    s = SMALL[1][1]
+    X, Wt, G = make_inputs(s, 1)
+    _, y, gw, gx = run_gpu_layer(X, Wt, G, s, "nvfp4", 5)
+    assert np.count_nonzero(y) > 0.9 * y.size and np.count_nonzero(gx) > 0.5 * gx.size
+    assert np.count_nonzero(gw) > 0.9 * gw.size
+
+
+def test_repeat_calls_are_deterministic():
+    s = O.ConvShape(16, 64, 64, 14, 14, 3, 3, 1, 1)
+    X, Wt, G = make_inputs(s, 2)
+    a = run_gpu_layer(X, Wt, G, s, "nvfp4", 3)
+    b = run_gpu_layer(X, Wt, G, s, "nvfp4", 3)
+    for u, v in zip(a[1:], b[1:]):
+        assert np.array_equal(u, v)
+
+
+# ------------------------------------------------------- full-size sampling
+
+class BandOracle:
+    """Oracle code values of single pixels of a big [H][W][C][N] tensor,
+    quantized band by band with the tensor's global amax and global SR
+    counter (so each band equals the same rows of a full quantization)."""
+
+    def __init__(self, t: np.ndarray, fmt, rnd, seed):
+        self.t, self.fmt, self.rnd, self.seed = t, fmt, rnd, seed
+        self.H, self.W, self.C, self.N = t.shape
+        self.amax = float(np.max(np.abs(t)))
+        self.T = np.float32(np.float32(self.amax) / np.float32(O.E4M3_MAX * O.element_max(fmt)))
+        self.cache = {}
+
+    def pix(self, h, w):
+        key = (h, w)
+        if key not in self.cache:
+            band = self.t[h, w].reshape(self.C, self.N)
+            q = O.quantize(band, self.fmt, self.rnd, self.seed, amax=self.amax,
+                           row_offset=(h * self.W + w) * self.C)
+            self.cache[key] = O.code_values(q)
+        return self.cache[key]
+
+
+def sampled_check(layer: workloads.Layer, nsamp=96, full_wgrad=False):
+    s = O.ConvShape(layer.N, layer.Cin, layer.Cout, layer.H, layer.W, layer.K, layer.K,
+                    layer.stride, layer.pad)
+    fmt = layer.fmt
+    seed = workloads.sr_seed(layer)
+    X, Wt, G = workloads.make_layer_inputs(layer)
+    (qx, qw, qg), y, gw, gx = run_gpu_layer(X, Wt, G, s, fmt, seed)
+    of = FMT[fmt]
+    oq_w = O.quantize(Wt.numpy().reshape(s.w_view()), of, O.RNE)
+    Wcv = O.code_values(oq_w).reshape(s.Cout, s.Kh, s.Kw, s.Cin)
+    bx = BandOracle(X.numpy(), of, O.RNE, 0)
+    bg = BandOracle(G.numpy(), of, O.SR, seed)
+    Tw, Tx, Tg = np.float64(oq_w.T), np.float64(bx.T), np.float64(bg.T)
+    assert np.float32(qx.tscale.item()) == bx.T and np.float32(qg.tscale.item()) == bg.T
+    rng = np.random.default_rng(layer.seed)
+    y = y.reshape(s.Ho, s.Wo, s.Cout, s.N)
+    gx = gx.reshape(s.H, s.W, s.Cin, s.N)
+    got, ref, S = [], [], []
+    for _ in range(nsamp):                                  # forward samples
+        ho, wo, co, n = (int(rng.integers(d)) for d in (s.Ho, s.Wo, s.Cout, s.N))
+        acc = sacc = 0.0
+        for kh in range(s.Kh):
+            for kw in range(s.Kw):
+                hi, wi = ho * s.stride + kh - s.pad, wo * s.stride + kw - s.pad
+                if 0 <= hi < s.H and 0 <= wi < s.W:
+                    p = Wcv[co, kh, kw, :] * bx.pix(hi, wi)[:, n]
+                    acc += p.sum()
+                    sacc += np.abs(p).sum()
+        got.append(y[ho, wo, co, n]); ref.append(acc * Tw * Tx); S.append(sacc * Tw * Tx)
+    assert_close(np.array(got), np.array(ref), np.array(S), f"{layer.name} fwd sampled")
+    got, ref, S = [], [], []
+    for _ in range(nsamp):                                  # input-gradient samples
+        hi, wi, ci, n = (int(rng.integers(d)) for d in (s.H, s.W, s.Cin, s.N))
+        acc = sacc = 0.0
+        for kh in range(s.Kh):
+            th = hi + s.pad - kh
+            if th < 0 or th % s.stride or th // s.stride >= s.Ho:
+                continue
+            for kw in range(s.Kw):
+                tw = wi + s.pad - kw
+                if tw < 0 or tw % s.stride or tw // s.stride >= s.Wo:
+                    continue
+                p = Wcv[:, kh, kw, ci] * bg.pix(th // s.stride, tw // s.stride)[:, n]
+                acc += p.sum()
+                sacc += np.abs(p).sum()
+        got.append(gx[hi, wi, ci, n]); ref.append(acc * Tw * Tg); S.append(sacc * Tw * Tg)
+    assert_close(np.array(got), np.array(ref), np.array(S), f"{layer.name} dgrad sampled")
+    if full_wgrad:                                          # weight-gradient samples
+        Xcv = O.code_values(O.quantize(X.numpy().reshape(s.x_view()), of, O.RNE)).reshape(X.shape)
+        Gcv = O.code_values(O.quantize(G.numpy().reshape(s.gy_view()), of, O.SR, seed)).reshape(G.shape)
+        gw = gw.reshape(s.Cout, s.Kh, s.Kw, s.Cin)
+        got, ref, S = [], [], []
+        for _ in range(max(16, nsamp // 4)):
+            co, kh, kw, ci = (int(rng.integers(d)) for d in (s.Cout, s.Kh, s.Kw, s.Cin))
+            v, sa = O.wgrad_at(Gcv, Xcv, s, co, kh, kw, ci)
+            got.append(gw[co, kh, kw, ci]); ref.append(v * Tg * Tx); S.append(sa * Tg * Tx)
+        assert_close(np.array(got), np.array(ref), np.array(S), f"{layer.name} wgrad sampled")
+
+
+def test_resnet18_layer2_full_size_sampled():
+    sampled_check(workloads.resnet18_layer2(), nsamp=128, full_wgrad=True)
+
+
+BODY = workloads.resnet18_body()
+
+
+@pytest.mark.parametrize("layer", BODY, ids=[l.name for l in BODY])
+def test_resnet18_body_full_size_sampled(layer):
+    sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (4, 8, 15))
+
+
+YOLO = workloads.yolov8n_mix()
+
+
+@pytest.mark.parametrize("layer", YOLO, ids=[l.name for l in YOLO])
+def test_yolov8n_full_size_sampled(layer):
+    sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (3, 6, 17))

@@ -1,0 +1,164 @@
+"""GPU parity of the quantize-once kernels against the oracle: packed codes,
+E4M3 scales and the tensor scale must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import microscaling_quantized_convolution_b200 as mqv
+import workloads
+from oracle import mqv_oracle as O
+from tests.parity_utils import FMT, assert_quant_equal, gpu_quantize
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand(shape, seed, signed=True, scale=1.0, outliers=False):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(shape, generator=g) * scale
+    if not signed:
+        x = x.abs()
+    if outliers:
+        k = max(1, x.numel() // 1000)
+        idx = torch.randint(0, x.numel(), (k,), generator=g)
+        x.view(-1)[idx] *= 100
+    return x
+
+
+SHAPES = [(4, 4), (8, 84), (16, 64), (6 * 6 * 16, 4), (128, 1152), (7 * 7 * 64, 32), (400, 20)]
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+@pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_quantize_bit_exact(fmt, rnd, shape):
+    rows, cols = shape
+    for i, kw in enumerate([dict(), dict(signed=False), dict(outliers=True), dict(scale=1e-30)]):
+        x = _rand(shape, 10 + i, **kw)
+        q, c, s, T = gpu_quantize(x, rows, cols, fmt, rnd, seed=1234 + i)
+        assert_quant_equal(x.numpy(), rows, cols, fmt, rnd, 1234 + i, (c, s, T))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+def test_layer_tensors_bit_exact(fmt):
+    """X, W and G_Y of the tiny layer and the ResNet-18 layer2-shaped layer."""
+    for layer in (workloads.tiny_layer(), workloads.resnet18_layer2()):
+        X, Wt, G = workloads.make_layer_inputs(layer)
+        s = layer
+        for t, (r, c), rnd, seed in [(X, (s.H * s.W * s.Cin, s.N), mqv.RNE, 0),
+                                     (Wt, (s.Cout, s.K * s.K * s.Cin), mqv.RNE, 0),
+                                     (G, (s.Ho * s.Wo * s.Cout, s.N), mqv.SR, workloads.sr_seed(s))]:
+            q, cb, sb, T = gpu_quantize(t, r, c, fmt, rnd, seed)
+            assert_quant_equal(t.numpy(), r, c, fmt, rnd, seed, (cb, sb, T))
+
+
+def _tie_tensor(fmt, seed):
+    """T = 1 exactly (amax = 448·emax), then blocks whose max is emax·m for
+    chosen m (so B = CastE4M3(m)) and elements drawn from every tie point,
+    grid point and their fp32 neighbours."""
+    rng = np.random.default_rng(seed)
+    emax = O.element_max(FMT[fmt])
+    grid = O.element_grid(FMT[fmt])
+    mids = (grid[:-1] + grid[1:]) / 2
+    cand = np.concatenate([grid, mids, np.nextafter(mids.astype(np.float32), 0),
+                           np.nextafter(mids.astype(np.float32), 100)]).astype(np.float32)
+    e4 = O.E4M3_GRID
+    e4mids = ((e4[:-1] + e4[1:]) / 2).astype(np.float32)
+    ms = np.concatenate([e4[1:], e4mids, np.nextafter(e4mids, 0), np.nextafter(e4mids, 1000),
+                         rng.uniform(0.001, 448, 200)]).astype(np.float32)
+    nblocks = len(ms) + 512
+    x = np.zeros((4 * nblocks, 4), np.float32)
+    x[0, 0] = np.float32(448.0 * emax)
+    for b in range(1, nblocks):
+        blk = rng.choice(cand, size=16).astype(np.float32) * rng.choice([-1, 1], size=16)
+        if b <= len(ms):                       # scale-rounding block: max = emax·m
+            blk = (blk / emax * ms[b - 1]).astype(np.float32)
+            blk[rng.integers(16)] = np.float32(emax) * ms[b - 1]
+        else:                                  # element-rounding block: B = 1
+            blk[rng.integers(16)] = np.float32(emax)
+        x[4 * b:4 * b + 4] = blk.reshape(4, 4)
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+@pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
+def test_rounding_ties_bit_exact(fmt, rnd):
+    x = _tie_tensor(fmt, 3)
+    rows, cols = x.shape
+    q, c, s, T = gpu_quantize(torch.from_numpy(x), rows, cols, fmt, rnd, seed=99)
+    assert T == 1.0
+    assert_quant_equal(x, rows, cols, fmt, rnd, 99, (c, s, T))
+
+
+def test_zero_tensor_and_negative_zero():
+    x = torch.zeros(16, 8)
+    x[1, 1] = -0.0
+    for fmt in ("nvfp4", "nvfp6"):
+        q, c, s, T = gpu_quantize(x, 16, 8, fmt, mqv.RNE)
+        assert T == 0.0 and not s.any()
+        assert_quant_equal(x.numpy(), 16, 8, fmt, mqv.RNE, 0, (c, s, T))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+def test_dequantize_enumerates_every_code_and_scale(fmt):
+    """Every (code, E4M3 scale) product decoded on the GPU equals the
+    oracle's exact value: code·B (and the fp32 product with T)."""
+    nbits = 4 if fmt == "nvfp4" else 6
+    ncodes = 1 << nbits
+    cols = ncodes                     # one view row holds every code once
+    rows = 4 * 127                    # one block row per finite scale code
+    codes = np.tile(np.arange(ncodes), (rows, 1))
+    scales = np.repeat(np.arange(127, dtype=np.uint8)[:, None], cols // 4, axis=1)
+    for T in (1.0, 0.1234567):
+        q = mqv.QTensor.empty(rows, cols, fmt)
+        q.codes.copy_(torch.from_numpy(O.pack_codes(codes, FMT[fmt])))
+        q.scales.copy_(torch.from_numpy(scales.reshape(-1)))
+        q.tscale.fill_(T)
+        got = mqv.dequantize(q).cpu().numpy().reshape(rows, cols)
+        oq = O.QTensor(codes.astype(np.int64), scales, np.float32(T), FMT[fmt])
+        ref = (O.code_values(oq) * np.float64(np.float32(T))).astype(np.float32)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_split_amax_path_matches_fused():
+    x = _rand((28 * 28 * 32, 64), 5, outliers=True)
+    xd = x.cuda().view(-1)
+    a = mqv.amax(xd, *x.shape)
+    assert a.item() == float(x.abs().max())
+    q1 = mqv.quantize(xd, *x.shape, "nvfp4", mqv.SR, 7)
+    q2 = mqv.quantize_with_amax(xd, *x.shape, "nvfp4", mqv.SR, 7, a)
+    torch.cuda.synchronize()
+    for f in ("codes", "scales", "tscale"):
+        assert torch.equal(getattr(q1, f), getattr(q2, f))
+
+
+@pytest.mark.parametrize("C,H,N,signed,outliers,rnd", [
+    (256, 7, 84, False, False, mqv.RNE), (512, 7, 256, True, True, mqv.SR),
+    (512, 14, 256, False, True, mqv.RNE)])
+def test_replay_shapes_full_tensor(C, H, N, signed, outliers, rnd):
+    x = workloads.make_replay_input(C, H, N, signed=signed, outliers=outliers, seed=1)
+    rows, cols = H * H * C, N
+    q, c, s, T = gpu_quantize(x, rows, cols, "nvfp4", rnd, seed=17)
+    assert_quant_equal(x.numpy(), rows, cols, "nvfp4", rnd, 17, (c, s, T))
+
+
+@pytest.mark.parametrize("C,H,N,rnd", [(512, 14, 2560, mqv.SR), (512, 14, 10240, mqv.RNE)])
+def test_replay_shapes_large_sampled_bands(C, H, N, rnd):
+    """1/4-G-element and 1-G-element replay buffers: every tensor scale bit,
+    then code/scale bytes of 6 row bands (checked against the oracle with the
+    global amax and the global SR counter), in the launch the bench times."""
+    rows, cols = H * H * C, N
+    x = workloads.make_replay_input(C, H, N, outliers=True, seed=2, device="cuda").view(-1)
+    q = mqv.quantize(x, rows, cols, "nvfp4", rnd, 23)
+    torch.cuda.synchronize()
+    amax = float(x.abs().max())
+    rng = np.random.default_rng(0)
+    T = q.tscale.item()
+    rb = cols // 2
+    for band in [0, rows - 8] + list(4 * rng.integers(0, rows // 4 - 2, 4)):
+        band = int(band)
+        xb = x[band * cols:(band + 8) * cols].cpu().numpy().reshape(8, cols)
+        cb = q.codes[band * rb:(band + 8) * rb].cpu().numpy()
+        sb = q.scales[band // 4 * (cols // 4):(band // 4 + 2) * (cols // 4)].cpu().numpy()
+        assert_quant_equal(xb, 8, cols, "nvfp4", rnd, 23, (cb, sb, T), amax=amax, row_offset=band)
+    del x, q
+    torch.cuda.empty_cache()
