@@ -1,0 +1,429 @@
+"""Benchmark of the quantize-once convolution hot path on B200.
+
+One step = one pass of the whole path for one conv layer: quantize X and W
+(round-to-nearest-even) and G_Y (Philox stochastic rounding) into square-block
+NVFP4/NVFP6 form, then the implicit-GEMM forward, weight-gradient and
+input-gradient passes.  `value` is conv TFLOP/s (fwd + wgrad + dgrad FLOPs of
+all ranks / device time of the timed steps, max over ranks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, bounded sample
+
+Under torchrun (N > 1) each rank runs its own batch of the same layer (weak
+scaling, data parallel): the per-tensor max|x| of X and G_Y is MAX-all-reduced
+before quantizing (so every rank uses the global tensor scale) and G_W is
+SUM-all-reduced after the weight-gradient pass, both over NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "quantize GB/s and conv fwd+wgrad+dgrad TFLOP/s at 1 B200, as fraction of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pick_layer(name: str) -> workloads.Layer:
+    table = {l.name: l for l in [workloads.tiny_layer(), workloads.resnet18_layer2()]
+             + workloads.resnet18_body() + workloads.yolov8n_mix()}
+    if name not in table:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
+    return table[name]
+
+
+def layer_bytes(layer: workloads.Layer):
+    """Algorithmic bytes: quantize = 2 fp32 reads + codes + scales written;
+    conv pass = both quantized operands read once + fp32 output written once."""
+    eb = 0.5 if layer.fmt == "nvfp4" else 0.75
+    qb = eb + 1.0 / 16
+    x = layer.H * layer.W * layer.Cin * layer.N
+    w = layer.Cout * layer.K * layer.K * layer.Cin
+    g = layer.Ho * layer.Wo * layer.Cout * layer.N
+    quant = {"x": x * (8 + qb), "w": w * (8 + qb), "g": g * (8 + qb)}
+    conv = {"fwd": (w + x) * qb + g * 4, "wgrad": (g + x) * qb + w * 4, "dgrad": (w + g) * qb + x * 4}
+    return quant, conv, (x, w, g)
+
+
+class Clocks:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    mqv.lib()
+
+    layer = pick_layer(args.workload)
+    fmt = layer.fmt
+    d = mqv.conv_desc(**layer.dims(), fmt=fmt)
+    Ho, Wo = layer.Ho, layer.Wo
+    xr, xc = layer.H * layer.W * layer.Cin, layer.N
+    wr, wc = layer.Cout, layer.K * layer.K * layer.Cin
+    gr, gc = Ho * Wo * layer.Cout, layer.N
+    dev = torch.device("cuda", local)
+
+    # Inputs resident in HBM, rotated over enough sets to exceed the 126 MB L2
+    quant_b, conv_b, (nx, nw, ng) = layer_bytes(layer)
+    per_set = 4 * (nx + nw + ng) + 4 * (nx + nw + ng)        # fp32 inputs + outputs
+    nsets = max(2, min(16, -(-400_000_000 // per_set)))
+    sets = []
+    for i in range(nsets):
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 * rank + i)
+        X = torch.randn((layer.H, layer.W, layer.Cin, layer.N), generator=g, device=dev)
+        X = torch.relu(X) if layer.x_dist == "relu" else (torch.nn.functional.silu(X) if layer.x_dist == "silu" else X)
+        Wt = torch.randn((layer.Cout, layer.K, layer.K, layer.Cin), generator=g, device=dev) * (2.0 / wc) ** 0.5
+        G = torch.randn((Ho, Wo, layer.Cout, layer.N), generator=g, device=dev) * layer.gy_std
+        sets.append(dict(X=X.view(-1), W=Wt.view(-1), G=G.view(-1),
+                         qx=mqv.QTensor.empty(xr, xc, fmt, dev), qw=mqv.QTensor.empty(wr, wc, fmt, dev),
+                         qg=mqv.QTensor.empty(gr, gc, fmt, dev),
+                         y=torch.empty(Ho * Wo * layer.Cout * layer.N, device=dev),
+                         gw=torch.empty(wr * wc, device=dev),
+                         gx=torch.empty(xr * xc, device=dev)))
+    ws_q = [torch.empty(mqv.quantize_workspace_bytes(r, c), dtype=torch.uint8, device=dev)
+            for r, c in ((xr, xc), (wr, wc), (gr, gc))]
+    ws_w = mqv.conv_workspace_bytes(d, mqv.OP_WGRAD)
+    ws_wgrad = torch.empty(max(ws_w, 16), dtype=torch.uint8, device=dev)
+    amax_buf = torch.empty(3, dtype=torch.float32, device=dev)
+    seed = workloads.sr_seed(layer)
+    splits_reduce = 1 if ws_w > 0 else 0
+
+    def quantize_all(s, step):
+        if world == 1:
+            mqv.quantize(s["X"], xr, xc, fmt, mqv.RNE, 0, out=s["qx"], ws=ws_q[0])
+            mqv.quantize(s["W"], wr, wc, fmt, mqv.RNE, 0, out=s["qw"], ws=ws_q[1])
+            mqv.quantize(s["G"], gr, gc, fmt, mqv.SR, seed + step, out=s["qg"], ws=ws_q[2])
+        else:
+            mqv.amax(s["X"], xr, xc, out=amax_buf[0:1], ws=ws_q[0])
+            mqv.amax(s["G"], gr, gc, out=amax_buf[2:3], ws=ws_q[2])
+            dist.all_reduce(amax_buf, op=dist.ReduceOp.MAX)
+            mqv.quantize_with_amax(s["X"], xr, xc, fmt, mqv.RNE, 0, amax_buf[0:1], out=s["qx"])
+            mqv.quantize(s["W"], wr, wc, fmt, mqv.RNE, 0, out=s["qw"], ws=ws_q[1])
+            mqv.quantize_with_amax(s["G"], gr, gc, fmt, mqv.SR, seed + step, amax_buf[2:3], out=s["qg"])
+
+    def step(i, ev=None):
+        s = sets[i % nsets]
+        if ev is not None:
+            ev[0].record()
+        quantize_all(s, i)
+        if ev is not None:
+            ev[1].record()
+        mqv.conv_fwd(d, s["qw"], s["qx"], y=s["y"])
+        if ev is not None:
+            ev[2].record()
+        mqv.conv_wgrad(d, s["qg"], s["qx"], gw=s["gw"], ws=ws_wgrad)
+        if world > 1:
+            dist.all_reduce(s["gw"])
+        if ev is not None:
+            ev[3].record()
+        mqv.conv_dgrad(d, s["qw"], s["qg"], gx=s["gx"])
+        if ev is not None:
+            ev[4].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    flags = mqv.device_errors()
+    if flags:
+        raise SystemExit(f"device wait timeout flags {flags:#x}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.15)
+    t0.record()
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    parts = {"quantize": [], "fwd": [], "wgrad": [], "dgrad": []}
+    for e in evs:
+        parts["quantize"].append(e[0].elapsed_time(e[1]))
+        parts["fwd"].append(e[1].elapsed_time(e[2]))
+        parts["wgrad"].append(e[2].elapsed_time(e[3]))
+        parts["dgrad"].append(e[3].elapsed_time(e[4]))
+    mean = {k: sum(v) / len(v) for k, v in parts.items()}
+    if world > 1:
+        t = torch.tensor([total_ms] + [mean[k] for k in parts], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t[0].item()
+        mean = {k: t[1 + j].item() for j, k in enumerate(parts)}
+    flags = mqv.device_errors()
+
+    # end-to-end through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hX = sets[0]["X"].cpu().pin_memory(); hW = sets[0]["W"].cpu().pin_memory()
+        hG = sets[0]["G"].cpu().pin_memory()
+        hy = torch.empty(sets[0]["y"].numel()).pin_memory()
+        hgw = torch.empty(sets[0]["gw"].numel()).pin_memory()
+        hgx = torch.empty(sets[0]["gx"].numel()).pin_memory()
+        s = sets[0]
+        def e2e_step(i):
+            s["X"].copy_(hX, non_blocking=True); s["W"].copy_(hW, non_blocking=True)
+            s["G"].copy_(hG, non_blocking=True)
+            step(i)
+            hy.copy_(s["y"], non_blocking=True); hgw.copy_(s["gw"], non_blocking=True)
+            hgx.copy_(s["gx"], non_blocking=True)
+        for i in range(3):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        h2d = 4 * (nx + nw + ng)
+        e2e = {"value": round(3 * layer.flops() * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d, "ms_per_step": round(e2e_ms, 4)}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    flops = layer.flops()
+    ms_step = total_ms / args.steps
+    value = 3 * flops * world / (ms_step * 1e-3) / 1e12
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops"]              # f16 and bf16 dense MMA have the same nominal rate
+    kern = {}
+    for name in ("fwd", "wgrad", "dgrad"):
+        t = mean[name] * 1e-3
+        tflops = flops / t / 1e12
+        gbs = conv_b[name] / t / 1e9
+        roof_t = max(flops / (tc * 1e12), conv_b[name] / (hbm * 1e9))
+        bound = "tensor" if flops / (tc * 1e12) >= conv_b[name] / (hbm * 1e9) else "hbm"
+        kern[name] = {"ms": round(mean[name], 5), "tflops": round(tflops, 2), "gbs": round(gbs, 1),
+                      "bound": bound, "frac_of_roofline": round(roof_t / t, 4)}
+    qbytes = sum(quant_b.values())
+    qt = mean["quantize"] * 1e-3
+    kern["quantize"] = {"ms": round(mean["quantize"], 5), "gbs": round(qbytes / qt / 1e9, 1),
+                        "bound": "hbm", "frac_of_roofline": round(qbytes / qt / 1e9 / hbm, 4),
+                        "launches": 6 if world == 1 else 8}
+    dom = max(("fwd", "wgrad", "dgrad", "quantize"), key=lambda k: mean[k])
+    if dom == "quantize":
+        roof = {"kernel": "quantize (amax + block quantizer, X, W, G_Y)", "bound": "hbm",
+                "achieved": kern["quantize"]["gbs"], "peak": hbm, "unit": "GB/s",
+                "frac": round(kern["quantize"]["gbs"] / hbm, 4)}
+    else:
+        k = kern[dom]
+        if k["bound"] == "tensor":
+            roof = {"kernel": f"conv_{dom}", "bound": "tensor", "achieved": k["tflops"], "peak": tc,
+                    "unit": "TFLOP/s", "frac": round(k["tflops"] / tc, 4)}
+        else:
+            roof = {"kernel": f"conv_{dom}", "bound": "hbm", "achieved": k["gbs"], "peak": hbm,
+                    "unit": "GB/s", "frac": round(k["gbs"] / hbm, 4)}
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json burst' if peak_src == 'measured' else 'recipe fallback'})"
+    roof["traffic"] = args.traffic.get(roof["kernel"]) if args.traffic else None
+    launches_per_step = (3 + 3 if world == 1 else 4 + 2 + 2) + 3 + splits_reduce
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic",
+        "config": {"workload": layer.name, "N": layer.N, "Cin": layer.Cin, "Cout": layer.Cout,
+                   "H": layer.H, "W": layer.W, "K": layer.K, "stride": layer.stride, "pad": layer.pad,
+                   "storage": f"{layer.fmt} (4x4 blocks, e4m3 block scales, fp32 tensor scale)",
+                   "step": "quantize X,W (RNE) and G_Y (SR); conv fwd, wgrad, dgrad",
+                   "l2": f"inputs rotated over {nsets} resident sets ({nsets * per_set / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "quantize_gbs": kern["quantize"]["gbs"],
+        "kernels": kern,
+        "roofline": roof,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "device_error_flags": flags,
+    }
+    if e2e:
+        out["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(layer, budget_s=args.cpu_budget)
+    print(json.dumps(out), flush=True)
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_sample_layer(layer: workloads.Layer, n_batch: int, hw: int) -> workloads.Layer:
+    """The same layer with the batch cut to n_batch and the input to hw x hw."""
+    return workloads.Layer(layer.name + f"_sample_n{n_batch}_{hw}px", n_batch, layer.Cin, layer.Cout,
+                           hw, hw, layer.K, layer.stride, layer.pad, layer.fmt, layer.x_dist,
+                           layer.gy_std, layer.seed, layer.cin_real)
+
+
+def oracle_step(sample: workloads.Layer):
+    from oracle import mqv_oracle as O
+    X, Wt, G = workloads.make_layer_inputs(sample)
+    s = O.ConvShape(sample.N, sample.Cin, sample.Cout, sample.H, sample.W, sample.K, sample.K,
+                    sample.stride, sample.pad)
+    f = O.FP4 if sample.fmt == "nvfp4" else O.FP6
+    qx, qw, qg = O.quantize_layer(X.numpy(), Wt.numpy(), G.numpy(), s, f, workloads.sr_seed(sample))
+    O.layer_outputs(qx, qw, qg, s)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(layer: workloads.Layer, budget_s: float = 15.0):
+    """The oracle as it stands, timed on the host on a bounded sample of the
+    same layer: the batch cut to 4 and the input to 14 x 14 pixels."""
+    sample = oracle_sample_layer(layer, 4, min(layer.H, 14))
+    oracle_step(sample)                      # warm-up
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(sample)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(3 * sample.flops() / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{sample.name}: quantize X,W,G_Y + fp64 im2col fwd/wgrad/dgrad with |ab| sums, "
+                      f"{3 * sample.flops() / 1e9:.3f} GFLOP per step, {n} steps in {n * dt:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is the bounded sample."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    layer = pick_layer(args.workload)
+    total = args.steps + args.warmup
+    hw = 8 if total > 200 else 14
+    sample = oracle_sample_layer(layer, 4, min(layer.H, hw))
+    for _ in range(args.warmup):
+        oracle_step(sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sample)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = round(3 * sample.flops() / dt / 1e12, 6)
+    out = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": layer.name, "sample": sample.name},
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                            "sample": f"{sample.name} per step"},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default=workloads.resnet18_layer2().name)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    args.traffic = None
+    if os.path.exists(args.traffic_json):
+        with open(args.traffic_json) as f:
+            args.traffic = json.load(f).get(args.workload)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
