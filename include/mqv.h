@@ -149,6 +149,28 @@ mqv_status mqv_conv_fwd(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_
 mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const mqv_qtensor* x,
                           float* gw, void* ws, size_t ws_bytes, void* stream);
 
+/* Weight gradient exactly as mqv_conv_wgrad (same split plan, same
+ * results), for callers that cannot allocate device memory at all: code
+ * that runs where every byte of device memory is owned by someone else's
+ * fixed pool (an inference server or framework plugin that may not grow its
+ * footprint), or that has no allocator to ask for a workspace.  The paper
+ * has no counterpart; this is an interface convenience of this library.
+ *   - Allocates nothing: the split-K partial sums go to one file-scope
+ *     device array of 32 MiB inside the library, which every GPU that loads
+ *     the library holds until the process exits.  Layers whose partials
+ *     need more (mqv_conv_workspace_size(d, MQV_OP_WGRAD) > 32 MiB) are
+ *     rejected with MQV_ERR_UNSUPPORTED and a message; use mqv_conv_wgrad.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     every partial a call reads was written by the same call, so nothing
+ *     needs clearing.  Calls that overlap on the GPU (other streams, other
+ *     host threads) race on the array: serialize them.
+ * gy, x, gw and stream as in mqv_conv_wgrad. */
+mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
+                                  const mqv_qtensor* x, float* gw, void* stream);
+
 /* Input-gradient G_X = col2im(W^T·G_Y), computed directly as an implicit
  * transposed convolution: gx[hi][wi][ci][n] = T_w·T_g·sum over (kh, kw, co)
  * and every (ho, wo) with ho·stride + kh - pad = hi, wo·stride + kw - pad = wi.

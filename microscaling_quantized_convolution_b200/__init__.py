@@ -79,6 +79,8 @@ _SIGS = {
                                       ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_device_errors": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_void_p]),
+    "mqv_conv_wgrad_noalloc": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                              ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -261,6 +263,18 @@ def conv_dgrad(d: ConvDesc, w: QTensor, gy: QTensor, gx: torch.Tensor | None = N
     _check(lib().mqv_conv_dgrad(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(gc), gx.data_ptr(),
                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return gx
+
+
+def conv_wgrad_noalloc(d: ConvDesc, gy: QTensor, x: QTensor, gw: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """As conv_wgrad, but the library's built-in scratch replaces the
+    workspace (for callers that cannot allocate; see mqv_conv_wgrad_noalloc)."""
+    gw = gw if gw is not None else torch.empty((d.Cout, d.Kh, d.Kw, d.Cin), dtype=torch.float32,
+                                               device=x.codes.device)
+    gc, xc = gy.c(), x.c()
+    _check(lib().mqv_conv_wgrad_noalloc(ctypes.byref(d), ctypes.byref(gc), ctypes.byref(xc),
+                                        gw.data_ptr(), _stream(stream)))
+    return gw
 
 
 def device_errors(stream=None) -> int:

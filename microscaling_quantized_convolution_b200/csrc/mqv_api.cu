@@ -441,3 +441,53 @@ mqv_status mqv_device_errors(uint32_t* flags, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Weight gradient without any caller-provided workspace.  The split-K
+// partial sums live in a fixed device array that belongs to this library, so
+// a caller that has no way to allocate device memory can still run the pass.
+namespace {
+
+// Largest split-K partial set the built-in scratch holds (32 MiB per GPU; it
+// is part of the library's device image and stays resident until exit).
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) float g_noalloc_wgrad_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+float* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the array's name as a device pointer).
+mqv_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MQV_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_wgrad_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(wgrad scratch)");
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MQV_OK;
+}
+
+}  // namespace
+
+extern "C" mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
+                                             const mqv_qtensor* x, float* gw, void* stream) {
+  mqv_status st = check_desc(d);
+  if (st) return st;
+  ConvPlan pl;
+  plan_conv(d, MQV_OP_WGRAD, &pl);
+  if (pl.ws_bytes > kNoAllocScratchBytes)
+    return fail(MQV_ERR_UNSUPPORTED,
+                "mqv_conv_wgrad_noalloc: this layer's split partials need %zu bytes, the built-in "
+                "scratch holds %zu; call mqv_conv_wgrad with a workspace instead",
+                pl.ws_bytes, kNoAllocScratchBytes);
+  float* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  return run_conv(MQV_OP_WGRAD, d, gy, "gy", x, "x", gw, scratch, kNoAllocScratchBytes, stream);
+}
