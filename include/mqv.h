@@ -122,10 +122,16 @@ mqv_status mqv_amax(const float* src, int64_t rows, int64_t cols, float* amax,
                     void* ws, size_t ws_bytes, void* stream);
 
 /* The quantize step alone, given a device fp32 amax (from mqv_amax, possibly
- * combined across processes).  Same arithmetic as mqv_quantize_cbf. */
+ * combined across processes).  Same arithmetic as mqv_quantize_cbf.  For a
+ * batch shard the view holds columns [sr_col0, sr_col0 + cols) of a view
+ * with sr_cols columns; stochastic rounding then numbers element (r, c) as
+ * r·sr_cols + sr_col0 + c, so the shard draws the same Philox words as the
+ * whole tensor would (sr_cols = 0 means an unsharded view: sr_cols = cols).
+ * sr_col0 must be a multiple of 4. */
 mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols,
                                   int32_t fmt, int32_t rounding, uint64_t seed,
-                                  const float* amax, const mqv_qtensor* out, void* stream);
+                                  const float* amax, int64_t sr_col0, int64_t sr_cols,
+                                  const mqv_qtensor* out, void* stream);
 
 /* dst[r][c] = code·B·T of a quantized view, fp32 (code·B is exact in fp16;
  * the product with T is one fp32 rounding).  Reads a stored (for example
@@ -156,10 +162,11 @@ mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const m
  * footprint), or that has no allocator to ask for a workspace.  The paper
  * has no counterpart; this is an interface convenience of this library.
  *   - Allocates nothing: the split-K partial sums go to one file-scope
- *     device array of 32 MiB inside the library, which every GPU that loads
+ *     device array of 16 MiB inside the library, which every GPU that loads
  *     the library holds until the process exits.  Layers whose partials
- *     need more (mqv_conv_workspace_size(d, MQV_OP_WGRAD) > 32 MiB) are
- *     rejected with MQV_ERR_UNSUPPORTED and a message; use mqv_conv_wgrad.
+ *     would need more (mqv_conv_workspace_size(d, MQV_OP_WGRAD) > 16 MiB)
+ *     are rejected with MQV_ERR_UNSUPPORTED and a message; the current split
+ *     planner stays below 9.7 MB for every shape.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

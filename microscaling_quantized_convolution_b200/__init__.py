@@ -65,7 +65,8 @@ _SIGS = {
                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_quantize_with_amax": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_uint64,
-                                              ctypes.c_void_p, ctypes.POINTER(QTensorC), ctypes.c_void_p]),
+                                              ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.POINTER(QTensorC), ctypes.c_void_p]),
     "mqv_dequantize": (ctypes.c_int, [ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_conv_workspace_size": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_int32,
                                                ctypes.POINTER(ctypes.c_size_t)]),
@@ -188,13 +189,17 @@ def amax(src: torch.Tensor, rows: int, cols: int, out: torch.Tensor | None = Non
 
 
 def quantize_with_amax(src: torch.Tensor, rows: int, cols: int, fmt, rounding: int, seed: int,
-                       amax_dev: torch.Tensor, out: QTensor | None = None, stream=None) -> QTensor:
+                       amax_dev: torch.Tensor, out: QTensor | None = None, sr_col0: int = 0,
+                       sr_cols: int = 0, stream=None) -> QTensor:
+    """Quantize with a given device amax; (sr_col0, sr_cols) place a batch
+    shard inside the full view for stochastic rounding."""
     _require_cuda(src, "src", torch.float32)
     _require_cuda(amax_dev, "amax", torch.float32)
     out = out or QTensor.empty(rows, cols, fmt, src.device)
     qc = out.c()
     _check(lib().mqv_quantize_with_amax(src.data_ptr(), rows, cols, _fmt(fmt), rounding, seed,
-                                        amax_dev.data_ptr(), ctypes.byref(qc), _stream(stream)))
+                                        amax_dev.data_ptr(), sr_col0, sr_cols, ctypes.byref(qc),
+                                        _stream(stream)))
     return out
 
 

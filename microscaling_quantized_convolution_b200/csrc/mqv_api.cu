@@ -1,6 +1,6 @@
 // C ABI of the MicroQonv hot path (declared in include/mqv.h): argument
 // validation, launch geometry and error reporting.  Every compute step runs
-// in the kernels of mqv_quantize.cuh and mqv_conv.cuh; this file only checks
+// in the kernels of mqv_quantize.cuh and mqv_conv_kernels.cuh; this file only checks
 // arguments and enqueues launches on the caller's stream.
 #include <cuda_runtime.h>
 
@@ -10,7 +10,8 @@
 #include <mutex>
 
 #include "../../include/mqv.h"
-#include "mqv_conv.cuh"
+#include "mqv_conv_common.cuh"
+#include "mqv_conv_kernels.cuh"
 #include "mqv_quantize.cuh"
 
 namespace {
@@ -110,21 +111,30 @@ mqv_status check_qtensor(const mqv_qtensor* q, const char* name) {
 
 template <int FMT, int RND>
 void launch_quantize(const float* src, int64_t rows, int64_t cols, const float* amax_src,
-                     int amax_count, uint64_t seed, const mqv_qtensor* out, cudaStream_t st) {
-  quantize_kernel<FMT, RND><<<(unsigned)quant_ctas(rows, cols), kQuantThreads, 0, st>>>(
-      src, rows, cols, amax_src, amax_count, seed, static_cast<uint8_t*>(out->codes), out->scales,
-      out->tscale);
+                     int amax_count, uint64_t seed, int64_t sr_cols, int64_t sr_col0,
+                     const mqv_qtensor* out, cudaStream_t st) {
+  uint8_t* codes = static_cast<uint8_t*>(out->codes);
+  if ((cols / 4) % 2 == 0) {
+    const unsigned g = (unsigned)quant_ctas(rows, cols / 2);
+    quantize_kernel<FMT, RND, 2><<<g, kQuantThreads, 0, st>>>(
+        src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes, out->scales, out->tscale);
+  } else {
+    const unsigned g = (unsigned)quant_ctas(rows, cols);
+    quantize_kernel<FMT, RND, 1><<<g, kQuantThreads, 0, st>>>(
+        src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes, out->scales, out->tscale);
+  }
 }
 
 mqv_status enqueue_quantize(const float* src, int64_t rows, int64_t cols, int32_t fmt,
                             int32_t rounding, uint64_t seed, const float* amax_src,
-                            int amax_count, const mqv_qtensor* out, cudaStream_t st) {
+                            int amax_count, int64_t sr_cols, int64_t sr_col0,
+                            const mqv_qtensor* out, cudaStream_t st) {
   if (fmt == MQV_NVFP4)
-    rounding == MQV_RNE ? launch_quantize<0, 0>(src, rows, cols, amax_src, amax_count, seed, out, st)
-                        : launch_quantize<0, 1>(src, rows, cols, amax_src, amax_count, seed, out, st);
+    rounding == MQV_RNE ? launch_quantize<0, 0>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st)
+                        : launch_quantize<0, 1>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st);
   else
-    rounding == MQV_RNE ? launch_quantize<1, 0>(src, rows, cols, amax_src, amax_count, seed, out, st)
-                        : launch_quantize<1, 1>(src, rows, cols, amax_src, amax_count, seed, out, st);
+    rounding == MQV_RNE ? launch_quantize<1, 0>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st)
+                        : launch_quantize<1, 1>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return ok();
@@ -149,14 +159,16 @@ mqv_status check_quantize_args(const float* src, int64_t rows, int64_t cols, int
 // ------------------------------------------------------------- conv geometry
 
 struct ConvPlan {
-  ConvArgs a;
-  dim3 grid;
-  int splits;
+  V2Args a;
+  int bn;               // 128 or 256 columns per tile
+  int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0
+  int grid;             // persistent CTAs
+  size_t image_bytes;   // fwd/dgrad: dequantized A image (workspace head)
+  size_t partial_bytes; // wgrad: split partials (workspace)
   size_t ws_bytes;
 };
 
-constexpr int kBN = 128;
-constexpr int kStages = 3;
+constexpr int kSMs = 148;
 
 mqv_status check_desc(const mqv_conv_desc* d) {
   if (!d) return fail(MQV_ERR_INVALID_ARG, "null conv descriptor");
@@ -177,7 +189,8 @@ mqv_status check_desc(const mqv_conv_desc* d) {
   const int64_t lim = int64_t(1) << 30;
   if (d->H * d->W > lim || d->Cin > 65536 || d->Cout > 65536 || d->N > 65536 || d->Kh > 64 ||
       d->Kw > 64 || d->H * d->W * d->Cin * d->N > (int64_t(1) << 36) ||
-      Ho * Wo * d->Cout * d->N > (int64_t(1) << 36))
+      Ho * Wo * d->Cout * d->N > (int64_t(1) << 36) || Ho * Wo * d->N >= (int64_t(1) << 31) ||
+      d->H * d->W * d->N >= (int64_t(1) << 31) || d->Kh * d->Kw * (d->Cin + d->Cout) >= (int64_t(1) << 31))
     return fail(MQV_ERR_UNSUPPORTED, "conv shape exceeds the supported range");
   return MQV_OK;
 }
@@ -192,9 +205,20 @@ QView make_view(const mqv_qtensor* q) {
   return v;
 }
 
+// Multiplier and shift of mqv::fdiv for divisor d >= 1.
+FastDiv make_fastdiv(int64_t d) {
+  FastDiv f;
+  uint32_t s = 0;
+  while ((int64_t(1) << s) < d) ++s;
+  const unsigned __int128 num = (static_cast<unsigned __int128>(1) << (32 + s)) + (d - 1);
+  f.m = static_cast<uint32_t>(static_cast<uint64_t>(num / static_cast<unsigned __int128>(d)) - (uint64_t(1) << 32));
+  f.s = s;
+  return f;
+}
+
 // Geometry of one pass (no pointers needed for sizing).
 void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
-  ConvArgs& a = pl->a;
+  V2Args& a = pl->a;
   std::memset(&a, 0, sizeof(a));
   a.N = (int)d->N; a.Cin = (int)d->Cin; a.Cout = (int)d->Cout; a.H = (int)d->H; a.W = (int)d->W;
   a.Kh = (int)d->Kh; a.Kw = (int)d->Kw; a.stride = (int)d->stride; a.pad = (int)d->pad;
@@ -202,25 +226,37 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   a.Wo = (int)((d->W + 2 * d->pad - d->Kw) / d->stride + 1);
   const int64_t taps = d->Kh * d->Kw;
   if (op == MQV_OP_FWD) {
-    a.M = a.Cout;
+    a.M = a.Cout; a.Cred = a.Cin;
     a.Ncols = (int64_t)a.Ho * a.Wo * a.N;
     a.Kdim = taps * a.Cin;
   } else if (op == MQV_OP_WGRAD) {
-    a.M = a.Cout;
+    a.M = a.Cout; a.Cred = a.Cin;
     a.Ncols = taps * a.Cin;
     a.Kdim = (int64_t)a.Ho * a.Wo * a.N;
   } else {
-    a.M = a.Cin;
+    a.M = a.Cin; a.Cred = a.Cout;
     a.Ncols = (int64_t)a.H * a.W * a.N;
     a.Kdim = taps * a.Cout;
   }
-  a.ktiles = (int)((a.Kdim + kBK - 1) / kBK);
-  const int64_t tiles_n = (a.Ncols + kBN - 1) / kBN;
-  const int64_t tiles_m = (a.M + kBM - 1) / kBM;
+  a.ktiles = (int)((a.Kdim + 63) / 64);
+  a.mtiles = (int)((a.M + 127) / 128);
+  a.dN = make_fastdiv(a.N);
+  a.dWo = make_fastdiv(a.Wo);
+  a.dW = make_fastdiv(a.W);
+  a.dCred = make_fastdiv(a.Cred);
+  a.dKw = make_fastdiv(a.Kw);
+  a.dCin = make_fastdiv(a.Cin);
+  pl->nu = (d->N % 8 == 0) ? 8 : 4;
+  // Columns per tile: the option with the smaller (waves x tile width) over
+  // one persistent CTA per SM; ties go to the wider tile.
+  auto waves = [&](int bn) { return ((a.Ncols + bn - 1) / bn * a.mtiles + kSMs - 1) / kSMs; };
+  pl->bn = waves(256) * 256 <= waves(128) * 128 ? 256 : 128;
+  a.ntiles = (int)((a.Ncols + pl->bn - 1) / pl->bn);
+  const int64_t tiles_mn = (int64_t)a.ntiles * a.mtiles;
   int splits = 1;
   if (op == MQV_OP_WGRAD) {
-    const int64_t target = 2 * 148;
-    int64_t s = (target + tiles_n * tiles_m - 1) / (tiles_n * tiles_m);
+    // split the (ho, wo, n) contraction so that all tiles fit one wave
+    int64_t s = tiles_mn >= kSMs ? 1 : kSMs / tiles_mn;
     if (s > a.ktiles) s = a.ktiles;
     if (s < 1) s = 1;
     const int64_t per = (a.ktiles + s - 1) / s;
@@ -229,31 +265,80 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   } else {
     a.kt_per_split = a.ktiles;
   }
-  pl->splits = splits;
+  a.splits = splits;
+  a.tiles = (int)(tiles_mn * splits);
   a.scale_out = splits == 1;
-  pl->grid = dim3((unsigned)tiles_n, (unsigned)tiles_m, (unsigned)splits);
-  pl->ws_bytes = splits > 1 ? (size_t)splits * a.M * a.Ncols * sizeof(float) : 0;
+  pl->grid = a.tiles < kSMs ? a.tiles : kSMs;
+  pl->image_bytes = op == MQV_OP_WGRAD ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
+  pl->partial_bytes = splits > 1 ? (size_t)splits * a.M * a.Ncols * sizeof(float) : 0;
+  pl->ws_bytes = pl->image_bytes + pl->partial_bytes;
 }
 
-template <int PASS, int FMT>
-cudaError_t launch_conv(const ConvPlan& pl, cudaStream_t st) {
-  using L = ConvSmem<kBN, kStages>;
-  auto kern = conv_gemm_kernel<PASS, FMT, kBN, kStages>;
-  static bool attr_set[kMaxDevices] = {};
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+// `done` must be distinct for every kernel (one static per launcher instance).
+template <typename K>
+cudaError_t set_smem(K kern, int bytes, bool (&done)[kMaxDevices]) {
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    done[dev] = true;
   }
-  kern<<<pl.grid, kConvThreads, L::kBytes, st>>>(pl.a);
+  return cudaSuccess;
+}
+
+template <int PASS, int FMT, int BN, int NU>
+cudaError_t launch_fd(const ConvPlan& pl, cudaStream_t st) {
+  auto kern = conv_fd_kernel<PASS, FMT, BN, NU>;
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(kern, V2Smem<BN>::kBytes, done);
+  if (e != cudaSuccess) return e;
+  kern<<<pl.grid, kV2Threads, V2Smem<BN>::kBytes, st>>>(pl.a);
   return cudaGetLastError();
 }
 
+template <int FMT, int BN, int NU>
+cudaError_t launch_wg(const ConvPlan& pl, cudaStream_t st) {
+  auto kern = conv_wg_kernel<FMT, BN, NU>;
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(kern, V2Smem<BN>::kBytes, done);
+  if (e != cudaSuccess) return e;
+  kern<<<pl.grid, kV2Threads, V2Smem<BN>::kBytes, st>>>(pl.a);
+  return cudaGetLastError();
+}
+
+template <int PASS, int FMT>
+cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
+  if (PASS == kWgrad) {
+    if (pl.bn == 256) return pl.nu == 8 ? launch_wg<FMT, 256, 8>(pl, st) : launch_wg<FMT, 256, 4>(pl, st);
+    return pl.nu == 8 ? launch_wg<FMT, 128, 8>(pl, st) : launch_wg<FMT, 128, 4>(pl, st);
+  }
+  constexpr int P = PASS == kWgrad ? kFwd : PASS;
+  if (pl.bn == 256) return pl.nu == 8 ? launch_fd<P, FMT, 256, 8>(pl, st) : launch_fd<P, FMT, 256, 4>(pl, st);
+  return pl.nu == 8 ? launch_fd<P, FMT, 128, 8>(pl, st) : launch_fd<P, FMT, 128, 4>(pl, st);
+}
+
 template <int PASS>
-cudaError_t launch_conv_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
-  return fmt == MQV_NVFP4 ? launch_conv<PASS, 0>(pl, st) : launch_conv<PASS, 1>(pl, st);
+cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
+  return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
+}
+
+cudaError_t launch_prep(int op, int fmt, const ConvPlan& pl, const QView& w, uint8_t* image, cudaStream_t st) {
+  const V2Args& a = pl.a;
+  const int64_t chunks = (int64_t)a.mtiles * 128 * a.ktiles * 8;
+  int64_t g = (chunks + 255) / 256;
+  if (g > kSMs * 8) g = kSMs * 8;
+  if (op == MQV_OP_FWD) {
+    if (fmt == MQV_NVFP4) prep_image_kernel<0, false><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+    else prep_image_kernel<1, false><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+  } else {
+    if (fmt == MQV_NVFP4) prep_image_kernel<0, true><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+    else prep_image_kernel<1, true><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+  }
+  return cudaGetLastError();
 }
 
 mqv_status check_operand(const mqv_qtensor* q, const char* name, int64_t rows, int64_t cols, int32_t fmt) {
@@ -289,25 +374,39 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
                 pl.ws_bytes, ws ? ws_bytes : (size_t)0);
   uint32_t* err = nullptr;
   if ((st = device_error_word(&err))) return st;
-  pl.a.a = make_view(qa);
-  pl.a.b = make_view(qb);
-  pl.a.err = err;
-  pl.a.out = pl.splits > 1 ? static_cast<float*>(ws) : out;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  pl.a.err = err;
   cudaError_t e;
-  if (op == MQV_OP_FWD) e = launch_conv_fmt<kFwd>(d->fmt, pl, s);
-  else if (op == MQV_OP_WGRAD) e = launch_conv_fmt<kWgrad>(d->fmt, pl, s);
-  else e = launch_conv_fmt<kDgrad>(d->fmt, pl, s);
-  if (e != cudaSuccess) return cuda_fail(e, "conv launch");
-  if (pl.splits > 1) {
-    const int64_t n4 = (int64_t)pl.a.M * pl.a.Ncols / 4;
-    int64_t g = (n4 + 255) / 256;
-    if (g > 148 * 8) g = 148 * 8;
-    wgrad_reduce_kernel<<<(unsigned)g, 256, 0, s>>>(reinterpret_cast<const float4*>(ws), pl.splits, n4,
-                                                     qa->tscale, qb->tscale, reinterpret_cast<float4*>(out));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "wgrad reduce launch");
+  if (op == MQV_OP_WGRAD) {
+    pl.a.a = make_view(qa);
+    pl.a.b = make_view(qb);
+    pl.a.ta = qa->tscale;
+    pl.a.tb = qb->tscale;
+    pl.a.out = pl.a.splits > 1 ? reinterpret_cast<float*>(wsb) : out;
+    e = launch_pass_fmt<kWgrad>(d->fmt, pl, s);
+    if (e != cudaSuccess) return cuda_fail(e, "wgrad launch");
+    if (pl.a.splits > 1) {
+      const int64_t n4 = (int64_t)pl.a.M * pl.a.Ncols / 4;
+      int64_t g = (n4 + 255) / 256;
+      if (g > kSMs * 8) g = kSMs * 8;
+      wgrad_reduce_kernel<<<(unsigned)g, 256, 0, s>>>(reinterpret_cast<const float4*>(wsb), pl.a.splits, n4,
+                                                       qa->tscale, qb->tscale, reinterpret_cast<float4*>(out));
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "wgrad reduce launch");
+    }
+    return ok();
   }
+  // fwd / dgrad: qa is W, qb is X (fwd) or G_Y (dgrad)
+  e = launch_prep(op, d->fmt, pl, make_view(qa), wsb, s);
+  if (e != cudaSuccess) return cuda_fail(e, "operand image launch");
+  pl.a.image = wsb;
+  pl.a.b = make_view(qb);
+  pl.a.ta = qa->tscale;
+  pl.a.tb = qb->tscale;
+  pl.a.out = out;
+  e = op == MQV_OP_FWD ? launch_pass_fmt<kFwd>(d->fmt, pl, s) : launch_pass_fmt<kDgrad>(d->fmt, pl, s);
+  if (e != cudaSuccess) return cuda_fail(e, "conv launch");
   return ok();
 }
 
@@ -369,16 +468,21 @@ mqv_status mqv_quantize_cbf(const float* src, int64_t rows, int64_t cols, int32_
   amax_partial_kernel<<<(unsigned)g, kAmaxThreads, 0, s>>>(reinterpret_cast<const float4*>(src), rows * cols / 4, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "amax launch");
-  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, part, (int)g, out, s);
+  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, part, (int)g, cols, 0, out, s);
 }
 
 mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols, int32_t fmt,
                                   int32_t rounding, uint64_t seed, const float* amax,
-                                  const mqv_qtensor* out, void* stream) {
+                                  int64_t sr_col0, int64_t sr_cols, const mqv_qtensor* out,
+                                  void* stream) {
   mqv_status st = check_quantize_args(src, rows, cols, fmt, rounding, out);
   if (st) return st;
   if (!amax || (reinterpret_cast<uintptr_t>(amax) & 3u)) return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
-  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, amax, 1, out,
+  if (sr_cols == 0) sr_cols = cols;
+  if (sr_col0 < 0 || sr_col0 % 4 || sr_cols < cols || sr_col0 + cols > sr_cols)
+    return fail(MQV_ERR_INVALID_ARG, "columns [%lld, %lld) are not a 4-aligned window of %lld SR columns",
+                (long long)sr_col0, (long long)(sr_col0 + cols), (long long)sr_cols);
+  return enqueue_quantize(src, rows, cols, fmt, rounding, seed, amax, 1, sr_cols, sr_col0, out,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -448,9 +552,12 @@ mqv_status mqv_device_errors(uint32_t* flags, void* stream) {
 // a caller that has no way to allocate device memory can still run the pass.
 namespace {
 
-// Largest split-K partial set the built-in scratch holds (32 MiB per GPU; it
-// is part of the library's device image and stays resident until exit).
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+// Largest split-K partial set the built-in scratch holds (16 MiB per GPU; it
+// is part of the library's device image and stays resident until exit).  The
+// split planner only splits layers with at most 74 output tiles of 128 x 128
+// and fills at most one tile per SM, so its partials stay below
+// 148 x 128 x 128 x 4 B = 9.7 MB; the size check below guards that bound.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) float g_noalloc_wgrad_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 float* g_noalloc_ptr[kMaxDevices] = {};

@@ -1,0 +1,680 @@
+// Persistent, warp-specialized implicit-GEMM kernels for the three conv
+// GEMMs on square-block quantized operands (MicroQonv summary,
+// onedev.kr/papers/182, section "무엇과 다른가": Y = W·X', G_W = G_Y·X'^T,
+// G_X' = W^T·G_Y; im2col built on chip, section "어떻게 동작하나").
+//
+// Forward and input-gradient (conv_fd_kernel): D[m][col] = sum_k A[m][k]·B[col][k]
+//   m   = output channel of the pass (co for fwd, ci for dgrad), 128 per tile
+//   col = (output pixel, n) of the pass, BN per tile
+//   k   = (kh, kw, reduced channel)
+//   A = W (fwd) or W^T (dgrad): small, dequantized once per call by
+//       prep_image_kernel into an fp16 image laid out exactly like the
+//       swizzled K-major shared-memory tile, then brought in 16 KB per stage
+//       with one plain bulk copy.
+//   B = the im2col rows of X (fwd) or the transposed-conv gather of G_Y
+//       (dgrad), dequantized on chip by 8 producer warps straight from the
+//       channel-batch-first codes into an MN-major tile: for one channel the
+//       codes of consecutive batch items are consecutive, which is exactly
+//       the MN-major order, so no transpose is needed.
+// Weight gradient (conv_wg_kernel): D[co][(kh,kw,ci)] = sum over (ho,wo,n)
+//   A = G_Y and B = X', both gathered K-major (their codes run along n, the
+//   contraction), split over CTAs along (ho, wo, n).
+//
+// Roles (one CTA per SM, persistent over tiles):
+//   warps 0-3 epilogue (tcgen05.ld from TMEM lane quarter = warp, scale by
+//             T_a·T_b, fp32 store), double-buffered accumulators so a tile's
+//             epilogue overlaps the next tile's MMAs;
+//   warp  4   tensor-memory allocation and the single MMA-issuing thread;
+//   warp  5   bulk-copy loader of the A image (fwd/dgrad);
+//   warps 6-13 producers (gather + dequantize).
+// Every wait is bounded (see mbar_wait_bounded); nothing waits on another
+// CTA or GPU.
+#pragma once
+
+#include <cstdint>
+
+#include "mqv_conv_common.cuh"
+#include "mqv_ptx.cuh"
+
+namespace mqv {
+
+constexpr int kV2EpiWarps = 4;
+constexpr int kV2MmaWarp = 4;
+constexpr int kV2LoadWarp = 5;
+constexpr int kV2ProdWarp0 = 6;
+constexpr int kV2ProdThreads = 256;
+constexpr int kV2Threads = (kV2ProdWarp0 + kV2ProdThreads / 32) * 32;   // 448
+constexpr int kV2Stages = 4;
+constexpr uint32_t kATileBytes = 128 * 64 * 2;                             // 16 KB
+
+// Division of dividends below 2^31 by an invariant positive divisor with one
+// multiply-high, one add and one shift (Granlund & Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994, round-up variant):
+// s = ceil(log2 d), m = ceil(2^(32+s) / d) - 2^32, q = (umulhi(k, m) + k) >> s.
+struct FastDiv {
+  uint32_t m, s;
+};
+
+__device__ __forceinline__ int fdiv(int k, FastDiv f) {
+  const uint32_t u = static_cast<uint32_t>(k);
+  return static_cast<int>((__umulhi(u, f.m) + u) >> f.s);
+}
+
+struct V2Args {
+  const uint8_t* image;   // fwd/dgrad: A image [mtiles][ktiles] x 16 KB
+  QView a;                // wgrad: G_Y
+  QView b;                // fwd: X, dgrad: G_Y, wgrad: X
+  const float* ta;
+  const float* tb;
+  float* out;
+  uint32_t* err;
+  int N, Cin, Cout, H, W, Kh, Kw, stride, pad, Ho, Wo;
+  int M;                  // GEMM rows (channels)
+  int Cred;               // fwd: Cin, dgrad: Cout (channels of the reduction)
+  int64_t Ncols;          // GEMM columns
+  int64_t Kdim;           // contraction length
+  int ktiles;             // K tiles of 64 over the whole contraction
+  int kt_per_split;       // wgrad: K tiles per split
+  int splits;
+  int mtiles, ntiles;
+  int tiles;              // mtiles * ntiles * splits
+  int scale_out;          // multiply by T_a·T_b (0 for wgrad split partials)
+  FastDiv dN, dWo, dW, dCred, dKw, dCin;
+};
+
+template <int BN>
+struct V2Smem {
+  static constexpr int kBTile = BN * 128;
+  static constexpr int kStage = kATileBytes + kBTile;
+  static constexpr int kBarOffset = kV2Stages * kStage;
+  static constexpr int kBytes = kBarOffset + 256 + 1024;
+};
+
+// MN-major 128B-swizzled fp16 tile of BN rows (MN) x 64 K: atoms of 64 MN x
+// 8 K (1 KB); the 8 K-atoms of one MN-atom are consecutive (SBO = 1 KB), the
+// MN-atoms 8 KB apart (LBO).
+__device__ __forceinline__ uint32_t mn_offset(uint32_t mn, uint32_t k) {
+  return (mn >> 6) * 8192u + (k >> 3) * 1024u + (k & 7u) * 128u +
+         ((((mn & 63u) >> 3) ^ (k & 7u)) << 4) + (mn & 7u) * 2u;
+}
+
+// ---------------------------------------------------------------------------
+// Code decoding helpers.  code·scale is exact in fp16: an E2M1 (E2M3) value
+// has at most 2 (4) significant bits, an E4M3 scale 4, and every product lies
+// between 2^-12 and 3360, inside the fp16 range; the tensor scales are applied
+// in the epilogue.
+
+// 8 FP4 codes of one source row (n0..n0+7) times their two block scales
+// (n0..n0+3 use s2lo, n0+4..n0+7 use s2hi) -> 4 fp16x2 in n order.
+__device__ __forceinline__ void dq8_fp4(uint32_t w, uint32_t s2lo, uint32_t s2hi, uint32_t (&h)[4]) {
+  e2m1x8_to_f16x2(w, h);
+  h[0] = hmul2_u32(h[0], s2lo);
+  h[1] = hmul2_u32(h[1], s2lo);
+  h[2] = hmul2_u32(h[2], s2hi);
+  h[3] = hmul2_u32(h[3], s2hi);
+}
+
+// 4 FP6 codes in the low 24 bits of q -> 2 fp16x2.
+__device__ __forceinline__ void dq4_fp6(uint32_t q, uint32_t s2, uint32_t& h01, uint32_t& h23) {
+  h01 = hmul2_u32(e2m3x2_to_f16x2((q & 0x3F) | ((q << 2) & 0x3F00)), s2);
+  h23 = hmul2_u32(e2m3x2_to_f16x2(((q >> 12) & 0x3F) | ((q >> 10) & 0x3F00)), s2);
+}
+
+__device__ __forceinline__ uint32_t scale2(uint32_t s) { return e4m3x2_to_f16x2(s | (s << 8)); }
+
+// Load the codes of `nu` (8 or 4) consecutive columns starting at column c
+// of view row `row` (c a multiple of nu).  FP4: nu/2 bytes; FP6: 3·nu/4 bytes.
+template <int FMT, int NU>
+__device__ __forceinline__ uint32_t load_codes(const QView& v, int64_t row, int64_t c, uint32_t& hi) {
+  const uint8_t* p = v.codes + row * v.row_bytes;
+  hi = 0;
+  if (FMT == 0) {
+    if (NU == 8) return __ldg(reinterpret_cast<const uint32_t*>(p + (c >> 1)));
+    return __ldg(reinterpret_cast<const unsigned short*>(p + (c >> 1)));
+  } else {
+    const uint8_t* q = p + ((c * 3) >> 2);
+    if (NU == 8) {   // 6 bytes, 2-byte aligned
+      const unsigned short* q16 = reinterpret_cast<const unsigned short*>(q);
+      const uint32_t a = __ldg(q16), b = __ldg(q16 + 1), d = __ldg(q16 + 2);
+      const uint32_t lo = a | (b << 16);          // bytes 0-3
+      hi = d;                                      // bytes 4-5
+      return lo;
+    }
+    return static_cast<uint32_t>(__ldg(q)) | (static_cast<uint32_t>(__ldg(q + 1)) << 8) |
+           (static_cast<uint32_t>(__ldg(q + 2)) << 16);
+  }
+}
+
+// Dequantize NU codes of one source row into NU/2 fp16x2 (column order).
+template <int FMT, int NU>
+__device__ __forceinline__ void dequant_run(uint32_t lo, uint32_t hi, uint32_t s2lo, uint32_t s2hi,
+                                            uint32_t (&h)[4]) {
+  if (FMT == 0) {
+    if (NU == 8) {
+      dq8_fp4(lo, s2lo, s2hi, h);
+    } else {
+      h[0] = hmul2_u32(e2m1x2_to_f16x2(lo & 0xFF), s2lo);
+      h[1] = hmul2_u32(e2m1x2_to_f16x2((lo >> 8) & 0xFF), s2lo);
+    }
+  } else {
+    dq4_fp6(lo & 0xFFFFFF, s2lo, h[0], h[1]);
+    if (NU == 8) dq4_fp6((lo >> 24) | (hi << 8), s2hi, h[2], h[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// A image: [mtiles][ktiles] tiles, each 128 rows x 64 fp16, K-major, rows of
+// 128 B with the 16-byte chunks XOR-swizzled by (row & 7), i.e. byte for byte
+// the shared-memory tile the MMA reads.  fwd: A[co][k] = W[co][k];
+// dgrad: A[ci][(tap, co)] = W[co][tap·Cin + ci].  Rows/columns past the
+// matrix are zero.  One thread per 16-byte chunk.
+template <int FMT, bool TRANS>
+__global__ void __launch_bounds__(256)
+prep_image_kernel(QView w, int M, int64_t Kdim, int ktiles, int mtiles, int Cin, int Cout,
+                  uint8_t* __restrict__ image) {
+  const int64_t chunks = static_cast<int64_t>(mtiles) * 128 * ktiles * 8;
+  for (int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; id < chunks;
+       id += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t m = id / (static_cast<int64_t>(ktiles) * 8);
+    const int64_t k0 = (id - m * ktiles * 8) * 8;
+    uint32_t h[4] = {0u, 0u, 0u, 0u};
+    if (m < M) {
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const int64_t k = k0 + e;
+        if (k >= Kdim) break;
+        int64_t row, col;
+        if (!TRANS) {
+          row = m;
+          col = k;
+        } else {
+          const int64_t tap = k / Cout, co = k - tap * Cout;
+          row = co;
+          col = tap * Cin + m;
+        }
+        const uint32_t s = __ldg(w.scales + (row >> 2) * w.scale_cols + (col >> 2));
+        uint32_t c0, c1;
+        const uint8_t* p = w.codes + row * w.row_bytes;
+        const int64_t row2 = TRANS ? row + 1 : row;       // second element: next co (dgrad)
+        const int64_t col2 = TRANS ? col : col + 1;
+        const uint8_t* p2 = w.codes + row2 * w.row_bytes;
+        if (FMT == 0) {
+          c0 = (__ldg(p + (col >> 1)) >> ((col & 1) * 4)) & 0xF;
+          c1 = (__ldg(p2 + (col2 >> 1)) >> ((col2 & 1) * 4)) & 0xF;
+          h[e >> 1] = hmul2_u32(e2m1x2_to_f16x2(c0 | (c1 << 4)), scale2(s));
+        } else {
+          auto code6 = [](const uint8_t* base, int64_t c) -> uint32_t {
+            const uint8_t* q = base + (c >> 2) * 3;
+            const uint32_t v = static_cast<uint32_t>(__ldg(q)) | (static_cast<uint32_t>(__ldg(q + 1)) << 8) |
+                               (static_cast<uint32_t>(__ldg(q + 2)) << 16);
+            return (v >> ((c & 3) * 6)) & 0x3F;
+          };
+          c0 = code6(p, col);
+          c1 = code6(p2, col2);
+          h[e >> 1] = hmul2_u32(e2m3x2_to_f16x2(c0 | (c1 << 8)), scale2(s));
+        }
+      }
+    }
+    const int64_t mt = m >> 7, r = m & 127, kt = k0 >> 6, kc = (k0 & 63) >> 3;
+    uint8_t* dst = image + (mt * ktiles + kt) * kATileBytes + r * 128 + ((kc ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shared control block of the persistent kernels.
+struct V2Bars {
+  uint64_t full[kV2Stages];
+  uint64_t empty[kV2Stages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem;
+};
+
+template <int BN>
+__device__ __forceinline__ V2Bars* v2_setup(uint8_t* smem, int full_count) {
+  V2Bars* bars = reinterpret_cast<V2Bars*>(smem + V2Smem<BN>::kBarOffset);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kV2Stages; ++s) {
+      mbar_init(&bars->full[s], full_count);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], kV2EpiWarps * 32);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kV2MmaWarp) {
+    tmem_alloc(&bars->tmem, 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return bars;
+}
+
+template <int BN>
+__device__ __forceinline__ void v2_teardown(V2Bars* bars) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kV2MmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(bars->tmem, 2 * BN);
+  }
+}
+
+// Epilogue of one tile: TMEM accumulator buffer `acc` -> fp32 output.
+// FD=true: out[(pixel·M + m)·N + n] with col = pixel·N + n;
+// FD=false (wgrad): out[(split·M + m)·Ncols + col].
+template <int BN, bool FD>
+__device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int acc, int64_t m0,
+                                            int64_t col0, int split, bool has_k) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m = m0 + warp * 32 + lane;
+  const float scale = p.scale_out ? __fmul_rn(*p.ta, *p.tb) : 1.0f;
+  const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * BN;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c, r);
+    tmem_ld_wait();
+    if (m < p.M) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t col = col0 + c + 4 * j;
+        if (col >= p.Ncols) continue;
+        float4 o;
+        o.x = has_k ? __uint_as_float(r[4 * j + 0]) * scale : 0.f;
+        o.y = has_k ? __uint_as_float(r[4 * j + 1]) * scale : 0.f;
+        o.z = has_k ? __uint_as_float(r[4 * j + 2]) * scale : 0.f;
+        o.w = has_k ? __uint_as_float(r[4 * j + 3]) * scale : 0.f;
+        int64_t idx;
+        if (FD) {
+          const int64_t pix = col / p.N;
+          idx = (pix * p.M + m) * p.N + (col - pix * p.N);
+        } else {
+          idx = (static_cast<int64_t>(split) * p.M + m) * p.Ncols + col;
+        }
+        *reinterpret_cast<float4*>(p.out + idx) = o;
+      }
+    }
+  }
+  tc_fence_before();
+  mbar_arrive(&bars->acc_empty[acc]);
+}
+
+// ---------------------------------------------------------------------------
+// Raw codes of one producer unit: 4 view rows (consecutive channels) x NU
+// consecutive batch items, plus the one or two E4M3 scales that cover them.
+template <int FMT, int NU>
+struct UnitRaw {
+  uint32_t lo[4];
+  uint32_t hi[4];          // FP6 with NU = 8: bytes 4-5 of each run
+  uint32_t ss;             // scale byte(s)
+  bool ok;
+};
+
+template <int FMT, int NU>
+__device__ __forceinline__ void load_unit(const QView& v, int64_t row, int n, bool ok, UnitRaw<FMT, NU>& u) {
+  u.ok = ok;
+  if (!ok) return;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) u.lo[j] = load_codes<FMT, NU>(v, row + j, n, u.hi[j]);
+  const uint8_t* sp = v.scales + (row >> 2) * v.scale_cols + (n >> 2);
+  u.ss = NU == 8 ? static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(sp))) : __ldg(sp);
+}
+
+// Dequantize a unit and store it: MN-major (the unit's NU batch items are
+// consecutive MN rows of K column kl + j) or K-major (tile row r0 + j gets
+// NU consecutive K values at kl).
+template <int FMT, int NU, bool MN_MAJOR>
+__device__ __forceinline__ void store_unit(const UnitRaw<FMT, NU>& u, uint32_t tile, uint32_t a, uint32_t kl) {
+  const uint32_t s2lo = u.ok ? scale2(u.ss & 0xFF) : 0u;
+  const uint32_t s2hi = (u.ok && NU == 8) ? scale2(u.ss >> 8) : 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t h[4] = {0u, 0u, 0u, 0u};
+    if (u.ok) dequant_run<FMT, NU>(u.lo[j], u.hi[j], s2lo, s2hi, h);
+    const uint32_t off = MN_MAJOR ? mn_offset(a, kl + j) : sw128_offset(a + j, kl);
+    if (NU == 8) st_shared_v4(tile + off, h[0], h[1], h[2], h[3]);
+    else st_shared_v2(tile + off, h[0], h[1]);
+  }
+}
+
+// Forward / input-gradient B producer.  Unit u of a K tile: column group
+// g = u % G (NU batch items of one output pixel), channel quad kq = u / G.
+// Consecutive lanes take consecutive column groups, so the 4-byte code loads
+// of a warp are contiguous and each 8-lane phase of a 16-byte shared store
+// lands on 8 different swizzled chunks.
+template <int PASS, int FMT, int BN, int NU>
+struct FdProducer {
+  static constexpr int G = BN / NU;
+  static constexpr int UNITS = G * 16;
+  static constexpr int PER = UNITS / kV2ProdThreads;
+  static_assert(kV2ProdThreads % G == 0 && UNITS % kV2ProdThreads == 0, "producer mapping");
+  UnitRaw<FMT, NU> raw[PER];
+
+  __device__ __forceinline__ void load(const V2Args& p, int64_t col0, int kt, int t) {
+    const int g = t % G;
+    const int64_t col = col0 + static_cast<int64_t>(g) * NU;
+    const bool col_ok = col < p.Ncols;
+    const int c32 = col_ok ? static_cast<int>(col) : 0;
+    const int pix = fdiv(c32, p.dN);
+    const int n = c32 - pix * p.N;
+    const int ph = fdiv(pix, PASS == kFwd ? p.dWo : p.dW);
+    const int pw = pix - ph * (PASS == kFwd ? p.Wo : p.W);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int kq = t / G + (kV2ProdThreads / G) * i;
+      const int k = kt * 64 + 4 * kq;
+      bool ok = col_ok && k < p.Kdim;
+      int64_t row = 0;
+      if (ok) {
+        const int tap = fdiv(k, p.dCred);
+        const int c = k - tap * p.Cred;
+        const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
+        if (PASS == kFwd) {
+          const int sh = ph * p.stride + kh - p.pad, sw = pw * p.stride + kw - p.pad;
+          ok = sh >= 0 && sh < p.H && sw >= 0 && sw < p.W;
+          row = (static_cast<int64_t>(sh) * p.W + sw) * p.Cred + c;
+        } else {
+          const int th = ph + p.pad - kh, tw = pw + p.pad - kw;
+          const int sh = th / p.stride, sw = tw / p.stride;
+          ok = th >= 0 && tw >= 0 && sh * p.stride == th && sw * p.stride == tw && sh < p.Ho && sw < p.Wo;
+          row = (static_cast<int64_t>(sh) * p.Wo + sw) * p.Cred + c;
+        }
+      }
+      load_unit<FMT, NU>(p.b, row, n, ok, raw[i]);
+    }
+  }
+
+  __device__ __forceinline__ void store(uint32_t tile, int t) const {
+    const int g = t % G;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int kq = t / G + (kV2ProdThreads / G) * i;
+      store_unit<FMT, NU, true>(raw[i], tile, static_cast<uint32_t>(g * NU), static_cast<uint32_t>(4 * kq));
+    }
+  }
+};
+
+// Producer warps signal a filled stage once per warp: every lane makes its
+// shared stores visible to the async proxy, the warp converges, lane 0 arrives.
+__device__ __forceinline__ void producer_warp_arrive(uint64_t* bar) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+template <int PASS, int FMT, int BN, int NU>
+__global__ void __launch_bounds__(kV2Threads, 1)
+conv_fd_kernel(const V2Args p) {
+  using L = V2Smem<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  V2Bars* bars = v2_setup<BN>(smem, kV2ProdThreads / 32 + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp < kV2EpiWarps) {
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
+      tc_fence_after();
+      const int mt = tile / p.ntiles, nt = tile - mt * p.ntiles;
+      v2_epilogue<BN, true>(p, bars, acc, static_cast<int64_t>(mt) * 128,
+                            static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0);
+    }
+  } else if (warp == kV2MmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32_bmn(128, BN);
+      int it = 0, kit = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
+        tc_fence_after();
+        const uint32_t dt = bars->tmem + acc * BN;
+        for (int kt = 0; kt < p.ktiles; ++kt, ++kit) {
+          const int s = kit % kV2Stages;
+          mbar_wait_bounded(&bars->full[s], (kit / kV2Stages) & 1, p.err, kErrWaitFull);
+          tc_fence_after();
+          const uint32_t a_tile = sbase + s * L::kStage;
+          const uint64_t adesc = smem_desc_sw128(a_tile);
+          const uint64_t bdesc = smem_desc_sw128_mn(a_tile + kATileBytes, 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(dt, adesc + 2 * kk, bdesc + 128 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars->empty[s]);
+        }
+        mma_commit(&bars->acc_full[acc]);
+      }
+    }
+  } else if (warp == kV2LoadWarp) {
+    if (lane == 0) {
+      int kit = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
+        const int mt = tile / p.ntiles;
+        const uint8_t* src = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
+        for (int kt = 0; kt < p.ktiles; ++kt, ++kit) {
+          const int s = kit % kV2Stages;
+          mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
+          mbar_arrive_expect_tx(&bars->full[s], kATileBytes);
+          bulk_copy_g2s(sbase + s * L::kStage, src + static_cast<int64_t>(kt) * kATileBytes,
+                        kATileBytes, &bars->full[s]);
+        }
+      }
+    }
+  } else {
+    // producers: the codes of stage i + kLookahead are requested right after
+    // stage i is stored, so each load has kLookahead stages of work (and of
+    // waiting for free stages) to arrive in.  The ring of raw registers is
+    // indexed at compile time (unrolled by kLookahead).
+    const int t = threadIdx.x - kV2ProdWarp0 * 32;
+    const int total = p.ktiles * ((p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                                  static_cast<int>(gridDim.x));
+    using Prod = FdProducer<PASS, FMT, BN, NU>;
+    constexpr int kLookahead = Prod::PER >= 4 ? 2 : 3;      // keep the ring in registers
+    Prod ring[kLookahead];
+    int ltile = blockIdx.x, lkt = 0;          // load cursor
+    auto load_next = [&](Prod& pr) {
+      pr.load(p, static_cast<int64_t>(ltile % p.ntiles) * BN, lkt, t);
+      if (++lkt == p.ktiles) { lkt = 0; ltile += gridDim.x; }
+    };
+#pragma unroll
+    for (int r = 0; r < kLookahead; ++r)
+      if (r < total) load_next(ring[r]);
+    for (int kit = 0; kit < total;) {
+#pragma unroll
+      for (int r = 0; r < kLookahead; ++r, ++kit) {
+        if (kit >= total) break;
+        const int s = kit % kV2Stages;
+        mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
+        ring[r].store(sbase + s * L::kStage + kATileBytes, t);
+        producer_warp_arrive(&bars->full[s]);
+        if (kit + kLookahead < total) load_next(ring[r]);
+      }
+    }
+  }
+  v2_teardown<BN>(bars);
+}
+
+// ---------------------------------------------------------------------------
+// Weight-gradient producer: the K-major A (G_Y) and B (X') tiles of one K
+// tile.  Unit = 4 view rows x NU consecutive batch items of one pixel; lane
+// order runs along K first (KG units per tile row), so a warp reads
+// contiguous code bytes of each row.
+template <int FMT, int NU, int ROWS>
+struct WgOperand {
+  static constexpr int KG = 64 / NU;
+  static constexpr int UNITS = (ROWS / 4) * KG;
+  static constexpr int PER = UNITS / kV2ProdThreads;
+  static_assert(UNITS % kV2ProdThreads == 0, "producer mapping");
+  UnitRaw<FMT, NU> raw[PER];
+
+  template <bool IS_A>
+  __device__ __forceinline__ void load(const V2Args& p, const QView& v, int row_base, int kt, int t) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int u = t + kV2ProdThreads * i;
+      const int kg = u % KG, rq = u / KG;
+      const int q = kt * 64 + kg * NU;              // (pixel, n) contraction index
+      const int r0 = row_base + 4 * rq;
+      bool ok = q < p.Kdim;
+      int64_t row = 0;
+      int n = 0;
+      if (ok) {
+        const int pix = fdiv(q, p.dN);
+        n = q - pix * p.N;
+        if (IS_A) {
+          ok = r0 < p.M;
+          row = static_cast<int64_t>(pix) * p.Cout + r0;
+        } else {
+          ok = r0 < p.Ncols;
+          const int tap = fdiv(r0, p.dCin), ci = r0 - tap * p.Cin;
+          const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
+          const int ho = fdiv(pix, p.dWo), wo = pix - ho * p.Wo;
+          const int hi = ho * p.stride + kh - p.pad, wi = wo * p.stride + kw - p.pad;
+          ok = ok && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
+          row = (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci;
+        }
+      }
+      load_unit<FMT, NU>(v, row, n, ok, raw[i]);
+    }
+  }
+
+  __device__ __forceinline__ void store(uint32_t tile, int t) const {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int u = t + kV2ProdThreads * i;
+      const int kg = u % KG, rq = u / KG;
+      store_unit<FMT, NU, false>(raw[i], tile, static_cast<uint32_t>(4 * rq), static_cast<uint32_t>(kg * NU));
+    }
+  }
+};
+
+template <int FMT, int BN, int NU>
+struct WgProducer {
+  WgOperand<FMT, NU, 128> a;
+  WgOperand<FMT, NU, BN> b;
+  static constexpr int PER = WgOperand<FMT, NU, 128>::PER + WgOperand<FMT, NU, BN>::PER;
+  __device__ __forceinline__ void load(const V2Args& p, int mt, int nt, int kt, int t) {
+    a.template load<true>(p, p.a, mt * 128, kt, t);
+    b.template load<false>(p, p.b, nt * BN, kt, t);
+  }
+  __device__ __forceinline__ void store(uint32_t a_tile, int t) const {
+    a.store(a_tile, t);
+    b.store(a_tile + kATileBytes, t);
+  }
+};
+
+template <int FMT, int BN, int NU>
+__global__ void __launch_bounds__(kV2Threads, 1)
+conv_wg_kernel(const V2Args p) {
+  using L = V2Smem<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  V2Bars* bars = v2_setup<BN>(smem, kV2ProdThreads / 32);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+
+  auto decode = [&](int tile, int& mt, int& nt, int& sp) {
+    sp = tile % p.splits;
+    const int r = tile / p.splits;
+    mt = r / p.ntiles;
+    nt = r - mt * p.ntiles;
+  };
+
+  if (warp < kV2EpiWarps) {
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      int mt, nt, sp;
+      decode(tile, mt, nt, sp);
+      const int kt0 = sp * p.kt_per_split;
+      const bool has_k = min(p.ktiles, kt0 + p.kt_per_split) > kt0;
+      mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
+      tc_fence_after();
+      v2_epilogue<BN, false>(p, bars, acc, static_cast<int64_t>(mt) * 128,
+                             static_cast<int64_t>(nt) * BN, sp, has_k);
+    }
+  } else if (warp == kV2MmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, BN);
+      int it = 0, kit = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+        int mt, nt, sp;
+        decode(tile, mt, nt, sp);
+        const int kt0 = sp * p.kt_per_split, kt1 = min(p.ktiles, kt0 + p.kt_per_split);
+        const int acc = it & 1;
+        mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
+        tc_fence_after();
+        const uint32_t dt = bars->tmem + acc * BN;
+        for (int kt = kt0; kt < kt1; ++kt, ++kit) {
+          const int s = kit % kV2Stages;
+          mbar_wait_bounded(&bars->full[s], (kit / kV2Stages) & 1, p.err, kErrWaitFull);
+          tc_fence_after();
+          const uint32_t a_tile = sbase + s * L::kStage;
+          const uint64_t adesc = smem_desc_sw128(a_tile);
+          const uint64_t bdesc = smem_desc_sw128(a_tile + kATileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(dt, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kt > kt0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars->empty[s]);
+        }
+        mma_commit(&bars->acc_full[acc]);
+      }
+    }
+  } else if (warp >= kV2ProdWarp0) {
+    // producers with a kLookahead-deep load ring, as in conv_fd_kernel; the
+    // load cursor walks this CTA's (tile, K tile) sequence, skipping tiles
+    // with an empty K range (none with the host's split plan).
+    const int t = threadIdx.x - kV2ProdWarp0 * 32;
+    int total = 0;
+    for (int tl = blockIdx.x; tl < p.tiles; tl += gridDim.x) {
+      int m_, n_, s_;
+      decode(tl, m_, n_, s_);
+      const int k0 = s_ * p.kt_per_split;
+      total += max(0, min(p.ktiles, k0 + p.kt_per_split) - k0);
+    }
+    using Prod = WgProducer<FMT, BN, NU>;
+    constexpr int kLookahead = Prod::PER >= 4 ? 2 : 3;      // keep the ring in registers
+    Prod ring[kLookahead];
+    int ltile = blockIdx.x, lkt = 0, lkt1 = 0, lmt = 0, lnt = 0;
+    auto seek = [&]() {                        // first tile at or after ltile with work
+      while (ltile < p.tiles) {
+        int sp_;
+        decode(ltile, lmt, lnt, sp_);
+        lkt = sp_ * p.kt_per_split;
+        lkt1 = min(p.ktiles, lkt + p.kt_per_split);
+        if (lkt < lkt1) return;
+        ltile += gridDim.x;
+      }
+    };
+    seek();
+    auto load_next = [&](Prod& pr) {
+      pr.load(p, lmt, lnt, lkt, t);
+      if (++lkt == lkt1) { ltile += gridDim.x; seek(); }
+    };
+#pragma unroll
+    for (int r = 0; r < kLookahead; ++r)
+      if (r < total) load_next(ring[r]);
+    for (int kit = 0; kit < total;) {
+#pragma unroll
+      for (int r = 0; r < kLookahead; ++r, ++kit) {
+        if (kit >= total) break;
+        const int s = kit % kV2Stages;
+        mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
+        ring[r].store(sbase + s * L::kStage, t);
+        producer_warp_arrive(&bars->full[s]);
+        if (kit + kLookahead < total) load_next(ring[r]);
+      }
+    }
+  }
+  v2_teardown<BN>(bars);
+}
+
+}  // namespace mqv

@@ -35,46 +35,48 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
 }
 
 // ------------------------------------------------- element rounding (a >= 0)
-// Each element grid is piecewise uniform: E2M1 steps 0.5 on [0,2), 1 on
-// [2,4), 2 on [4,6]; E2M3 steps 1/8 on [0,2), 1/4 on [2,4), 1/2 on [4,7.5].
-// Within a piece, magnitude code = piece base + (a - start)/step, and the
-// scaling by a power of two and the subtraction are exact, so rintf's
-// ties-to-even gives ties to the even code.
-template <int FMT>
-__device__ __forceinline__ uint32_t round_rne_mag(float a) {
-  if (FMT == 0) {
-    if (!(a <= 6.0f)) return 7u;
-    if (a < 2.0f) return static_cast<uint32_t>(rintf(a * 2.0f));
-    if (a < 4.0f) return 4u + static_cast<uint32_t>(rintf(a - 2.0f));
-    return 6u + static_cast<uint32_t>(rintf((a - 4.0f) * 0.5f));
-  } else {
-    if (!(a <= 7.5f)) return 31u;
-    if (a < 2.0f) return static_cast<uint32_t>(rintf(a * 8.0f));
-    if (a < 4.0f) return 16u + static_cast<uint32_t>(rintf((a - 2.0f) * 4.0f));
-    return 24u + static_cast<uint32_t>(rintf((a - 4.0f) * 2.0f));
-  }
-}
-
+// Round-to-nearest-even onto the element grid is the hardware conversion
+// (cvt.rn.satfinite.e2m1x2 / e2m3x2, see mqv_ptx.cuh).  For stochastic
+// rounding each grid is used as piecewise uniform: E2M1 steps 0.5 on [0,2),
+// 1 on [2,4), 2 on [4,6]; E2M3 steps 1/8 on [0,2), 1/4 on [2,4), 1/2 on
+// [4,7.5]; within a piece, code = piece base + (a - start)/step, where the
+// subtraction and the power-of-two scaling are exact.
 // Stochastic rounding: q = position in units of the local step, round up
-// iff u < frac(q) (frac is exact: q is an exact rescaling of a).
+// iff u < frac(q) (frac is exact: q is an exact rescaling of a).  Selects
+// instead of branches, since neighbouring lanes land in different pieces.
 template <int FMT>
 __device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
   float q;
   uint32_t base;
   if (FMT == 0) {
-    if (!(a < 6.0f)) return 7u;
-    if (a < 2.0f) { q = a * 2.0f; base = 0u; }
-    else if (a < 4.0f) { q = a - 2.0f; base = 4u; }
-    else { q = (a - 4.0f) * 0.5f; base = 6u; }
+    const bool p0 = a < 2.0f, p1 = a < 4.0f;
+    q = p0 ? a * 2.0f : (p1 ? a - 2.0f : (a - 4.0f) * 0.5f);
+    base = p0 ? 0u : (p1 ? 4u : 6u);
   } else {
-    if (!(a < 7.5f)) return 31u;
-    if (a < 2.0f) { q = a * 8.0f; base = 0u; }
-    else if (a < 4.0f) { q = (a - 2.0f) * 4.0f; base = 16u; }
-    else { q = (a - 4.0f) * 2.0f; base = 24u; }
+    const bool p0 = a < 2.0f, p1 = a < 4.0f;
+    q = p0 ? a * 8.0f : (p1 ? (a - 2.0f) * 4.0f : (a - 4.0f) * 2.0f);
+    base = p0 ? 0u : (p1 ? 16u : 24u);
   }
   const float fl = floorf(q);
   const float f = q - fl;
-  return base + static_cast<uint32_t>(fl) + (u < f ? 1u : 0u);
+  const uint32_t mag = base + static_cast<uint32_t>(fl) + (u < f ? 1u : 0u);
+  const float top = FMT == 0 ? 6.0f : 7.5f;
+  return a < top ? mag : (FMT == 0 ? 7u : 31u);
+}
+
+// Correctly rounded a / d for the elements of a block, which share d, by
+// Markstein's method (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also
+// Muller et al., Handbook of Floating-Point Arithmetic, 2nd ed., 2018,
+// sec. 4.9): with y = RN(1/d) and q0 = RN(a·y) within one ulp of a/d, the
+// remainder r = a - d·q0 is exact (one FMA) and RN(q0 + r·y) = RN(a/d).
+// The theorem assumes no underflow, so tiny nonzero quotients take the IEEE
+// divide (a = 0 gives q1 = 0 exactly and stays on the fast path).
+__device__ __forceinline__ float div_shared_divisor(float a, float d, float y) {
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-d, q0, a);
+  const float q1 = __fmaf_rn(r, y, q0);
+  return (q0 >= 1.0e-30f || a == 0.0f) ? q1 : __fdiv_rn(a, d);
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
@@ -143,13 +145,48 @@ amax_finish_kernel(const float* __restrict__ partial, int count, float* __restri
 }
 
 // ----------------------------------------------------------- quantize
-// One thread per 4 x 4 block of the rows x cols view, consecutive threads on
-// consecutive column blocks (coalesced float4 reads of each of the 4 rows).
-// `amax_src` holds `amax_count` partial maxima; every CTA reduces them.
+// One thread per QB horizontally adjacent 4 x 4 blocks of the rows x cols
+// view (QB = 2 when the view has an even number of column blocks, so each
+// thread keeps eight float4 loads in flight and stores 32-bit code words);
+// consecutive threads take consecutive column blocks, so each of the 4 rows
+// is read as one coalesced run.  `amax_src` holds `amax_count` partial
+// maxima; every CTA reduces them.  Stochastic rounding numbers element
+// (r, c) as r·sr_cols + sr_col0 + c, so a column slice of a wider view (a
+// batch shard) draws the words the whole view would (sr_cols = cols,
+// sr_col0 = 0 for an unsharded tensor).
 template <int FMT, int RND>
+__device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d, float y, const float (&u)[4]) {
+  float v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = d > 0.0f ? div_shared_divisor(fabsf(xv[j]), d, y) : 0.0f;
+  uint32_t mag[4];
+  if (RND == 0) {
+    if (FMT == 0) {
+      const uint32_t b01 = f32x2_to_e2m1x2(v[0], v[1]), b23 = f32x2_to_e2m1x2(v[2], v[3]);
+      mag[0] = b01 & 0xF; mag[1] = b01 >> 4; mag[2] = b23 & 0xF; mag[3] = b23 >> 4;
+    } else {
+      const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
+      mag[0] = b01 & 0x3F; mag[1] = (b01 >> 8) & 0x3F; mag[2] = b23 & 0x3F; mag[3] = (b23 >> 8) & 0x3F;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mag[j] = round_sr_mag<FMT>(v[j], u[j]);
+  }
+  uint32_t packed = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
+    const uint32_t code = FMT == 0 ? (mag[j] | (sgn << 3)) : (mag[j] | (sgn << 5));
+    packed |= code << (j * (FMT == 0 ? 4 : 6));
+  }
+  return packed;
+}
+
+template <int FMT, int RND, int QB>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
                 const float* __restrict__ amax_src, int amax_count, uint64_t seed,
+                int64_t sr_cols, int64_t sr_col0,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                 float* __restrict__ tscale) {
   __shared__ float red[32];
@@ -159,66 +196,81 @@ quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
   const float Temax = __fmul_rn(T, emax);
   if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = T;
 
-  const int64_t cb = cols >> 2;
-  const int64_t nblocks = (rows >> 2) * cb;
+  const int64_t cb = cols >> 2;                       // column blocks per block row
+  const int64_t cu = cb / QB;                         // work units per block row
+  const int64_t nunits = (rows >> 2) * cu;
   const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
 
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; b < nblocks;
-       b += stride) {
-    const int64_t br = b / cb, bc = b - br * cb;
-    const float* p = src + (br * 4) * cols + bc * 4;
-    float4 x[4];
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; w < nunits;
+       w += stride) {
+    const int64_t br = w / cu;
+    const int64_t bc0 = (w - br * cu) * QB;
+    const float* p = src + (br * 4) * cols + bc0 * 4;
+    float4 x[QB][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) x[r] = __ldg(reinterpret_cast<const float4*>(p + r * cols));
-    float bmax = 0.0f;
+    for (int q = 0; q < QB; ++q)
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-      bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[r].x), fabsf(x[r].y)),
-                               fmaxf(fabsf(x[r].z), fabsf(x[r].w))));
-    uint32_t scode = 0;
-    float d = 0.0f;
-    if (T > 0.0f) {
-      scode = f32_to_e4m3_satfinite(__fdiv_rn(bmax, Temax));
-      d = __fmul_rn(e4m3_to_f32(scode), T);
+      for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
+    uint32_t scode[QB];
+    float d[QB], y[QB];
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      float bmax = 0.0f;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[q][r].x), fabsf(x[q][r].y)),
+                                 fmaxf(fabsf(x[q][r].z), fabsf(x[q][r].w))));
+      scode[q] = 0;
+      d[q] = 0.0f;
+      y[q] = 0.0f;
+      if (T > 0.0f) {
+        scode[q] = f32_to_e4m3_satfinite(__fdiv_rn(bmax, Temax));
+        d[q] = __fmul_rn(e4m3_to_f32(scode[q]), T);
+        y[q] = d[q] > 0.0f ? __frcp_rn(d[q]) : 0.0f;
+      }
     }
-    scales[b] = static_cast<uint8_t>(scode);
+    const int64_t b = br * cb + bc0;
+    if (QB == 2) *reinterpret_cast<uint16_t*>(scales + b) = static_cast<uint16_t>(scode[0] | (scode[1] << 8));
+    else scales[b] = static_cast<uint8_t>(scode[0]);
 
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float xv[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
-      float u[4] = {0.f, 0.f, 0.f, 0.f};
-      if (RND == 1) {
-        const uint64_t g = static_cast<uint64_t>((br * 4 + r) * cols + bc * 4) >> 2;
-        const uint4 w = philox4x32_10(
-            make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), k0, k1);
-        const float s24 = 5.9604644775390625e-08f;   // 2^-24
-        u[0] = __uint2float_rn(w.x >> 8) * s24;
-        u[1] = __uint2float_rn(w.y >> 8) * s24;
-        u[2] = __uint2float_rn(w.z >> 8) * s24;
-        u[3] = __uint2float_rn(w.w >> 8) * s24;
-      }
-      uint32_t packed = 0;
+      uint32_t packed[QB];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t mag = 0;
-        if (d > 0.0f) {
-          const float v = __fdiv_rn(fabsf(xv[j]), d);
-          mag = RND == 0 ? round_rne_mag<FMT>(v) : round_sr_mag<FMT>(v, u[j]);
+      for (int q = 0; q < QB; ++q) {
+        const float xv[4] = {x[q][r].x, x[q][r].y, x[q][r].z, x[q][r].w};
+        float u[4] = {0.f, 0.f, 0.f, 0.f};
+        if (RND == 1) {
+          // element index in the (possibly wider) view the SR stream is defined on
+          const uint64_t g = static_cast<uint64_t>((br * 4 + r) * sr_cols + sr_col0 + (bc0 + q) * 4) >> 2;
+          const uint4 wd = philox4x32_10(
+              make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), k0, k1);
+          const float s24 = 5.9604644775390625e-08f;   // 2^-24
+          u[0] = __uint2float_rn(wd.x >> 8) * s24;
+          u[1] = __uint2float_rn(wd.y >> 8) * s24;
+          u[2] = __uint2float_rn(wd.z >> 8) * s24;
+          u[3] = __uint2float_rn(wd.w >> 8) * s24;
         }
-        const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
-        const uint32_t code = FMT == 0 ? (mag | (sgn << 3)) : (mag | (sgn << 5));
-        packed |= code << (j * (FMT == 0 ? 4 : 6));
+        packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], u);
       }
       uint8_t* out = codes + (br * 4 + r) * row_bytes;
       if (FMT == 0) {
-        *reinterpret_cast<uint16_t*>(out + bc * 2) = static_cast<uint16_t>(packed);
+        if (QB == 2) *reinterpret_cast<uint32_t*>(out + bc0 * 2) = packed[0] | (packed[1] << 16);
+        else *reinterpret_cast<uint16_t*>(out + bc0 * 2) = static_cast<uint16_t>(packed[0]);
       } else {
-        out += bc * 3;
-        out[0] = static_cast<uint8_t>(packed);
-        out[1] = static_cast<uint8_t>(packed >> 8);
-        out[2] = static_cast<uint8_t>(packed >> 16);
+        if (QB == 2) {   // 48 bits at a 6-byte (2-aligned) offset
+          uint16_t* o16 = reinterpret_cast<uint16_t*>(out + bc0 * 3);
+          o16[0] = static_cast<uint16_t>(packed[0]);
+          o16[1] = static_cast<uint16_t>((packed[0] >> 16) | (packed[1] << 8));
+          o16[2] = static_cast<uint16_t>(packed[1] >> 8);
+        } else {
+          out += bc0 * 3;
+          out[0] = static_cast<uint8_t>(packed[0]);
+          out[1] = static_cast<uint8_t>(packed[0] >> 8);
+          out[2] = static_cast<uint8_t>(packed[0] >> 16);
+        }
       }
     }
   }

@@ -226,18 +226,28 @@ def tensor_scale(x: np.ndarray, fmt: str) -> np.float32:
     return np.float32(amax / np.float32(E4M3_MAX * element_max(fmt)))
 
 
-def quantize(x2d: np.ndarray, fmt: str, rounding: str, seed: int = 0) -> QTensor:
+def quantize(x2d: np.ndarray, fmt: str, rounding: str, seed: int = 0,
+             amax: float | None = None, row_offset: int = 0,
+             col_offset: int = 0, total_cols: int | None = None) -> QTensor:
     """Square-block (4 x 4) two-level quantization of a 2D fp32 view.
 
     Follows the NVFP4 formulas of section "무엇과 다른가": tensor scale,
     then per 4x4 block B = CastE4M3(blockmax / (T × emax)), then every
     element x -> Round(x / (B × T)).  Rounding is RNE or SR (reading R8).
-    """
+
+    `amax`/`row_offset` quantize a band of rows of a larger view whose
+    max|x| is `amax` and whose first row here is row `row_offset` (used to
+    spot-check very large tensors band by band; the SR counter uses the
+    element's index in the full view).  `col_offset`/`total_cols` do the same
+    for a window of columns (a batch shard of a wider view)."""
     x = np.ascontiguousarray(x2d, dtype=np.float32)
     rows, cols = x.shape
-    assert rows % 4 == 0 and cols % 4 == 0
+    assert rows % 4 == 0 and cols % 4 == 0 and row_offset % 4 == 0
     emax = np.float32(element_max(fmt))
-    T = tensor_scale(x, fmt)
+    if amax is None:
+        T = tensor_scale(x, fmt)
+    else:
+        T = np.float32(np.float32(amax) / np.float32(E4M3_MAX * element_max(fmt)))
     blocks = np.abs(x).reshape(rows // 4, 4, cols // 4, 4)
     bmax = blocks.max(axis=(1, 3)).astype(np.float32)
     mbits = element_bits(fmt) - 1
@@ -254,7 +264,10 @@ def quantize(x2d: np.ndarray, fmt: str, rounding: str, seed: int = 0) -> QTensor
     if rounding == RNE:
         mag = round_rne(v, fmt)
     else:
-        u = sr_uniforms(seed, np.arange(rows * cols, dtype=np.uint64)).reshape(rows, cols)
+        tc = cols if total_cols is None else total_cols
+        r_idx = np.arange(rows, dtype=np.uint64)[:, None] + np.uint64(row_offset)
+        c_idx = np.arange(cols, dtype=np.uint64)[None, :] + np.uint64(col_offset)
+        u = sr_uniforms(seed, (r_idx * np.uint64(tc) + c_idx).reshape(-1)).reshape(rows, cols)
         mag = round_sr(v, u, fmt)
     mag = np.where(d == 0, 0, mag)
     return QTensor(sign | mag, scales, T, fmt)

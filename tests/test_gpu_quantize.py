@@ -89,6 +89,39 @@ def test_rounding_ties_bit_exact(fmt, rnd):
     assert_quant_equal(x, rows, cols, fmt, rnd, 99, (c, s, T))
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+@pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
+def test_division_near_grid_points_with_arbitrary_scales(fmt, rnd):
+    """Elements within a few ulps of RN(m·d) for every grid value and grid
+    midpoint m, with block divisors d = B·T that are not powers of two, so
+    the quotient x/d must be correctly rounded for the code to match."""
+    rng = np.random.default_rng(11 if fmt == "nvfp4" else 12)
+    f = FMT[fmt]
+    emax = np.float32(O.element_max(f))
+    grid = O.element_grid(f)
+    targets = np.concatenate([(grid[:-1] + grid[1:]) / 2, grid[1:]])
+    amax = np.float32(3.7)
+    T = np.float32(amax / np.float32(448.0 * O.element_max(f)))
+    nblocks = 4096
+    x = np.zeros((4 * nblocks, 4), np.float32)
+    x[0, 0] = amax
+    for b in range(1, nblocks):
+        bmax = np.float32(rng.uniform(0.05, 1.0) * amax)
+        B = np.float32(O.E4M3_GRID[O.cast_e4m3(np.array([bmax / np.float32(T * emax)], np.float32))[0]])
+        d = np.float32(B * T)
+        ok = targets[targets * float(d) < float(bmax)]
+        t = rng.choice(ok, 15)
+        v = (t * np.float64(d)).astype(np.float32)
+        steps = rng.integers(-3, 4, 15).astype(np.int32)
+        v = np.where(v > 0, (v.view(np.int32) + steps).view(np.float32), v)
+        v = np.minimum(np.abs(v), bmax)
+        blk = np.concatenate([[bmax], v]).astype(np.float32) * rng.choice([-1.0, 1.0], 16).astype(np.float32)
+        x[4 * b:4 * b + 4] = blk.reshape(4, 4)
+    rows, cols = x.shape
+    q, c, sc, Tg = gpu_quantize(torch.from_numpy(x), rows, cols, fmt, rnd, seed=5)
+    assert_quant_equal(x, rows, cols, fmt, rnd, 5, (c, sc, Tg))
+
+
 def test_zero_tensor_and_negative_zero():
     x = torch.zeros(16, 8)
     x[1, 1] = -0.0
@@ -162,3 +195,24 @@ def test_replay_shapes_large_sampled_bands(C, H, N, rnd):
         assert_quant_equal(xb, 8, cols, "nvfp4", rnd, 23, (cb, sb, T), amax=amax, row_offset=band)
     del x, q
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+def test_batch_shard_quantization_matches_whole_tensor(fmt):
+    """A batch shard quantized with the global amax and its SR column window
+    (as the data-parallel step does) equals the matching columns of the
+    whole tensor's quantization, and the oracle's."""
+    rows, N, world = 7 * 7 * 32, 64, 4
+    x = _rand((rows, N), 21, outliers=True)
+    xd = x.cuda()
+    amax = mqv.amax(xd.view(-1), rows, N)
+    n = N // world
+    for rank in range(world):
+        part = xd[:, rank * n:(rank + 1) * n].contiguous().view(-1)
+        q = mqv.quantize_with_amax(part, rows, n, fmt, mqv.SR, 41, amax, sr_col0=rank * n, sr_cols=N)
+        torch.cuda.synchronize()
+        gq = (q.codes.cpu().numpy(), q.scales.cpu().numpy(), q.tscale.item())
+        oq = O.quantize(x.numpy()[:, rank * n:(rank + 1) * n], FMT[fmt], O.SR, 41,
+                        amax=float(x.abs().max()), col_offset=rank * n, total_cols=N)
+        assert np.array_equal(gq[0], O.pack_codes(oq.codes, FMT[fmt]))
+        assert np.array_equal(gq[1], oq.scales.reshape(-1)) and np.float32(gq[2]) == oq.T
