@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/mqv.h"
+#include "mqv.h"
 #include "mqv_conv_common.cuh"
 #include "mqv_conv_kernels.cuh"
 #include "mqv_quantize.cuh"
@@ -246,6 +246,7 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   a.dCred = make_fastdiv(a.Cred);
   a.dKw = make_fastdiv(a.Kw);
   a.dCin = make_fastdiv(a.Cin);
+  a.dS = make_fastdiv(a.stride);
   pl->nu = (d->N % 8 == 0) ? 8 : 4;
   // Columns per tile: the option with the smaller (waves x tile width) over
   // one persistent CTA per SM; ties go to the wider tile.

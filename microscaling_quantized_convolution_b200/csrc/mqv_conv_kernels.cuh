@@ -79,15 +79,21 @@ struct V2Args {
   int mtiles, ntiles;
   int tiles;              // mtiles * ntiles * splits
   int scale_out;          // multiply by T_a·T_b (0 for wgrad split partials)
-  FastDiv dN, dWo, dW, dCred, dKw, dCin;
+  FastDiv dN, dWo, dW, dCred, dKw, dCin, dS;
 };
+
+// Entries of the per-CTA K-tile table of the forward / input-gradient
+// producers (16 per K tile): larger contractions decode on the fly.
+constexpr int kKtabEntries = 4096;
+constexpr uint32_t kKtabInvalid = 0xFFFFFFFFu;
 
 template <int BN>
 struct V2Smem {
   static constexpr int kBTile = BN * 128;
   static constexpr int kStage = kATileBytes + kBTile;
   static constexpr int kBarOffset = kV2Stages * kStage;
-  static constexpr int kBytes = kBarOffset + 256 + 1024;
+  static constexpr int kKtabOffset = kBarOffset + 256;
+  static constexpr int kBytes = kKtabOffset + kKtabEntries * 4 + 1024;
 };
 
 // MN-major 128B-swizzled fp16 tile of BN rows (MN) x 64 K: atoms of 64 MN x
@@ -344,11 +350,51 @@ __device__ __forceinline__ void store_unit(const UnitRaw<FMT, NU>& u, uint32_t t
   }
 }
 
-// Forward / input-gradient B producer.  Unit u of a K tile: column group
-// g = u % G (NU batch items of one output pixel), channel quad kq = u / G.
-// Consecutive lanes take consecutive column groups, so the 4-byte code loads
-// of a warp are contiguous and each 8-lane phase of a 16-byte shared store
-// lands on 8 different swizzled chunks.
+// Forward / input-gradient B producer.
+//
+// K index k = (kh, kw, c) of the reduction decomposes the same way in every
+// output tile, so each CTA tabulates it once per (K tile, channel quad):
+// entry = (dh + 128) | (dw + 128) << 8 | c << 16 with (dh, dw) = (kh - pad,
+// kw - pad) for the forward pass and (pad - kh, pad - kw) for the input
+// gradient, or kKtabInvalid past the contraction.
+template <int PASS>
+__device__ __forceinline__ uint32_t ktab_entry(const V2Args& p, int kt, int kq) {
+  const int k = kt * 64 + 4 * kq;
+  if (k >= p.Kdim) return kKtabInvalid;
+  const int tap = fdiv(k, p.dCred);
+  const int c = k - tap * p.Cred;
+  const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
+  const int dh = PASS == kFwd ? kh - p.pad : p.pad - kh;
+  const int dw = PASS == kFwd ? kw - p.pad : p.pad - kw;
+  return static_cast<uint32_t>(dh + 128) | (static_cast<uint32_t>(dw + 128) << 8) |
+         (static_cast<uint32_t>(c) << 16);
+}
+
+// Output-tile column of a producer thread: NU batch items of one pixel.
+struct TileCol {
+  int h, w;       // fwd: ho·s, wo·s;  dgrad: hi, wi
+  int n;
+  bool ok;
+};
+
+template <int PASS>
+__device__ __forceinline__ TileCol tile_col(const V2Args& p, int64_t col) {
+  TileCol c;
+  c.ok = col < p.Ncols;
+  const int c32 = c.ok ? static_cast<int>(col) : 0;
+  const int pix = fdiv(c32, p.dN);
+  c.n = c32 - pix * p.N;
+  const int ph = fdiv(pix, PASS == kFwd ? p.dWo : p.dW);
+  const int pw = pix - ph * (PASS == kFwd ? p.Wo : p.W);
+  c.h = PASS == kFwd ? ph * p.stride : ph;
+  c.w = PASS == kFwd ? pw * p.stride : pw;
+  return c;
+}
+
+// Unit u of a K tile: column group g = u % G (NU batch items of one output
+// pixel), channel quad kq = u / G.  Consecutive lanes take consecutive
+// column groups, so the 4-byte code loads of a warp are contiguous and each
+// 8-lane phase of a 16-byte shared store lands on 8 different swizzled chunks.
 template <int PASS, int FMT, int BN, int NU>
 struct FdProducer {
   static constexpr int G = BN / NU;
@@ -357,37 +403,32 @@ struct FdProducer {
   static_assert(kV2ProdThreads % G == 0 && UNITS % kV2ProdThreads == 0, "producer mapping");
   UnitRaw<FMT, NU> raw[PER];
 
-  __device__ __forceinline__ void load(const V2Args& p, int64_t col0, int kt, int t) {
-    const int g = t % G;
-    const int64_t col = col0 + static_cast<int64_t>(g) * NU;
-    const bool col_ok = col < p.Ncols;
-    const int c32 = col_ok ? static_cast<int>(col) : 0;
-    const int pix = fdiv(c32, p.dN);
-    const int n = c32 - pix * p.N;
-    const int ph = fdiv(pix, PASS == kFwd ? p.dWo : p.dW);
-    const int pw = pix - ph * (PASS == kFwd ? p.Wo : p.W);
+  __device__ __forceinline__ void load(const V2Args& p, const TileCol& tc, int kt, int t,
+                                       const uint32_t* ktab) {
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int kq = t / G + (kV2ProdThreads / G) * i;
-      const int k = kt * 64 + 4 * kq;
-      bool ok = col_ok && k < p.Kdim;
-      int64_t row = 0;
-      if (ok) {
-        const int tap = fdiv(k, p.dCred);
-        const int c = k - tap * p.Cred;
-        const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
-        if (PASS == kFwd) {
-          const int sh = ph * p.stride + kh - p.pad, sw = pw * p.stride + kw - p.pad;
-          ok = sh >= 0 && sh < p.H && sw >= 0 && sw < p.W;
-          row = (static_cast<int64_t>(sh) * p.W + sw) * p.Cred + c;
-        } else {
-          const int th = ph + p.pad - kh, tw = pw + p.pad - kw;
-          const int sh = th / p.stride, sw = tw / p.stride;
-          ok = th >= 0 && tw >= 0 && sh * p.stride == th && sw * p.stride == tw && sh < p.Ho && sw < p.Wo;
-          row = (static_cast<int64_t>(sh) * p.Wo + sw) * p.Cred + c;
+      const uint32_t e = ktab ? ktab[kt * 16 + kq] : ktab_entry<PASS>(p, kt, kq);
+      bool ok = tc.ok && e != kKtabInvalid;
+      const int dh = static_cast<int>(e & 0xFF) - 128, dw = static_cast<int>((e >> 8) & 0xFF) - 128;
+      const int c = static_cast<int>(e >> 16);
+      int pix = 0;
+      if (PASS == kFwd) {
+        const int sh = tc.h + dh, sw = tc.w + dw;
+        ok = ok && sh >= 0 && sh < p.H && sw >= 0 && sw < p.W;
+        pix = sh * p.W + sw;
+      } else {
+        const int th = tc.h + dh, tw = tc.w + dw;     // = hi + pad - kh, wi + pad - kw
+        int sh = th, sw = tw;
+        if (p.stride != 1) {
+          sh = th >= 0 ? fdiv(th, p.dS) : -1;
+          sw = tw >= 0 ? fdiv(tw, p.dS) : -1;
+          ok = ok && sh * p.stride == th && sw * p.stride == tw;
         }
+        ok = ok && sh >= 0 && sh < p.Ho && sw >= 0 && sw < p.Wo;
+        pix = sh * p.Wo + sw;
       }
-      load_unit<FMT, NU>(p.b, row, n, ok, raw[i]);
+      load_unit<FMT, NU>(p.b, static_cast<int64_t>(pix) * p.Cred + c, tc.n, ok, raw[i]);
     }
   }
 
@@ -479,10 +520,22 @@ conv_fd_kernel(const V2Args p) {
     using Prod = FdProducer<PASS, FMT, BN, NU>;
     constexpr int kLookahead = Prod::PER >= 4 ? 2 : 3;      // keep the ring in registers
     Prod ring[kLookahead];
+    // the CTA's K-tile table, built once by the producer warps
+    uint32_t* ktab = nullptr;
+    if (p.ktiles * 16 <= kKtabEntries) {
+      ktab = reinterpret_cast<uint32_t*>(smem + L::kKtabOffset);
+      for (int e = t; e < p.ktiles * 16; e += kV2ProdThreads) ktab[e] = ktab_entry<PASS>(p, e >> 4, e & 15);
+      asm volatile("bar.sync 1, %0;" ::"n"(kV2ProdThreads) : "memory");
+    }
     int ltile = blockIdx.x, lkt = 0;          // load cursor
+    TileCol tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
     auto load_next = [&](Prod& pr) {
-      pr.load(p, static_cast<int64_t>(ltile % p.ntiles) * BN, lkt, t);
-      if (++lkt == p.ktiles) { lkt = 0; ltile += gridDim.x; }
+      pr.load(p, tc, lkt, t, ktab);
+      if (++lkt == p.ktiles) {
+        lkt = 0;
+        ltile += gridDim.x;
+        tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
+      }
     };
 #pragma unroll
     for (int r = 0; r < kLookahead; ++r)
@@ -507,42 +560,71 @@ conv_fd_kernel(const V2Args p) {
 // tile.  Unit = 4 view rows x NU consecutive batch items of one pixel; lane
 // order runs along K first (KG units per tile row), so a warp reads
 // contiguous code bytes of each row.
+// Contraction position of a producer thread in the weight-gradient pass:
+// q = kt·64 + kg·NU = (pixel, n); stepped from one K tile to the next without
+// divisions (q grows by 64 per tile).
+struct WgPos {
+  int ho, wo, n;
+  bool ok;
+};
+
+__device__ __forceinline__ WgPos wg_pos(const V2Args& p, int q) {
+  WgPos w;
+  w.ok = q < p.Kdim;
+  const int qq = w.ok ? q : 0;
+  const int pix = fdiv(qq, p.dN);
+  w.n = qq - pix * p.N;
+  w.ho = fdiv(pix, p.dWo);
+  w.wo = pix - w.ho * p.Wo;
+  return w;
+}
+
+__device__ __forceinline__ void wg_advance(const V2Args& p, WgPos& w, int q_next) {
+  w.ok = q_next < p.Kdim;
+  w.n += 64;
+  while (w.n >= p.N) {
+    w.n -= p.N;
+    if (++w.wo == p.Wo) {
+      w.wo = 0;
+      ++w.ho;
+    }
+  }
+}
+
+// Weight-gradient producer: the K-major A (G_Y) and B (X') tiles of one K
+// tile.  Unit = 4 view rows x NU consecutive batch items of one pixel; lane
+// order runs along K first (KG units per tile row), so a warp reads
+// contiguous code bytes of each row and every unit of a thread has the same
+// contraction position.
 template <int FMT, int NU, int ROWS>
 struct WgOperand {
   static constexpr int KG = 64 / NU;
   static constexpr int UNITS = (ROWS / 4) * KG;
   static constexpr int PER = UNITS / kV2ProdThreads;
-  static_assert(UNITS % kV2ProdThreads == 0, "producer mapping");
+  static_assert(UNITS % kV2ProdThreads == 0 && kV2ProdThreads % KG == 0, "producer mapping");
   UnitRaw<FMT, NU> raw[PER];
 
   template <bool IS_A>
-  __device__ __forceinline__ void load(const V2Args& p, const QView& v, int row_base, int kt, int t) {
+  __device__ __forceinline__ void load(const V2Args& p, const QView& v, int row_base, const WgPos& w, int t) {
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int u = t + kV2ProdThreads * i;
-      const int kg = u % KG, rq = u / KG;
-      const int q = kt * 64 + kg * NU;              // (pixel, n) contraction index
+      const int rq = u / KG;
       const int r0 = row_base + 4 * rq;
-      bool ok = q < p.Kdim;
+      bool ok = w.ok;
       int64_t row = 0;
-      int n = 0;
-      if (ok) {
-        const int pix = fdiv(q, p.dN);
-        n = q - pix * p.N;
-        if (IS_A) {
-          ok = r0 < p.M;
-          row = static_cast<int64_t>(pix) * p.Cout + r0;
-        } else {
-          ok = r0 < p.Ncols;
-          const int tap = fdiv(r0, p.dCin), ci = r0 - tap * p.Cin;
-          const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
-          const int ho = fdiv(pix, p.dWo), wo = pix - ho * p.Wo;
-          const int hi = ho * p.stride + kh - p.pad, wi = wo * p.stride + kw - p.pad;
-          ok = ok && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
-          row = (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci;
-        }
+      if (IS_A) {
+        ok = ok && r0 < p.M;
+        row = static_cast<int64_t>(w.ho * p.Wo + w.wo) * p.Cout + r0;
+      } else {
+        ok = ok && r0 < p.Ncols;
+        const int tap = fdiv(r0, p.dCin), ci = r0 - tap * p.Cin;
+        const int kh = fdiv(tap, p.dKw), kw = tap - kh * p.Kw;
+        const int hi = w.ho * p.stride + kh - p.pad, wi = w.wo * p.stride + kw - p.pad;
+        ok = ok && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
+        row = (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci;
       }
-      load_unit<FMT, NU>(v, row, n, ok, raw[i]);
+      load_unit<FMT, NU>(v, row, w.n, ok, raw[i]);
     }
   }
 
@@ -561,9 +643,9 @@ struct WgProducer {
   WgOperand<FMT, NU, 128> a;
   WgOperand<FMT, NU, BN> b;
   static constexpr int PER = WgOperand<FMT, NU, 128>::PER + WgOperand<FMT, NU, BN>::PER;
-  __device__ __forceinline__ void load(const V2Args& p, int mt, int nt, int kt, int t) {
-    a.template load<true>(p, p.a, mt * 128, kt, t);
-    b.template load<false>(p, p.b, nt * BN, kt, t);
+  __device__ __forceinline__ void load(const V2Args& p, int mt, int nt, const WgPos& w, int t) {
+    a.template load<true>(p, p.a, mt * 128, w, t);
+    b.template load<false>(p, p.b, nt * BN, w, t);
   }
   __device__ __forceinline__ void store(uint32_t a_tile, int t) const {
     a.store(a_tile, t);
@@ -655,9 +737,17 @@ conv_wg_kernel(const V2Args p) {
       }
     };
     seek();
+    const int kg_off = (t % WgOperand<FMT, NU, 128>::KG) * NU;   // this thread's K offset in a tile
+    WgPos wpos = wg_pos(p, lkt * 64 + kg_off);
     auto load_next = [&](Prod& pr) {
-      pr.load(p, lmt, lnt, lkt, t);
-      if (++lkt == lkt1) { ltile += gridDim.x; seek(); }
+      pr.load(p, lmt, lnt, wpos, t);
+      if (++lkt == lkt1) {
+        ltile += gridDim.x;
+        seek();
+        wpos = wg_pos(p, lkt * 64 + kg_off);
+      } else {
+        wg_advance(p, wpos, lkt * 64 + kg_off);
+      }
     };
 #pragma unroll
     for (int r = 0; r < kLookahead; ++r)
