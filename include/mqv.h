@@ -133,6 +133,28 @@ mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols,
                                   const float* amax, int64_t sr_col0, int64_t sr_cols,
                                   const mqv_qtensor* out, void* stream);
 
+/* One tensor of a mqv_quantize_many call: the arguments of mqv_quantize_cbf. */
+typedef struct {
+  const float* src;
+  int64_t rows, cols;
+  int32_t fmt, rounding;
+  uint64_t seed;
+  mqv_qtensor out;
+} mqv_quantize_job;
+
+/* Workspace bytes of mqv_quantize_many for these jobs.  Host-only. */
+mqv_status mqv_quantize_many_workspace_size(const mqv_quantize_job* jobs, int32_t count,
+                                            size_t* bytes);
+
+/* Quantize 1..8 tensors (for a layer: X and W with RNE, G_Y with SR) in two
+ * launches: one amax pass over all of them, then one quantize pass.  Each
+ * tensor's codes, scales and T are bit-identical to mqv_quantize_cbf on it
+ * alone.  jobs: host array; every job is validated as mqv_quantize_cbf's
+ * arguments are; outputs must not overlap.  ws: at least
+ * mqv_quantize_many_workspace_size bytes, 16-byte aligned. */
+mqv_status mqv_quantize_many(const mqv_quantize_job* jobs, int32_t count, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* dst[r][c] = code·B·T of a quantized view, fp32 (code·B is exact in fp16;
  * the product with T is one fp32 rounding).  Reads a stored (for example
  * latent-replay) tensor back.  dst: rows x cols fp32, 16-byte aligned. */

@@ -49,6 +49,12 @@ class QTensorC(ctypes.Structure):
                 ("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class QuantJobC(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("fmt", ctypes.c_int32), ("rounding", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("out", QTensorC)]
+
+
 _lib = None
 
 _SIGS = {
@@ -80,6 +86,10 @@ _SIGS = {
                                       ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_device_errors": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_void_p]),
+    "mqv_quantize_many_workspace_size": (ctypes.c_int, [ctypes.POINTER(QuantJobC), ctypes.c_int32,
+                                                        ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_quantize_many": (ctypes.c_int, [ctypes.POINTER(QuantJobC), ctypes.c_int32, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_conv_wgrad_noalloc": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                               ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
 }
@@ -174,6 +184,34 @@ def quantize(src: torch.Tensor, rows: int, cols: int, fmt, rounding: int = RNE, 
     _check(lib().mqv_quantize_cbf(src.data_ptr(), rows, cols, _fmt(fmt), rounding, seed,
                                   ctypes.byref(qc), ws.data_ptr(), ws.numel(), _stream(stream)))
     return out
+
+
+def quantize_many(jobs, ws: torch.Tensor | None = None, stream=None) -> list[QTensor]:
+    """Quantize several tensors in two launches (see mqv_quantize_many).
+    jobs: (src, rows, cols, fmt, rounding, seed[, out QTensor]) tuples."""
+    outs, cjobs = [], []
+    for j in jobs:
+        src, rows, cols, fmt, rnd, seed = j[:6]
+        _require_cuda(src, "src", torch.float32)
+        out = j[6] if len(j) > 6 and j[6] is not None else QTensor.empty(rows, cols, fmt, src.device)
+        outs.append(out)
+        cjobs.append(QuantJobC(src.data_ptr(), rows, cols, _fmt(fmt), rnd, seed, out.c()))
+    arr = (QuantJobC * len(cjobs))(*cjobs)
+    if ws is None:
+        b = ctypes.c_size_t()
+        _check(lib().mqv_quantize_many_workspace_size(arr, len(cjobs), ctypes.byref(b)))
+        ws = torch.empty(b.value, dtype=torch.uint8, device=jobs[0][0].device)
+    _check(lib().mqv_quantize_many(arr, len(cjobs), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return outs
+
+
+def quantize_many_workspace_bytes(jobs) -> int:
+    cjobs = [QuantJobC(0, j[1], j[2], _fmt(j[3]), j[4], j[5], QTensorC(16, 16, 16, j[1], j[2], _fmt(j[3]), 0))
+             for j in jobs]
+    arr = (QuantJobC * len(cjobs))(*cjobs)
+    b = ctypes.c_size_t()
+    _check(lib().mqv_quantize_many_workspace_size(arr, len(cjobs), ctypes.byref(b)))
+    return b.value
 
 
 def amax(src: torch.Tensor, rows: int, cols: int, out: torch.Tensor | None = None,

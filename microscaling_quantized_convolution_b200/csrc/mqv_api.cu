@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <string>
 
 #include "mqv.h"
 #include "mqv_conv_common.cuh"
@@ -411,6 +412,47 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
   return ok();
 }
 
+// CTA ranges of every job; pointers are checked only when the plan launches.
+static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count, QuantJobs* plan,
+                                     int* amax_total, int* quant_total, bool check_pointers) {
+  if (!jobs || count < 1 || count > kMaxQuantJobs)
+    return fail(MQV_ERR_INVALID_ARG, "mqv_quantize_many: 1..%d jobs, got %d", kMaxQuantJobs, count);
+  std::memset(plan, 0, sizeof(*plan));
+  plan->count = count;
+  int a = 0, q = 0;
+  for (int i = 0; i < count; ++i) {
+    const mqv_quantize_job& j = jobs[i];
+    mqv_status st = MQV_OK;
+    if (check_pointers) {
+      st = check_quantize_args(j.src, j.rows, j.cols, j.fmt, j.rounding, &j.out);
+    } else if (!(st = check_view(j.rows, j.cols)) && !(st = check_fmt(j.fmt)) &&
+               j.rounding != MQV_RNE && j.rounding != MQV_SR) {
+      st = fail(MQV_ERR_INVALID_ARG, "unknown rounding %d", j.rounding);
+    }
+    if (st) return fail(st, "job %d: %s", i, std::string(g_msg).c_str());
+    QuantJob& qj = plan->job[i];
+    qj.src = j.src;
+    qj.rows = j.rows;
+    qj.cols = j.cols;
+    qj.codes = static_cast<uint8_t*>(j.out.codes);
+    qj.scales = j.out.scales;
+    qj.tscale = j.out.tscale;
+    qj.seed = j.seed;
+    qj.fmt = j.fmt;
+    qj.rounding = j.rounding;
+    qj.qb = (j.cols / 4) % 2 == 0 ? 2 : 1;
+    qj.amax_cta0 = a;
+    qj.amax_ctas = (int)amax_ctas(j.rows, j.cols);
+    qj.quant_cta0 = q;
+    qj.quant_ctas = (int)quant_ctas(j.rows, qj.qb == 2 ? j.cols / 2 : j.cols);
+    a += qj.amax_ctas;
+    q += qj.quant_ctas;
+  }
+  *amax_total = a;
+  *quant_total = q;
+  return MQV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -485,6 +527,34 @@ mqv_status mqv_quantize_with_amax(const float* src, int64_t rows, int64_t cols, 
                 (long long)sr_col0, (long long)(sr_col0 + cols), (long long)sr_cols);
   return enqueue_quantize(src, rows, cols, fmt, rounding, seed, amax, 1, sr_cols, sr_col0, out,
                           static_cast<cudaStream_t>(stream));
+}
+
+mqv_status mqv_quantize_many_workspace_size(const mqv_quantize_job* jobs, int32_t count,
+                                            size_t* bytes) {
+  if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  QuantJobs plan;
+  int a = 0, q = 0;
+  mqv_status st = plan_quantize_many(jobs, count, &plan, &a, &q, false);
+  if (st) return st;
+  *bytes = (size_t)((a * sizeof(float) + 255) / 256 * 256);
+  return ok();
+}
+
+mqv_status mqv_quantize_many(const mqv_quantize_job* jobs, int32_t count, void* ws, size_t ws_bytes,
+                             void* stream) {
+  QuantJobs plan;
+  int a = 0, q = 0;
+  mqv_status st = plan_quantize_many(jobs, count, &plan, &a, &q, true);
+  if (st) return st;
+  if (!ws || ws_bytes < (size_t)a * sizeof(float) || !aligned16(ws))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes required", (size_t)a * sizeof(float));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  amax_many_kernel<<<a, kAmaxThreads, 0, s>>>(plan, part);
+  quantize_many_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_many launch");
+  return ok();
 }
 
 mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream) {

@@ -84,12 +84,13 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 }
 
 // ------------------------------------------------------------- amax
-// Pass 1: each CTA writes max|x| over its grid-stride share to partial[cta].
-__global__ void __launch_bounds__(kAmaxThreads)
-amax_partial_kernel(const float4* __restrict__ src, int64_t n4, float* __restrict__ partial) {
+// Pass 1: CTA `cta` of `nctas` writes max|x| over its grid-stride share of
+// the n4 float4 of src to *partial.
+__device__ __forceinline__ void amax_partial_body(const float4* __restrict__ src, int64_t n4,
+                                                  float* __restrict__ partial, int cta, int nctas) {
   float m = 0.0f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kAmaxThreads;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * kAmaxThreads + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(nctas) * kAmaxThreads;
+  int64_t i = static_cast<int64_t>(cta) * kAmaxThreads + threadIdx.x;
   for (; i + 3 * stride < n4; i += 4 * stride) {
     const float4 a = __ldg(src + i), b = __ldg(src + i + stride);
     const float4 c = __ldg(src + i + 2 * stride), d = __ldg(src + i + 3 * stride);
@@ -111,8 +112,13 @@ amax_partial_kernel(const float4* __restrict__ src, int64_t n4, float* __restric
     m = threadIdx.x < kAmaxThreads / 32 ? warp_max[threadIdx.x] : 0.0f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (threadIdx.x == 0) partial[blockIdx.x] = m;
+    if (threadIdx.x == 0) *partial = m;
   }
+}
+
+__global__ void __launch_bounds__(kAmaxThreads)
+amax_partial_kernel(const float4* __restrict__ src, int64_t n4, float* __restrict__ partial) {
+  amax_partial_body(src, n4, partial + blockIdx.x, blockIdx.x, gridDim.x);
 }
 
 // Block-wide max over `count` floats (every thread gets the result).
@@ -183,27 +189,26 @@ __device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d,
 }
 
 template <int FMT, int RND, int QB>
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
-                const float* __restrict__ amax_src, int amax_count, uint64_t seed,
-                int64_t sr_cols, int64_t sr_col0,
-                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                float* __restrict__ tscale) {
+__device__ __forceinline__ void quantize_body(const float* __restrict__ src, int64_t rows, int64_t cols,
+                                              const float* __restrict__ amax_src, int amax_count,
+                                              uint64_t seed, int64_t sr_cols, int64_t sr_col0,
+                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                              float* __restrict__ tscale, int cta, int nctas) {
   __shared__ float red[32];
   const float amax = block_max_of(amax_src, amax_count, red);
   const float emax = FMT == 0 ? 6.0f : 7.5f;
   const float T = __fdiv_rn(amax, 448.0f * emax);         // 2688 or 3360, exact
   const float Temax = __fmul_rn(T, emax);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *tscale = T;
+  if (cta == 0 && threadIdx.x == 0) *tscale = T;
 
   const int64_t cb = cols >> 2;                       // column blocks per block row
   const int64_t cu = cb / QB;                         // work units per block row
   const int64_t nunits = (rows >> 2) * cu;
   const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kQuantThreads;
+  const int64_t stride = static_cast<int64_t>(nctas) * kQuantThreads;
 
-  for (int64_t w = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; w < nunits;
+  for (int64_t w = static_cast<int64_t>(cta) * kQuantThreads + threadIdx.x; w < nunits;
        w += stride) {
     const int64_t br = w / cu;
     const int64_t bc0 = (w - br * cu) * QB;
@@ -274,6 +279,72 @@ quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
       }
     }
   }
+}
+
+template <int FMT, int RND, int QB>
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
+                const float* __restrict__ amax_src, int amax_count, uint64_t seed,
+                int64_t sr_cols, int64_t sr_col0,
+                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                float* __restrict__ tscale) {
+  quantize_body<FMT, RND, QB>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes,
+                              scales, tscale, blockIdx.x, gridDim.x);
+}
+
+// ------------------------------------------------ several tensors at once
+// The quantize-once step of a layer (X, W, G_Y) in two launches instead of
+// six: every CTA of a launch serves one tensor ("job"), CTAs are assigned to
+// jobs in contiguous ranges.  Results are bit-identical to one
+// amax_partial_kernel + quantize_kernel pair per tensor with the same CTA
+// counts.
+constexpr int kMaxQuantJobs = 8;
+
+struct QuantJob {
+  const float* src;
+  int64_t rows, cols;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* tscale;
+  uint64_t seed;
+  int32_t fmt, rounding, qb;
+  int32_t amax_cta0, amax_ctas;     // this job's range of amax CTAs (= its partials)
+  int32_t quant_cta0, quant_ctas;   // this job's range of quantize CTAs
+};
+
+struct QuantJobs {
+  QuantJob job[kMaxQuantJobs];
+  int32_t count;
+};
+
+__device__ __forceinline__ int job_of(const QuantJobs& jobs, int cta, bool quant) {
+  int j = 0;
+  for (int i = 1; i < jobs.count; ++i)
+    if (cta >= (quant ? jobs.job[i].quant_cta0 : jobs.job[i].amax_cta0)) j = i;
+  return j;
+}
+
+__global__ void __launch_bounds__(kAmaxThreads)
+amax_many_kernel(const __grid_constant__ QuantJobs jobs, float* __restrict__ partial) {
+  const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, false)];
+  amax_partial_body(reinterpret_cast<const float4*>(jb.src), jb.rows * jb.cols / 4, partial + blockIdx.x,
+                    blockIdx.x - jb.amax_cta0, jb.amax_ctas);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_many_kernel(const __grid_constant__ QuantJobs jobs, const float* __restrict__ partial) {
+  const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, true)];
+  const int cta = blockIdx.x - jb.quant_cta0;
+  const float* amax = partial + jb.amax_cta0;
+#define MQV_QUANT_CASE(F, R, Q)                                                                   \
+  if (jb.fmt == F && jb.rounding == R && jb.qb == Q) {                                            \
+    quantize_body<F, R, Q>(jb.src, jb.rows, jb.cols, amax, jb.amax_ctas, jb.seed, jb.cols, 0,     \
+                           jb.codes, jb.scales, jb.tscale, cta, jb.quant_ctas);                   \
+    return;                                                                                       \
+  }
+  MQV_QUANT_CASE(0, 0, 2) MQV_QUANT_CASE(0, 1, 2) MQV_QUANT_CASE(1, 0, 2) MQV_QUANT_CASE(1, 1, 2)
+  MQV_QUANT_CASE(0, 0, 1) MQV_QUANT_CASE(0, 1, 1) MQV_QUANT_CASE(1, 0, 1) MQV_QUANT_CASE(1, 1, 1)
+#undef MQV_QUANT_CASE
 }
 
 // ---------------------------------------------------------- dequantize

@@ -216,3 +216,26 @@ def test_batch_shard_quantization_matches_whole_tensor(fmt):
                         amax=float(x.abs().max()), col_offset=rank * n, total_cols=N)
         assert np.array_equal(gq[0], O.pack_codes(oq.codes, FMT[fmt]))
         assert np.array_equal(gq[1], oq.scales.reshape(-1)) and np.float32(gq[2]) == oq.T
+
+
+@pytest.mark.parametrize("layer", [workloads.resnet18_layer2(), workloads.yolov8n_mix()[6],
+                                   workloads.tiny_layer()], ids=lambda l: l.name)
+def test_quantize_many_equals_one_call_per_tensor(layer):
+    """The layer's X, W (RNE) and G_Y (SR) in one two-launch call are bit for
+    bit the three single-tensor quantizations (and so the oracle's)."""
+    X, Wt, G = workloads.make_layer_inputs(layer)
+    s = layer
+    views = [(X, s.H * s.W * s.Cin, s.N, mqv.RNE, 0),
+             (Wt, s.Cout, s.K * s.K * s.Cin, mqv.RNE, 0),
+             (G, s.Ho * s.Wo * s.Cout, s.N, mqv.SR, workloads.sr_seed(s)),
+             (_rand((8, 84), 4), 8, 84, mqv.SR, 9)]                     # odd column blocks
+    jobs = [(t.cuda().contiguous().view(-1), r, c, s.fmt, rnd, seed) for t, r, c, rnd, seed in views]
+    many = mqv.quantize_many(jobs)
+    torch.cuda.synchronize()
+    for (t, r, c, rnd, seed), q in zip(views, many):
+        one = mqv.quantize(t.cuda().contiguous().view(-1), r, c, s.fmt, rnd, seed)
+        torch.cuda.synchronize()
+        for f in ("codes", "scales", "tscale"):
+            assert torch.equal(getattr(q, f), getattr(one, f)), f
+    assert_quant_equal(views[3][0].numpy(), 8, 84, s.fmt, mqv.SR, 9,
+                       (many[3].codes.cpu().numpy(), many[3].scales.cpu().numpy(), many[3].tscale.item()))
