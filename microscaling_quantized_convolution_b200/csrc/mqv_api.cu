@@ -13,6 +13,7 @@
 #include "mqv.h"
 #include "mqv_conv_common.cuh"
 #include "mqv_conv_kernels.cuh"
+#include "mqv_conv_halo.cuh"
 #include "mqv_quantize.cuh"
 
 namespace {
@@ -161,6 +162,8 @@ mqv_status check_quantize_args(const float* src, int64_t rows, int64_t cols, int
 
 struct ConvPlan {
   V2Args a;
+  bool halo;            // stride-1 fwd/dgrad with the on-chip halo (conv_halo_kernel)
+  HaloGeom g;
   int bn;               // 128 or 256 columns per tile
   int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0
   int grid;             // persistent CTAs
@@ -269,6 +272,22 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   }
   a.splits = splits;
   a.tiles = (int)(tiles_mn * splits);
+  // Stride-1 fwd/dgrad on NVFP4 with N | 256, N % 8 == 0, a halo of at most
+  // 384 rows and whole 64-channel chunks: the kernel-row halo path.
+  pl->halo = op != MQV_OP_WGRAD && d->fmt == MQV_NVFP4 && d->stride == 1 && d->N % 8 == 0 &&
+             256 % d->N == 0 && (d->Kw - 1) * d->N <= 128 && a.Cred % 64 == 0;
+  if (pl->halo) {
+    HaloGeom& g = pl->g;
+    g.bw = (int)(256 / d->N);
+    g.rows = (int)((g.bw + d->Kw - 1) * d->N);
+    g.out_h = op == MQV_OP_FWD ? a.Ho : a.H;
+    g.out_w = op == MQV_OP_FWD ? a.Wo : a.W;
+    g.src_h = op == MQV_OP_FWD ? a.H : a.Ho;
+    g.src_w = op == MQV_OP_FWD ? a.W : a.Wo;
+    g.tpr = (g.out_w + g.bw - 1) / g.bw;
+    g.cchunks = a.Cred / 64;
+    a.tiles = a.mtiles * g.out_h * g.tpr;
+  }
   a.scale_out = splits == 1;
   pl->grid = a.tiles < kSMs ? a.tiles : kSMs;
   pl->image_bytes = op == MQV_OP_WGRAD ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
@@ -324,7 +343,18 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
 }
 
 template <int PASS>
+cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
+  auto kern = conv_halo_kernel<PASS>;
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
+  if (e != cudaSuccess) return e;
+  kern<<<pl.grid, kV2Threads, HaloSmem::kBytes, st>>>(pl.a, pl.g);
+  return cudaGetLastError();
+}
+
+template <int PASS>
 cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
+  if (PASS != kWgrad && pl.halo) return launch_halo<PASS == kWgrad ? kFwd : PASS>(pl, st);
   return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
 }
 

@@ -1,0 +1,331 @@
+// Stride-1 forward and input-gradient convolution with the im2col tile built
+// once per kernel row on chip (MicroQonv summary, onedev.kr/papers/182,
+// section "어떻게 동작하나": the channel-batch-first layout lets the window
+// slide over channel/batch runs read once and reused on chip).
+//
+// A CTA owns an output tile of BW = 256/N consecutive pixels of one output
+// row x all N batch items (256 GEMM columns) x 128 output channels.  For
+// each kernel row kh and 64-channel chunk of the reduction, the producer
+// warps dequantize the BW + Kw - 1 source pixels the window touches (the
+// "halo") into one K-major shared tile; the Kw taps of that kernel row are
+// then Kw MMA groups on the same tile, each starting kw·N rows further on
+// (a descriptor offset: N % 8 == 0 keeps it on the 8-row swizzle atom).  So
+// every source pixel is dequantized once per kernel row instead of once per
+// tap, and every MMA is 128 x 256 x 16.
+//
+// Forward:        source = X,   row  hi = ho + kh - pad,  columns wi = wo0 - pad + q,
+//                 tap kw uses halo pixels q = j + kw.
+// Input gradient: source = G_Y, row  ho = hi + pad - kh,  columns wo = wi0 + pad - (Kw-1) + q,
+//                 tap kw uses halo pixels q = j + (Kw - 1 - kw).
+// The weight operand is the fp16 image of prep_image_kernel (tap-major K, so
+// the tile of (tap, chunk) is image tile tap·(Cred/64) + chunk), one 16 KB
+// bulk copy per tap.  Roles, bounded waits and the double-buffered
+// accumulators are those of conv_fd_kernel.
+#pragma once
+
+#include <cstdint>
+
+#include "mqv_conv_common.cuh"
+#include "mqv_conv_kernels.cuh"
+#include "mqv_ptx.cuh"
+
+namespace mqv {
+
+constexpr int kHaloBN = 256;                  // GEMM columns per tile
+constexpr int kHaloMaxRows = 384;             // halo rows: 256 + (Kw - 1)·N <= 384
+constexpr int kHaloBStages = 2;
+constexpr int kHaloAStages = 6;
+constexpr uint32_t kHaloBTile = kHaloMaxRows * 128;   // 48 KB
+
+struct HaloSmem {
+  static constexpr int kAOffset = 0;
+  static constexpr int kBOffset = kHaloAStages * kATileBytes;
+  static constexpr int kBarOffset = kBOffset + kHaloBStages * kHaloBTile;
+  static constexpr int kBytes = kBarOffset + 512 + 1024;
+};
+
+struct HaloBars {
+  uint64_t afull[kHaloAStages];
+  uint64_t aempty[kHaloAStages];
+  uint64_t bfull[kHaloBStages];
+  uint64_t bempty[kHaloBStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem;
+};
+
+// Geometry of the halo pass (filled by the host).
+struct HaloGeom {
+  int bw;             // output pixels per tile (256 / N)
+  int rows;           // halo rows (bw + Kw - 1)·N
+  int tpr;            // tiles per output row
+  int cchunks;        // 64-channel chunks of the reduction
+  int out_h, out_w;   // output pixel grid of the pass
+  int src_h, src_w;   // source pixel grid
+};
+
+// Raw codes of one halo unit: 8 batch items (rows) x 8 channels (K).
+struct HaloRaw {
+  uint32_t w[2][8];   // per unit: codes of channel c0 + j for the 8 batch items
+  uint32_t s[2][2];   // per unit: scales of channel blocks 0/1, batch blocks 0/1
+  bool ok[2];
+};
+
+// Transposed dequantize + store of one unit: row n0 + r of the tile gets the
+// 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
+// channel words is interleaved nibble-wise first, so one cvt.e2m1x2 per
+// byte yields the (channel 2i, channel 2i+1) pair of one batch item.
+__device__ __forceinline__ void halo_store_unit(const uint32_t (&w)[8], const uint32_t (&s)[2], bool ok,
+                                                uint32_t tile, uint32_t row0, uint32_t kg) {
+  uint32_t out[8][4];
+  if (ok) {
+    const uint32_t sc[2][2] = {{scale2(s[0] & 0xFF), scale2(s[0] >> 8)},    // [channel block][batch block]
+                               {scale2(s[1] & 0xFF), scale2(s[1] >> 8)}};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {                         // channel pair (2i, 2i+1)
+      const uint32_t a = w[2 * i], b = w[2 * i + 1];
+      const uint32_t even = (a & 0x0F0F0F0Fu) | ((b & 0x0F0F0F0Fu) << 4);   // batch items 0,2,4,6
+      const uint32_t odd = ((a >> 4) & 0x0F0F0F0Fu) | (b & 0xF0F0F0F0u);    // batch items 1,3,5,7
+      uint32_t he[4], ho[4];
+      e2m1x8_to_f16x2(even, he);
+      e2m1x8_to_f16x2(odd, ho);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t s2 = sc[i >> 1][q >> 1];             // batch items 2q, 2q+1: block q/2
+        out[2 * q][i] = hmul2_u32(he[q], s2);
+        out[2 * q + 1][i] = hmul2_u32(ho[q], s2);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) out[r][0] = out[r][1] = out[r][2] = out[r][3] = 0u;
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    st_shared_v4(tile + sw128_offset(row0 + r, 8 * kg), out[r][0], out[r][1], out[r][2], out[r][3]);
+}
+
+template <int PASS>
+struct HaloProducer {
+  // per-tile state of this thread's (up to) two units
+  int sc[2], n0[2];
+  bool cok[2];
+  HaloRaw raw;
+
+  // t: producer thread; u = t + 256·i: kg = u % 8 (K chunk of 8 channels),
+  // rg = u / 8 (8-row group of the halo).
+  __device__ __forceinline__ void begin_tile(const V2Args& p, const HaloGeom& g, int tile, int t) {
+    const int oh = tile / g.tpr;
+    const int ow0 = (tile - oh * g.tpr) * g.bw;
+    (void)oh;
+    const int base = PASS == kFwd ? ow0 - p.pad : ow0 + p.pad - (p.Kw - 1);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int u = t + kV2ProdThreads * i;
+      const int r = 8 * (u >> 3);
+      const int q = fdiv(r, p.dN);
+      n0[i] = r - q * p.N;
+      sc[i] = base + q;
+      cok[i] = u < g.rows && sc[i] >= 0 && sc[i] < g.src_w;      // unit u covers halo rows 8(u/8)..
+    }
+  }
+
+  __device__ __forceinline__ void load(const V2Args& p, const HaloGeom& g, int tile, int kh, int c, int t) {
+    const int oh = tile / g.tpr;
+    const int sr = PASS == kFwd ? oh + kh - p.pad : oh + p.pad - kh;
+    const bool rok = sr >= 0 && sr < g.src_h;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int u = t + kV2ProdThreads * i;
+      const int kg = u & 7;
+      raw.ok[i] = rok && cok[i];
+      if (!raw.ok[i]) continue;
+      const int64_t row0 = (static_cast<int64_t>(sr) * g.src_w + sc[i]) * p.Cred + 64 * c + 8 * kg;
+      const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + (n0[i] >> 1);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) raw.w[i][j] = __ldg(reinterpret_cast<const uint32_t*>(cp + j * p.b.row_bytes));
+      const uint8_t* sp = p.b.scales + (row0 >> 2) * p.b.scale_cols + (n0[i] >> 2);
+      raw.s[i][0] = __ldg(reinterpret_cast<const unsigned short*>(sp));
+      raw.s[i][1] = __ldg(reinterpret_cast<const unsigned short*>(sp + p.b.scale_cols));
+    }
+  }
+
+  __device__ __forceinline__ void store(const HaloGeom& g, uint32_t tile, int t) const {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int u = t + kV2ProdThreads * i;
+      if ((u >> 3) * 8 >= g.rows) continue;
+      halo_store_unit(raw.w[i], raw.s[i], raw.ok[i], tile, static_cast<uint32_t>(8 * (u >> 3)),
+                      static_cast<uint32_t>(u & 7));
+    }
+  }
+};
+
+template <int PASS>
+__global__ void __launch_bounds__(kV2Threads, 1)
+conv_halo_kernel(const V2Args p, const HaloGeom g) {
+  using L = HaloSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  HaloBars* bars = reinterpret_cast<HaloBars*>(smem + L::kBarOffset);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kHaloAStages; ++s) {
+      mbar_init(&bars->afull[s], 1);
+      mbar_init(&bars->aempty[s], 1);
+    }
+    for (int s = 0; s < kHaloBStages; ++s) {
+      mbar_init(&bars->bfull[s], kV2ProdThreads / 32);
+      mbar_init(&bars->bempty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars->acc_full[a], 1);
+      mbar_init(&bars->acc_empty[a], kV2EpiWarps * 32);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kV2MmaWarp) {
+    tmem_alloc(&bars->tmem, 2 * kHaloBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t sbase = smem_u32(smem);
+  const int stages_per_tile = p.Kh * g.cchunks;
+
+  if (warp < kV2EpiWarps) {
+    // epilogue: column lc of the tile = (pixel j, batch item n) -> output
+    // pixel (oh, ow0 + j), skipped past the end of the output row.
+    int it = 0;
+    const int64_t m = static_cast<int64_t>(0) + warp * 32 + lane;
+    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
+      tc_fence_after();
+      const int mt = tile / (g.out_h * g.tpr);
+      const int rest = tile - mt * g.out_h * g.tpr;
+      const int oh = rest / g.tpr;
+      const int ow0 = (rest - oh * g.tpr) * g.bw;
+      const int64_t mrow = static_cast<int64_t>(mt) * 128 + m;
+      const float scale = __fmul_rn(*p.ta, *p.tb);
+      const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * kHaloBN;
+#pragma unroll 1
+      for (int c = 0; c < kHaloBN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c, r);
+        tmem_ld_wait();
+        if (mrow < p.M) {
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const int lc = c + 4 * j4;
+            const int j = fdiv(lc, p.dN);
+            const int n = lc - j * p.N;
+            const int ow = ow0 + j;
+            if (j >= g.bw || ow >= g.out_w) continue;
+            float4 o;
+            o.x = __uint_as_float(r[4 * j4 + 0]) * scale;
+            o.y = __uint_as_float(r[4 * j4 + 1]) * scale;
+            o.z = __uint_as_float(r[4 * j4 + 2]) * scale;
+            o.w = __uint_as_float(r[4 * j4 + 3]) * scale;
+            const int64_t idx = ((static_cast<int64_t>(oh) * g.out_w + ow) * p.M + mrow) * p.N + n;
+            *reinterpret_cast<float4*>(p.out + idx) = o;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty[acc]);
+    }
+  } else if (warp == kV2MmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, kHaloBN);
+      int it = 0, bit = 0, ait = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
+        tc_fence_after();
+        const uint32_t dt = bars->tmem + acc * kHaloBN;
+        bool first = true;
+        for (int st = 0; st < stages_per_tile; ++st, ++bit) {
+          const int sb = bit % kHaloBStages;
+          mbar_wait_bounded(&bars->bfull[sb], (bit / kHaloBStages) & 1, p.err, kErrWaitFull);
+          tc_fence_after();
+          const uint32_t b_tile = sbase + L::kBOffset + sb * kHaloBTile;
+          for (int kw = 0; kw < p.Kw; ++kw, ++ait) {
+            const int sa = ait % kHaloAStages;
+            mbar_wait_bounded(&bars->afull[sa], (ait / kHaloAStages) & 1, p.err, kErrWaitFull);
+            tc_fence_after();
+            const int shift = PASS == kFwd ? kw : p.Kw - 1 - kw;
+            const uint64_t adesc = smem_desc_sw128(sbase + L::kAOffset + sa * kATileBytes);
+            const uint64_t bdesc = smem_desc_sw128(b_tile + static_cast<uint32_t>(shift * p.N) * 128u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_f16_ss(dt, adesc + 2 * kk, bdesc + 2 * kk, idesc, first ? 0u : 1u);
+              first = false;
+            }
+            mma_commit(&bars->aempty[sa]);
+          }
+          mma_commit(&bars->bempty[sb]);
+        }
+        mma_commit(&bars->acc_full[acc]);
+      }
+    }
+  } else if (warp == kV2LoadWarp) {
+    if (lane == 0) {
+      int ait = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
+        const int mt = tile / (g.out_h * g.tpr);
+        const uint8_t* img = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
+        for (int kh = 0; kh < p.Kh; ++kh)
+          for (int c = 0; c < g.cchunks; ++c)
+            for (int kw = 0; kw < p.Kw; ++kw, ++ait) {
+              const int sa = ait % kHaloAStages;
+              mbar_wait_bounded(&bars->aempty[sa], ((ait / kHaloAStages) & 1) ^ 1, p.err, kErrWaitEmpty);
+              mbar_arrive_expect_tx(&bars->afull[sa], kATileBytes);
+              const int kt = (kh * p.Kw + kw) * g.cchunks + c;
+              bulk_copy_g2s(sbase + L::kAOffset + sa * kATileBytes, img + static_cast<int64_t>(kt) * kATileBytes,
+                            kATileBytes, &bars->afull[sa]);
+            }
+      }
+    }
+  } else {
+    // producers: one stage ahead in registers (two units of 8 x 8 per thread)
+    const int t = threadIdx.x - kV2ProdWarp0 * 32;
+    const int ntile_cta = (p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                          static_cast<int>(gridDim.x);
+    const int total = ntile_cta * stages_per_tile;
+    HaloProducer<PASS> cur, nxt;
+    int ltile = blockIdx.x, lkh = 0, lc = 0;
+    auto tile_in_grid = [&](int tl) { return tl % (g.out_h * g.tpr); };
+    if (total > 0) {
+      cur.begin_tile(p, g, tile_in_grid(ltile), t);
+      nxt = cur;
+      cur.load(p, g, tile_in_grid(ltile), lkh, lc, t);
+    }
+    for (int kit = 0; kit < total; ++kit) {
+      // advance the load cursor and prefetch the next stage
+      if (++lc == g.cchunks) {
+        lc = 0;
+        if (++lkh == p.Kh) {
+          lkh = 0;
+          ltile += gridDim.x;
+          if (kit + 1 < total) nxt.begin_tile(p, g, tile_in_grid(ltile), t);
+        }
+      }
+      if (kit + 1 < total) nxt.load(p, g, tile_in_grid(ltile), lkh, lc, t);
+      const int sb = kit % kHaloBStages;
+      mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
+      cur.store(g, sbase + L::kBOffset + sb * kHaloBTile, t);
+      producer_warp_arrive(&bars->bfull[sb]);
+      cur = nxt;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kV2MmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(bars->tmem, 2 * kHaloBN);
+  }
+}
+
+}  // namespace mqv

@@ -50,6 +50,12 @@ SMALL = [
     ("n12_c8", O.ConvShape(12, 8, 8, 5, 5, 3, 3, 1, 1), "nvfp6"),
     ("wide_k_s2_p2", O.ConvShape(4, 72, 68, 11, 11, 5, 5, 2, 2), "nvfp4"),
     ("deep_cin", O.ConvShape(8, 256, 32, 4, 4, 3, 3, 1, 1), "nvfp4"),
+    # stride-1 shapes of the kernel-row halo path (N | 256, N % 8 == 0, 64-channel chunks)
+    ("halo_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp4"),
+    ("halo_n32_two_m_tiles", O.ConvShape(32, 128, 192, 5, 9, 3, 3, 1, 1), "nvfp4"),
+    ("halo_n16_pad0", O.ConvShape(16, 64, 64, 7, 7, 3, 3, 1, 0), "nvfp4"),
+    ("halo_n8_5x5", O.ConvShape(8, 64, 128, 9, 9, 5, 5, 1, 2), "nvfp4"),
+    ("halo_1x1_n64", O.ConvShape(64, 128, 64, 5, 5, 1, 1, 1, 0), "nvfp4"),
 ]
 
 
