@@ -348,7 +348,7 @@ cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<pl.grid, kV2Threads, HaloSmem::kBytes, st>>>(pl.a, pl.g);
+  kern<<<pl.grid, kHaloThreads, HaloSmem::kBytes, st>>>(pl.a, pl.g);
   return cudaGetLastError();
 }
 

@@ -35,6 +35,10 @@ constexpr int kHaloBN = 256;                  // GEMM columns per tile
 constexpr int kHaloMaxRows = 384;             // halo rows: 256 + (Kw - 1)·N <= 384
 constexpr int kHaloBStages = 2;
 constexpr int kHaloAStages = 6;
+constexpr int kHaloProdWarps = 12;                       // one 8 x 8 unit per thread per stage
+constexpr int kHaloProdThreads = kHaloProdWarps * 32;    // 384 = the largest halo
+constexpr int kHaloThreads = (kV2ProdWarp0 + kHaloProdWarps) * 32;
+constexpr int kHaloLookahead = 2;                        // stages of codes in flight per thread
 constexpr uint32_t kHaloBTile = kHaloMaxRows * 128;   // 48 KB
 
 struct HaloSmem {
@@ -65,25 +69,24 @@ struct HaloGeom {
 };
 
 // Raw codes of one halo unit: 8 batch items (rows) x 8 channels (K).
-struct HaloRaw {
-  uint32_t w[2][8];   // per unit: codes of channel c0 + j for the 8 batch items
-  uint32_t s[2][2];   // per unit: scales of channel blocks 0/1, batch blocks 0/1
-  bool ok[2];
+struct HaloUnit {
+  uint32_t w[8];      // codes of channel c0 + j for the 8 batch items
+  uint32_t s[2];      // scales of channel blocks 0/1 (low byte: batch block 0)
+  bool ok;
 };
 
-// Transposed dequantize + store of one unit: row n0 + r of the tile gets the
-// 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
+// Transposed dequantize + store of one unit: row row0 + r of the tile gets
+// the 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
 // channel words is interleaved nibble-wise first, so one cvt.e2m1x2 per
 // byte yields the (channel 2i, channel 2i+1) pair of one batch item.
-__device__ __forceinline__ void halo_store_unit(const uint32_t (&w)[8], const uint32_t (&s)[2], bool ok,
-                                                uint32_t tile, uint32_t row0, uint32_t kg) {
+__device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile, uint32_t row0, uint32_t kg) {
   uint32_t out[8][4];
-  if (ok) {
-    const uint32_t sc[2][2] = {{scale2(s[0] & 0xFF), scale2(s[0] >> 8)},    // [channel block][batch block]
-                               {scale2(s[1] & 0xFF), scale2(s[1] >> 8)}};
+  if (u.ok) {
+    const uint32_t sc[2][2] = {{scale2(u.s[0] & 0xFF), scale2(u.s[0] >> 8)},    // [channel block][batch block]
+                               {scale2(u.s[1] & 0xFF), scale2(u.s[1] >> 8)}};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {                         // channel pair (2i, 2i+1)
-      const uint32_t a = w[2 * i], b = w[2 * i + 1];
+      const uint32_t a = u.w[2 * i], b = u.w[2 * i + 1];
       const uint32_t even = (a & 0x0F0F0F0Fu) | ((b & 0x0F0F0F0Fu) << 4);   // batch items 0,2,4,6
       const uint32_t odd = ((a >> 4) & 0x0F0F0F0Fu) | (b & 0xF0F0F0F0u);    // batch items 1,3,5,7
       uint32_t he[4], ho[4];
@@ -105,64 +108,43 @@ __device__ __forceinline__ void halo_store_unit(const uint32_t (&w)[8], const ui
     st_shared_v4(tile + sw128_offset(row0 + r, 8 * kg), out[r][0], out[r][1], out[r][2], out[r][3]);
 }
 
+// Producer thread t owns unit t of every stage: K chunk kg = t % 8 (8
+// channels), rows 8(t/8)..8(t/8)+7 of the halo.  Lanes of an 8-lane phase
+// differ in kg, so their 16-byte stores hit 8 different swizzled chunks.
 template <int PASS>
-struct HaloProducer {
-  // per-tile state of this thread's (up to) two units
-  int sc[2], n0[2];
-  bool cok[2];
-  HaloRaw raw;
+struct HaloCursor {
+  int sc, n0;         // halo pixel column in the source, first batch item
+  bool cok;           // unit inside the halo and its column inside the source
 
-  // t: producer thread; u = t + 256·i: kg = u % 8 (K chunk of 8 channels),
-  // rg = u / 8 (8-row group of the halo).
   __device__ __forceinline__ void begin_tile(const V2Args& p, const HaloGeom& g, int tile, int t) {
     const int oh = tile / g.tpr;
     const int ow0 = (tile - oh * g.tpr) * g.bw;
-    (void)oh;
     const int base = PASS == kFwd ? ow0 - p.pad : ow0 + p.pad - (p.Kw - 1);
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = t + kV2ProdThreads * i;
-      const int r = 8 * (u >> 3);
-      const int q = fdiv(r, p.dN);
-      n0[i] = r - q * p.N;
-      sc[i] = base + q;
-      cok[i] = u < g.rows && sc[i] >= 0 && sc[i] < g.src_w;      // unit u covers halo rows 8(u/8)..
-    }
+    const int r = 8 * (t >> 3);
+    const int q = fdiv(r, p.dN);
+    n0 = r - q * p.N;
+    sc = base + q;
+    cok = t < g.rows && sc >= 0 && sc < g.src_w;
   }
 
-  __device__ __forceinline__ void load(const V2Args& p, const HaloGeom& g, int tile, int kh, int c, int t) {
+  __device__ __forceinline__ void load(const V2Args& p, const HaloGeom& g, int tile, int kh, int c, int t,
+                                       HaloUnit& u) const {
     const int oh = tile / g.tpr;
     const int sr = PASS == kFwd ? oh + kh - p.pad : oh + p.pad - kh;
-    const bool rok = sr >= 0 && sr < g.src_h;
+    u.ok = cok && sr >= 0 && sr < g.src_h;
+    if (!u.ok) return;
+    const int64_t row0 = (static_cast<int64_t>(sr) * g.src_w + sc) * p.Cred + 64 * c + 8 * (t & 7);
+    const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + (n0 >> 1);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = t + kV2ProdThreads * i;
-      const int kg = u & 7;
-      raw.ok[i] = rok && cok[i];
-      if (!raw.ok[i]) continue;
-      const int64_t row0 = (static_cast<int64_t>(sr) * g.src_w + sc[i]) * p.Cred + 64 * c + 8 * kg;
-      const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + (n0[i] >> 1);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) raw.w[i][j] = __ldg(reinterpret_cast<const uint32_t*>(cp + j * p.b.row_bytes));
-      const uint8_t* sp = p.b.scales + (row0 >> 2) * p.b.scale_cols + (n0[i] >> 2);
-      raw.s[i][0] = __ldg(reinterpret_cast<const unsigned short*>(sp));
-      raw.s[i][1] = __ldg(reinterpret_cast<const unsigned short*>(sp + p.b.scale_cols));
-    }
-  }
-
-  __device__ __forceinline__ void store(const HaloGeom& g, uint32_t tile, int t) const {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int u = t + kV2ProdThreads * i;
-      if ((u >> 3) * 8 >= g.rows) continue;
-      halo_store_unit(raw.w[i], raw.s[i], raw.ok[i], tile, static_cast<uint32_t>(8 * (u >> 3)),
-                      static_cast<uint32_t>(u & 7));
-    }
+    for (int j = 0; j < 8; ++j) u.w[j] = __ldg(reinterpret_cast<const uint32_t*>(cp + j * p.b.row_bytes));
+    const uint8_t* sp = p.b.scales + (row0 >> 2) * p.b.scale_cols + (n0 >> 2);
+    u.s[0] = __ldg(reinterpret_cast<const unsigned short*>(sp));
+    u.s[1] = __ldg(reinterpret_cast<const unsigned short*>(sp + p.b.scale_cols));
   }
 };
 
 template <int PASS>
-__global__ void __launch_bounds__(kV2Threads, 1)
+__global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
   using L = HaloSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -175,7 +157,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       mbar_init(&bars->aempty[s], 1);
     }
     for (int s = 0; s < kHaloBStages; ++s) {
-      mbar_init(&bars->bfull[s], kV2ProdThreads / 32);
+      mbar_init(&bars->bfull[s], kHaloProdWarps);
       mbar_init(&bars->bempty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -289,35 +271,43 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       }
     }
   } else {
-    // producers: one stage ahead in registers (two units of 8 x 8 per thread)
+    // producers: kHaloLookahead stages of codes in flight per thread (a ring
+    // of registers indexed at compile time)
     const int t = threadIdx.x - kV2ProdWarp0 * 32;
     const int ntile_cta = (p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                           static_cast<int>(gridDim.x);
     const int total = ntile_cta * stages_per_tile;
-    HaloProducer<PASS> cur, nxt;
+    const int spatial = g.out_h * g.tpr;
+    HaloCursor<PASS> cursor;
+    HaloUnit ring[kHaloLookahead];
     int ltile = blockIdx.x, lkh = 0, lc = 0;
-    auto tile_in_grid = [&](int tl) { return tl % (g.out_h * g.tpr); };
-    if (total > 0) {
-      cur.begin_tile(p, g, tile_in_grid(ltile), t);
-      nxt = cur;
-      cur.load(p, g, tile_in_grid(ltile), lkh, lc, t);
-    }
-    for (int kit = 0; kit < total; ++kit) {
-      // advance the load cursor and prefetch the next stage
+    if (total > 0) cursor.begin_tile(p, g, ltile % spatial, t);
+    auto load_next = [&](HaloUnit& u) {
+      cursor.load(p, g, ltile % spatial, lkh, lc, t, u);
       if (++lc == g.cchunks) {
         lc = 0;
         if (++lkh == p.Kh) {
           lkh = 0;
           ltile += gridDim.x;
-          if (kit + 1 < total) nxt.begin_tile(p, g, tile_in_grid(ltile), t);
+          if (ltile < p.tiles) cursor.begin_tile(p, g, ltile % spatial, t);
         }
       }
-      if (kit + 1 < total) nxt.load(p, g, tile_in_grid(ltile), lkh, lc, t);
-      const int sb = kit % kHaloBStages;
-      mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
-      cur.store(g, sbase + L::kBOffset + sb * kHaloBTile, t);
-      producer_warp_arrive(&bars->bfull[sb]);
-      cur = nxt;
+    };
+#pragma unroll
+    for (int r = 0; r < kHaloLookahead; ++r)
+      if (r < total) load_next(ring[r]);
+    for (int kit = 0; kit < total;) {
+#pragma unroll
+      for (int r = 0; r < kHaloLookahead; ++r, ++kit) {
+        if (kit >= total) break;
+        const int sb = kit % kHaloBStages;
+        mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
+        if (t < g.rows)
+          halo_store_unit(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
+                          static_cast<uint32_t>(t & 7));
+        producer_warp_arrive(&bars->bfull[sb]);
+        if (kit + kHaloLookahead < total) load_next(ring[r]);
+      }
     }
   }
   tc_fence_before();
