@@ -184,11 +184,11 @@ mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const m
  * footprint), or that has no allocator to ask for a workspace.  The paper
  * has no counterpart; this is an interface convenience of this library.
  *   - Allocates nothing: the split-K partial sums go to one file-scope
- *     device array of 16 MiB inside the library, which every GPU that loads
+ *     device array of 32 MiB inside the library, which every GPU that loads
  *     the library holds until the process exits.  Layers whose partials
- *     would need more (mqv_conv_workspace_size(d, MQV_OP_WGRAD) > 16 MiB)
+ *     would need more (mqv_conv_workspace_size(d, MQV_OP_WGRAD) > 32 MiB)
  *     are rejected with MQV_ERR_UNSUPPORTED and a message; the current split
- *     planner stays below 9.7 MB for every shape.
+ *     planner stays below 29.1 MB for every shape.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

@@ -14,6 +14,7 @@
 #include "mqv_conv_common.cuh"
 #include "mqv_conv_kernels.cuh"
 #include "mqv_conv_halo.cuh"
+#include "mqv_conv_wgk.cuh"
 #include "mqv_quantize.cuh"
 
 namespace {
@@ -164,6 +165,8 @@ struct ConvPlan {
   V2Args a;
   bool halo;            // stride-1 fwd/dgrad with the on-chip halo (conv_halo_kernel)
   HaloGeom g;
+  bool wgk;             // stride-1 wgrad with the taps of a kernel row sharing operands
+  WgkGeom wg;
   int bn;               // 128 or 256 columns per tile
   int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0
   int grid;             // persistent CTAs
@@ -288,6 +291,25 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
     g.cchunks = a.Cred / 64;
     a.tiles = a.mtiles * g.out_h * g.tpr;
   }
+  // Stride-1 weight gradient with N % 16 == 0 and Kw <= 3 whose taps reach
+  // at most two 64-element chunks further: the kernel-row path.
+  pl->wgk = op == MQV_OP_WGRAD && d->stride == 1 && d->N % 16 == 0 && d->Kw <= kWgkMaxTaps &&
+            (48 + (d->Kw - 1) * d->N) / 64 <= 2;
+  if (pl->wgk) {
+    WgkGeom& w = pl->wg;
+    w.chunks = (int)((a.Wo * d->N + 63) / 64);
+    w.sx = (int)((48 + (d->Kw - 1) * d->N) / 64);
+    w.ctiles = (a.Cin + 127) / 128;
+    w.base_tiles = a.mtiles * w.ctiles * a.Kh;
+    const int64_t total_q = (int64_t)a.Ho * w.chunks;
+    int64_t s = w.base_tiles >= kSMs ? 1 : kSMs / w.base_tiles;
+    if (s > total_q) s = total_q;
+    const int64_t per = (total_q + s - 1) / s;
+    w.q_per_split = (int)per;
+    splits = (int)((total_q + per - 1) / per);
+    a.splits = splits;
+    a.tiles = w.base_tiles * splits;
+  }
   a.scale_out = splits == 1;
   pl->grid = a.tiles < kSMs ? a.tiles : kSMs;
   pl->image_bytes = op == MQV_OP_WGRAD ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
@@ -352,9 +374,20 @@ cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int FMT>
+cudaError_t launch_wgk(const ConvPlan& pl, cudaStream_t st) {
+  auto kern = conv_wgk_kernel<FMT>;
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(kern, WgkSmem::kBytes, done);
+  if (e != cudaSuccess) return e;
+  kern<<<pl.grid, kV2Threads, WgkSmem::kBytes, st>>>(pl.a, pl.wg);
+  return cudaGetLastError();
+}
+
 template <int PASS>
 cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
   if (PASS != kWgrad && pl.halo) return launch_halo<PASS == kWgrad ? kFwd : PASS>(pl, st);
+  if (PASS == kWgrad && pl.wgk) return fmt == MQV_NVFP4 ? launch_wgk<0>(pl, st) : launch_wgk<1>(pl, st);
   return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
 }
 
@@ -653,12 +686,13 @@ mqv_status mqv_device_errors(uint32_t* flags, void* stream) {
 // a caller that has no way to allocate device memory can still run the pass.
 namespace {
 
-// Largest split-K partial set the built-in scratch holds (16 MiB per GPU; it
+// Largest split-K partial set the built-in scratch holds (32 MiB per GPU; it
 // is part of the library's device image and stays resident until exit).  The
-// split planner only splits layers with at most 74 output tiles of 128 x 128
-// and fills at most one tile per SM, so its partials stay below
-// 148 x 128 x 128 x 4 B = 9.7 MB; the size check below guards that bound.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+// split planner splits only while the tiles fit one wave of one tile per SM,
+// and a tile's partial is at most 128 output channels x 3 taps x 128 input
+// channels, so partials stay below 148 x 128 x 384 x 4 B = 29.1 MB; the size
+// check below guards that bound.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) float g_noalloc_wgrad_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 float* g_noalloc_ptr[kMaxDevices] = {};

@@ -35,9 +35,23 @@ wgrad_reduce_kernel(const float4* __restrict__ partial, int splits, int64_t n4,
                     float4* __restrict__ out) {
   const float scale = __fmul_rn(*ta, *tb);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  constexpr int kBatch = 8;     // loads in flight per thread; the adds stay in split order
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
     float4 acc = __ldg(partial + i);
-    for (int s = 1; s < splits; ++s) {
+    int s = 1;
+    for (; s + kBatch <= splits; s += kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) v[b] = __ldg(partial + (s + b) * n4 + i);
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        acc.x += v[b].x;
+        acc.y += v[b].y;
+        acc.z += v[b].z;
+        acc.w += v[b].w;
+      }
+    }
+    for (; s < splits; ++s) {
       const float4 v = __ldg(partial + s * n4 + i);
       acc.x += v.x;
       acc.y += v.y;

@@ -56,6 +56,13 @@ SMALL = [
     ("halo_n16_pad0", O.ConvShape(16, 64, 64, 7, 7, 3, 3, 1, 0), "nvfp4"),
     ("halo_n8_5x5", O.ConvShape(8, 64, 128, 9, 9, 5, 5, 1, 2), "nvfp4"),
     ("halo_1x1_n64", O.ConvShape(64, 128, 64, 5, 5, 1, 1, 1, 0), "nvfp4"),
+    # stride-1 weight-gradient shapes whose kernel-row taps share operands
+    # (N % 16 == 0): ragged rows and channels, split ranges that end inside a
+    # row, several channel tiles, a 2 x 2 kernel
+    ("wgk_n16_ragged_c", O.ConvShape(16, 24, 40, 9, 7, 3, 3, 1, 1), "nvfp4"),
+    ("wgk_n32_fp6_two_tiles", O.ConvShape(32, 200, 136, 6, 5, 3, 3, 1, 0), "nvfp6"),
+    ("wgk_n48_2x2", O.ConvShape(48, 16, 20, 8, 8, 2, 2, 1, 0), "nvfp4"),
+    ("wgk_rows_split", O.ConvShape(16, 256, 512, 10, 10, 3, 3, 1, 1), "nvfp4"),
 ]
 
 

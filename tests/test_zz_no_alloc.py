@@ -3,7 +3,7 @@
 Some callers cannot allocate device memory at all (their device memory is
 owned by a fixed pool they may not grow, or they have no allocator to ask for
 a workspace).  mqv_conv_wgrad_noalloc serves them: its split-K partial sums go
-to a fixed 16 MiB array inside the library instead of a caller workspace.
+to a fixed 32 MiB array inside the library instead of a caller workspace.
 These tests call it through the C ABI and check it against mqv_conv_wgrad
 (the allocating entry point) within the parity tolerance, twice in a row,
 since the array keeps the previous call's contents.  This file is collected
@@ -53,7 +53,7 @@ LAYERS = [workloads.tiny_layer(),
 def test_noalloc_wgrad_matches_allocating_entry_point(layer):
     d, qx, qg, S = _layer_case(layer)
     ref = mqv.conv_wgrad(d, qg, qx).cpu().numpy().astype(np.float64).reshape(S.shape)
-    assert mqv.conv_workspace_bytes(d, mqv.OP_WGRAD) <= 16 << 20
+    assert mqv.conv_workspace_bytes(d, mqv.OP_WGRAD) <= 32 << 20
     lim = 1e-5 * S + 1e-7
     for call in range(2):                       # the scratch keeps the last call's data
         gw = torch.full((d.Cout, d.Kh, d.Kw, d.Cin), float("nan"), device="cuda")
@@ -80,8 +80,8 @@ def test_noalloc_wgrad_after_other_layer_reuses_scratch():
 
 
 def test_noalloc_scratch_covers_every_planned_layer():
-    """The split planner keeps wgrad partials under the 16 MiB built-in scratch
-    for every shape (at most 148 tiles of 128 x 128 fp32); so no layer of the
+    """The split planner keeps wgrad partials under the 32 MiB built-in scratch
+    for every shape (at most 148 tiles of 128 x 384 fp32); so no layer of the
     benchmarked workloads, nor any shape of a wide sweep, is rejected."""
     shapes = [l.dims() | {"fmt": l.fmt} for l in
               [workloads.tiny_layer(), workloads.resnet18_layer2()] + workloads.resnet18_body()
@@ -92,4 +92,4 @@ def test_noalloc_scratch_covers_every_planned_layer():
                 shapes.append(dict(N=32, Cin=cin, Cout=cout, H=14, W=14, Kh=k, Kw=k, stride=1,
                                    pad=k // 2, fmt="nvfp4"))
     worst = max(mqv.conv_workspace_bytes(mqv.conv_desc(**s), mqv.OP_WGRAD) for s in shapes)
-    assert 0 < worst <= 148 * 128 * 128 * 4 < 16 << 20
+    assert 0 < worst <= 148 * 128 * 384 * 4 < 32 << 20
