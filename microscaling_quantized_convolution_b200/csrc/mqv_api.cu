@@ -311,7 +311,9 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
     a.tiles = w.base_tiles * splits;
   }
   a.scale_out = splits == 1;
-  pl->grid = a.tiles < kSMs ? a.tiles : kSMs;
+  // persistent kernels: one CTA per SM at most; the kernel-row weight
+  // gradient runs one tile per CTA
+  pl->grid = pl->wgk ? a.tiles : (a.tiles < kSMs ? a.tiles : kSMs);
   pl->image_bytes = op == MQV_OP_WGRAD ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
   pl->partial_bytes = splits > 1 ? (size_t)splits * a.M * a.Ncols * sizeof(float) : 0;
   pl->ws_bytes = pl->image_bytes + pl->partial_bytes;
@@ -374,20 +376,32 @@ cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int FMT>
+template <int FMT, int KW, bool PAIR>
 cudaError_t launch_wgk(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_wgk_kernel<FMT>;
+  auto kern = conv_wgk_kernel<FMT, KW, PAIR>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, WgkSmem::kBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<pl.grid, kV2Threads, WgkSmem::kBytes, st>>>(pl.a, pl.wg);
+  kern<<<pl.grid, kWgkThreads, WgkSmem::kBytes, st>>>(pl.a, pl.wg);
   return cudaGetLastError();
+}
+
+// Batch 64 puts each tap of a kernel row exactly one X chunk further, so the
+// taps share one run of B rows (paired MMAs); other batches use one MMA per tap.
+template <int FMT>
+cudaError_t launch_wgk_kw(const ConvPlan& pl, cudaStream_t st) {
+  const bool pair = pl.a.N == 64;
+  switch (pl.a.Kw) {
+    case 1: return launch_wgk<FMT, 1, false>(pl, st);
+    case 2: return pair ? launch_wgk<FMT, 2, true>(pl, st) : launch_wgk<FMT, 2, false>(pl, st);
+    default: return pair ? launch_wgk<FMT, 3, true>(pl, st) : launch_wgk<FMT, 3, false>(pl, st);
+  }
 }
 
 template <int PASS>
 cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
   if (PASS != kWgrad && pl.halo) return launch_halo<PASS == kWgrad ? kFwd : PASS>(pl, st);
-  if (PASS == kWgrad && pl.wgk) return fmt == MQV_NVFP4 ? launch_wgk<0>(pl, st) : launch_wgk<1>(pl, st);
+  if (PASS == kWgrad && pl.wgk) return fmt == MQV_NVFP4 ? launch_wgk_kw<0>(pl, st) : launch_wgk_kw<1>(pl, st);
   return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
 }
 

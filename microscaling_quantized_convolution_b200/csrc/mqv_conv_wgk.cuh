@@ -7,17 +7,23 @@
 // accumulator per tap kw.  The contraction runs over the output rows ho and,
 // along each row, over 64-element chunks of its (wo, n) elements.  For tap
 // kw the X' elements of output chunk j are X elements (wo + kw - pad, n), the
-// same X row shifted by kw·N elements; so the producers dequantize each
-// X chunk (128 channels x 64 elements of the row hi = ho + kh - pad) and each
-// G_Y chunk once, and the Kw taps are MMA groups whose 16-element K slices
-// point at the right X chunk and slice (N % 16 == 0 keeps every slice whole).
+// same X row shifted by kw·N elements; so each X chunk (128 channels x 64
+// elements of the row hi = ho + kh - pad) is dequantized once into shared
+// memory, and the Kw taps are MMA groups whose 16-element K slices point at
+// the right X chunk and slice (N % 16 == 0 keeps every slice whole).
 //
-// Stage t of a row segment [j0, j1) produces G_Y chunk t (t < j1) and X
-// chunk t (t < j1 + SX, SX = the furthest X chunk a tap reaches) into ring
-// slot t, and for t >= j0 + SX runs output chunk j = t - SX, which reads G_Y
-// chunk j and X chunks j..j+SX; slot j is released after that.  Splits of
-// the (ho, j) chunk range across CTAs make the partial sums that
-// wgrad_reduce_kernel adds in split order.
+// The G_Y chunk (128 output channels x the 64 elements of output chunk j) is
+// the MMA's A operand and lives in tensor memory: its producer threads own
+// one channel row each, dequantize the row's 64 codes and write them with
+// tcgen05.st.  Each MMA then reads only its B tile from shared memory, which
+// halves the shared-memory traffic of the 128 x 128 MMAs.
+//
+// X stage t of a row segment [j0, j1) fills X chunk t for t in
+// [j0, j1 + SX), SX = the furthest X chunk a tap reaches; output chunk
+// j = t - SX runs at stage t >= j0 + SX and reads X chunks j..j+SX.  The X
+// and G_Y rings advance independently.  Splits of the (ho, j) chunk range
+// across CTAs make the partial sums that wgrad_reduce_kernel adds in split
+// order.
 #pragma once
 
 #include <cstdint>
@@ -28,8 +34,24 @@
 
 namespace mqv {
 
-constexpr int kWgkSlots = 5;            // SX + 1 + producer lookahead, SX <= 2
+constexpr int kWgkXSlots = 8;           // X chunks in shared memory (a power of two)
+constexpr int kWgkXMirrors = 2;         // copies of slots 0 and 1 after the ring (paired taps)
+constexpr int kWgkASlots = 4;           // G_Y chunks in tensor memory
 constexpr int kWgkMaxTaps = 3;
+constexpr int kWgkACol = kWgkMaxTaps * 128;     // first TMEM column of the G_Y ring
+constexpr int kWgkLookahead = 2;        // stages of codes in flight per producer thread
+// Roles: warps 0-3 produce the first half of each G_Y chunk and run the
+// epilogue between tiles; warp 4 issues the MMAs; warps 8-11 produce the
+// second G_Y half (each G_Y warp owns its TMEM lane quarter, warp % 4);
+// warps 6, 7 and 12-17 produce X.  Warp 5 has no role.
+constexpr int kWgkWarps = 18;
+constexpr int kWgkThreads = kWgkWarps * 32;
+constexpr int kWgkXWarps = 8;
+constexpr int kWgkGWarps = 8;
+
+__device__ __forceinline__ int wgk_x_index(int warp) {   // X producer number of a warp, or -1
+  return warp == 6 ? 0 : warp == 7 ? 1 : (warp >= 12 && warp < 18) ? warp - 10 : -1;
+}
 
 struct WgkGeom {
   int chunks;         // 64-element chunks per output row, ceil(Wo·N / 64)
@@ -40,18 +62,19 @@ struct WgkGeom {
 };
 
 struct WgkSmem {
-  static constexpr int kSlot = 2 * kATileBytes;              // G_Y chunk + X chunk
-  static constexpr int kEpiOffset = kWgkSlots * kSlot;       // 32 x 32 fp32 per epilogue warp
+  static constexpr int kXSlot = kATileBytes;                 // 128 channels x 64 fp16
+  static constexpr int kEpiOffset = (kWgkXSlots + kWgkXMirrors) * kXSlot;   // 32 x 32 fp32 per epilogue warp
   static constexpr int kEpiWarpBytes = 32 * 128;
-  static constexpr int kBarOffset = kEpiOffset + kV2EpiWarps * kEpiWarpBytes;
+  static constexpr int kBarOffset = kEpiOffset + 4 * kEpiWarpBytes;
   static constexpr int kBytes = kBarOffset + 256 + 1024;
 };
 
 struct WgkBars {
-  uint64_t full[kWgkSlots];
-  uint64_t empty[kWgkSlots];
-  uint64_t done;        // all MMAs of a tile completed (tcgen05.commit)
-  uint64_t acc_empty;   // the epilogue has read the accumulators of a tile
+  uint64_t xfull[kWgkXSlots];
+  uint64_t xempty[kWgkXSlots];
+  uint64_t afull[kWgkASlots];
+  uint64_t aempty[kWgkASlots];
+  uint64_t done;        // all MMAs of the tile completed (tcgen05.commit)
   uint32_t tmem;
 };
 
@@ -71,55 +94,184 @@ __device__ __forceinline__ WgkTile wgk_tile(const V2Args& p, const WgkGeom& g, i
   return w;
 }
 
-// Fill one stage: G_Y chunk (rows co, K = 64 (wo, n) elements of output row ho)
-// and X chunk (rows ci, K = 64 (wi, n) elements of input row hi, starting
-// at wi = -pad).  Unit = 4 rows x 8 batch items of one pixel (K-major,
-// natural order: the codes run along n).
-template <int FMT>
-__device__ __forceinline__ void wgk_fill(const V2Args& p, uint32_t slot, const WgkTile& w, int ho, int t,
-                                         bool with_a, int chunk) {
-  constexpr int NU = 8;
-  constexpr int KG = 64 / NU;
-  constexpr int PER = 128 / 4 * KG / kV2ProdThreads;   // units per thread per operand
-  const int hi = ho + w.kh - p.pad;
-  UnitRaw<FMT, NU> raw[2][PER];
-  // all loads of the stage first, then the dequantize + stores
-#pragma unroll
-  for (int op = 0; op < 2; ++op) {
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int u = t + kV2ProdThreads * i;
-      const int kg = u % KG, rq = u / KG;
-      const int e = chunk * 64 + kg * NU;           // element of the row: (pixel, n)
-      const int pix = fdiv(e, p.dN);
-      const int n = e - pix * p.N;
-      if (op == 0) {                                 // G_Y[ho][wo = pix][co][n]
-        const int co = w.mt * 128 + 4 * rq;
-        const bool ok = with_a && co < p.Cout && pix < p.Wo;
-        load_unit<FMT, NU>(p.a, (static_cast<int64_t>(ho) * p.Wo + pix) * p.Cout + co, n, ok, raw[0][i]);
-      } else {                                       // X[hi][wi = pix - pad][ci][n]
-        const int ci = w.ct * 128 + 4 * rq;
-        const int wi = pix - p.pad;
-        const bool ok = ci < p.Cin && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
-        load_unit<FMT, NU>(p.b, (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci, n, ok, raw[1][i]);
-      }
-    }
+// Walk over the stages of this CTA's tile (one tile per CTA): each row
+// segment [j0, j1) of the tile's chunk range yields stages t = j0 .. j1 +
+// ext - 1 (ext = SX for the X ring and the MMA, 0 for the G_Y ring).
+struct WgkCursor {
+  int q, q1, ho, j0, j1, t;
+  bool valid;
+
+  __device__ __forceinline__ void segment(const WgkGeom& g) {
+    ho = q / g.chunks;
+    j0 = q - ho * g.chunks;
+    j1 = min(g.chunks, j0 + (q1 - q));
+    t = j0;
   }
+  __device__ __forceinline__ void begin(const V2Args& p, const WgkGeom& g, const WgkTile& w) {
+    q = w.sp * g.q_per_split;
+    q1 = min(p.Ho * g.chunks, q + g.q_per_split);
+    valid = q < q1;
+    if (valid) segment(g);
+  }
+  __device__ __forceinline__ void advance(const WgkGeom& g, int ext) {
+    if (++t < j1 + ext) return;
+    q += j1 - j0;
+    valid = q < q1;
+    if (valid) segment(g);
+  }
+};
+
+// X producer: one unit (4 channels x 8 consecutive (pixel, n) elements) per
+// thread per stage; 256 units fill a 128-channel x 64-element chunk.
+template <int FMT>
+__device__ __forceinline__ void wgk_x_load(const V2Args& p, const WgkTile& w, const WgkCursor& c, int tid,
+                                           UnitRaw<FMT, 8>& r) {
+  const int hi = c.ho + w.kh - p.pad;
+  const int kg = tid & 7, rq = tid >> 3;
+  const int e = c.t * 64 + kg * 8;              // element (pixel, n) of the padded X row
+  const int pix = fdiv(e, p.dN);
+  const int n = e - pix * p.N;
+  const int ci = w.ct * 128 + 4 * rq;
+  const int wi = pix - p.pad;
+  const bool ok = ci < p.Cin && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
+  load_unit<FMT, 8>(p.b, (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci, n, ok, r);
+}
+
+// Dequantize the unit into X slot `slot` and, when `mirror` is nonzero, into
+// that second slot as well.
+template <int FMT>
+__device__ __forceinline__ void wgk_x_store(const UnitRaw<FMT, 8>& un, uint32_t slot, uint32_t mirror, int tid) {
+  const uint32_t row0 = static_cast<uint32_t>(4 * (tid >> 3)), kl = static_cast<uint32_t>(8 * (tid & 7));
+  const uint32_t s2lo = un.ok ? scale2(un.ss & 0xFF) : 0u;
+  const uint32_t s2hi = un.ok ? scale2(un.ss >> 8) : 0u;
 #pragma unroll
-  for (int op = 0; op < 2; ++op) {
-    if (op == 0 && !with_a) continue;
+  for (int j = 0; j < 4; ++j) {
+    uint32_t h[4] = {0u, 0u, 0u, 0u};
+    if (un.ok) dequant_run<FMT, 8>(un.lo[j], un.hi[j], s2lo, s2hi, h);
+    const uint32_t off = sw128_offset(row0 + j, kl);
+    st_shared_v4(slot + off, h[0], h[1], h[2], h[3]);
+    if (mirror) st_shared_v4(mirror + off, h[0], h[1], h[2], h[3]);
+  }
+}
+
+// G_Y producer: 32 of the 64 codes of one output-channel row of an output
+// chunk (half h: elements 32h..32h+31), as two 16-element pieces, each inside
+// one pixel since N % 16 == 0.
+struct WgkGRaw {
+  uint32_t c[2][3];     // FP4: 8 bytes in c[.][0..1]; FP6: 12 bytes
+  uint32_t s[2];        // the four E4M3 block scales of a piece
+  uint32_t ok;          // bit per piece
+};
+
+template <int FMT>
+__device__ __forceinline__ void wgk_g_load(const V2Args& p, const WgkTile& w, const WgkCursor& c, int row, int half,
+                                           WgkGRaw& r) {
+  const int co = w.mt * 128 + row;
+  r.ok = 0;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int u = t + kV2ProdThreads * i;
-      const int kg = u % KG, rq = u / KG;
-      store_unit<FMT, NU, false>(raw[op][i], slot + op * kATileBytes, static_cast<uint32_t>(4 * rq),
-                                 static_cast<uint32_t>(kg * NU));
+  for (int pc = 0; pc < 2; ++pc) {
+    const int e = c.t * 64 + 32 * half + 16 * pc;
+    const int pix = fdiv(e, p.dN);
+    const int n = e - pix * p.N;
+    if (co < p.Cout && pix < p.Wo) {
+      r.ok |= 1u << pc;
+      const int64_t vrow = (static_cast<int64_t>(c.ho) * p.Wo + pix) * p.Cout + co;
+      const uint8_t* cp = p.a.codes + vrow * p.a.row_bytes;
+      if (FMT == 0) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(cp + (n >> 1)));
+        r.c[pc][0] = v.x;
+        r.c[pc][1] = v.y;
+      } else {
+        const uint32_t* q = reinterpret_cast<const uint32_t*>(cp + ((n * 3) >> 2));
+        r.c[pc][0] = __ldg(q);
+        r.c[pc][1] = __ldg(q + 1);
+        r.c[pc][2] = __ldg(q + 2);
+      }
+      r.s[pc] = __ldg(reinterpret_cast<const uint32_t*>(p.a.scales + (vrow >> 2) * p.a.scale_cols + (n >> 2)));
     }
   }
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kV2Threads, 1)
+__device__ __forceinline__ void wgk_g_dequant(const WgkGRaw& r, uint32_t (&h)[16]) {
+#pragma unroll
+  for (int pc = 0; pc < 2; ++pc) {
+    uint32_t* o = h + 8 * pc;
+    if (!((r.ok >> pc) & 1u)) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = 0u;
+      continue;
+    }
+    const uint32_t s = r.s[pc];
+    const uint32_t s0 = scale2(s & 0xFF), s1 = scale2((s >> 8) & 0xFF);
+    const uint32_t s2 = scale2((s >> 16) & 0xFF), s3 = scale2(s >> 24);
+    if (FMT == 0) {
+      uint32_t a[4], b[4];
+      dq8_fp4(r.c[pc][0], s0, s1, a);
+      dq8_fp4(r.c[pc][1], s2, s3, b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o[j] = a[j];
+        o[4 + j] = b[j];
+      }
+    } else {
+      const uint32_t c0 = r.c[pc][0], c1 = r.c[pc][1], c2 = r.c[pc][2];
+      dq4_fp6(c0 & 0xFFFFFF, s0, o[0], o[1]);
+      dq4_fp6((c0 >> 24) | ((c1 & 0xFFFF) << 8), s1, o[2], o[3]);
+      dq4_fp6((c1 >> 16) | ((c2 & 0xFF) << 16), s2, o[4], o[5]);
+      dq4_fp6(c2 >> 8, s3, o[6], o[7]);
+    }
+  }
+}
+
+// Epilogue of one tile (warps 0-3, one TMEM lane quarter each): accumulator
+// rows are read with tcgen05.ld, transposed through a swizzled 32 x 32 buffer
+// in shared memory, and stored as whole 128-byte row pieces.
+__device__ __forceinline__ void wgk_epilogue(const V2Args& e, const WgkTile& w, WgkBars* bars, uint32_t tmem,
+                                             uint32_t wbuf, int warp, int lane) {
+  const int sp = w.sp, kh = w.kh, ct = w.ct, mt = w.mt;
+  mbar_wait_bounded(&bars->done, 0, e.err, kErrWaitDone);
+  tc_fence_after();
+  const float scale = e.scale_out ? __fmul_rn(*e.ta, *e.tb) : 1.0f;
+  const int rsub = lane >> 3, q = lane & 7;
+  for (int kw = 0; kw < e.Kw; ++kw) {
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(warp * 32) << 16) + kw * 128;
+    const int64_t col_base = (static_cast<int64_t>(kh) * e.Kw + kw) * e.Cin + ct * 128;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {     // 16 columns at a time keeps the register count low
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tbase + c + 16 * hf, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
+                       __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
+                       __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
+                       __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
+                       __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
+        }
+      }
+      __syncwarp();
+      const int ci = ct * 128 + c + 4 * q;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = 4 * i + rsub;
+        const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+        const int co = mt * 128 + warp * 32 + row;
+        if (co < e.Cout && ci < e.Cin) {
+          const int64_t idx = (static_cast<int64_t>(sp) * e.M + co) * e.Ncols + col_base + c + 4 * q;
+          *reinterpret_cast<float4*>(e.out + idx) = o;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+template <int FMT, int KW, bool PAIR>
+__global__ void __launch_bounds__(kWgkThreads, 1)
 conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   using L = WgkSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -127,12 +279,15 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   WgkBars* bars = reinterpret_cast<WgkBars*>(smem + L::kBarOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kWgkSlots; ++s) {
-      mbar_init(&bars->full[s], kV2ProdThreads / 32);
-      mbar_init(&bars->empty[s], 1);
+    for (int s = 0; s < kWgkXSlots; ++s) {
+      mbar_init(&bars->xfull[s], kWgkXWarps);
+      mbar_init(&bars->xempty[s], 1);
+    }
+    for (int s = 0; s < kWgkASlots; ++s) {
+      mbar_init(&bars->afull[s], kWgkGWarps);
+      mbar_init(&bars->aempty[s], 1);
     }
     mbar_init(&bars->done, 1);
-    mbar_init(&bars->acc_empty, kV2EpiWarps * 32);
     fence_mbar_init();
   }
   if (warp == kV2MmaWarp) {
@@ -143,131 +298,160 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   __syncthreads();
   tc_fence_after();
   const uint32_t sbase = smem_u32(smem);
-  const int total_q = p.Ho * g.chunks;
+  const uint32_t tmem = bars->tmem;
 
-  // The same (tile, segment, stage) walk in every role: f(tile, w, ho, t, j0, j1)
-  // per stage, t running over j0 .. j1 + sx - 1 of each row segment.
-  auto walk = [&](auto&& f) {
-    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
-      const WgkTile w = wgk_tile(p, g, tile);
-      const int q0 = w.sp * g.q_per_split;
-      const int q1 = min(total_q, q0 + g.q_per_split);
-      for (int q = q0; q < q1;) {
-        const int ho = q / g.chunks;
-        const int j0 = q - ho * g.chunks;
-        const int j1 = min(g.chunks, j0 + (q1 - q));
-        for (int t = j0; t < j1 + g.sx; ++t) f(tile, w, ho, t, j0, j1);
-        q += j1 - j0;
+  const WgkTile w = wgk_tile(p, g, blockIdx.x);
+  const int xi = wgk_x_index(warp);
+  if (xi >= 0) {
+    // X producer: kWgkLookahead stages of codes in flight (a ring of
+    // registers indexed at compile time)
+    const int tid = xi * 32 + lane;
+    WgkCursor cur, ld;
+    cur.begin(p, g, w);
+    ld = cur;
+    UnitRaw<FMT, 8> ring[kWgkLookahead];
+#pragma unroll
+    for (int r = 0; r < kWgkLookahead; ++r)
+      if (ld.valid) {
+        wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
+        ld.advance(g, g.sx);
+      }
+    int kit = 0;
+    while (cur.valid) {
+#pragma unroll
+      for (int r = 0; r < kWgkLookahead; ++r) {
+        if (!cur.valid) break;
+        const int s = kit % kWgkXSlots;
+        mbar_wait_bounded(&bars->xempty[s], ((kit / kWgkXSlots) & 1) ^ 1, p.err, kErrWaitEmpty);
+        const uint32_t mirror = (PAIR && s < kWgkXMirrors) ? sbase + (kWgkXSlots + s) * L::kXSlot : 0u;
+        wgk_x_store<FMT>(ring[r], sbase + s * L::kXSlot, mirror, tid);
+        producer_warp_arrive(&bars->xfull[s]);
+        if (ld.valid) {
+          wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
+          ld.advance(g, g.sx);
+        }
+        cur.advance(g, g.sx);
+        ++kit;
       }
     }
-  };
-
-  if (warp >= kV2ProdWarp0) {
-    const int t_id = threadIdx.x - kV2ProdWarp0 * 32;
-    int kit = 0;
-    walk([&](int, const WgkTile& w, int ho, int t, int, int j1) {
-      const int s = kit % kWgkSlots;
-      mbar_wait_bounded(&bars->empty[s], ((kit / kWgkSlots) & 1) ^ 1, p.err, kErrWaitEmpty);
-      wgk_fill<FMT>(p, sbase + s * L::kSlot, w, ho, t_id, t < j1, t);
-      producer_warp_arrive(&bars->full[s]);
-      ++kit;
-    });
+  } else if (warp < 4 || (warp >= 8 && warp < 12)) {
+    // G_Y producer: thread = output-channel row (this warp's TMEM lane
+    // quarter); warps 0-3 write columns 0-15 of a slot, warps 8-11 columns
+    // 16-31.  Warps 0-3 then run the epilogue.
+    const int quarter = warp & 3, half = warp < 4 ? 0 : 1;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    WgkCursor cur, ld;
+    cur.begin(p, g, w);
+    ld = cur;
+    WgkGRaw ring[kWgkLookahead];
+#pragma unroll
+    for (int r = 0; r < kWgkLookahead; ++r)
+      if (ld.valid) {
+        wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
+        ld.advance(g, 0);
+      }
+    int ait = 0;
+    while (cur.valid) {
+#pragma unroll
+      for (int r = 0; r < kWgkLookahead; ++r) {
+        if (!cur.valid) break;
+        const int s = ait % kWgkASlots;
+        uint32_t h[16];
+        wgk_g_dequant<FMT>(ring[r], h);
+        mbar_wait_bounded(&bars->aempty[s], ((ait / kWgkASlots) & 1) ^ 1, p.err, kErrWaitEmpty);
+        tc_fence_after();
+        tmem_st_32x32b_x16(tmem + lane_base + kWgkACol + s * 32 + 16 * half, h);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->afull[s]);
+        if (ld.valid) {
+          wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
+          ld.advance(g, 0);
+        }
+        cur.advance(g, 0);
+        ++ait;
+      }
+    }
+    if (half == 0) wgk_epilogue(p, w, bars, tmem, sbase + L::kEpiOffset + quarter * L::kEpiWarpBytes, warp, lane);
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, 128);
-      int kit = 0, cur_tile = -1, tiles_seen = 0;
-      bool started[kWgkMaxTaps] = {false, false, false};
-      walk([&](int tile, const WgkTile&, int, int t, int j0, int j1) {
-        if (tile != cur_tile) {
-          if (cur_tile >= 0) mma_commit(&bars->done);   // previous tile finished: hand over
-          if (tiles_seen > 0) {                         // its accumulators must be read first
-            mbar_wait_bounded(&bars->acc_empty, (tiles_seen - 1) & 1, p.err, kErrWaitEmpty);
-            tc_fence_after();
-          }
-          ++tiles_seen;
-          cur_tile = tile;
-          for (int kw = 0; kw < kWgkMaxTaps; ++kw) started[kw] = false;
+      // The B operand of tap kw, K slice kk is X chunk j + o / 64, slice
+      // (o % 64) / 16, o = 16·kk + kw·N: a fixed slot delta and descriptor
+      // offset per (kw, kk), so each MMA costs a few integer operations.
+      uint32_t bdelta[KW][4], boff[KW][4];
+#pragma unroll
+      for (int kw = 0; kw < KW; ++kw)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t o = 16u * kk + static_cast<uint32_t>(kw * p.N);
+          bdelta[kw][kk] = o >> 6;
+          boff[kw][kk] = 2u * ((o & 63u) >> 4);
         }
-        const int s = kit % kWgkSlots;
-        mbar_wait_bounded(&bars->full[s], (kit / kWgkSlots) & 1, p.err, kErrWaitFull);
+      const uint64_t desc0 = smem_desc_sw128(sbase);
+      constexpr uint32_t kSlotDesc = L::kXSlot >> 4;
+      int kit = 0, ait = 0;
+      bool started = false;     // an output chunk has been issued
+      WgkCursor c;
+      for (c.begin(p, g, w); c.valid; c.advance(g, g.sx)) {
+        const int s = kit % kWgkXSlots;
+        mbar_wait_bounded(&bars->xfull[s], (kit / kWgkXSlots) & 1, p.err, kErrWaitFull);
         tc_fence_after();
-        if (t >= j0 + g.sx) {
-          // output chunk j = t - sx: G_Y chunk in slot (kit - sx), X chunks in slots kit - sx .. kit
-          const int sj = (kit - g.sx) % kWgkSlots;
-          const uint64_t adesc = smem_desc_sw128(sbase + sj * L::kSlot);
-          for (int kw = 0; kw < p.Kw; ++kw) {
+        if (c.t >= c.j0 + g.sx) {
+          // output chunk j = t - sx: G_Y chunk in A slot ait, X chunks in X slots kit - sx .. kit
+          const int as = ait % kWgkASlots;
+          mbar_wait_bounded(&bars->afull[as], (ait / kWgkASlots) & 1, p.err, kErrWaitFull);
+          tc_fence_after();
+          const uint32_t a_t = tmem + kWgkACol + as * 32;
+          const uint32_t xbase = static_cast<uint32_t>(kit - g.sx);
+          if (PAIR) {
+            // N = 64: tap kw reads X chunk j + kw whole, and chunks j..j+KW-1
+            // sit in consecutive slots (slots 0 and 1 are mirrored after the
+            // ring), so the taps' B operands are one run of KW·128 rows:
+            // two N = 192 MMAs for three taps, one N = 256 MMA for two.
+            const uint64_t b = desc0 + (xbase & (kWgkXSlots - 1)) * kSlotDesc;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const int o = 16 * kk + kw * p.N;     // element offset from X chunk j
-              const int sx = (kit - g.sx + o / 64) % kWgkSlots;
-              const uint64_t bdesc = smem_desc_sw128(sbase + sx * L::kSlot + kATileBytes) + 2 * ((o & 63) >> 4);
-              mma_f16_ss(bars->tmem + kw * 128, adesc + 2 * kk, bdesc, idesc, started[kw] ? 1u : 0u);
-              started[kw] = true;
+              const uint32_t acc = (started || kk > 0) ? 1u : 0u;
+              if (KW == 3) {
+                mma_f16_ts(tmem, a_t + 8 * kk, b + 2 * kk, idesc_f16_f32(128, 192), acc);
+                mma_f16_ts(tmem + 192, a_t + 8 * kk, b + (192 * 128 >> 4) + 2 * kk, idesc_f16_f32(128, 192), acc);
+              } else {
+                mma_f16_ts(tmem, a_t + 8 * kk, b + 2 * kk, idesc_f16_f32(128, 256), acc);
+              }
             }
+          } else {
+#pragma unroll
+            for (int kw = 0; kw < KW; ++kw)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t slot = (xbase + bdelta[kw][kk]) & (kWgkXSlots - 1);
+                const uint64_t bdesc = desc0 + (slot * kSlotDesc + boff[kw][kk]);
+                mma_f16_ts(tmem + kw * 128, a_t + 8 * kk, bdesc, idesc, (started || kk > 0) ? 1u : 0u);
+              }
           }
-          mma_commit(&bars->empty[sj]);
+          started = true;
+          mma_commit(&bars->aempty[as]);
+          mma_commit(&bars->xempty[xbase & (kWgkXSlots - 1)]);
+          ++ait;
         }
-        if (t == j1 + g.sx - 1) {
+        if (c.t == c.j1 + g.sx - 1) {
           // end of the segment (always an MMA stage): its last sx slots hold
           // X chunks no later output chunk of this row reads
-          for (int k = kit - g.sx + 1; k <= kit; ++k) mma_commit(&bars->empty[k % kWgkSlots]);
+          for (int k = kit - g.sx + 1; k <= kit; ++k) mma_commit(&bars->xempty[k % kWgkXSlots]);
         }
         ++kit;
-      });
-      if (cur_tile >= 0) mma_commit(&bars->done);
-    }
-  } else if (warp < kV2EpiWarps) {
-    int it = 0;
-    for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
-      const WgkTile w = wgk_tile(p, g, tile);
-      mbar_wait_bounded(&bars->done, it & 1, p.err, kErrWaitDone);
-      tc_fence_after();
-      const float scale = p.scale_out ? __fmul_rn(*p.ta, *p.tb) : 1.0f;
-      // Each lane reads one accumulator row (output channel) from TMEM; a
-      // swizzled 32 x 32 transpose in shared memory turns that into stores of
-      // four whole 128-byte row pieces per warp instruction.
-      const uint32_t wbuf = sbase + L::kEpiOffset + warp * L::kEpiWarpBytes;
-      const int rsub = lane >> 3, q = lane & 7;
-      for (int kw = 0; kw < p.Kw; ++kw) {
-        const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + kw * 128;
-        const int64_t col_base = (static_cast<int64_t>(w.kh) * p.Kw + kw) * p.Cin + w.ct * 128;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            st_shared_v4(wbuf + lane * 128 + ((j ^ (lane & 7)) << 4),
-                         __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
-          }
-          __syncwarp();
-          const int ci = w.ct * 128 + c + 4 * q;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int row = 4 * i + rsub;
-            const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
-            const int co = w.mt * 128 + warp * 32 + row;
-            if (co < p.Cout && ci < p.Cin) {
-              const int64_t idx = (static_cast<int64_t>(w.sp) * p.M + co) * p.Ncols + col_base + c + 4 * q;
-              *reinterpret_cast<float4*>(p.out + idx) = o;
-            }
-          }
-          __syncwarp();
-        }
       }
-      tc_fence_before();
-      mbar_arrive(&bars->acc_empty);     // the next tile may overwrite the accumulators
+      mma_commit(&bars->done);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == kV2MmaWarp) {
     tc_fence_after();
-    tmem_dealloc(bars->tmem, 512);
+    tmem_dealloc(tmem, 512);
   }
 }
 

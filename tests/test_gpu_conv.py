@@ -63,6 +63,9 @@ SMALL = [
     ("wgk_n32_fp6_two_tiles", O.ConvShape(32, 200, 136, 6, 5, 3, 3, 1, 0), "nvfp6"),
     ("wgk_n48_2x2", O.ConvShape(48, 16, 20, 8, 8, 2, 2, 1, 0), "nvfp4"),
     ("wgk_rows_split", O.ConvShape(16, 256, 512, 10, 10, 3, 3, 1, 1), "nvfp4"),
+    # batch 64: the taps of a kernel row share one run of B rows (paired MMAs)
+    ("wgk_n64_pair_2x2", O.ConvShape(64, 200, 72, 6, 7, 2, 2, 1, 0), "nvfp4"),
+    ("wgk_n64_pair_fp6", O.ConvShape(64, 136, 40, 5, 6, 3, 3, 1, 1), "nvfp6"),
 ]
 
 
