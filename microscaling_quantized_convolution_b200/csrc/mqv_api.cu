@@ -467,9 +467,8 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
     if (e != cudaSuccess) return cuda_fail(e, "wgrad launch");
     if (pl.a.splits > 1) {
       const int64_t n4 = (int64_t)pl.a.M * pl.a.Ncols / 4;
-      int64_t g = (n4 + 255) / 256;
-      if (g > kSMs * 8) g = kSMs * 8;
-      wgrad_reduce_kernel<<<(unsigned)g, 256, 0, s>>>(reinterpret_cast<const float4*>(wsb), pl.a.splits, n4,
+      const int64_t g = (n4 + kReduceCols - 1) / kReduceCols;
+      wgrad_reduce_kernel<<<(unsigned)g, kReduceCols * kReduceGroups, 0, s>>>(reinterpret_cast<const float4*>(wsb), pl.a.splits, n4,
                                                        qa->tscale, qb->tscale, reinterpret_cast<float4*>(out));
       e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(e, "wgrad reduce launch");

@@ -28,21 +28,30 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t k) {
   return row * 128u + ((((k >> 3) ^ (row & 7u)) << 4) | ((k & 4u) << 1));
 }
 
-// G_W = T_g·T_x·sum over splits of the partial tiles, in split order.
-__global__ void __launch_bounds__(256)
+// G_W = T_g·T_x·sum over splits of the partial tiles.  A block takes 64
+// float4 columns; four thread groups each add a contiguous quarter of the
+// splits in split order, and the four group sums are added in group order, so
+// the result is the same on every run.  Sixteen independent loads per thread
+// keep enough bytes in flight to run at memory speed.
+constexpr int kReduceCols = 64, kReduceGroups = 4;
+__global__ void __launch_bounds__(kReduceCols * kReduceGroups)
 wgrad_reduce_kernel(const float4* __restrict__ partial, int splits, int64_t n4,
                     const float* __restrict__ ta, const float* __restrict__ tb,
                     float4* __restrict__ out) {
-  const float scale = __fmul_rn(*ta, *tb);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  constexpr int kBatch = 8;     // loads in flight per thread; the adds stay in split order
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
-    float4 acc = __ldg(partial + i);
-    int s = 1;
-    for (; s + kBatch <= splits; s += kBatch) {
+  __shared__ float4 part[kReduceGroups][kReduceCols];
+  const int col = threadIdx.x % kReduceCols, grp = threadIdx.x / kReduceCols;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kReduceCols + col;
+  const int per = (splits + kReduceGroups - 1) / kReduceGroups;
+  const int s0 = grp * per, s1 = min(splits, s0 + per);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (i < n4 && s0 < s1) {
+    acc = __ldg(partial + static_cast<int64_t>(s0) * n4 + i);
+    int s = s0 + 1;
+    constexpr int kBatch = 16;
+    for (; s + kBatch <= s1; s += kBatch) {
       float4 v[kBatch];
 #pragma unroll
-      for (int b = 0; b < kBatch; ++b) v[b] = __ldg(partial + (s + b) * n4 + i);
+      for (int b = 0; b < kBatch; ++b) v[b] = __ldg(partial + static_cast<int64_t>(s + b) * n4 + i);
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
         acc.x += v[b].x;
@@ -51,18 +60,32 @@ wgrad_reduce_kernel(const float4* __restrict__ partial, int splits, int64_t n4,
         acc.w += v[b].w;
       }
     }
-    for (; s < splits; ++s) {
-      const float4 v = __ldg(partial + s * n4 + i);
+    for (; s < s1; ++s) {
+      const float4 v = __ldg(partial + static_cast<int64_t>(s) * n4 + i);
       acc.x += v.x;
       acc.y += v.y;
       acc.z += v.z;
       acc.w += v.w;
     }
-    acc.x *= scale;
-    acc.y *= scale;
-    acc.z *= scale;
-    acc.w *= scale;
-    out[i] = acc;
+  }
+  part[grp][col] = acc;
+  __syncthreads();
+  if (grp == 0 && i < n4) {
+    float4 t = part[0][col];
+#pragma unroll
+    for (int g = 1; g < kReduceGroups; ++g) {
+      const float4 v = part[g][col];
+      t.x += v.x;
+      t.y += v.y;
+      t.z += v.z;
+      t.w += v.w;
+    }
+    const float scale = __fmul_rn(*ta, *tb);
+    t.x *= scale;
+    t.y *= scale;
+    t.z *= scale;
+    t.w *= scale;
+    out[i] = t;
   }
 }
 

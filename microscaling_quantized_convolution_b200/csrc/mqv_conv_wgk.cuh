@@ -22,8 +22,8 @@
 // [j0, j1 + SX), SX = the furthest X chunk a tap reaches; output chunk
 // j = t - SX runs at stage t >= j0 + SX and reads X chunks j..j+SX.  The X
 // and G_Y rings advance independently.  Splits of the (ho, j) chunk range
-// across CTAs make the partial sums that wgrad_reduce_kernel adds in split
-// order.
+// across CTAs make the partial sums that wgrad_reduce_kernel adds in a
+// fixed order.
 #pragma once
 
 #include <cstdint>
@@ -40,10 +40,10 @@ constexpr int kWgkASlots = 4;           // G_Y chunks in tensor memory
 constexpr int kWgkMaxTaps = 3;
 constexpr int kWgkACol = kWgkMaxTaps * 128;     // first TMEM column of the G_Y ring
 constexpr int kWgkLookahead = 2;        // stages of codes in flight per producer thread
-// Roles: warps 0-3 produce the first half of each G_Y chunk and run the
-// epilogue between tiles; warp 4 issues the MMAs; warps 8-11 produce the
-// second G_Y half (each G_Y warp owns its TMEM lane quarter, warp % 4);
-// warps 6, 7 and 12-17 produce X.  Warp 5 has no role.
+// Roles: warps 0-3 produce the first half of each G_Y chunk, warps 8-11 the
+// second (each G_Y warp owns its TMEM lane quarter, warp % 4); warps 6, 7 and
+// 12-17 produce X; warp 4 issues the MMAs; warp 5 has no role.  All 16
+// producer warps then run the epilogue.
 constexpr int kWgkWarps = 18;
 constexpr int kWgkThreads = kWgkWarps * 32;
 constexpr int kWgkXWarps = 8;
@@ -63,18 +63,23 @@ struct WgkGeom {
 
 struct WgkSmem {
   static constexpr int kXSlot = kATileBytes;                 // 128 channels x 64 fp16
-  static constexpr int kEpiOffset = (kWgkXSlots + kWgkXMirrors) * kXSlot;   // 32 x 32 fp32 per epilogue warp
-  static constexpr int kEpiWarpBytes = 32 * 128;
-  static constexpr int kBarOffset = kEpiOffset + 4 * kEpiWarpBytes;
+  static constexpr int kEpiWarpBytes = 32 * 128;                  // epilogue transpose buffer per warp,
+                                                                   // inside the X ring once it is idle
+  static constexpr int kBarOffset = (kWgkXSlots + kWgkXMirrors) * kXSlot;
   static constexpr int kBytes = kBarOffset + 256 + 1024;
 };
 
+// One full and one done barrier per stage of the X ring: both producers
+// arrive on full[n % 8] for every stage n (the G_Y warps with the A chunk
+// of an MMA stage, immediately otherwise), and the MMA thread commits
+// done[n % 8] after every stage, so it waits once and commits once a stage.
+// X stage n reuses its slot once stage n - 8 + SX (the last that reads the
+// previous X chunk in it) is done; G_Y chunk a reuses A slot a % 4 once the
+// stage four earlier is done (chunk a - 4 ran no later than that).
 struct WgkBars {
-  uint64_t xfull[kWgkXSlots];
-  uint64_t xempty[kWgkXSlots];
-  uint64_t afull[kWgkASlots];
-  uint64_t aempty[kWgkASlots];
-  uint64_t done;        // all MMAs of the tile completed (tcgen05.commit)
+  uint64_t full[kWgkXSlots];
+  uint64_t done[kWgkXSlots];
+  uint64_t tile_done;   // all MMAs of the tile completed (tcgen05.commit)
   uint32_t tmem;
 };
 
@@ -101,24 +106,26 @@ struct WgkCursor {
   int q, q1, ho, j0, j1, t;
   bool valid;
 
-  __device__ __forceinline__ void segment(const WgkGeom& g) {
+  __device__ __forceinline__ void begin(const V2Args& p, const WgkGeom& g, const WgkTile& w) {
+    q = w.sp * g.q_per_split;
+    q1 = min(p.Ho * g.chunks, q + g.q_per_split);
+    valid = q < q1;
     ho = q / g.chunks;
     j0 = q - ho * g.chunks;
     j1 = min(g.chunks, j0 + (q1 - q));
     t = j0;
   }
-  __device__ __forceinline__ void begin(const V2Args& p, const WgkGeom& g, const WgkTile& w) {
-    q = w.sp * g.q_per_split;
-    q1 = min(p.Ho * g.chunks, q + g.q_per_split);
-    valid = q < q1;
-    if (valid) segment(g);
-  }
+  // after the first segment every segment starts a new output row
   __device__ __forceinline__ void advance(const WgkGeom& g, int ext) {
     if (++t < j1 + ext) return;
     q += j1 - j0;
     valid = q < q1;
-    if (valid) segment(g);
+    ++ho;
+    j0 = 0;
+    j1 = min(g.chunks, q1 - q);
+    t = 0;
   }
+  __device__ __forceinline__ bool mma_stage(const WgkGeom& g) const { return t >= j0 + g.sx; }
 };
 
 // X producer: one unit (4 channels x 8 consecutive (pixel, n) elements) per
@@ -224,49 +231,50 @@ __device__ __forceinline__ void wgk_g_dequant(const WgkGRaw& r, uint32_t (&h)[16
   }
 }
 
-// Epilogue of one tile (warps 0-3, one TMEM lane quarter each): accumulator
-// rows are read with tcgen05.ld, transposed through a swizzled 32 x 32 buffer
-// in shared memory, and stored as whole 128-byte row pieces.
+// Epilogue of the tile, run by all 16 producer warps once the last MMA has
+// completed: four warps per TMEM lane quarter (warp % 4), each taking every
+// fourth 32-column block of the Kw·128 accumulator columns.  Rows are read
+// with tcgen05.ld, transposed through a swizzled 32 x 32 buffer in shared
+// memory (the X ring is free by then), and stored as whole 128-byte row
+// pieces.
 __device__ __forceinline__ void wgk_epilogue(const V2Args& e, const WgkTile& w, WgkBars* bars, uint32_t tmem,
-                                             uint32_t wbuf, int warp, int lane) {
-  const int sp = w.sp, kh = w.kh, ct = w.ct, mt = w.mt;
-  mbar_wait_bounded(&bars->done, 0, e.err, kErrWaitDone);
+                                             uint32_t wbuf, int quarter, int cpart, int lane) {
+  mbar_wait_bounded(&bars->tile_done, 0, e.err, kErrWaitDone);
   tc_fence_after();
   const float scale = e.scale_out ? __fmul_rn(*e.ta, *e.tb) : 1.0f;
   const int rsub = lane >> 3, q = lane & 7;
-  for (int kw = 0; kw < e.Kw; ++kw) {
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(warp * 32) << 16) + kw * 128;
-    const int64_t col_base = (static_cast<int64_t>(kh) * e.Kw + kw) * e.Cin + ct * 128;
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 32) {
+  for (int blk = cpart; blk < 4 * e.Kw; blk += 4) {
+    const int kw = blk >> 2, c = (blk & 3) * 32;
+    const int64_t col_base = (static_cast<int64_t>(w.kh) * e.Kw + kw) * e.Cin + w.ct * 128;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {     // 16 columns at a time keeps the register count low
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tbase + c + 16 * hf, r);
-        tmem_ld_wait();
+    for (int hf = 0; hf < 2; ++hf) {     // 16 columns at a time keeps the register count low
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(tlane + kw * 128 + c + 16 * hf, r);
+      tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
-                       __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
-                       __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
-                       __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
-                       __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
-        }
+      for (int j = 0; j < 4; ++j) {
+        st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
+                     __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
       }
-      __syncwarp();
-      const int ci = ct * 128 + c + 4 * q;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int row = 4 * i + rsub;
-        const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
-        const int co = mt * 128 + warp * 32 + row;
-        if (co < e.Cout && ci < e.Cin) {
-          const int64_t idx = (static_cast<int64_t>(sp) * e.M + co) * e.Ncols + col_base + c + 4 * q;
-          *reinterpret_cast<float4*>(e.out + idx) = o;
-        }
-      }
-      __syncwarp();
     }
+    __syncwarp();
+    const int ci = w.ct * 128 + c + 4 * q;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = 4 * i + rsub;
+      const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+      const int co = w.mt * 128 + quarter * 32 + row;
+      if (co < e.Cout && ci < e.Cin) {
+        const int64_t idx = (static_cast<int64_t>(w.sp) * e.M + co) * e.Ncols + col_base + c + 4 * q;
+        *reinterpret_cast<float4*>(e.out + idx) = o;
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -280,14 +288,10 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWgkXSlots; ++s) {
-      mbar_init(&bars->xfull[s], kWgkXWarps);
-      mbar_init(&bars->xempty[s], 1);
+      mbar_init(&bars->full[s], kWgkXWarps + kWgkGWarps);
+      mbar_init(&bars->done[s], 1);
     }
-    for (int s = 0; s < kWgkASlots; ++s) {
-      mbar_init(&bars->afull[s], kWgkGWarps);
-      mbar_init(&bars->aempty[s], 1);
-    }
-    mbar_init(&bars->done, 1);
+    mbar_init(&bars->tile_done, 1);
     fence_mbar_init();
   }
   if (warp == kV2MmaWarp) {
@@ -302,6 +306,10 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
 
   const WgkTile w = wgk_tile(p, g, blockIdx.x);
   const int xi = wgk_x_index(warp);
+  // wait until stage m's MMAs have completed
+  auto wait_done = [&](int m) {
+    mbar_wait_bounded(&bars->done[m % kWgkXSlots], (m / kWgkXSlots) & 1, p.err, kErrWaitEmpty);
+  };
   if (xi >= 0) {
     // X producer: kWgkLookahead stages of codes in flight (a ring of
     // registers indexed at compile time)
@@ -316,28 +324,29 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
         wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
         ld.advance(g, g.sx);
       }
-    int kit = 0;
+    int n = 0;
     while (cur.valid) {
 #pragma unroll
       for (int r = 0; r < kWgkLookahead; ++r) {
         if (!cur.valid) break;
-        const int s = kit % kWgkXSlots;
-        mbar_wait_bounded(&bars->xempty[s], ((kit / kWgkXSlots) & 1) ^ 1, p.err, kErrWaitEmpty);
+        const int s = n % kWgkXSlots;
+        if (n >= kWgkXSlots) wait_done(n - kWgkXSlots + g.sx);
         const uint32_t mirror = (PAIR && s < kWgkXMirrors) ? sbase + (kWgkXSlots + s) * L::kXSlot : 0u;
         wgk_x_store<FMT>(ring[r], sbase + s * L::kXSlot, mirror, tid);
-        producer_warp_arrive(&bars->xfull[s]);
+        producer_warp_arrive(&bars->full[s]);
         if (ld.valid) {
           wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
           ld.advance(g, g.sx);
         }
         cur.advance(g, g.sx);
-        ++kit;
+        ++n;
       }
     }
   } else if (warp < 4 || (warp >= 8 && warp < 12)) {
     // G_Y producer: thread = output-channel row (this warp's TMEM lane
     // quarter); warps 0-3 write columns 0-15 of a slot, warps 8-11 columns
-    // 16-31.  Warps 0-3 then run the epilogue.
+    // 16-31.  It walks the X stages, loading ahead along the output chunks.
+    // All producer warps run the epilogue afterwards.
     const int quarter = warp & 3, half = warp < 4 ? 0 : 1;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -351,30 +360,35 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
         wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
         ld.advance(g, 0);
       }
-    int ait = 0;
+    int n = 0, a = 0;
     while (cur.valid) {
 #pragma unroll
       for (int r = 0; r < kWgkLookahead; ++r) {
+        while (cur.valid && !cur.mma_stage(g)) {    // stages with no G_Y chunk
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->full[n % kWgkXSlots]);
+          cur.advance(g, g.sx);
+          ++n;
+        }
         if (!cur.valid) break;
-        const int s = ait % kWgkASlots;
         uint32_t h[16];
         wgk_g_dequant<FMT>(ring[r], h);
-        mbar_wait_bounded(&bars->aempty[s], ((ait / kWgkASlots) & 1) ^ 1, p.err, kErrWaitEmpty);
+        if (n >= kWgkASlots) wait_done(n - kWgkASlots);
         tc_fence_after();
-        tmem_st_32x32b_x16(tmem + lane_base + kWgkACol + s * 32 + 16 * half, h);
+        tmem_st_32x32b_x16(tmem + lane_base + kWgkACol + (a % kWgkASlots) * 32 + 16 * half, h);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->afull[s]);
+        if (lane == 0) mbar_arrive(&bars->full[n % kWgkXSlots]);
         if (ld.valid) {
           wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
           ld.advance(g, 0);
         }
-        cur.advance(g, 0);
-        ++ait;
+        cur.advance(g, g.sx);
+        ++n;
+        ++a;
       }
     }
-    if (half == 0) wgk_epilogue(p, w, bars, tmem, sbase + L::kEpiOffset + quarter * L::kEpiWarpBytes, warp, lane);
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, 128);
@@ -392,20 +406,17 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
         }
       const uint64_t desc0 = smem_desc_sw128(sbase);
       constexpr uint32_t kSlotDesc = L::kXSlot >> 4;
-      int kit = 0, ait = 0;
-      bool started = false;     // an output chunk has been issued
+      int n = 0, a = 0;
       WgkCursor c;
-      for (c.begin(p, g, w); c.valid; c.advance(g, g.sx)) {
-        const int s = kit % kWgkXSlots;
-        mbar_wait_bounded(&bars->xfull[s], (kit / kWgkXSlots) & 1, p.err, kErrWaitFull);
+      for (c.begin(p, g, w); c.valid; c.advance(g, g.sx), ++n) {
+        const int s = n % kWgkXSlots;
+        mbar_wait_bounded(&bars->full[s], (n / kWgkXSlots) & 1, p.err, kErrWaitFull);
         tc_fence_after();
-        if (c.t >= c.j0 + g.sx) {
-          // output chunk j = t - sx: G_Y chunk in A slot ait, X chunks in X slots kit - sx .. kit
-          const int as = ait % kWgkASlots;
-          mbar_wait_bounded(&bars->afull[as], (ait / kWgkASlots) & 1, p.err, kErrWaitFull);
-          tc_fence_after();
-          const uint32_t a_t = tmem + kWgkACol + as * 32;
-          const uint32_t xbase = static_cast<uint32_t>(kit - g.sx);
+        if (c.mma_stage(g)) {
+          // output chunk j = t - sx: G_Y chunk in A slot a % 4, X chunks in X slots n - sx .. n
+          const uint32_t a_t = tmem + kWgkACol + (a % kWgkASlots) * 32;
+          const uint32_t xbase = static_cast<uint32_t>(n - g.sx);
+          const uint32_t first = a == 0 ? 0u : 1u;
           if (PAIR) {
             // N = 64: tap kw reads X chunk j + kw whole, and chunks j..j+KW-1
             // sit in consecutive slots (slots 0 and 1 are mirrored after the
@@ -414,7 +425,7 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
             const uint64_t b = desc0 + (xbase & (kWgkXSlots - 1)) * kSlotDesc;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (started || kk > 0) ? 1u : 0u;
+              const uint32_t acc = kk > 0 ? 1u : first;
               if (KW == 3) {
                 mma_f16_ts(tmem, a_t + 8 * kk, b + 2 * kk, idesc_f16_f32(128, 192), acc);
                 mma_f16_ts(tmem + 192, a_t + 8 * kk, b + (192 * 128 >> 4) + 2 * kk, idesc_f16_f32(128, 192), acc);
@@ -429,23 +440,20 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
               for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t slot = (xbase + bdelta[kw][kk]) & (kWgkXSlots - 1);
                 const uint64_t bdesc = desc0 + (slot * kSlotDesc + boff[kw][kk]);
-                mma_f16_ts(tmem + kw * 128, a_t + 8 * kk, bdesc, idesc, (started || kk > 0) ? 1u : 0u);
+                mma_f16_ts(tmem + kw * 128, a_t + 8 * kk, bdesc, idesc, kk > 0 ? 1u : first);
               }
           }
-          started = true;
-          mma_commit(&bars->aempty[as]);
-          mma_commit(&bars->xempty[xbase & (kWgkXSlots - 1)]);
-          ++ait;
+          ++a;
         }
-        if (c.t == c.j1 + g.sx - 1) {
-          // end of the segment (always an MMA stage): its last sx slots hold
-          // X chunks no later output chunk of this row reads
-          for (int k = kit - g.sx + 1; k <= kit; ++k) mma_commit(&bars->xempty[k % kWgkXSlots]);
-        }
-        ++kit;
+        mma_commit(&bars->done[s]);
       }
-      mma_commit(&bars->done);
+      mma_commit(&bars->tile_done);
     }
+  }
+  if (xi >= 0 || warp < 4 || (warp >= 8 && warp < 12)) {
+    // column part: G_Y warps 0-3 -> 0, 8-11 -> 1; X warps 6, 7, 12, 13 -> 2; 14-17 -> 3
+    const int cpart = warp < 4 ? 0 : warp < 12 && warp >= 8 ? 1 : (warp < 14 ? 2 : 3);
+    wgk_epilogue(p, w, bars, tmem, sbase + warp * L::kEpiWarpBytes, warp & 3, cpart, lane);
   }
   tc_fence_before();
   __syncthreads();
