@@ -84,11 +84,21 @@ int64_t quant_ctas(int64_t rows, int64_t cols) {
   return g < kMaxQuantCtas ? g : kMaxQuantCtas;
 }
 
+FastDiv make_fastdiv(int64_t d) {
+  FastDiv f;
+  uint32_t s = 0;
+  while ((int64_t(1) << s) < d) ++s;
+  const unsigned __int128 num = (static_cast<unsigned __int128>(1) << (32 + s)) + (d - 1);
+  f.m = static_cast<uint32_t>(static_cast<uint64_t>(num / static_cast<unsigned __int128>(d)) - (uint64_t(1) << 32));
+  f.s = s;
+  return f;
+}
+
 mqv_status check_view(int64_t rows, int64_t cols) {
   if (rows <= 0 || cols <= 0 || rows % 4 || cols % 4)
     return fail(MQV_ERR_INVALID_ARG, "view %lld x %lld: rows and cols must be positive multiples of 4",
                 (long long)rows, (long long)cols);
-  if (rows > (int64_t(1) << 40) / cols)
+  if (rows > (int64_t(1) << 34) / cols)     // quantize work units (4 x 4 blocks) stay below 2^30
     return fail(MQV_ERR_UNSUPPORTED, "view %lld x %lld too large", (long long)rows, (long long)cols);
   return MQV_OK;
 }
@@ -112,32 +122,53 @@ mqv_status check_qtensor(const mqv_qtensor* q, const char* name) {
   return MQV_OK;
 }
 
-template <int FMT, int RND>
-void launch_quantize(const float* src, int64_t rows, int64_t cols, const float* amax_src,
-                     int amax_count, uint64_t seed, int64_t sr_cols, int64_t sr_col0,
-                     const mqv_qtensor* out, cudaStream_t st) {
-  uint8_t* codes = static_cast<uint8_t*>(out->codes);
-  if ((cols / 4) % 2 == 0) {
-    const unsigned g = (unsigned)quant_ctas(rows, cols / 2);
-    quantize_kernel<FMT, RND, 2><<<g, kQuantThreads, 0, st>>>(
-        src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes, out->scales, out->tscale);
-  } else {
-    const unsigned g = (unsigned)quant_ctas(rows, cols);
-    quantize_kernel<FMT, RND, 1><<<g, kQuantThreads, 0, st>>>(
-        src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes, out->scales, out->tscale);
+// Round keys of Philox4x32-10 for a 64-bit seed (key = low, high word).
+PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys k;
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    k.k0[r] = k0;
+    k.k1[r] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
   }
+  return k;
+}
+
+// One 4 x 4 block per work unit (QB = 1): the fewest registers per thread.
+QuantArgs make_quant_args(const float* src, int64_t rows, int64_t cols, uint64_t seed, int64_t sr_cols,
+                          int64_t sr_col0, const mqv_qtensor* out) {
+  QuantArgs qa;
+  qa.src = src;
+  qa.rows = rows;
+  qa.cols = cols;
+  qa.codes = static_cast<uint8_t*>(out->codes);
+  qa.scales = out->scales;
+  qa.tscale = out->tscale;
+  qa.keys = philox_keys(seed);
+  qa.sr_cols = sr_cols;
+  qa.sr_col0 = sr_col0;
+  qa.dcu = make_fastdiv(cols / 4);
+  return qa;
+}
+
+template <int FMT, int RND>
+void launch_quantize(const QuantArgs& qa, const float* amax_src, int amax_count, cudaStream_t st) {
+  const unsigned g = (unsigned)quant_ctas(qa.rows, qa.cols);
+  quantize_kernel<FMT, RND, 1><<<g, kQuantThreads, 0, st>>>(qa, amax_src, amax_count);
 }
 
 mqv_status enqueue_quantize(const float* src, int64_t rows, int64_t cols, int32_t fmt,
                             int32_t rounding, uint64_t seed, const float* amax_src,
                             int amax_count, int64_t sr_cols, int64_t sr_col0,
                             const mqv_qtensor* out, cudaStream_t st) {
+  const QuantArgs qa = make_quant_args(src, rows, cols, seed, sr_cols, sr_col0, out);
   if (fmt == MQV_NVFP4)
-    rounding == MQV_RNE ? launch_quantize<0, 0>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st)
-                        : launch_quantize<0, 1>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st);
+    rounding == MQV_RNE ? launch_quantize<0, 0>(qa, amax_src, amax_count, st)
+                        : launch_quantize<0, 1>(qa, amax_src, amax_count, st);
   else
-    rounding == MQV_RNE ? launch_quantize<1, 0>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st)
-                        : launch_quantize<1, 1>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, out, st);
+    rounding == MQV_RNE ? launch_quantize<1, 0>(qa, amax_src, amax_count, st)
+                        : launch_quantize<1, 1>(qa, amax_src, amax_count, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return ok();
@@ -213,15 +244,6 @@ QView make_view(const mqv_qtensor* q) {
 }
 
 // Multiplier and shift of mqv::fdiv for divisor d >= 1.
-FastDiv make_fastdiv(int64_t d) {
-  FastDiv f;
-  uint32_t s = 0;
-  while ((int64_t(1) << s) < d) ++s;
-  const unsigned __int128 num = (static_cast<unsigned __int128>(1) << (32 + s)) + (d - 1);
-  f.m = static_cast<uint32_t>(static_cast<uint64_t>(num / static_cast<unsigned __int128>(d)) - (uint64_t(1) << 32));
-  f.s = s;
-  return f;
-}
 
 // Geometry of one pass (no pointers needed for sizing).
 void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
@@ -507,20 +529,14 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
     }
     if (st) return fail(st, "job %d: %s", i, std::string(g_msg).c_str());
     QuantJob& qj = plan->job[i];
-    qj.src = j.src;
-    qj.rows = j.rows;
-    qj.cols = j.cols;
-    qj.codes = static_cast<uint8_t*>(j.out.codes);
-    qj.scales = j.out.scales;
-    qj.tscale = j.out.tscale;
-    qj.seed = j.seed;
+    qj.qa = make_quant_args(j.src, j.rows, j.cols, j.seed, j.cols, 0, &j.out);
     qj.fmt = j.fmt;
     qj.rounding = j.rounding;
-    qj.qb = (j.cols / 4) % 2 == 0 ? 2 : 1;
+    qj.qb = 1;
     qj.amax_cta0 = a;
     qj.amax_ctas = (int)amax_ctas(j.rows, j.cols);
     qj.quant_cta0 = q;
-    qj.quant_ctas = (int)quant_ctas(j.rows, qj.qb == 2 ? j.cols / 2 : j.cols);
+    qj.quant_ctas = (int)quant_ctas(j.rows, j.cols);
     a += qj.amax_ctas;
     q += qj.quant_ctas;
   }

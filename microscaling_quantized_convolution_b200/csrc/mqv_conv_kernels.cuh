@@ -47,19 +47,6 @@ constexpr int kV2Threads = (kV2ProdWarp0 + kV2ProdThreads / 32) * 32;   // 448
 constexpr int kV2Stages = 4;
 constexpr uint32_t kATileBytes = 128 * 64 * 2;                             // 16 KB
 
-// Division of dividends below 2^31 by an invariant positive divisor with one
-// multiply-high, one add and one shift (Granlund & Montgomery, "Division by
-// invariant integers using multiplication", PLDI 1994, round-up variant):
-// s = ceil(log2 d), m = ceil(2^(32+s) / d) - 2^32, q = (umulhi(k, m) + k) >> s.
-struct FastDiv {
-  uint32_t m, s;
-};
-
-__device__ __forceinline__ int fdiv(int k, FastDiv f) {
-  const uint32_t u = static_cast<uint32_t>(k);
-  return static_cast<int>((__umulhi(u, f.m) + u) >> f.s);
-}
-
 struct V2Args {
   const uint8_t* image;   // fwd/dgrad: A image [mtiles][ktiles] x 16 KB
   QView a;                // wgrad: G_Y

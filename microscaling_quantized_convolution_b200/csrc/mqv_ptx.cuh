@@ -8,6 +8,19 @@
 
 namespace mqv {
 
+// Division by a runtime constant d < 2^31 (Granlund and Montgomery, "Division
+// by invariant integers using multiplication", PLDI 1994): with s = ceil(log2 d)
+// and m = ceil(2^(32+s) / d) - 2^32, k / d = (umulhi(k, m) + k) >> s for
+// 0 <= k < 2^31.
+struct FastDiv {
+  uint32_t m, s;
+};
+
+__device__ __forceinline__ int fdiv(int k, FastDiv f) {
+  const uint32_t u = static_cast<uint32_t>(k);
+  return static_cast<int>((__umulhi(u, f.m) + u) >> f.s);
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -295,7 +308,7 @@ __device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float x) {
   return r & 0xFF;
 }
 
-// Two non-negative fp32 -> two E2M1 codes (RNE, saturating at 6):
+// Two fp32 -> two E2M1 codes (RNE, saturating at +-6, sign bit kept):
 // low nibble from lo, high nibble from hi.
 __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
   uint32_t r;
@@ -308,8 +321,8 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
   return r;
 }
 
-// Two non-negative fp32 -> two E2M3 codes (RNE, saturating at 7.5), one per
-// byte: low byte from lo, high byte from hi.
+// Two fp32 -> two E2M3 codes (RNE, saturating at +-7.5, sign bit kept), one
+// per byte: low byte from lo, high byte from hi.
 __device__ __forceinline__ uint32_t f32x2_to_e2m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e2m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));

@@ -19,17 +19,19 @@ constexpr int kQuantThreads = 256;
 
 // ---------------------------------------------------------------- Philox
 // Philox4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64-bit
-// multiplies with the round keys bumped by the Weyl constants.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+// multiplies; round r XORs in the key (k0 + r·0x9E3779B9, k1 + r·0xBB67AE85),
+// precomputed on the host from the seed so each round is two wide multiplies
+// and two three-input XORs.
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& k) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
     const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
     const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    c = make_uint4(hi1 ^ c.y ^ k.k0[r], lo1, hi0 ^ c.w ^ k.k1[r], lo0);
   }
   return c;
 }
@@ -79,6 +81,14 @@ __device__ __forceinline__ float div_shared_divisor(float a, float d, float y) {
   return (q0 >= 1.0e-30f || a == 0.0f) ? q1 : __fdiv_rn(a, d);
 }
 
+// The same for a signed a (d > 0), keeping the sign of a zero a.
+__device__ __forceinline__ float div_shared_divisor_signed(float a, float d, float y) {
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-d, q0, a);
+  const float q1 = __fmaf_rn(r, y, q0);
+  return fabsf(q0) >= 1.0e-30f ? q1 : (a == 0.0f ? a : __fdiv_rn(a, d));
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return f16_lo_to_f32(e4m3x2_to_f16x2(code));
 }
@@ -88,20 +98,20 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 // the n4 float4 of src to *partial.
 __device__ __forceinline__ void amax_partial_body(const float4* __restrict__ src, int64_t n4,
                                                   float* __restrict__ partial, int cta, int nctas) {
+  // chunks of kAmaxThreads x 8 float4, eight independent loads per thread
+  constexpr int kPer = 8;
   float m = 0.0f;
-  const int64_t stride = static_cast<int64_t>(nctas) * kAmaxThreads;
-  int64_t i = static_cast<int64_t>(cta) * kAmaxThreads + threadIdx.x;
-  for (; i + 3 * stride < n4; i += 4 * stride) {
-    const float4 a = __ldg(src + i), b = __ldg(src + i + stride);
-    const float4 c = __ldg(src + i + 2 * stride), d = __ldg(src + i + 3 * stride);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(c.x), fabsf(c.y)), fmaxf(fabsf(c.z), fabsf(c.w))));
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(d.x), fabsf(d.y)), fmaxf(fabsf(d.z), fabsf(d.w))));
-  }
-  for (; i < n4; i += stride) {
-    const float4 a = __ldg(src + i);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+  const int64_t chunk = static_cast<int64_t>(kAmaxThreads) * kPer;
+  for (int64_t base = static_cast<int64_t>(cta) * chunk; base < n4; base += static_cast<int64_t>(nctas) * chunk) {
+    float4 v[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int64_t i = base + k * kAmaxThreads + threadIdx.x;
+      v[k] = i < n4 ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -162,134 +172,153 @@ amax_finish_kernel(const float* __restrict__ partial, int count, float* __restri
 // sr_col0 = 0 for an unsharded tensor).
 template <int FMT, int RND>
 __device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d, float y, const float (&u)[4]) {
-  float v[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = d > 0.0f ? div_shared_divisor(fabsf(xv[j]), d, y) : 0.0f;
-  uint32_t mag[4];
   if (RND == 0) {
-    if (FMT == 0) {
-      const uint32_t b01 = f32x2_to_e2m1x2(v[0], v[1]), b23 = f32x2_to_e2m1x2(v[2], v[3]);
-      mag[0] = b01 & 0xF; mag[1] = b01 >> 4; mag[2] = b23 & 0xF; mag[3] = b23 >> 4;
-    } else {
-      const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
-      mag[0] = b01 & 0x3F; mag[1] = (b01 >> 8) & 0x3F; mag[2] = b23 & 0x3F; mag[3] = (b23 >> 8) & 0x3F;
-    }
-  } else {
+    // RNE: the conversion of the signed quotient gives sign bit and
+    // magnitude together (the sign of x, also for a zero quotient)
+    float v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) mag[j] = round_sr_mag<FMT>(v[j], u[j]);
+    for (int j = 0; j < 4; ++j) v[j] = d > 0.0f ? div_shared_divisor_signed(xv[j], d, y) : xv[j];
+    if (FMT == 0) return f32x2_to_e2m1x2(v[0], v[1]) | (f32x2_to_e2m1x2(v[2], v[3]) << 8);
+    const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
+    return (b01 & 0x3F) | ((b01 >> 2) & 0xFC0) | ((b23 & 0x3F) << 12) | ((b23 & 0x3F00) << 10);
   }
   uint32_t packed = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
+    const float v = d > 0.0f ? div_shared_divisor(fabsf(xv[j]), d, y) : 0.0f;
+    const uint32_t mag = round_sr_mag<FMT>(v, u[j]);
     const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
-    const uint32_t code = FMT == 0 ? (mag[j] | (sgn << 3)) : (mag[j] | (sgn << 5));
+    const uint32_t code = FMT == 0 ? (mag | (sgn << 3)) : (mag | (sgn << 5));
     packed |= code << (j * (FMT == 0 ? 4 : 6));
   }
   return packed;
 }
 
+// Scale constants of a tensor from its amax (every scale step one IEEE fp32
+// operation in the formula's order).
+template <int FMT>
+struct TensorScale {
+  float T, Temax;
+  __device__ __forceinline__ explicit TensorScale(float amax) {
+    const float emax = FMT == 0 ? 6.0f : 7.5f;
+    T = __fdiv_rn(amax, 448.0f * emax);         // 2688 or 3360, exact
+    Temax = __fmul_rn(T, emax);
+  }
+};
+
+// Quantize QB horizontally adjacent 4 x 4 blocks (block row br, first column
+// block bc0) whose 4 rows are x[q][r], and store their scales and codes.
 template <int FMT, int RND, int QB>
-__device__ __forceinline__ void quantize_body(const float* __restrict__ src, int64_t rows, int64_t cols,
-                                              const float* __restrict__ amax_src, int amax_count,
-                                              uint64_t seed, int64_t sr_cols, int64_t sr_col0,
-                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                              float* __restrict__ tscale, int cta, int nctas) {
-  __shared__ float red[32];
-  const float amax = block_max_of(amax_src, amax_count, red);
-  const float emax = FMT == 0 ? 6.0f : 7.5f;
-  const float T = __fdiv_rn(amax, 448.0f * emax);         // 2688 or 3360, exact
-  const float Temax = __fmul_rn(T, emax);
-  if (cta == 0 && threadIdx.x == 0) *tscale = T;
-
-  const int64_t cb = cols >> 2;                       // column blocks per block row
-  const int64_t cu = cb / QB;                         // work units per block row
-  const int64_t nunits = (rows >> 2) * cu;
-  const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
-  const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
-  const int64_t stride = static_cast<int64_t>(nctas) * kQuantThreads;
-
-  for (int64_t w = static_cast<int64_t>(cta) * kQuantThreads + threadIdx.x; w < nunits;
-       w += stride) {
-    const int64_t br = w / cu;
-    const int64_t bc0 = (w - br * cu) * QB;
-    const float* p = src + (br * 4) * cols + bc0 * 4;
-    float4 x[QB][4];
+__device__ __forceinline__ void quantize_unit(const float4 (&x)[QB][4], const TensorScale<FMT>& ts, int64_t br,
+                                              int64_t bc0, int64_t cb, int64_t row_bytes, const PhiloxKeys& keys,
+                                              int64_t sr_cols, int64_t sr_col0,
+                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const float T = ts.T;
+  uint32_t scode[QB];
+  float d[QB], y[QB];
 #pragma unroll
-    for (int q = 0; q < QB; ++q)
+  for (int q = 0; q < QB; ++q) {
+    float bmax = 0.0f;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
-    uint32_t scode[QB];
-    float d[QB], y[QB];
+    for (int r = 0; r < 4; ++r)
+      bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[q][r].x), fabsf(x[q][r].y)),
+                               fmaxf(fabsf(x[q][r].z), fabsf(x[q][r].w))));
+    scode[q] = 0;
+    d[q] = 0.0f;
+    y[q] = 0.0f;
+    if (T > 0.0f) {
+      scode[q] = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
+      d[q] = __fmul_rn(e4m3_to_f32(scode[q]), T);
+      y[q] = d[q] > 0.0f ? __frcp_rn(d[q]) : 0.0f;
+    }
+  }
+  const int64_t b = br * cb + bc0;
+  if (QB == 2) *reinterpret_cast<uint16_t*>(scales + b) = static_cast<uint16_t>(scode[0] | (scode[1] << 8));
+  else scales[b] = static_cast<uint8_t>(scode[0]);
+
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    uint32_t packed[QB];
 #pragma unroll
     for (int q = 0; q < QB; ++q) {
-      float bmax = 0.0f;
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[q][r].x), fabsf(x[q][r].y)),
-                                 fmaxf(fabsf(x[q][r].z), fabsf(x[q][r].w))));
-      scode[q] = 0;
-      d[q] = 0.0f;
-      y[q] = 0.0f;
-      if (T > 0.0f) {
-        scode[q] = f32_to_e4m3_satfinite(__fdiv_rn(bmax, Temax));
-        d[q] = __fmul_rn(e4m3_to_f32(scode[q]), T);
-        y[q] = d[q] > 0.0f ? __frcp_rn(d[q]) : 0.0f;
+      const float xv[4] = {x[q][r].x, x[q][r].y, x[q][r].z, x[q][r].w};
+      float u[4] = {0.f, 0.f, 0.f, 0.f};
+      if (RND == 1) {
+        // element index in the (possibly wider) view the SR stream is defined on
+        const uint64_t g = static_cast<uint64_t>((br * 4 + r) * sr_cols + sr_col0 + (bc0 + q) * 4) >> 2;
+        const uint4 wd = philox4x32_10(make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), keys);
+        const float s24 = 5.9604644775390625e-08f;   // 2^-24
+        u[0] = __uint2float_rn(wd.x >> 8) * s24;
+        u[1] = __uint2float_rn(wd.y >> 8) * s24;
+        u[2] = __uint2float_rn(wd.z >> 8) * s24;
+        u[3] = __uint2float_rn(wd.w >> 8) * s24;
       }
+      packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], u);
     }
-    const int64_t b = br * cb + bc0;
-    if (QB == 2) *reinterpret_cast<uint16_t*>(scales + b) = static_cast<uint16_t>(scode[0] | (scode[1] << 8));
-    else scales[b] = static_cast<uint8_t>(scode[0]);
-
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      uint32_t packed[QB];
-#pragma unroll
-      for (int q = 0; q < QB; ++q) {
-        const float xv[4] = {x[q][r].x, x[q][r].y, x[q][r].z, x[q][r].w};
-        float u[4] = {0.f, 0.f, 0.f, 0.f};
-        if (RND == 1) {
-          // element index in the (possibly wider) view the SR stream is defined on
-          const uint64_t g = static_cast<uint64_t>((br * 4 + r) * sr_cols + sr_col0 + (bc0 + q) * 4) >> 2;
-          const uint4 wd = philox4x32_10(
-              make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), k0, k1);
-          const float s24 = 5.9604644775390625e-08f;   // 2^-24
-          u[0] = __uint2float_rn(wd.x >> 8) * s24;
-          u[1] = __uint2float_rn(wd.y >> 8) * s24;
-          u[2] = __uint2float_rn(wd.z >> 8) * s24;
-          u[3] = __uint2float_rn(wd.w >> 8) * s24;
-        }
-        packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], u);
-      }
-      uint8_t* out = codes + (br * 4 + r) * row_bytes;
-      if (FMT == 0) {
-        if (QB == 2) *reinterpret_cast<uint32_t*>(out + bc0 * 2) = packed[0] | (packed[1] << 16);
-        else *reinterpret_cast<uint16_t*>(out + bc0 * 2) = static_cast<uint16_t>(packed[0]);
+    uint8_t* out = codes + (br * 4 + r) * row_bytes;
+    if (FMT == 0) {
+      if (QB == 2) *reinterpret_cast<uint32_t*>(out + bc0 * 2) = packed[0] | (packed[1] << 16);
+      else *reinterpret_cast<uint16_t*>(out + bc0 * 2) = static_cast<uint16_t>(packed[0]);
+    } else {
+      if (QB == 2) {   // 48 bits at a 6-byte (2-aligned) offset
+        uint16_t* o16 = reinterpret_cast<uint16_t*>(out + bc0 * 3);
+        o16[0] = static_cast<uint16_t>(packed[0]);
+        o16[1] = static_cast<uint16_t>((packed[0] >> 16) | (packed[1] << 8));
+        o16[2] = static_cast<uint16_t>(packed[1] >> 8);
       } else {
-        if (QB == 2) {   // 48 bits at a 6-byte (2-aligned) offset
-          uint16_t* o16 = reinterpret_cast<uint16_t*>(out + bc0 * 3);
-          o16[0] = static_cast<uint16_t>(packed[0]);
-          o16[1] = static_cast<uint16_t>((packed[0] >> 16) | (packed[1] << 8));
-          o16[2] = static_cast<uint16_t>(packed[1] >> 8);
-        } else {
-          out += bc0 * 3;
-          out[0] = static_cast<uint8_t>(packed[0]);
-          out[1] = static_cast<uint8_t>(packed[0] >> 8);
-          out[2] = static_cast<uint8_t>(packed[0] >> 16);
-        }
+        out += bc0 * 3;
+        out[0] = static_cast<uint8_t>(packed[0]);
+        out[1] = static_cast<uint8_t>(packed[0] >> 8);
+        out[2] = static_cast<uint8_t>(packed[0] >> 16);
       }
     }
   }
 }
 
+// Per-tensor parameters of the quantize pass.
+struct QuantArgs {
+  const float* src;
+  int64_t rows, cols;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* tscale;
+  PhiloxKeys keys;
+  int64_t sr_cols, sr_col0;
+  FastDiv dcu;          // division by the work units per block row (unit count < 2^31)
+};
+
+template <int FMT, int RND, int QB>
+__device__ __forceinline__ void quantize_body(const QuantArgs& qa, const float* __restrict__ amax_src, int amax_count,
+                                              int cta, int nctas) {
+  __shared__ float red[32];
+  const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
+  if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
+
+  const int64_t cols = qa.cols;
+  const int64_t cb = cols >> 2;                       // column blocks per block row
+  const int cu = static_cast<int>(cb / QB);           // work units per block row
+  const int nunits = static_cast<int>((qa.rows >> 2) * cu);
+  const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
+  const int stride = nctas * kQuantThreads;
+
+  for (int w = cta * kQuantThreads + static_cast<int>(threadIdx.x); w < nunits; w += stride) {
+    const int br = fdiv(w, qa.dcu);
+    const int64_t bc0 = static_cast<int64_t>(w - br * cu) * QB;
+    const float* p = qa.src + (static_cast<int64_t>(br) * 4) * cols + bc0 * 4;
+    float4 x[QB][4];
+#pragma unroll
+    for (int q = 0; q < QB; ++q)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
+    quantize_unit<FMT, RND, QB>(x, ts, br, bc0, cb, row_bytes, qa.keys, qa.sr_cols, qa.sr_col0, qa.codes,
+                                qa.scales);
+  }
+}
+
 template <int FMT, int RND, int QB>
 __global__ void __launch_bounds__(kQuantThreads)
-quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
-                const float* __restrict__ amax_src, int amax_count, uint64_t seed,
-                int64_t sr_cols, int64_t sr_col0,
-                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                float* __restrict__ tscale) {
-  quantize_body<FMT, RND, QB>(src, rows, cols, amax_src, amax_count, seed, sr_cols, sr_col0, codes,
-                              scales, tscale, blockIdx.x, gridDim.x);
+quantize_kernel(const __grid_constant__ QuantArgs qa, const float* __restrict__ amax_src, int amax_count) {
+  quantize_body<FMT, RND, QB>(qa, amax_src, amax_count, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------ several tensors at once
@@ -301,12 +330,7 @@ quantize_kernel(const float* __restrict__ src, int64_t rows, int64_t cols,
 constexpr int kMaxQuantJobs = 8;
 
 struct QuantJob {
-  const float* src;
-  int64_t rows, cols;
-  uint8_t* codes;
-  uint8_t* scales;
-  float* tscale;
-  uint64_t seed;
+  QuantArgs qa;
   int32_t fmt, rounding, qb;
   int32_t amax_cta0, amax_ctas;     // this job's range of amax CTAs (= its partials)
   int32_t quant_cta0, quant_ctas;   // this job's range of quantize CTAs
@@ -327,7 +351,7 @@ __device__ __forceinline__ int job_of(const QuantJobs& jobs, int cta, bool quant
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_many_kernel(const __grid_constant__ QuantJobs jobs, float* __restrict__ partial) {
   const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, false)];
-  amax_partial_body(reinterpret_cast<const float4*>(jb.src), jb.rows * jb.cols / 4, partial + blockIdx.x,
+  amax_partial_body(reinterpret_cast<const float4*>(jb.qa.src), jb.qa.rows * jb.qa.cols / 4, partial + blockIdx.x,
                     blockIdx.x - jb.amax_cta0, jb.amax_ctas);
 }
 
@@ -338,11 +362,9 @@ quantize_many_kernel(const __grid_constant__ QuantJobs jobs, const float* __rest
   const float* amax = partial + jb.amax_cta0;
 #define MQV_QUANT_CASE(F, R, Q)                                                                   \
   if (jb.fmt == F && jb.rounding == R && jb.qb == Q) {                                            \
-    quantize_body<F, R, Q>(jb.src, jb.rows, jb.cols, amax, jb.amax_ctas, jb.seed, jb.cols, 0,     \
-                           jb.codes, jb.scales, jb.tscale, cta, jb.quant_ctas);                   \
+    quantize_body<F, R, Q>(jb.qa, amax, jb.amax_ctas, cta, jb.quant_ctas);                         \
     return;                                                                                       \
   }
-  MQV_QUANT_CASE(0, 0, 2) MQV_QUANT_CASE(0, 1, 2) MQV_QUANT_CASE(1, 0, 2) MQV_QUANT_CASE(1, 1, 2)
   MQV_QUANT_CASE(0, 0, 1) MQV_QUANT_CASE(0, 1, 1) MQV_QUANT_CASE(1, 0, 1) MQV_QUANT_CASE(1, 1, 1)
 #undef MQV_QUANT_CASE
 }
