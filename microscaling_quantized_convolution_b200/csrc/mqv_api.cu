@@ -300,7 +300,7 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   // Stride-1 fwd/dgrad on NVFP4 with N | 256, N % 8 == 0, a halo of at most
   // 384 rows and whole 64-channel chunks: the kernel-row halo path.
   pl->halo = op != MQV_OP_WGRAD && d->fmt == MQV_NVFP4 && d->stride == 1 && d->N % 8 == 0 &&
-             256 % d->N == 0 && (d->Kw - 1) * d->N <= 128 && a.Cred % 64 == 0;
+             256 % d->N == 0 && (d->Kw - 1) * d->N <= 128 && a.Cred % 64 == 0 && d->Kw <= kHaloAStages;
   if (pl->halo) {
     HaloGeom& g = pl->g;
     g.bw = (int)(256 / d->N);

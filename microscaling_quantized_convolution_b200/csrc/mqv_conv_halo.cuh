@@ -19,8 +19,9 @@
 //                 tap kw uses halo pixels q = j + (Kw - 1 - kw).
 // The weight operand is the fp16 image of prep_image_kernel (tap-major K, so
 // the tile of (tap, chunk) is image tile tap·(Cred/64) + chunk), one 16 KB
-// bulk copy per tap.  Roles, bounded waits and the double-buffered
-// accumulators are those of conv_fd_kernel.
+// bulk copy per tap, the Kw tiles of a stage under one barrier.  Roles,
+// bounded waits and the double-buffered accumulators are those of
+// conv_fd_kernel.
 #pragma once
 
 #include <cstdint>
@@ -42,9 +43,10 @@ constexpr int kHaloLookahead = 2;                        // stages of codes in f
 constexpr uint32_t kHaloBTile = kHaloMaxRows * 128;   // 48 KB
 
 struct HaloSmem {
-  static constexpr int kAOffset = 0;
+  static constexpr int kAOffset = 0;                                  // kHaloAStages weight tiles
   static constexpr int kBOffset = kHaloAStages * kATileBytes;
-  static constexpr int kBarOffset = kBOffset + kHaloBStages * kHaloBTile;
+  static constexpr int kEpiOffset = kBOffset + kHaloBStages * kHaloBTile;   // 32 x 32 fp32 per epilogue warp
+  static constexpr int kBarOffset = kEpiOffset + kV2EpiWarps * 4096;
   static constexpr int kBytes = kBarOffset + 512 + 1024;
 };
 
@@ -175,12 +177,14 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
   tc_fence_after();
   const uint32_t sbase = smem_u32(smem);
   const int stages_per_tile = p.Kh * g.cchunks;
+  const int na = kHaloAStages / p.Kw;     // weight stages in the ring (Kw <= kHaloAStages)
 
   if (warp < kV2EpiWarps) {
     // epilogue: column lc of the tile = (pixel j, batch item n) -> output
     // pixel (oh, ow0 + j), skipped past the end of the output row.
     int it = 0;
-    const int64_t m = static_cast<int64_t>(0) + warp * 32 + lane;
+    const uint32_t wbuf = sbase + L::kEpiOffset + warp * 4096;
+    const int rsub = lane >> 3, q = lane & 7;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
@@ -189,31 +193,42 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       const int rest = tile - mt * g.out_h * g.tpr;
       const int oh = rest / g.tpr;
       const int ow0 = (rest - oh * g.tpr) * g.bw;
-      const int64_t mrow = static_cast<int64_t>(mt) * 128 + m;
       const float scale = __fmul_rn(*p.ta, *p.tb);
       const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * kHaloBN;
+      // Each lane reads one accumulator row from TMEM; a swizzled 32 x 32
+      // transpose in shared memory turns that into stores of 128-byte runs of
+      // one (pixel, channel) row's batch items.
 #pragma unroll 1
       for (int c = 0; c < kHaloBN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + c, r);
-        tmem_ld_wait();
-        if (mrow < p.M) {
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const int lc = c + 4 * j4;
-            const int j = fdiv(lc, p.dN);
-            const int n = lc - j * p.N;
-            const int ow = ow0 + j;
-            if (j >= g.bw || ow >= g.out_w) continue;
-            float4 o;
-            o.x = __uint_as_float(r[4 * j4 + 0]) * scale;
-            o.y = __uint_as_float(r[4 * j4 + 1]) * scale;
-            o.z = __uint_as_float(r[4 * j4 + 2]) * scale;
-            o.w = __uint_as_float(r[4 * j4 + 3]) * scale;
-            const int64_t idx = ((static_cast<int64_t>(oh) * g.out_w + ow) * p.M + mrow) * p.N + n;
-            *reinterpret_cast<float4*>(p.out + idx) = o;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tbase + c + 16 * hf, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
+                         __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
+                         __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
+                         __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
+                         __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
+        }
+        __syncwarp();
+        const int lc = c + 4 * q;
+        const int j = fdiv(lc, p.dN);
+        const int n = lc - j * p.N;
+        const int ow = ow0 + j;
+        if (j < g.bw && ow < g.out_w) {
+          const int64_t pix = static_cast<int64_t>(oh) * g.out_w + ow;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int row = 4 * i + rsub;
+            const int64_t mrow = static_cast<int64_t>(mt) * 128 + warp * 32 + row;
+            const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+            if (mrow < p.M) *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
@@ -221,7 +236,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, kHaloBN);
-      int it = 0, bit = 0, ait = 0;
+      int it = 0, bit = 0;
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
@@ -230,23 +245,23 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         bool first = true;
         for (int st = 0; st < stages_per_tile; ++st, ++bit) {
           const int sb = bit % kHaloBStages;
+          const int sa = bit % na;
           mbar_wait_bounded(&bars->bfull[sb], (bit / kHaloBStages) & 1, p.err, kErrWaitFull);
+          mbar_wait_bounded(&bars->afull[sa], (bit / na) & 1, p.err, kErrWaitFull);
           tc_fence_after();
           const uint32_t b_tile = sbase + L::kBOffset + sb * kHaloBTile;
-          for (int kw = 0; kw < p.Kw; ++kw, ++ait) {
-            const int sa = ait % kHaloAStages;
-            mbar_wait_bounded(&bars->afull[sa], (ait / kHaloAStages) & 1, p.err, kErrWaitFull);
-            tc_fence_after();
+          const uint32_t a_stage = sbase + L::kAOffset + sa * p.Kw * kATileBytes;
+          for (int kw = 0; kw < p.Kw; ++kw) {
             const int shift = PASS == kFwd ? kw : p.Kw - 1 - kw;
-            const uint64_t adesc = smem_desc_sw128(sbase + L::kAOffset + sa * kATileBytes);
+            const uint64_t adesc = smem_desc_sw128(a_stage + kw * kATileBytes);
             const uint64_t bdesc = smem_desc_sw128(b_tile + static_cast<uint32_t>(shift * p.N) * 128u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               mma_f16_ss(dt, adesc + 2 * kk, bdesc + 2 * kk, idesc, first ? 0u : 1u);
               first = false;
             }
-            mma_commit(&bars->aempty[sa]);
           }
+          mma_commit(&bars->aempty[sa]);
           mma_commit(&bars->bempty[sb]);
         }
         mma_commit(&bars->acc_full[acc]);
@@ -259,15 +274,17 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         const int mt = tile / (g.out_h * g.tpr);
         const uint8_t* img = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
         for (int kh = 0; kh < p.Kh; ++kh)
-          for (int c = 0; c < g.cchunks; ++c)
-            for (int kw = 0; kw < p.Kw; ++kw, ++ait) {
-              const int sa = ait % kHaloAStages;
-              mbar_wait_bounded(&bars->aempty[sa], ((ait / kHaloAStages) & 1) ^ 1, p.err, kErrWaitEmpty);
-              mbar_arrive_expect_tx(&bars->afull[sa], kATileBytes);
+          for (int c = 0; c < g.cchunks; ++c, ++ait) {
+            // the Kw weight tiles of the stage, under one barrier
+            const int sa = ait % na;
+            mbar_wait_bounded(&bars->aempty[sa], ((ait / na) & 1) ^ 1, p.err, kErrWaitEmpty);
+            mbar_arrive_expect_tx(&bars->afull[sa], p.Kw * kATileBytes);
+            for (int kw = 0; kw < p.Kw; ++kw) {
               const int kt = (kh * p.Kw + kw) * g.cchunks + c;
-              bulk_copy_g2s(sbase + L::kAOffset + sa * kATileBytes, img + static_cast<int64_t>(kt) * kATileBytes,
-                            kATileBytes, &bars->afull[sa]);
+              bulk_copy_g2s(sbase + L::kAOffset + (sa * p.Kw + kw) * kATileBytes,
+                            img + static_cast<int64_t>(kt) * kATileBytes, kATileBytes, &bars->afull[sa]);
             }
+          }
       }
     }
   } else {
