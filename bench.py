@@ -196,8 +196,8 @@ def run_gpu(args):
     def dgrad(s):
         mqv.conv_dgrad(d, s["qw"], s["qg"], gx=s["gx"], ws=ws_dgrad)
 
-    def step(i):
-        s = sets[i % nsets]
+    def step(i, s=None):
+        s = sets[i % nsets] if s is None else s
         quantize_all(s, i)
         fwd(s)
         wgrad(s)
@@ -285,28 +285,53 @@ def run_gpu(args):
         mean = {k: t[1 + j].item() for j, k in enumerate(parts)}
     flags = mqv.device_errors()
 
-    # end-to-end through the public API with pinned host buffers
+    # End to end through the public API with pinned host buffers, pipelined
+    # as a training loop would be: step i copies its inputs in on one stream,
+    # computes on the current stream and copies its outputs back on a third,
+    # alternating between two device slots, so the copies of neighbouring
+    # steps overlap each other and the compute.
     e2e = None
     if args.e2e_steps > 0:
         hX = sets[0]["X"].cpu().pin_memory(); hW = sets[0]["W"].cpu().pin_memory()
         hG = sets[0]["G"].cpu().pin_memory()
-        hy = torch.empty(sets[0]["y"].numel()).pin_memory()
-        hgw = torch.empty(sets[0]["gw"].numel()).pin_memory()
-        hgx = torch.empty(sets[0]["gx"].numel()).pin_memory()
-        s = sets[0]
+        hout = [{k: torch.empty(sets[0][k].numel()).pin_memory() for k in ("y", "gw", "gx")} for _ in range(2)]
+        cur = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = [{n: torch.cuda.Event() for n in ("in", "comp", "out")} for _ in range(2)]
+
         def e2e_step(i):
-            s["X"].copy_(hX, non_blocking=True); s["W"].copy_(hW, non_blocking=True)
-            s["G"].copy_(hG, non_blocking=True)
-            step(i)
-            hy.copy_(s["y"], non_blocking=True); hgw.copy_(s["gw"], non_blocking=True)
-            hgx.copy_(s["gx"], non_blocking=True)
-        for i in range(3):
+            k = i % 2
+            sk = sets[k]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev[k]["comp"])      # slot k's inputs are consumed
+                sk["X"].copy_(hX, non_blocking=True); sk["W"].copy_(hW, non_blocking=True)
+                sk["G"].copy_(hG, non_blocking=True)
+                ev[k]["in"].record(s_in)
+            cur.wait_event(ev[k]["in"])
+            if i >= 2:
+                cur.wait_event(ev[k]["out"])            # slot k's outputs are back on the host
+            step(i, sk)
+            ev[k]["comp"].record(cur)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev[k]["comp"])
+                for n in ("y", "gw", "gx"):
+                    hout[k][n].copy_(sk[n], non_blocking=True)
+                ev[k]["out"].record(s_out)
+
+        def drain(last):
+            for i in range(max(0, last - 1), last + 1):
+                cur.wait_event(ev[i % 2]["out"])
+
+        for i in range(4):
             e2e_step(i)
+        drain(3)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for i in range(args.e2e_steps):
             e2e_step(i)
+        drain(args.e2e_steps - 1)
         b.record()
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / args.e2e_steps
@@ -315,8 +340,10 @@ def run_gpu(args):
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = t.item()
         h2d = 4 * (nx + nw + ng)
+        d2h = 4 * sum(sets[0][n].numel() for n in ("y", "gw", "gx"))
         e2e = {"value": round(3 * layer.flops() * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d, "ms_per_step": round(e2e_ms, 4)}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+               "pipeline": "inputs in, compute, outputs out on three streams, two device slots"}
 
     del graphs
     torch.cuda.synchronize()
