@@ -429,15 +429,16 @@ cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
 
 cudaError_t launch_prep(int op, int fmt, const ConvPlan& pl, const QView& w, uint8_t* image, cudaStream_t st) {
   const V2Args& a = pl.a;
-  const int64_t chunks = (int64_t)a.mtiles * 128 * a.ktiles * 8;
-  int64_t g = (chunks + 255) / 256;
-  if (g > kSMs * 8) g = kSMs * 8;
+  const int chunks = a.mtiles * 128 * a.ktiles * 8;
+  const unsigned g = (unsigned)((chunks + kPrepThreads - 1) / kPrepThreads);
+  const FastDiv dkt8 = make_fastdiv((int64_t)a.ktiles * 8), dcout = make_fastdiv(a.Cout);
+  const int kd = (int)a.Kdim;
   if (op == MQV_OP_FWD) {
-    if (fmt == MQV_NVFP4) prep_image_kernel<0, false><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
-    else prep_image_kernel<1, false><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+    if (fmt == MQV_NVFP4) prep_image_kernel<0, false><<<g, kPrepThreads, 0, st>>>(w, a.M, kd, a.ktiles, a.mtiles, a.Cin, a.Cout, dkt8, dcout, image);
+    else prep_image_kernel<1, false><<<g, kPrepThreads, 0, st>>>(w, a.M, kd, a.ktiles, a.mtiles, a.Cin, a.Cout, dkt8, dcout, image);
   } else {
-    if (fmt == MQV_NVFP4) prep_image_kernel<0, true><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
-    else prep_image_kernel<1, true><<<(unsigned)g, 256, 0, st>>>(w, a.M, a.Kdim, a.ktiles, a.mtiles, a.Cin, a.Cout, image);
+    if (fmt == MQV_NVFP4) prep_image_kernel<0, true><<<g, kPrepThreads, 0, st>>>(w, a.M, kd, a.ktiles, a.mtiles, a.Cin, a.Cout, dkt8, dcout, image);
+    else prep_image_kernel<1, true><<<g, kPrepThreads, 0, st>>>(w, a.M, kd, a.ktiles, a.mtiles, a.Cin, a.Cout, dkt8, dcout, image);
   }
   return cudaGetLastError();
 }

@@ -161,42 +161,52 @@ __device__ __forceinline__ void dequant_run(uint32_t lo, uint32_t hi, uint32_t s
 // the shared-memory tile the MMA reads.  fwd: A[co][k] = W[co][k];
 // dgrad: A[ci][(tap, co)] = W[co][tap·Cin + ci].  Rows/columns past the
 // matrix are zero.  One thread per 16-byte chunk.
+constexpr int kPrepThreads = 128;
+
 template <int FMT, bool TRANS>
-__global__ void __launch_bounds__(256)
-prep_image_kernel(QView w, int M, int64_t Kdim, int ktiles, int mtiles, int Cin, int Cout,
-                  uint8_t* __restrict__ image) {
-  const int64_t chunks = static_cast<int64_t>(mtiles) * 128 * ktiles * 8;
-  for (int64_t id = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; id < chunks;
-       id += static_cast<int64_t>(gridDim.x) * 256) {
-    const int64_t m = id / (static_cast<int64_t>(ktiles) * 8);
-    const int64_t k0 = (id - m * ktiles * 8) * 8;
-    uint32_t h[4] = {0u, 0u, 0u, 0u};
-    if (m < M) {
+__global__ void __launch_bounds__(kPrepThreads)
+prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int Cout, FastDiv dkt8,
+                  FastDiv dcout, uint8_t* __restrict__ image) {
+  const int chunks = mtiles * 128 * ktiles * 8;
+  const int id = blockIdx.x * kPrepThreads + threadIdx.x;
+  if (id >= chunks) return;
+  const int m = fdiv(id, dkt8);
+  const int k0 = (id - m * ktiles * 8) * 8;
+  uint32_t h[4] = {0u, 0u, 0u, 0u};
+  if (m < M) {
+    if (!TRANS && k0 + 8 <= Kdim && (FMT == 0 ? (w.row_bytes & 3) == 0 : (w.row_bytes & 1) == 0)) {
+      // eight consecutive codes of one weight row: one word (FP4) or three
+      // half-words (FP6) and the two block scales
+      uint32_t hi = 0;
+      const uint32_t lo = load_codes<FMT, 8>(w, m, k0, hi);
+      const uint32_t ss = __ldg(reinterpret_cast<const unsigned short*>(w.scales + (m >> 2) * w.scale_cols + (k0 >> 2)));
+      dequant_run<FMT, 8>(lo, hi, scale2(ss & 0xFF), scale2(ss >> 8), h);
+    } else {
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        const int64_t k = k0 + e;
+        const int k = k0 + e;
         if (k >= Kdim) break;
-        int64_t row, col;
+        int row, col;
         if (!TRANS) {
           row = m;
           col = k;
         } else {
-          const int64_t tap = k / Cout, co = k - tap * Cout;
+          const int tap = fdiv(k, dcout), co = k - tap * Cout;
           row = co;
           col = tap * Cin + m;
         }
         const uint32_t s = __ldg(w.scales + (row >> 2) * w.scale_cols + (col >> 2));
         uint32_t c0, c1;
-        const uint8_t* p = w.codes + row * w.row_bytes;
-        const int64_t row2 = TRANS ? row + 1 : row;       // second element: next co (dgrad)
-        const int64_t col2 = TRANS ? col : col + 1;
-        const uint8_t* p2 = w.codes + row2 * w.row_bytes;
+        const uint8_t* p = w.codes + static_cast<int64_t>(row) * w.row_bytes;
+        const int row2 = TRANS ? row + 1 : row;       // second element: next co (dgrad)
+        const int col2 = TRANS ? col : col + 1;
+        const uint8_t* p2 = w.codes + static_cast<int64_t>(row2) * w.row_bytes;
         if (FMT == 0) {
           c0 = (__ldg(p + (col >> 1)) >> ((col & 1) * 4)) & 0xF;
           c1 = (__ldg(p2 + (col2 >> 1)) >> ((col2 & 1) * 4)) & 0xF;
           h[e >> 1] = hmul2_u32(e2m1x2_to_f16x2(c0 | (c1 << 4)), scale2(s));
         } else {
-          auto code6 = [](const uint8_t* base, int64_t c) -> uint32_t {
+          auto code6 = [](const uint8_t* base, int c) -> uint32_t {
             const uint8_t* q = base + (c >> 2) * 3;
             const uint32_t v = static_cast<uint32_t>(__ldg(q)) | (static_cast<uint32_t>(__ldg(q + 1)) << 8) |
                                (static_cast<uint32_t>(__ldg(q + 2)) << 16);
@@ -208,10 +218,10 @@ prep_image_kernel(QView w, int M, int64_t Kdim, int ktiles, int mtiles, int Cin,
         }
       }
     }
-    const int64_t mt = m >> 7, r = m & 127, kt = k0 >> 6, kc = (k0 & 63) >> 3;
-    uint8_t* dst = image + (mt * ktiles + kt) * kATileBytes + r * 128 + ((kc ^ (r & 7)) << 4);
-    *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
   }
+  const int mt = m >> 7, r = m & 127, kt = k0 >> 6, kc = (k0 & 63) >> 3;
+  uint8_t* dst = image + (static_cast<int64_t>(mt) * ktiles + kt) * kATileBytes + r * 128 + ((kc ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
 }
 
 // ---------------------------------------------------------------------------
