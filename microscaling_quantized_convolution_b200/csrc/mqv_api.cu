@@ -303,14 +303,35 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
              256 % d->N == 0 && (d->Kw - 1) * d->N <= 128 && a.Cred % 64 == 0 && d->Kw <= kHaloAStages;
   if (pl->halo) {
     HaloGeom& g = pl->g;
-    g.bw = (int)(256 / d->N);
-    g.rows = (int)((g.bw + d->Kw - 1) * d->N);
     g.out_h = op == MQV_OP_FWD ? a.Ho : a.H;
     g.out_w = op == MQV_OP_FWD ? a.Wo : a.W;
     g.src_h = op == MQV_OP_FWD ? a.H : a.Ho;
     g.src_w = op == MQV_OP_FWD ? a.W : a.Wo;
-    g.tpr = (g.out_w + g.bw - 1) / g.bw;
     g.cchunks = a.Cred / 64;
+    // Tile width: the persistent CTAs run ceil(tiles / SMs) tiles, each
+    // stage costing the longer of its MMAs (about BN/2 cycles per 16-deep
+    // slice and tap, at least the N = 128 cost) and its producers (about 6
+    // cycles per halo row); pick the width with the least total, ties to
+    // the wider tile.
+    int best_bw = 0;
+    int64_t best_cost = 0;
+    for (int bw = (int)(256 / d->N); bw >= 1; --bw) {
+      const int bn = bw * (int)d->N;
+      if (bn % 16) continue;
+      const int64_t tiles = (int64_t)a.mtiles * g.out_h * ((g.out_w + bw - 1) / bw);
+      const int64_t waves = (tiles + kSMs - 1) / kSMs;
+      const int64_t mma = (int64_t)d->Kw * 4 * ((bn > 128 ? bn : 128) / 2);
+      const int64_t prod = 6 * (int64_t)(bw + d->Kw - 1) * d->N;
+      const int64_t cost = waves * (mma > prod ? mma : prod);
+      if (best_bw == 0 || cost < best_cost) {
+        best_bw = bw;
+        best_cost = cost;
+      }
+    }
+    g.bw = best_bw;
+    g.bn = g.bw * (int)d->N;
+    g.rows = (int)((g.bw + d->Kw - 1) * d->N);
+    g.tpr = (g.out_w + g.bw - 1) / g.bw;
     a.tiles = a.mtiles * g.out_h * g.tpr;
   }
   // Stride-1 weight gradient with N % 16 == 0 and Kw <= 3 whose taps reach

@@ -3,15 +3,16 @@
 // section "어떻게 동작하나": the channel-batch-first layout lets the window
 // slide over channel/batch runs read once and reused on chip).
 //
-// A CTA owns an output tile of BW = 256/N consecutive pixels of one output
-// row x all N batch items (256 GEMM columns) x 128 output channels.  For
+// A CTA owns an output tile of BW consecutive pixels of one output row x all
+// N batch items (BW·N <= 256 GEMM columns) x 128 output channels; the host
+// picks BW to balance the tiles over the SMs.  For
 // each kernel row kh and 64-channel chunk of the reduction, the producer
 // warps dequantize the BW + Kw - 1 source pixels the window touches (the
 // "halo") into one K-major shared tile; the Kw taps of that kernel row are
 // then Kw MMA groups on the same tile, each starting kw·N rows further on
 // (a descriptor offset: N % 8 == 0 keeps it on the 8-row swizzle atom).  So
 // every source pixel is dequantized once per kernel row instead of once per
-// tap, and every MMA is 128 x 256 x 16.
+// tap, and every MMA is 128 x BW·N x 16.
 //
 // Forward:        source = X,   row  hi = ho + kh - pad,  columns wi = wo0 - pad + q,
 //                 tap kw uses halo pixels q = j + kw.
@@ -32,7 +33,7 @@
 
 namespace mqv {
 
-constexpr int kHaloBN = 256;                  // GEMM columns per tile
+constexpr int kHaloBN = 256;                  // most GEMM columns per tile (TMEM spacing of the accumulators)
 constexpr int kHaloMaxRows = 384;             // halo rows: 256 + (Kw - 1)·N <= 384
 constexpr int kHaloBStages = 2;
 constexpr int kHaloAStages = 6;
@@ -62,7 +63,8 @@ struct HaloBars {
 
 // Geometry of the halo pass (filled by the host).
 struct HaloGeom {
-  int bw;             // output pixels per tile (256 / N)
+  int bw;             // output pixels per tile
+  int bn;             // GEMM columns per tile, bw·N (a multiple of 16, <= 256)
   int rows;           // halo rows (bw + Kw - 1)·N
   int tpr;            // tiles per output row
   int cchunks;        // 64-channel chunks of the reduction
@@ -195,11 +197,12 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       const int ow0 = (rest - oh * g.tpr) * g.bw;
       const float scale = __fmul_rn(*p.ta, *p.tb);
       const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * kHaloBN;
+      // columns past bw·N hold no output (j >= bw below)
       // Each lane reads one accumulator row from TMEM; a swizzled 32 x 32
       // transpose in shared memory turns that into stores of 128-byte runs of
       // one (pixel, channel) row's batch items.
 #pragma unroll 1
-      for (int c = 0; c < kHaloBN; c += 32) {
+      for (int c = 0; c < g.bn; c += 32) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t r[16];
@@ -235,7 +238,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
     }
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(128, kHaloBN);
+      const uint32_t idesc = idesc_f16_f32(128, g.bn);
       int it = 0, bit = 0;
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
