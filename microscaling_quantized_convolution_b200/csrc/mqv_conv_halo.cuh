@@ -238,54 +238,73 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
     }
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
+      // The issuing thread's own instructions sit on the critical path of
+      // every stage, so everything per stage is a counter or an add:
+      // descriptors are base + offset in 16-byte units, ring slots and their
+      // phases are counters (no division).
       const uint32_t idesc = idesc_f16_f32(128, g.bn);
-      int it = 0, bit = 0;
+      const uint64_t adesc0 = smem_desc_sw128(sbase + L::kAOffset);
+      const uint64_t bdesc0 = smem_desc_sw128(sbase + L::kBOffset);
+      constexpr uint32_t kATileDesc = kATileBytes >> 4;
+      constexpr uint32_t kBTileDesc = kHaloBTile >> 4;
+      const uint32_t a_stage_desc = static_cast<uint32_t>(p.Kw) * kATileDesc;
+      const uint32_t tap_desc = static_cast<uint32_t>(p.N) * 8u;      // N rows of 128 B
+      int it = 0, sb = 0, sa = 0;
+      uint32_t pb = 0, pa = 0;                                         // ring phases
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
         tc_fence_after();
         const uint32_t dt = bars->tmem + acc * kHaloBN;
-        bool first = true;
-        for (int st = 0; st < stages_per_tile; ++st, ++bit) {
-          const int sb = bit % kHaloBStages;
-          const int sa = bit % na;
-          mbar_wait_bounded(&bars->bfull[sb], (bit / kHaloBStages) & 1, p.err, kErrWaitFull);
-          mbar_wait_bounded(&bars->afull[sa], (bit / na) & 1, p.err, kErrWaitFull);
+        for (int st = 0; st < stages_per_tile; ++st) {
+          mbar_wait_bounded(&bars->bfull[sb], pb, p.err, kErrWaitFull);
+          mbar_wait_bounded(&bars->afull[sa], pa, p.err, kErrWaitFull);
           tc_fence_after();
-          const uint32_t b_tile = sbase + L::kBOffset + sb * kHaloBTile;
-          const uint32_t a_stage = sbase + L::kAOffset + sa * p.Kw * kATileBytes;
+          const uint64_t ad = adesc0 + static_cast<uint32_t>(sa) * a_stage_desc;
+          const uint64_t bd = bdesc0 + static_cast<uint32_t>(sb) * kBTileDesc;
           for (int kw = 0; kw < p.Kw; ++kw) {
-            const int shift = PASS == kFwd ? kw : p.Kw - 1 - kw;
-            const uint64_t adesc = smem_desc_sw128(a_stage + kw * kATileBytes);
-            const uint64_t bdesc = smem_desc_sw128(b_tile + static_cast<uint32_t>(shift * p.N) * 128u);
+            const uint32_t shift = PASS == kFwd ? kw : p.Kw - 1 - kw;
+            const uint64_t a_k = ad + static_cast<uint32_t>(kw) * kATileDesc;
+            const uint64_t b_k = bd + shift * tap_desc;
+            const uint32_t acc0 = (st | kw) ? 1u : 0u;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_f16_ss(dt, adesc + 2 * kk, bdesc + 2 * kk, idesc, first ? 0u : 1u);
-              first = false;
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(dt, a_k + 2 * kk, b_k + 2 * kk, idesc, kk ? 1u : acc0);
           }
           mma_commit(&bars->aempty[sa]);
           mma_commit(&bars->bempty[sb]);
+          if (++sb == kHaloBStages) {
+            sb = 0;
+            pb ^= 1u;
+          }
+          if (++sa == na) {
+            sa = 0;
+            pa ^= 1u;
+          }
         }
         mma_commit(&bars->acc_full[acc]);
       }
     }
   } else if (warp == kV2LoadWarp) {
     if (lane == 0) {
-      int ait = 0;
+      int sa = 0;
+      uint32_t pa = 1;                 // first pass: the empty slots count as released
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
         const int mt = tile / (g.out_h * g.tpr);
         const uint8_t* img = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
         for (int kh = 0; kh < p.Kh; ++kh)
-          for (int c = 0; c < g.cchunks; ++c, ++ait) {
+          for (int c = 0; c < g.cchunks; ++c) {
             // the Kw weight tiles of the stage, under one barrier
-            const int sa = ait % na;
-            mbar_wait_bounded(&bars->aempty[sa], ((ait / na) & 1) ^ 1, p.err, kErrWaitEmpty);
+            mbar_wait_bounded(&bars->aempty[sa], pa, p.err, kErrWaitEmpty);
             mbar_arrive_expect_tx(&bars->afull[sa], p.Kw * kATileBytes);
             for (int kw = 0; kw < p.Kw; ++kw) {
               const int kt = (kh * p.Kw + kw) * g.cchunks + c;
               bulk_copy_g2s(sbase + L::kAOffset + (sa * p.Kw + kw) * kATileBytes,
                             img + static_cast<int64_t>(kt) * kATileBytes, kATileBytes, &bars->afull[sa]);
+            }
+            if (++sa == na) {
+              sa = 0;
+              pa ^= 1u;
             }
           }
       }
