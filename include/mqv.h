@@ -207,6 +207,22 @@ mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
 mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
                           float* gx, void* ws, size_t ws_bytes, void* stream);
 
+/* The baseline the method removes (section "무엇인가": quantize after the
+ * im2col expansion, once per GEMM direction), for measuring it on the same
+ * kernels.  Explicit im2col of fp32 X [H][W][Cin][N] into
+ *   xc[(ho, wo)][(kh, kw, ci)][n] = X[ho·stride + kh - pad][wo·stride + kw - pad][ci][n]
+ * (zero outside), i.e. fp32 [Ho][Wo][Kh·Kw·Cin][N]: the channel-batch-first
+ * tensor of a 1 x 1 convolution with Kh·Kw·Cin input channels whose forward
+ * pass is Y = W·X'.  x, xc: 16-byte aligned device buffers the caller owns;
+ * xc holds Ho·Wo·Kh·Kw·Cin·N floats (below 2^33).  Asynchronous on stream. */
+mqv_status mqv_im2col(const mqv_conv_desc* d, const float* x, float* xc, void* stream);
+
+/* The adjoint of mqv_im2col (reading R14): gx[hi][wi][ci][n] = sum, over
+ * the taps (kh, kw) and output pixels (ho, wo) with ho·stride + kh - pad = hi
+ * and wo·stride + kw - pad = wi, of gc[(ho, wo)][(kh, kw, ci)][n], added in
+ * (kh, kw) order.  gc: fp32 [Ho][Wo][Kh·Kw·Cin][N]; gx: fp32 [H][W][Cin][N]. */
+mqv_status mqv_col2im(const mqv_conv_desc* d, const float* gc, float* gx, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word that
  * bounded waits inside the conv kernels set when they give up
  * (*flags = 0: none).  Returns MQV_ERR_TIMEOUT if a flag was set. */

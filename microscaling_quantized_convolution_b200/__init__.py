@@ -92,6 +92,8 @@ _SIGS = {
                                          ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_conv_wgrad_noalloc": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                               ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_im2col": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_col2im": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -270,6 +272,28 @@ def _ws(d, op, ws, device):
     if ws is None and need:
         ws = torch.empty(need, dtype=torch.uint8, device=device)
     return ws
+
+
+def im2col(d: ConvDesc, x: torch.Tensor, xc: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Explicit im2col of fp32 X [H][W][Cin][N] -> [Ho][Wo][Kh·Kw·Cin][N]
+    (see mqv_im2col); for the quantize-after-im2col baseline."""
+    _require_cuda(x, "x", torch.float32)
+    Ho, Wo = out_hw(d)
+    xc = xc if xc is not None else torch.empty((Ho, Wo, d.Kh * d.Kw * d.Cin, d.N), dtype=torch.float32,
+                                               device=x.device)
+    _require_cuda(xc, "xc", torch.float32)
+    _check(lib().mqv_im2col(ctypes.byref(d), x.data_ptr(), xc.data_ptr(), _stream(stream)))
+    return xc
+
+
+def col2im(d: ConvDesc, gc: torch.Tensor, gx: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The adjoint of im2col: [Ho][Wo][Kh·Kw·Cin][N] -> G_X [H][W][Cin][N]
+    (see mqv_col2im)."""
+    _require_cuda(gc, "gc", torch.float32)
+    gx = gx if gx is not None else torch.empty((d.H, d.W, d.Cin, d.N), dtype=torch.float32, device=gc.device)
+    _require_cuda(gx, "gx", torch.float32)
+    _check(lib().mqv_col2im(ctypes.byref(d), gc.data_ptr(), gx.data_ptr(), _stream(stream)))
+    return gx
 
 
 def conv_fwd(d: ConvDesc, w: QTensor, x: QTensor, y: torch.Tensor | None = None,

@@ -15,6 +15,7 @@
 #include "mqv_conv_kernels.cuh"
 #include "mqv_conv_halo.cuh"
 #include "mqv_conv_wgk.cuh"
+#include "mqv_naive.cuh"
 #include "mqv_quantize.cuh"
 
 namespace {
@@ -768,6 +769,67 @@ mqv_status noalloc_scratch(float** out) {
 }
 
 }  // namespace
+
+namespace {
+
+mqv_status plan_im2col(const mqv_conv_desc* d, Im2colGeom* g, int64_t* xc_n4, int64_t* x_n4) {
+  mqv_status st = check_desc(d);
+  if (st) return st;
+  g->N = (int)d->N; g->Cin = (int)d->Cin; g->H = (int)d->H; g->W = (int)d->W;
+  g->Kh = (int)d->Kh; g->Kw = (int)d->Kw; g->stride = (int)d->stride; g->pad = (int)d->pad;
+  g->Ho = (int)((d->H + 2 * d->pad - d->Kh) / d->stride + 1);
+  g->Wo = (int)((d->W + 2 * d->pad - d->Kw) / d->stride + 1);
+  const int64_t K = d->Kh * d->Kw * d->Cin;
+  *xc_n4 = (int64_t)g->Ho * g->Wo * K * (d->N / 4);
+  *x_n4 = d->H * d->W * d->Cin * (d->N / 4);
+  if (*xc_n4 >= (int64_t(1) << 31) || (int64_t)g->Ho * g->Wo * K >= (int64_t(1) << 31))
+    return fail(MQV_ERR_UNSUPPORTED, "the expanded matrix exceeds 2^31 float4");
+  g->dn4 = make_fastdiv(d->N / 4);
+  g->dcin = make_fastdiv(d->Cin);
+  g->dk = make_fastdiv(K);
+  g->dkw = make_fastdiv(d->Kw);
+  g->dwo = make_fastdiv(g->Wo);
+  g->dw = make_fastdiv(d->W);
+  return MQV_OK;
+}
+
+unsigned naive_grid(int64_t n4) {
+  int64_t g = (n4 + kNaiveThreads - 1) / kNaiveThreads;
+  if (g > kSMs * 16) g = kSMs * 16;
+  return (unsigned)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+extern "C" mqv_status mqv_im2col(const mqv_conv_desc* d, const float* x, float* xc, void* stream) {
+  Im2colGeom g;
+  int64_t xc_n4 = 0, x_n4 = 0;
+  mqv_status st = plan_im2col(d, &g, &xc_n4, &x_n4);
+  if (st) return st;
+  if (!x || !xc || !aligned16(x) || !aligned16(xc))
+    return fail(MQV_ERR_INVALID_ARG, "x and xc must be 16-byte aligned device pointers");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  im2col_kernel<<<naive_grid(xc_n4), kNaiveThreads, 0, s>>>(g, reinterpret_cast<const float4*>(x),
+                                                              reinterpret_cast<float4*>(xc), xc_n4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "im2col launch");
+  return ok();
+}
+
+extern "C" mqv_status mqv_col2im(const mqv_conv_desc* d, const float* gc, float* gx, void* stream) {
+  Im2colGeom g;
+  int64_t xc_n4 = 0, x_n4 = 0;
+  mqv_status st = plan_im2col(d, &g, &xc_n4, &x_n4);
+  if (st) return st;
+  if (!gc || !gx || !aligned16(gc) || !aligned16(gx))
+    return fail(MQV_ERR_INVALID_ARG, "gc and gx must be 16-byte aligned device pointers");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  col2im_kernel<<<naive_grid(x_n4), kNaiveThreads, 0, s>>>(g, reinterpret_cast<const float4*>(gc),
+                                                             reinterpret_cast<float4*>(gx), x_n4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "col2im launch");
+  return ok();
+}
 
 extern "C" mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
                                              const mqv_qtensor* x, float* gw, void* stream) {
