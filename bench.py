@@ -113,6 +113,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     import microscaling_quantized_convolution_b200 as mqv
+    from microscaling_quantized_convolution_b200 import naive
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -285,6 +286,65 @@ def run_gpu(args):
         mean = {k: t[1 + j].item() for j, k in enumerate(parts)}
     flags = mqv.device_errors()
 
+    # The baseline the method removes (expand with im2col first, quantize each
+    # operand once per GEMM direction), timed the same way on one GPU.
+    naive_res = None
+    if world == 1 and args.naive_steps > 0:
+        nb = naive.plan(d, dev)
+        nout = {"y": torch.empty_like(sets[0]["y"]), "gw": torch.empty_like(sets[0]["gw"]),
+                "gx": torch.empty_like(sets[0]["gx"])}
+
+        def nphase(k, ph):
+            sk = sets[k]
+            if ph == "quant":
+                naive.quantize_all(nb, sk["X"], sk["W"], sk["G"], seed + k)
+            elif ph == "fwd":
+                naive.fwd(nb, nout["y"])
+            elif ph == "wgrad":
+                naive.wgrad(nb, nout["gw"])
+            else:
+                naive.dgrad(nb, nout["gx"])
+
+        nphases = ("quant", "fwd", "wgrad", "dgrad")
+        for k in range(nsets):
+            for ph in nphases:
+                nphase(k, ph)
+        torch.cuda.synchronize()
+        ngraphs = [{ph: capture(lambda k=k, ph=ph: nphase(k, ph)) for ph in nphases} for k in range(nsets)]
+        nev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.naive_steps)]
+
+        def nstep(i, ev):
+            g = ngraphs[i % nsets]
+            for j, ph in enumerate(nphases):
+                ev[j].record()
+                g[ph].replay()
+            ev[4].record()
+
+        for i in range(3):
+            nstep(i, nev[0])
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(args.naive_steps):
+            nstep(i, nev[i])
+        b.record()
+        torch.cuda.synchronize()
+        n_ms = a.elapsed_time(b) / args.naive_steps
+        nparts = {ph: sum(e[j].elapsed_time(e[j + 1]) for e in nev) / len(nev) for j, ph in enumerate(nphases)}
+        nbytes = naive.layer_bytes(d)
+        Ho_, Wo_ = mqv.out_hw(d)
+        ex = Ho_ * Wo_ * d.Kh * d.Kw * d.Cin * d.N          # elements of the expanded X
+        once_bytes = sum(quant_b.values()) + sum(conv_b.values())
+        naive_res = {"ms_per_step": round(n_ms, 4),
+                     "phase_ms": {ph: round(v, 4) for ph, v in nparts.items()},
+                     "step_time_ratio": None, "quantize_time_ratio": None,
+                     "algorithmic_bytes_ratio": round(sum(nbytes.values()) / once_bytes, 3),
+                     "quantized_elements_ratio": round((2 * ex + 2 * nw + 2 * ng) / (nx + nw + ng), 3),
+                     "expanded_x_ratio": round(ex / nx, 3),
+                     "flow": "im2col, every operand quantized once per GEMM direction, 1x1 GEMMs, col2im"}
+        del ngraphs
+        torch.cuda.synchronize()
+
     # End to end through the public API with pinned host buffers, pipelined
     # as a training loop would be: step i copies its inputs in on one stream,
     # computes on the current stream and copies its outputs back on a third,
@@ -410,6 +470,10 @@ def run_gpu(args):
     }
     if e2e:
         out["e2e"] = e2e
+    if naive_res:
+        naive_res["step_time_ratio"] = round(naive_res["ms_per_step"] / ms_step, 3)
+        naive_res["quantize_time_ratio"] = round(naive_res["phase_ms"]["quant"] / mean["quantize"], 3)
+        out["naive_baseline"] = naive_res
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(layer, budget_s=args.cpu_budget)
     print(json.dumps(out), flush=True)
@@ -498,6 +562,8 @@ def main():
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--workload", default=workloads.resnet18_layer2().name)
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--naive-steps", type=int, default=100,
+                    help="steps of the quantize-after-im2col baseline (0: skip)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
