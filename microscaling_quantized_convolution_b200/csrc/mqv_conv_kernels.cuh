@@ -170,8 +170,19 @@ prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int
   const int chunks = mtiles * 128 * ktiles * 8;
   const int id = blockIdx.x * kPrepThreads + threadIdx.x;
   if (id >= chunks) return;
-  const int m = fdiv(id, dkt8);
-  const int k0 = (id - m * ktiles * 8) * 8;
+  // forward: consecutive threads take consecutive K chunks of one weight row
+  // (contiguous codes); transposed: consecutive threads take consecutive rows
+  // m = ci of one K chunk, so a warp's code reads walk along a weight row
+  int m, k0;
+  if (!TRANS) {
+    m = fdiv(id, dkt8);
+    k0 = (id - m * ktiles * 8) * 8;
+  } else {
+    const int mrows = mtiles * 128;
+    const int kc = id / mrows;
+    m = id - kc * mrows;
+    k0 = kc * 8;
+  }
   uint32_t h[4] = {0u, 0u, 0u, 0u};
   if (m < M) {
     if (!TRANS && k0 + 8 <= Kdim && (FMT == 0 ? (w.row_bytes & 3) == 0 : (w.row_bytes & 1) == 0)) {
