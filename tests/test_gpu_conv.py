@@ -199,3 +199,50 @@ YOLO = workloads.yolov8n_mix()
 @pytest.mark.parametrize("layer", YOLO, ids=[l.name for l in YOLO])
 def test_yolov8n_full_size_sampled(layer):
     sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (3, 6, 17))
+
+
+def test_concurrent_passes_match_serial():
+    """fwd, wgrad and dgrad on three streams (as the bench runs them), with
+    G_Y quantized on a fourth beside X and W, give bit-identical outputs to
+    the same calls on one stream."""
+    layer = workloads.resnet18_layer2()
+    s = O.ConvShape(layer.N, layer.Cin, layer.Cout, layer.H, layer.W, layer.K, layer.K, layer.stride, layer.pad)
+    X, Wt, G = (t.cuda().contiguous() for t in workloads.make_layer_inputs(layer))
+    d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+    fmt, seed = layer.fmt, workloads.sr_seed(layer)
+
+    def run(concurrent):
+        qx = mqv.QTensor.empty(*s.x_view(), fmt)
+        qw = mqv.QTensor.empty(*s.w_view(), fmt)
+        qg = mqv.QTensor.empty(*s.gy_view(), fmt)
+        cur = torch.cuda.current_stream()
+        streams = [torch.cuda.Stream() for _ in range(4)] if concurrent else [cur] * 4
+        start = torch.cuda.Event()
+        start.record(cur)
+        for st in streams:
+            st.wait_event(start)
+        with torch.cuda.stream(streams[3]):
+            mqv.quantize_many([(G.view(-1), *s.gy_view(), fmt, mqv.SR, seed, qg)])
+            g_done = torch.cuda.Event()
+            g_done.record(streams[3])
+        mqv.quantize_many([(X.view(-1), *s.x_view(), fmt, mqv.RNE, 0, qx),
+                           (Wt.view(-1), *s.w_view(), fmt, mqv.RNE, 0, qw)])
+        xw_done = torch.cuda.Event()
+        xw_done.record(cur)
+        outs = {}
+        for i, (name, fn) in enumerate((("y", lambda: mqv.conv_fwd(d, qw, qx)),
+                                        ("gw", lambda: mqv.conv_wgrad(d, qg, qx)),
+                                        ("gx", lambda: mqv.conv_dgrad(d, qw, qg)))):
+            st = streams[i]
+            st.wait_event(xw_done)
+            if name != "y":
+                st.wait_event(g_done)
+            with torch.cuda.stream(st):
+                outs[name] = fn()
+        torch.cuda.synchronize()
+        return {k: v.cpu().numpy() for k, v in outs.items()}
+
+    a, b = run(False), run(True)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+    assert mqv.device_errors() == 0
