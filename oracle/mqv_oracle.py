@@ -51,6 +51,9 @@ Readings where the pages are silent (each also listed in the design notes):
   R15 stride/padding follow the usual conv2d meaning (zero padding, floor).
   R16 packing: FP4 two codes per byte, even column in the low nibble; FP6
       four 6-bit codes per 3 bytes, code j at bits [6j, 6j+6) little-endian.
+  R21 replay form of a post-ReLU tensor: magnitudes only (3 or 5 bits),
+      element i at bits [i·m, i·m + m) of a little-endian bit stream; the
+      E4M3 block scales and T are kept as they are.
 """
 from __future__ import annotations
 
@@ -314,6 +317,48 @@ def unpack_codes(packed: np.ndarray, rows: int, cols: int, fmt: str) -> np.ndarr
 
 def packed_row_bytes(cols: int, fmt: str) -> int:
     return cols // 2 if fmt == FP4 else cols * 3 // 4
+
+
+# ---------------------------------------------------------------------------
+# Latent-replay storage of post-ReLU tensors (reading R21)
+# ---------------------------------------------------------------------------
+
+
+def magnitude_bits(fmt: str) -> int:
+    """Bits of an element code without its sign: 3 (E2M1) or 5 (E2M3)."""
+    return element_bits(fmt) - 1
+
+
+def pack_unsigned(codes: np.ndarray, fmt: str):
+    """Sections "어떻게 쓰나" and "전제와 한계": an activation after ReLU is never
+    negative, so its E2M1 code needs no sign bit and 3 bits per pixel remain.
+    Reading R21: element i of the row-major view (its magnitude bits, least
+    significant first) fills bits [i·m, i·m + m) of a bit stream stored
+    little-endian, m = magnitude_bits(fmt).  A code with the sign bit and a
+    nonzero magnitude cannot be stored; it is stored as 0 (the ReLU of its
+    value) and counted.  Returns (bytes, count of such codes)."""
+    c = np.asarray(codes, dtype=np.int64).reshape(-1)
+    m = magnitude_bits(fmt)
+    mag = c & ((1 << m) - 1)
+    negative = (((c >> m) & 1) == 1) & (mag != 0)
+    mag = np.where(negative, 0, mag)
+    bits = (mag[:, None] >> np.arange(m)[None, :]) & 1
+    return np.packbits(bits.reshape(-1).astype(np.uint8), bitorder="little"), int(negative.sum())
+
+
+def unpack_unsigned(packed: np.ndarray, rows: int, cols: int, fmt: str) -> np.ndarray:
+    """Codes (sign bit 0) of the view stored by pack_unsigned."""
+    m = magnitude_bits(fmt)
+    n = rows * cols
+    bits = np.unpackbits(np.asarray(packed, dtype=np.uint8), bitorder="little")[:n * m]
+    mag = (bits.reshape(n, m).astype(np.int64) << np.arange(m)[None, :]).sum(axis=1)
+    return mag.reshape(rows, cols)
+
+
+def unsigned_bits_per_element(fmt: str) -> float:
+    """Stored bits per element of the replay form: magnitude plus one E4M3
+    byte per 16 elements (T is one float per tensor and is not counted)."""
+    return magnitude_bits(fmt) + 8.0 / 16.0
 
 
 # ---------------------------------------------------------------------------

@@ -243,6 +243,72 @@ def test_packing_bit_layout():
         assert np.array_equal(O.unpack_codes(p, 8, 12, fmt), c)
 
 
+# ------------------------------------- replay form of post-ReLU tensors (R21)
+
+def test_unsigned_pack_bit_layout_by_hand():
+    # E2M1 magnitudes 1..7, 0 at 3 bits each: 1 | 2<<3 | 3<<6 | 4<<9 | 5<<12
+    # | 6<<15 | 7<<18 = 2054353 = 0x1F58D1, little-endian bytes D1 58 1F.
+    p, neg = O.pack_unsigned(np.array([[1, 2, 3, 4], [5, 6, 7, 0]]), O.FP4)
+    assert list(p) == [0xD1, 0x58, 0x1F] and neg == 0
+    # E2M3 magnitudes 31, 1, 0, 17, 2, 3, 4, 5 at 5 bits each:
+    # 31 | 1<<5 | 17<<15 | 2<<20 | 3<<25 | 4<<30 | 5<<35 = 176196976703
+    # = 0x290628803F, little-endian bytes 3F 80 28 06 29.
+    p, neg = O.pack_unsigned(np.array([[31, 1, 0, 17], [2, 3, 4, 5]]), O.FP6)
+    assert list(p) == [0x3F, 0x80, 0x28, 0x06, 0x29] and neg == 0
+
+
+def test_unsigned_pack_drops_only_the_sign_bit():
+    rng = np.random.default_rng(1)
+    for fmt, hi in ((O.FP4, 8), (O.FP6, 32)):
+        c = rng.integers(0, hi, size=(8, 12))
+        p, neg = O.pack_unsigned(c, fmt)
+        assert neg == 0 and p.size == 8 * 12 * O.magnitude_bits(fmt) // 8
+        assert np.array_equal(O.unpack_unsigned(p, 8, 12, fmt), c)
+        # one stored element spans bits [i·m, i·m+m): flipping bit k of the
+        # stream changes element k // m by 2^(k % m) and nothing else
+        m = O.magnitude_bits(fmt)
+        for k in (0, m - 1, m, 5 * m + 2, 8 * 12 * m - 1):
+            q = p.copy()
+            q[k // 8] ^= 1 << (k % 8)
+            d = O.unpack_unsigned(q, 8, 12, fmt).reshape(-1) - c.reshape(-1)
+            assert np.count_nonzero(d) == 1 and abs(d[k // m]) == 1 << (k % m)
+
+
+def test_unsigned_pack_counts_negative_codes_and_stores_relu():
+    # sign bit set: -0 (mag 0) is fine, -1.5 (E2M1 0b1011) is counted and
+    # stored as 0, +6 (0b0111) stays.
+    p, neg = O.pack_unsigned(np.array([[0b1000, 0b1011, 0b0111, 0b1111]]), O.FP4)
+    assert neg == 2
+    assert list(O.unpack_unsigned(p, 1, 4, O.FP4)[0]) == [0, 0, 7, 0]
+
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+def test_replay_form_of_relu_activations_dequantizes_to_the_same_values(fmt):
+    """Quantizing ReLU(x) yields no negative code, and the replay form reads
+    back exactly the values of the full codes; on a signed tensor it reads
+    back max(x_hat, 0)."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((16, 32)).astype(np.float32)
+    for src, relu in ((np.maximum(x, 0), True), (x, False)):
+        q = O.quantize(src, fmt, O.RNE)
+        p, neg = O.pack_unsigned(q.codes, fmt)
+        back = O.QTensor(O.unpack_unsigned(p, 16, 32, fmt), q.scales, q.T, fmt)
+        if relu:
+            assert neg == 0
+            assert np.array_equal(O.dequantize(back), O.dequantize(q))
+        else:
+            assert neg == int(np.count_nonzero(O.dequantize(q) < 0))
+            assert np.array_equal(O.dequantize(back), np.maximum(O.dequantize(q), 0))
+
+
+def test_replay_bits_per_element():
+    # 3 magnitude bits + one E4M3 byte per 4 x 4 block = 3.5 bits (FP4); the
+    # signed form holds 4.5.  The pages' 3.125 would need one byte per 64.
+    assert O.unsigned_bits_per_element(O.FP4) == 3.5
+    assert O.unsigned_bits_per_element(O.FP6) == 5.5
+    assert O.bits_per_element(O.FP4) - O.unsigned_bits_per_element(O.FP4) == 1.0
+
+
 # --------------------------------- P9 dequantized products fit f16 / bf16
 
 @pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
