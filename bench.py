@@ -547,11 +547,159 @@ def run_gpu(args):
         naive_res["step_time_ratio"] = round(naive_res["ms_per_step"] / (serial_ms / args.steps), 3)
         naive_res["quantize_time_ratio"] = round(naive_res["phase_ms"]["quant"] / mean["quantize"], 3)
         out["naive_baseline"] = naive_res
+    if world == 1 and not args.no_sweeps:
+        out["sweeps"] = run_sweeps(args, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(layer, budget_s=args.cpu_budget)
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------- sweeps at 1 GPU
+
+def _timed(torch, fn, iters, flush):
+    """Mean device ms of fn over `iters` calls, each bracketed by its own
+    CUDA events on the current stream, with L2 flushed (a 256 MB write)
+    before each call, outside the events."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / iters
+
+
+def run_sweeps(args, dev, peaks):
+    """The other measured workloads, each as absolute throughput and as a
+    fraction of its roofline:
+      - replay_quantize: the quantize-only sweep over the latent-replay
+        buffer shapes (1M..1G elements), |N(0,1)| with 0.1 % outliers x100,
+        RNE and SR; 8.5625 algorithmic B/element (two fp32 reads, codes,
+        scales);
+      - replay_form: the magnitude-only replay form of the same quantized
+        buffers: pack (0.5 B read + 0.375 B written per element) and values
+        read straight back (0.375 + 1/16 B read, 4 B written), beside
+        mqv_dequantize of the full codes;
+      - resnet18_body and yolov8n_mix: every layer's step (quantize, fwd,
+        wgrad, dgrad) timed phase by phase with L2 flushed before each
+        phase; per-network sums against the sum of per-pass rooflines."""
+    import torch
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    res = {"l2": "256 MB written before every timed call", "timing": "CUDA events per call"}
+    launches = 0
+
+    rq, rf = [], []
+    for C, H, N in workloads.REPLAY_SHAPES:
+        rows, cols = H * H * C, N
+        n = rows * cols
+        iters = 20 if n < 100_000_000 else 5
+        x = workloads.make_replay_input(C, H, N, outliers=True, seed=3, device=dev).view(-1)
+        q = mqv.QTensor.empty(rows, cols, "nvfp4", dev)
+        ws = torch.empty(mqv.quantize_workspace_bytes(rows, cols), dtype=torch.uint8, device=dev)
+        ent = {"C": C, "H": H, "N": N, "elements": n}
+        for name, rnd in (("rne", mqv.RNE), ("sr", mqv.SR)):
+            def f(rnd=rnd):
+                mqv.quantize(x, rows, cols, "nvfp4", rnd, 11, out=q, ws=ws)
+            for _ in range(3):
+                f()
+            ms = _timed(torch, f, iters, flush)
+            launches += 2 * (iters + 3)
+            gbs = 8.5625 * n / (ms * 1e-3) / 1e9
+            ent[name] = {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+        rq.append(ent)
+        del x
+        # replay form of the (RNE-rounded last: SR) quantized buffer
+        mqv.quantize(workloads.make_replay_input(C, H, N, outliers=True, seed=3, device=dev).view(-1),
+                     rows, cols, "nvfp4", mqv.RNE, 0, out=q, ws=ws)
+        packed = torch.empty(mqv.replay_bytes(rows, cols, "nvfp4"), dtype=torch.uint8, device=dev)
+        vals = torch.empty(n, dtype=torch.float32, device=dev)
+        neg = torch.zeros(1, dtype=torch.int32, device=dev)
+        calls = {"pack": (lambda: mqv.replay_pack(q, out=packed, negatives=neg), 0.875),
+                 "read": (lambda: mqv.replay_dequantize(packed, q.scales, q.tscale, rows, cols, "nvfp4",
+                                                        out=vals), 0.375 + 0.0625 + 4),
+                 "dequantize_full_codes": (lambda: mqv.dequantize(q, out=vals), 0.5 + 0.0625 + 4)}
+        fe = {"C": C, "H": H, "N": N, "elements": n, "bytes": mqv.replay_bytes(rows, cols, "nvfp4"),
+              "bits_per_element": 3.5, "bits_per_element_signed": 4.5}
+        for name, (fn, bpe) in calls.items():
+            for _ in range(3):
+                fn()
+            ms = _timed(torch, fn, iters, flush)
+            launches += iters + 3
+            gbs = bpe * n / (ms * 1e-3) / 1e9
+            fe[name] = {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+        fe["negative_codes"] = int(neg.item())
+        rf.append(fe)
+        del q, ws, packed, vals
+        torch.cuda.empty_cache()
+    res["replay_quantize"] = rq
+    res["replay_form"] = rf
+
+    for net, layers in (("resnet18_body", workloads.resnet18_body()), ("yolov8n_mix", workloads.yolov8n_mix())):
+        tot = {"quantize": 0.0, "fwd": 0.0, "wgrad": 0.0, "dgrad": 0.0}
+        roof = {"quantize": 0.0, "conv": 0.0}
+        flops_all, per_layer = 0, []
+        for layer in layers:
+            X, Wt, G = (t.view(-1) for t in workloads.make_layer_inputs(layer, device=dev))
+            d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+            xr, xc = layer.H * layer.W * layer.Cin, layer.N
+            wr, wc = layer.Cout, layer.K * layer.K * layer.Cin
+            gr, gc = layer.Ho * layer.Wo * layer.Cout, layer.N
+            qx, qw, qg = (mqv.QTensor.empty(r, c, layer.fmt, dev) for r, c in ((xr, xc), (wr, wc), (gr, gc)))
+            jobs = [(X, xr, xc, layer.fmt, mqv.RNE, 0, qx), (Wt, wr, wc, layer.fmt, mqv.RNE, 0, qw),
+                    (G, gr, gc, layer.fmt, mqv.SR, workloads.sr_seed(layer), qg)]
+            wsq = torch.empty(mqv.quantize_many_workspace_bytes([j[:6] for j in jobs]), dtype=torch.uint8,
+                              device=dev)
+            wss = {op: torch.empty(max(16, mqv.conv_workspace_bytes(d, op)), dtype=torch.uint8, device=dev)
+                   for op in (mqv.OP_FWD, mqv.OP_WGRAD, mqv.OP_DGRAD)}
+            y = torch.empty(gr * gc, device=dev)
+            gw = torch.empty(wr * wc, device=dev)
+            gx = torch.empty(xr * xc, device=dev)
+            phases = {"quantize": lambda: mqv.quantize_many(jobs, ws=wsq),
+                      "fwd": lambda: mqv.conv_fwd(d, qw, qx, y=y, ws=wss[mqv.OP_FWD]),
+                      "wgrad": lambda: mqv.conv_wgrad(d, qg, qx, gw=gw, ws=wss[mqv.OP_WGRAD]),
+                      "dgrad": lambda: mqv.conv_dgrad(d, qw, qg, gx=gx, ws=wss[mqv.OP_DGRAD])}
+            for _ in range(3):
+                for fn in phases.values():
+                    fn()
+            ms = {k: _timed(torch, fn, 5, flush) for k, fn in phases.items()}
+            launches += 8 * (2 + 2 + 2 + 1 + (1 if mqv.conv_workspace_bytes(d, mqv.OP_WGRAD) else 0))
+            qbytes, cbytes, _ = layer_bytes(layer)
+            fl = layer.flops()
+            flops_all += 3 * fl
+            lr = {"layer": layer.name, "ms": {k: round(v, 5) for k, v in ms.items()}}
+            lroof = 0.0
+            for k in ("fwd", "wgrad", "dgrad"):
+                tot[k] += ms[k]
+                rt = max(fl / (tc * 1e12), cbytes[k] / (hbm * 1e9)) * 1e3
+                roof["conv"] += rt
+                lroof += rt
+            tot["quantize"] += ms["quantize"]
+            roof["quantize"] += sum(qbytes.values()) / (hbm * 1e9) * 1e3
+            lr["conv_frac"] = round(lroof / (ms["fwd"] + ms["wgrad"] + ms["dgrad"]), 4)
+            per_layer.append(lr)
+            del X, Wt, G, qx, qw, qg, wsq, wss, y, gw, gx
+        torch.cuda.empty_cache()
+        conv_ms = tot["fwd"] + tot["wgrad"] + tot["dgrad"]
+        res[net] = {"layers": len(layers), "conv_ms": round(conv_ms, 4),
+                    "conv_tflops": round(flops_all / (conv_ms * 1e-3) / 1e12, 2),
+                    "conv_frac_of_roofline": round(roof["conv"] / conv_ms, 4),
+                    "quantize_ms": round(tot["quantize"], 4),
+                    "quantize_frac_of_roofline": round(roof["quantize"] / tot["quantize"], 4),
+                    "phase_ms": {k: round(v, 4) for k, v in tot.items()},
+                    "per_layer": per_layer}
+    flags = mqv.device_errors()
+    if flags:
+        raise SystemExit(f"device wait timeout flags {flags:#x} in the sweeps")
+    res["launches"] = launches
+    return res
+
+
+# -------------------------------------------------------------- CPU oracle
 # -------------------------------------------------------------- CPU oracle
 
 def oracle_sample_layer(layer: workloads.Layer, n_batch: int, hw: int) -> workloads.Layer:
@@ -639,6 +787,8 @@ def main():
                     help="run fwd, wgrad and dgrad one after another on one stream")
     ap.add_argument("--naive-steps", type=int, default=100,
                     help="steps of the quantize-after-im2col baseline (0: skip)")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the replay-buffer and whole-network sweeps")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))

@@ -160,6 +160,35 @@ mqv_status mqv_quantize_many(const mqv_quantize_job* jobs, int32_t count, void* 
  * latent-replay) tensor back.  dst: rows x cols fp32, 16-byte aligned. */
 mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream);
 
+/* Latent-replay form of a post-ReLU tensor (sections "어떻게 쓰나" and
+ * "전제와 한계": an E2M1 activation takes 3 bits per pixel, and the replay
+ * buffer keeps quantized activations).  After ReLU no code is negative, so
+ * only the magnitude bits are kept, m = 3 (NVFP4) or 5 (NVFP6): element i of
+ * the row-major rows x cols view at bits [i·m, i·m + m) of a little-endian
+ * bit stream, rows·cols·m/8 bytes.  The scale plane and T are not part of it
+ * (keep them as they are).  With the scales that is 3.5 bits per element
+ * for NVFP4 and 5.5 for NVFP6.  rows and cols: positive multiples of 4. */
+mqv_status mqv_replay_bytes(int64_t rows, int64_t cols, int32_t fmt, size_t* bytes);
+
+/* Write the replay form of q's codes to `packed` (16-byte aligned device
+ * buffer of mqv_replay_bytes bytes).  A code with the sign bit and a nonzero
+ * magnitude (a negative value) is stored as 0, the ReLU of its value; if
+ * `negatives` is not NULL, the number of such codes is added to the device
+ * uint32 it points to (the caller zeroes it).  Reads q->codes only. */
+mqv_status mqv_replay_pack(const mqv_qtensor* q, void* packed, uint32_t* negatives, void* stream);
+
+/* Codes (standard packing, sign bit 0) of a rows x cols view from its
+ * replay form.  packed, codes: 16-byte aligned device buffers. */
+mqv_status mqv_replay_unpack(const void* packed, int64_t rows, int64_t cols, int32_t fmt, void* codes,
+                             void* stream);
+
+/* Read the replay form straight back to fp32: dst[r][c] = code·B·T with the
+ * arithmetic of mqv_dequantize (code·B exact in fp16, one fp32 rounding).
+ * scales: [rows/4][cols/4] E4M3 bytes; tscale: one device fp32; dst: rows x
+ * cols fp32, 16-byte aligned. */
+mqv_status mqv_replay_dequantize(const void* packed, const uint8_t* scales, const float* tscale, int64_t rows,
+                                 int64_t cols, int32_t fmt, float* dst, void* stream);
+
 /* Workspace bytes for a conv pass (op = mqv_op).  Host-only. */
 mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* bytes);
 

@@ -94,6 +94,14 @@ _SIGS = {
                                               ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_im2col": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_col2im": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_replay_bytes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_replay_pack": (ctypes.c_int, [ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p]),
+    "mqv_replay_unpack": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_replay_dequantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -248,6 +256,54 @@ def dequantize(q: QTensor, out: torch.Tensor | None = None, stream=None) -> torc
                                                   device=q.codes.device)
     qc = q.c()
     _check(lib().mqv_dequantize(ctypes.byref(qc), out.data_ptr(), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------- latent-replay form
+
+def replay_bytes(rows: int, cols: int, fmt) -> int:
+    """Bytes of the magnitude-only replay form of a rows x cols view."""
+    b = ctypes.c_size_t()
+    _check(lib().mqv_replay_bytes(rows, cols, _fmt(fmt), ctypes.byref(b)))
+    return b.value
+
+
+def replay_pack(q: QTensor, out: torch.Tensor | None = None, negatives: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """Magnitude-only form of a post-ReLU tensor's codes (see
+    mqv_replay_pack); `negatives` (int32 device scalar, zeroed by the
+    caller) receives the count of negative codes, which are stored as 0."""
+    out = out if out is not None else torch.empty(replay_bytes(q.rows, q.cols, q.fmt), dtype=torch.uint8,
+                                                  device=q.codes.device)
+    _require_cuda(out, "out", torch.uint8)
+    if negatives is not None:
+        _require_cuda(negatives, "negatives", torch.int32)
+    qc = q.c()
+    _check(lib().mqv_replay_pack(ctypes.byref(qc), out.data_ptr(), _ptr(negatives), _stream(stream)))
+    return out
+
+
+def replay_unpack(packed: torch.Tensor, rows: int, cols: int, fmt, codes: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Standard-packing codes (sign bit 0) from the replay form."""
+    _require_cuda(packed, "packed", torch.uint8)
+    codes = codes if codes is not None else torch.empty(qtensor_bytes(rows, cols, fmt)[0], dtype=torch.uint8,
+                                                        device=packed.device)
+    _require_cuda(codes, "codes", torch.uint8)
+    _check(lib().mqv_replay_unpack(packed.data_ptr(), rows, cols, _fmt(fmt), codes.data_ptr(), _stream(stream)))
+    return codes
+
+
+def replay_dequantize(packed: torch.Tensor, scales: torch.Tensor, tscale: torch.Tensor, rows: int, cols: int,
+                      fmt, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """fp32 values code·B·T read straight from the replay form."""
+    _require_cuda(packed, "packed", torch.uint8)
+    _require_cuda(scales, "scales", torch.uint8)
+    _require_cuda(tscale, "tscale", torch.float32)
+    out = out if out is not None else torch.empty(rows * cols, dtype=torch.float32, device=packed.device)
+    _require_cuda(out, "out", torch.float32)
+    _check(lib().mqv_replay_dequantize(packed.data_ptr(), scales.data_ptr(), tscale.data_ptr(), rows, cols,
+                                       _fmt(fmt), out.data_ptr(), _stream(stream)))
     return out
 
 

@@ -17,6 +17,7 @@
 #include "mqv_conv_wgk.cuh"
 #include "mqv_naive.cuh"
 #include "mqv_quantize.cuh"
+#include "mqv_replay.cuh"
 
 namespace {
 
@@ -685,6 +686,89 @@ mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream) {
     dequantize_kernel<1><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, dst);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return ok();
+}
+
+// ------------------------------------------------------------ replay form
+
+namespace {
+
+mqv_status check_replay_view(int64_t rows, int64_t cols, int32_t fmt) {
+  mqv_status st = check_view(rows, cols);
+  if (st) return st;
+  return check_fmt(fmt);
+}
+
+unsigned replay_ctas(int64_t n) {
+  const int64_t runs = (n + kReplayRun - 1) / kReplayRun;
+  const int64_t g = (runs + kReplayThreads - 1) / kReplayThreads;
+  return static_cast<unsigned>(g < kMaxQuantCtas ? g : kMaxQuantCtas);
+}
+
+}  // namespace
+
+mqv_status mqv_replay_bytes(int64_t rows, int64_t cols, int32_t fmt, size_t* bytes) {
+  mqv_status st = check_replay_view(rows, cols, fmt);
+  if (st) return st;
+  if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  *bytes = static_cast<size_t>(rows * cols / 8 * (fmt == MQV_NVFP4 ? 3 : 5));
+  return ok();
+}
+
+mqv_status mqv_replay_pack(const mqv_qtensor* q, void* packed, uint32_t* negatives, void* stream) {
+  mqv_status st = check_qtensor(q, "q");
+  if (st) return st;
+  if (!packed || !aligned16(packed)) return fail(MQV_ERR_INVALID_ARG, "packed must be a 16-byte aligned pointer");
+  if (negatives && (reinterpret_cast<uintptr_t>(negatives) & 3u))
+    return fail(MQV_ERR_INVALID_ARG, "negatives must be 4-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = q->rows * q->cols;
+  const uint8_t* c = static_cast<const uint8_t*>(q->codes);
+  uint8_t* o = static_cast<uint8_t*>(packed);
+  if (q->fmt == MQV_NVFP4)
+    replay_pack_kernel<0><<<replay_ctas(n), kReplayThreads, 0, s>>>(c, n, o, negatives);
+  else
+    replay_pack_kernel<1><<<replay_ctas(n), kReplayThreads, 0, s>>>(c, n, o, negatives);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "replay pack launch");
+  return ok();
+}
+
+mqv_status mqv_replay_unpack(const void* packed, int64_t rows, int64_t cols, int32_t fmt, void* codes,
+                             void* stream) {
+  mqv_status st = check_replay_view(rows, cols, fmt);
+  if (st) return st;
+  if (!packed || !aligned16(packed) || !codes || !aligned16(codes))
+    return fail(MQV_ERR_INVALID_ARG, "packed and codes must be 16-byte aligned pointers");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  const uint8_t* in = static_cast<const uint8_t*>(packed);
+  uint8_t* c = static_cast<uint8_t*>(codes);
+  if (fmt == MQV_NVFP4)
+    replay_unpack_kernel<0><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, n, c);
+  else
+    replay_unpack_kernel<1><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, n, c);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "replay unpack launch");
+  return ok();
+}
+
+mqv_status mqv_replay_dequantize(const void* packed, const uint8_t* scales, const float* tscale, int64_t rows,
+                                 int64_t cols, int32_t fmt, float* dst, void* stream) {
+  mqv_status st = check_replay_view(rows, cols, fmt);
+  if (st) return st;
+  if (!packed || !aligned16(packed) || !scales || !tscale || !dst || !aligned16(dst))
+    return fail(MQV_ERR_INVALID_ARG, "packed and dst must be 16-byte aligned, scales and tscale non-null");
+  if (reinterpret_cast<uintptr_t>(tscale) & 3u) return fail(MQV_ERR_INVALID_ARG, "tscale must be 4-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  const uint8_t* in = static_cast<const uint8_t*>(packed);
+  if (fmt == MQV_NVFP4)
+    replay_dequantize_kernel<0><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, n, dst);
+  else
+    replay_dequantize_kernel<1><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, n, dst);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "replay dequantize launch");
   return ok();
 }
 

@@ -127,6 +127,26 @@ def test_quantize_rejects_bad_arguments(lib):
     assert st == 1                                              # misaligned src
 
 
+@pytest.mark.parametrize("rows,cols,fmt,nbytes", [
+    (4, 4, mqv.NVFP4, 6), (4, 4, mqv.NVFP6, 10), (8, 16, mqv.NVFP4, 48),
+    (7 * 7 * 256, 84, mqv.NVFP4, 7 * 7 * 256 * 84 * 3 // 8)])
+def test_replay_bytes_are_magnitude_bits(lib, rows, cols, fmt, nbytes):
+    assert mqv.replay_bytes(rows, cols, fmt) == nbytes
+
+
+def test_replay_entry_points_reject_bad_arguments(lib):
+    q = mqv.QTensorC(16, 16, 16, 8, 8, 0, 0)
+    assert lib.mqv_replay_pack(ctypes.byref(q), None, None, None) == 1         # null output
+    assert lib.mqv_replay_pack(ctypes.byref(q), 8, None, None) == 1            # misaligned output
+    assert lib.mqv_replay_pack(ctypes.byref(q), 16, 2, None) == 1              # misaligned counter
+    bad = mqv.QTensorC(16, 16, 16, 6, 8, 0, 0)
+    assert lib.mqv_replay_pack(ctypes.byref(bad), 16, None, None) == 1         # rows not a multiple of 4
+    assert lib.mqv_replay_unpack(16, 8, 8, 2, 16, None) == 1                   # format
+    assert lib.mqv_replay_unpack(16, 8, 8, 0, 4, None) == 1                    # misaligned codes
+    assert lib.mqv_replay_dequantize(16, 16, None, 8, 8, 0, 16, None) == 1     # null tscale
+    assert lib.mqv_replay_dequantize(16, 16, 16, 8, 8, 0, 8, None) == 1        # misaligned dst
+
+
 def test_cuda_path_has_no_cpu_fallback():
     import torch
     x = torch.zeros(16)
