@@ -578,9 +578,9 @@ def run_sweeps(args, dev, peaks):
         RNE and SR; 8.5625 algorithmic B/element (two fp32 reads, codes,
         scales);
       - replay_form: the magnitude-only replay form of the same quantized
-        buffers: pack (0.5 B read + 0.375 B written per element) and values
-        read straight back (0.375 + 1/16 B read, 4 B written), beside
-        mqv_dequantize of the full codes;
+        buffers: pack and unpack (0.5 + 0.375 B moved per element) and
+        values read straight back (0.375 + 1/16 B read, 4 B written),
+        beside mqv_dequantize of the full codes;
       - resnet18_body and yolov8n_mix: every layer's step (quantize, fwd,
         wgrad, dgrad) timed phase by phase with L2 flushed before each
         phase; per-network sums against the sum of per-pass rooflines."""
@@ -619,7 +619,9 @@ def run_sweeps(args, dev, peaks):
         packed = torch.empty(mqv.replay_bytes(rows, cols, "nvfp4"), dtype=torch.uint8, device=dev)
         vals = torch.empty(n, dtype=torch.float32, device=dev)
         neg = torch.zeros(1, dtype=torch.int32, device=dev)
+        codes2 = torch.empty_like(q.codes)
         calls = {"pack": (lambda: mqv.replay_pack(q, out=packed, negatives=neg), 0.875),
+                 "unpack": (lambda: mqv.replay_unpack(packed, rows, cols, "nvfp4", codes=codes2), 0.875),
                  "read": (lambda: mqv.replay_dequantize(packed, q.scales, q.tscale, rows, cols, "nvfp4",
                                                         out=vals), 0.375 + 0.0625 + 4),
                  "dequantize_full_codes": (lambda: mqv.dequantize(q, out=vals), 0.5 + 0.0625 + 4)}
@@ -634,7 +636,7 @@ def run_sweeps(args, dev, peaks):
             fe[name] = {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)}
         fe["negative_codes"] = int(neg.item())
         rf.append(fe)
-        del q, ws, packed, vals
+        del q, ws, packed, vals, codes2
         torch.cuda.empty_cache()
     res["replay_quantize"] = rq
     res["replay_form"] = rf

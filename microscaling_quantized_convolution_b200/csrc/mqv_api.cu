@@ -700,8 +700,8 @@ mqv_status check_replay_view(int64_t rows, int64_t cols, int32_t fmt) {
 }
 
 unsigned replay_ctas(int64_t n) {
-  const int64_t runs = (n + kReplayRun - 1) / kReplayRun;
-  const int64_t g = (runs + kReplayThreads - 1) / kReplayThreads;
+  const int64_t segs = (n + kReplaySeg - 1) / kReplaySeg;
+  const int64_t g = (segs + kReplayWarps - 1) / kReplayWarps;
   return static_cast<unsigned>(g < kMaxQuantCtas ? g : kMaxQuantCtas);
 }
 
@@ -763,10 +763,11 @@ mqv_status mqv_replay_dequantize(const void* packed, const uint8_t* scales, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n = rows * cols;
   const uint8_t* in = static_cast<const uint8_t*>(packed);
+  const FastDiv dc4 = make_fastdiv(cols / 4);
   if (fmt == MQV_NVFP4)
-    replay_dequantize_kernel<0><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, n, dst);
+    replay_dequantize_kernel<0><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, dc4, n, dst);
   else
-    replay_dequantize_kernel<1><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, n, dst);
+    replay_dequantize_kernel<1><<<replay_ctas(n), kReplayThreads, 0, s>>>(in, scales, tscale, cols, dc4, n, dst);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "replay dequantize launch");
   return ok();
