@@ -548,6 +548,7 @@ def run_gpu(args):
         naive_res["quantize_time_ratio"] = round(naive_res["phase_ms"]["quant"] / mean["quantize"], 3)
         out["naive_baseline"] = naive_res
     if world == 1 and not args.no_sweeps:
+        out["fused_epilogue"] = run_fused(dev, layer, peaks)
         out["sweeps"] = run_sweeps(args, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(layer, budget_s=args.cpu_budget)
@@ -698,6 +699,76 @@ def run_sweeps(args, dev, peaks):
     if flags:
         raise SystemExit(f"device wait timeout flags {flags:#x} in the sweeps")
     res["launches"] = launches
+    return res
+
+
+def run_fused(dev, layer, peaks):
+    """Producer epilogue fused with the next quantization's max pass, on the
+    benchmarked layer: fwd writes ReLU(Y) and max|Y| and the next layer's
+    X = ReLU(Y) is quantized in one pass (mqv_quantize_with_amax), against
+    the plain chain fwd, ReLU written back, amax pass, quantize pass; and
+    dgrad with max|G_X| fused, then the SR quantization of G_X, against
+    dgrad, amax pass, quantize pass.  Each chain is timed whole, L2 flushed
+    before each call."""
+    import torch
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    X, Wt, G = (t.view(-1) for t in workloads.make_layer_inputs(layer, device=dev))
+    d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+    fmt = layer.fmt
+    xr, xc = layer.H * layer.W * layer.Cin, layer.N
+    wr, wc = layer.Cout, layer.K * layer.K * layer.Cin
+    yr = layer.Ho * layer.Wo * layer.Cout
+    qx = mqv.quantize(X, xr, xc, fmt, mqv.RNE)
+    qw = mqv.quantize(Wt, wr, wc, fmt, mqv.RNE)
+    qg = mqv.quantize(G, yr, xc, fmt, mqv.SR, 3)
+    y = torch.empty(yr * xc, device=dev)
+    gx = torch.empty(xr * xc, device=dev)
+    amax = torch.empty(1, device=dev)
+    qy = mqv.QTensor.empty(yr, xc, fmt, dev)
+    qgx = mqv.QTensor.empty(xr, xc, fmt, dev)
+    wsf = torch.empty(max(16, mqv.conv_workspace_bytes(d, mqv.OP_FWD)), dtype=torch.uint8, device=dev)
+    wsd = torch.empty(max(16, mqv.conv_workspace_bytes(d, mqv.OP_DGRAD)), dtype=torch.uint8, device=dev)
+    wsy = torch.empty(mqv.quantize_workspace_bytes(yr, xc), dtype=torch.uint8, device=dev)
+    wsx = torch.empty(mqv.quantize_workspace_bytes(xr, xc), dtype=torch.uint8, device=dev)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+
+    def fwd_plain():
+        mqv.conv_fwd(d, qw, qx, y=y, ws=wsf)
+        torch.relu_(y)
+        mqv.quantize(y, yr, xc, fmt, mqv.RNE, 0, out=qy, ws=wsy)
+
+    def fwd_fused():
+        mqv.conv_fwd_fused(d, qw, qx, relu=True, y=y, y_amax=amax, ws=wsf)
+        mqv.quantize_with_amax(y, yr, xc, fmt, mqv.RNE, 0, amax, out=qy)
+
+    def dgrad_plain():
+        mqv.conv_dgrad(d, qw, qg, gx=gx, ws=wsd)
+        mqv.quantize(gx, xr, xc, fmt, mqv.SR, 4, out=qgx, ws=wsx)
+
+    def dgrad_fused():
+        mqv.conv_dgrad_fused(d, qw, qg, gx=gx, gx_amax=amax, ws=wsd)
+        mqv.quantize_with_amax(gx, xr, xc, fmt, mqv.SR, 4, amax, out=qgx)
+
+    res = {"layer": layer.name, "l2": "256 MB written before every timed chain"}
+    for name, fn in (("fwd_relu_quantize", (fwd_plain, fwd_fused)), ("dgrad_quantize", (dgrad_plain, dgrad_fused))):
+        plain, fused = fn
+        for f in (plain, fused):
+            for _ in range(3):
+                f()
+        tp = _timed(torch, plain, 50, flush)
+        tf = _timed(torch, fused, 50, flush)
+        res[name] = {"plain_ms": round(tp, 5), "fused_ms": round(tf, 5), "speedup": round(tp / tf, 3)}
+    ne = yr * xc
+    res["fwd_relu_quantize"]["note"] = ("plain: conv writes Y, a ReLU pass reads and writes it, an amax pass "
+                                        "reads it, the quantizer reads it; fused: conv writes ReLU(Y) and its "
+                                        "max, the quantizer reads it once")
+    res["fwd_relu_quantize"]["bytes_removed"] = 12 * ne
+    res["dgrad_quantize"]["bytes_removed"] = 4 * xr * xc
+    flags = mqv.device_errors()
+    if flags:
+        raise SystemExit(f"device wait timeout flags {flags:#x} in the fused chains")
     return res
 
 

@@ -236,6 +236,29 @@ mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
 mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
                           float* gx, void* ws, size_t ws_bytes, void* stream);
 
+/* Forward pass with the next quantization's first step fused into its
+ * epilogue.  Quantize-once needs the global max|x| of a tensor before any
+ * block can be scaled (section "무엇과 다른가": T = max|X| / (448·emax)); the
+ * tensor the next layer quantizes is this pass's output, so the epilogue
+ * that writes it can also reduce it, and the separate max pass (a full fp32
+ * read) disappears.  Outputs as mqv_conv_fwd, plus:
+ *   relu   0: y as mqv_conv_fwd; 1: y = max(conv, 0) (-0 and NaN become +0),
+ *          the next layer's post-ReLU input X.
+ *   y_amax NULL, or a device fp32 that receives max|y| over the stored
+ *          values (exactly what mqv_amax of y would return).  The call
+ *          enqueues a 4-byte clear of it, then the kernels' atomic updates;
+ *          read it after the stream reaches that point.  Feed it to
+ *          mqv_quantize_with_amax to quantize y in one pass with codes
+ *          bit-identical to mqv_quantize_cbf of y. */
+mqv_status mqv_conv_fwd_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x, float* y,
+                              int32_t relu, float* y_amax, void* ws, size_t ws_bytes, void* stream);
+
+/* Input-gradient pass with max|gx| fused into its epilogue (gx_amax as
+ * y_amax above); gx is the G_Y of the layer before, which the backward pass
+ * quantizes next with stochastic rounding. */
+mqv_status mqv_conv_dgrad_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy, float* gx,
+                                float* gx_amax, void* ws, size_t ws_bytes, void* stream);
+
 /* The baseline the method removes (section "무엇인가": quantize after the
  * im2col expansion, once per GEMM direction), for measuring it on the same
  * kernels.  Explicit im2col of fp32 X [H][W][Cin][N] into

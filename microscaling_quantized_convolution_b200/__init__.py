@@ -94,6 +94,12 @@ _SIGS = {
                                               ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_im2col": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_col2im": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_conv_fwd_fused": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                          ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_int32,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_dgrad_fused": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                            ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_replay_bytes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
                                         ctypes.POINTER(ctypes.c_size_t)]),
     "mqv_replay_pack": (ctypes.c_int, [ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
@@ -386,6 +392,40 @@ def conv_dgrad(d: ConvDesc, w: QTensor, gy: QTensor, gx: torch.Tensor | None = N
     _check(lib().mqv_conv_dgrad(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(gc), gx.data_ptr(),
                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return gx
+
+
+def conv_fwd_fused(d: ConvDesc, w: QTensor, x: QTensor, relu: bool = False, y: torch.Tensor | None = None,
+                   y_amax: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                   stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """conv_fwd with optional ReLU and max|y| fused into the epilogue (see
+    mqv_conv_fwd_fused); returns (y, y_amax), y_amax a device fp32 scalar."""
+    Ho, Wo = out_hw(d)
+    dev = x.codes.device
+    y = y if y is not None else torch.empty((Ho, Wo, d.Cout, d.N), dtype=torch.float32, device=dev)
+    y_amax = y_amax if y_amax is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    _require_cuda(y_amax, "y_amax", torch.float32)
+    ws = _ws(d, OP_FWD, ws, dev)
+    wc, xc = w.c(), x.c()
+    _check(lib().mqv_conv_fwd_fused(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), y.data_ptr(),
+                                    1 if relu else 0, y_amax.data_ptr(), _ptr(ws),
+                                    0 if ws is None else ws.numel(), _stream(stream)))
+    return y, y_amax
+
+
+def conv_dgrad_fused(d: ConvDesc, w: QTensor, gy: QTensor, gx: torch.Tensor | None = None,
+                     gx_amax: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """conv_dgrad with max|gx| fused into the epilogue; returns (gx, gx_amax)."""
+    dev = gy.codes.device
+    gx = gx if gx is not None else torch.empty((d.H, d.W, d.Cin, d.N), dtype=torch.float32, device=dev)
+    gx_amax = gx_amax if gx_amax is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    _require_cuda(gx_amax, "gx_amax", torch.float32)
+    ws = _ws(d, OP_DGRAD, ws, dev)
+    wc, gc = w.c(), gy.c()
+    _check(lib().mqv_conv_dgrad_fused(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(gc), gx.data_ptr(),
+                                      gx_amax.data_ptr(), _ptr(ws), 0 if ws is None else ws.numel(),
+                                      _stream(stream)))
+    return gx, gx_amax
 
 
 def conv_wgrad_noalloc(d: ConvDesc, gy: QTensor, x: QTensor, gw: torch.Tensor | None = None,

@@ -477,7 +477,7 @@ mqv_status check_operand(const mqv_qtensor* q, const char* name, int64_t rows, i
 
 mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const char* na,
                     const mqv_qtensor* qb, const char* nb, float* out, void* ws, size_t ws_bytes,
-                    void* stream) {
+                    void* stream, int32_t relu = 0, float* amax = nullptr) {
   mqv_status st = check_desc(d);
   if (st) return st;
   const int64_t Ho = (d->H + 2 * d->pad - d->Kh) / d->stride + 1;
@@ -492,6 +492,9 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
     if ((st = check_operand(qa, na, wr, wc, d->fmt)) || (st = check_operand(qb, nb, gr, d->N, d->fmt))) return st;
   }
   if (!out || !aligned16(out)) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
+  if (relu != 0 && relu != 1) return fail(MQV_ERR_INVALID_ARG, "relu must be 0 or 1");
+  if (amax && (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
   ConvPlan pl;
   plan_conv(d, op, &pl);
   if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)))
@@ -522,6 +525,12 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
     return ok();
   }
   // fwd / dgrad: qa is W, qb is X (fwd) or G_Y (dgrad)
+  if (amax) {
+    e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax clear");
+  }
+  pl.a.relu = relu;
+  pl.a.amax_out = reinterpret_cast<uint32_t*>(amax);
   e = launch_prep(op, d->fmt, pl, make_view(qa), wsb, s);
   if (e != cudaSuccess) return cuda_fail(e, "operand image launch");
   pl.a.image = wsb;
@@ -798,6 +807,16 @@ mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const m
 mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
                           float* gx, void* ws, size_t ws_bytes, void* stream) {
   return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", gx, ws, ws_bytes, stream);
+}
+
+mqv_status mqv_conv_fwd_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x, float* y,
+                              int32_t relu, float* y_amax, void* ws, size_t ws_bytes, void* stream) {
+  return run_conv(MQV_OP_FWD, d, w, "w", x, "x", y, ws, ws_bytes, stream, relu, y_amax);
+}
+
+mqv_status mqv_conv_dgrad_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy, float* gx,
+                                float* gx_amax, void* ws, size_t ws_bytes, void* stream) {
+  return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", gx, ws, ws_bytes, stream, 0, gx_amax);
 }
 
 mqv_status mqv_device_errors(uint32_t* flags, void* stream) {

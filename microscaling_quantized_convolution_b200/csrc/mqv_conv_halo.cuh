@@ -185,6 +185,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
     // epilogue: column lc of the tile = (pixel j, batch item n) -> output
     // pixel (oh, ow0 + j), skipped past the end of the output row.
     int it = 0;
+    float amax = 0.f;
     const uint32_t wbuf = sbase + L::kEpiOffset + warp * 4096;
     const int rsub = lane >> 3, q = lane & 7;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
@@ -227,8 +228,12 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
           for (int i = 0; i < 8; ++i) {
             const int row = 4 * i + rsub;
             const int64_t mrow = static_cast<int64_t>(mt) * 128 + warp * 32 + row;
-            const float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
-            if (mrow < p.M) *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
+            float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+            if (mrow < p.M) {
+              if (p.relu) o = epi_relu(o);
+              amax = epi_absmax(amax, o);
+              *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
+            }
           }
         }
         __syncwarp();
@@ -236,6 +241,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
     }
+    epi_amax_flush(p.amax_out, amax);
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
       // The issuing thread's own instructions sit on the critical path of

@@ -66,6 +66,11 @@ struct V2Args {
   int mtiles, ntiles;
   int tiles;              // mtiles * ntiles * splits
   int scale_out;          // multiply by T_a·T_b (0 for wgrad split partials)
+  // Fused producer epilogue (fwd/dgrad only): relu != 0 stores max(v, 0);
+  // amax_out != nullptr receives max|stored value| as fp32 bits through
+  // atomicMax (non-negative floats order like their bit patterns).
+  uint32_t* amax_out;
+  int relu;
   FastDiv dN, dWo, dW, dCred, dKw, dCin, dS;
 };
 
@@ -283,9 +288,30 @@ __device__ __forceinline__ void v2_teardown(V2Bars* bars) {
 // Epilogue of one tile: TMEM accumulator buffer `acc` -> fp32 output.
 // FD=true: out[(pixel·M + m)·N + n] with col = pixel·N + n;
 // FD=false (wgrad): out[(split·M + m)·Ncols + col].
+// ReLU that maps -0 and NaN to +0, and the running max of |v|.
+__device__ __forceinline__ float4 epi_relu(float4 o) {
+  o.x = o.x > 0.f ? o.x : 0.f;
+  o.y = o.y > 0.f ? o.y : 0.f;
+  o.z = o.z > 0.f ? o.z : 0.f;
+  o.w = o.w > 0.f ? o.w : 0.f;
+  return o;
+}
+
+__device__ __forceinline__ float epi_absmax(float m, float4 o) {
+  return fmaxf(m, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+}
+
+// One atomic per warp: the warp's largest |v| into *amax_out.
+__device__ __forceinline__ void epi_amax_flush(uint32_t* amax_out, float m) {
+  if (amax_out == nullptr) return;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_out, __float_as_uint(m));
+}
+
 template <int BN, bool FD>
 __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int acc, int64_t m0,
-                                            int64_t col0, int split, bool has_k) {
+                                            int64_t col0, int split, bool has_k, float& amax) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m = m0 + warp * 32 + lane;
   const float scale = p.scale_out ? __fmul_rn(*p.ta, *p.tb) : 1.0f;
@@ -307,6 +333,8 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
         o.w = has_k ? __uint_as_float(r[4 * j + 3]) * scale : 0.f;
         int64_t idx;
         if (FD) {
+          if (p.relu) o = epi_relu(o);
+          amax = epi_absmax(amax, o);
           const int64_t pix = col / p.N;
           idx = (pix * p.M + m) * p.N + (col - pix * p.N);
         } else {
@@ -470,14 +498,16 @@ conv_fd_kernel(const V2Args p) {
 
   if (warp < kV2EpiWarps) {
     int it = 0;
+    float amax = 0.f;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const int mt = tile / p.ntiles, nt = tile - mt * p.ntiles;
       v2_epilogue<BN, true>(p, bars, acc, static_cast<int64_t>(mt) * 128,
-                            static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0);
+                            static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0, amax);
     }
+    epi_amax_flush(p.amax_out, amax);
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32_bmn(128, BN);
@@ -688,8 +718,9 @@ conv_wg_kernel(const V2Args p) {
       const bool has_k = min(p.ktiles, kt0 + p.kt_per_split) > kt0;
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
+      float unused = 0.f;
       v2_epilogue<BN, false>(p, bars, acc, static_cast<int64_t>(mt) * 128,
-                             static_cast<int64_t>(nt) * BN, sp, has_k);
+                             static_cast<int64_t>(nt) * BN, sp, has_k, unused);
     }
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {

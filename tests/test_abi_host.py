@@ -147,6 +147,19 @@ def test_replay_entry_points_reject_bad_arguments(lib):
     assert lib.mqv_replay_dequantize(16, 16, 16, 8, 8, 0, 8, None) == 1        # misaligned dst
 
 
+def test_fused_passes_reject_bad_epilogue_arguments(lib):
+    d = mqv.conv_desc(64, 128, 128, 28, 28, 3, 3, 1, 1, "nvfp4")
+    w = mqv.QTensorC(16, 16, 16, 128, 1152, 0, 0)
+    x = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, 0)
+    ws = mqv.conv_workspace_bytes(d, mqv.OP_FWD)
+    st = lib.mqv_conv_fwd_fused(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 2, None, 16, ws, None)
+    assert st == 1                                              # relu must be 0 or 1
+    st = lib.mqv_conv_fwd_fused(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 1, 18, 16, ws, None)
+    assert st == 1                                              # misaligned amax
+    st = lib.mqv_conv_dgrad_fused(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 18, 16, ws, None)
+    assert st == 1                                              # misaligned gx_amax
+
+
 def test_cuda_path_has_no_cpu_fallback():
     import torch
     x = torch.zeros(16)
