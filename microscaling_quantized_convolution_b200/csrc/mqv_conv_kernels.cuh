@@ -316,8 +316,10 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
   const int64_t m = m0 + warp * 32 + lane;
   const float scale = p.scale_out ? __fmul_rn(*p.ta, *p.tb) : 1.0f;
   const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * BN;
+  // a warp whose 32 accumulator rows all lie past the M channels has nothing to store
+  const int cend = m0 + warp * 32 < p.M ? BN : 0;
 #pragma unroll 1
-  for (int c = 0; c < BN; c += 32) {
+  for (int c = 0; c < cend; c += 32) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(tbase + c, r);
     tmem_ld_wait();
@@ -335,8 +337,9 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
         if (FD) {
           if (p.relu) o = epi_relu(o);
           amax = epi_absmax(amax, o);
-          const int64_t pix = col / p.N;
-          idx = (pix * p.M + m) * p.N + (col - pix * p.N);
+          const int c32 = static_cast<int>(col);           // GEMM columns stay below 2^31
+          const int pix = fdiv(c32, p.dN);
+          idx = (static_cast<int64_t>(pix) * p.M + m) * p.N + (c32 - pix * p.N);
         } else {
           idx = (static_cast<int64_t>(split) * p.M + m) * p.Ncols + col;
         }
