@@ -200,6 +200,7 @@ struct ConvPlan {
   HaloGeom g;
   bool wgk;             // stride-1 wgrad with the taps of a kernel row sharing operands
   WgkGeom wg;
+  bool tr;              // generic fwd/dgrad on transposed tiles (M <= 128)
   int bn;               // 128 or 256 columns per tile
   int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0
   int grid;             // persistent CTAs
@@ -279,10 +280,16 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   a.dCin = make_fastdiv(a.Cin);
   a.dS = make_fastdiv(a.stride);
   pl->nu = (d->N % 8 == 0) ? 8 : 4;
+  // Generic fwd/dgrad with at most 128 output channels: transposed tiles,
+  // 128 GEMM columns x the channels rounded up to 16, so the MMA does no
+  // work on absent channels and every column's channels are stored by one
+  // lane.
+  pl->tr = op != MQV_OP_WGRAD && a.M <= 128;
+  a.nc = pl->tr ? (a.M + 15) / 16 * 16 : 0;
   // Columns per tile: the option with the smaller (waves x tile width) over
   // one persistent CTA per SM; ties go to the wider tile.
   auto waves = [&](int bn) { return ((a.Ncols + bn - 1) / bn * a.mtiles + kSMs - 1) / kSMs; };
-  pl->bn = waves(256) * 256 <= waves(128) * 128 ? 256 : 128;
+  pl->bn = pl->tr ? 128 : (waves(256) * 256 <= waves(128) * 128 ? 256 : 128);
   a.ntiles = (int)((a.Ncols + pl->bn - 1) / pl->bn);
   const int64_t tiles_mn = (int64_t)a.ntiles * a.mtiles;
   int splits = 1;
@@ -380,9 +387,9 @@ cudaError_t set_smem(K kern, int bytes, bool (&done)[kMaxDevices]) {
   return cudaSuccess;
 }
 
-template <int PASS, int FMT, int BN, int NU>
+template <int PASS, int FMT, int BN, int NU, bool TR>
 cudaError_t launch_fd(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_fd_kernel<PASS, FMT, BN, NU>;
+  auto kern = conv_fd_kernel<PASS, FMT, BN, NU, TR>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, V2Smem<BN>::kBytes, done);
   if (e != cudaSuccess) return e;
@@ -407,8 +414,10 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
     return pl.nu == 8 ? launch_wg<FMT, 128, 8>(pl, st) : launch_wg<FMT, 128, 4>(pl, st);
   }
   constexpr int P = PASS == kWgrad ? kFwd : PASS;
-  if (pl.bn == 256) return pl.nu == 8 ? launch_fd<P, FMT, 256, 8>(pl, st) : launch_fd<P, FMT, 256, 4>(pl, st);
-  return pl.nu == 8 ? launch_fd<P, FMT, 128, 8>(pl, st) : launch_fd<P, FMT, 128, 4>(pl, st);
+  if (pl.tr) return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, true>(pl, st) : launch_fd<P, FMT, 128, 4, true>(pl, st);
+  if (pl.bn == 256)
+    return pl.nu == 8 ? launch_fd<P, FMT, 256, 8, false>(pl, st) : launch_fd<P, FMT, 256, 4, false>(pl, st);
+  return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, false>(pl, st) : launch_fd<P, FMT, 128, 4, false>(pl, st);
 }
 
 template <int PASS>

@@ -71,6 +71,10 @@ struct V2Args {
   // atomicMax (non-negative floats order like their bit patterns).
   uint32_t* amax_out;
   int relu;
+  // Transposed tiles of the generic fwd/dgrad kernel (TR): the MMA's 128
+  // rows are GEMM columns (pixel, n) and its N = nc (M rounded up to 16)
+  // columns are the output channels.
+  int nc;
   FastDiv dN, dWo, dW, dCred, dKw, dCin, dS;
 };
 
@@ -351,6 +355,44 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
   mbar_arrive(&bars->acc_empty[acc]);
 }
 
+// Epilogue of a transposed tile: TMEM lane = GEMM column (pixel, n), TMEM
+// column = output channel.  Each lane stores its column's channels one by
+// one; for one channel the 32 lanes of a warp write consecutive batch items,
+// so every store of a warp covers runs of N contiguous floats.
+template <int BN>
+__device__ __forceinline__ void v2_epilogue_tr(const V2Args& p, V2Bars* bars, int acc, int64_t col0,
+                                               float& amax) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t col = col0 + warp * 32 + lane;
+  const bool ok = col < p.Ncols;
+  const int c32 = ok ? static_cast<int>(col) : 0;     // GEMM columns stay below 2^31
+  const int pix = fdiv(c32, p.dN);
+  float* out = p.out + static_cast<int64_t>(pix) * p.M * p.N + (c32 - pix * p.N);
+  const float scale = __fmul_rn(*p.ta, *p.tb);
+  const bool has_k = p.ktiles > 0;
+  const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * BN;
+#pragma unroll 1
+  for (int c = 0; c < p.nc; c += 16) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(tbase + c, r);
+    tmem_ld_wait();
+    if (ok) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int m = c + j;
+        if (m < p.M) {
+          float v = has_k ? __uint_as_float(r[j]) * scale : 0.f;
+          if (p.relu) v = v > 0.f ? v : 0.f;
+          amax = fmaxf(amax, fabsf(v));
+          out[static_cast<int64_t>(m) * p.N] = v;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  mbar_arrive(&bars->acc_empty[acc]);
+}
+
 // ---------------------------------------------------------------------------
 // Raw codes of one producer unit: 4 view rows (consecutive channels) x NU
 // consecutive batch items, plus the one or two E4M3 scales that cover them.
@@ -489,9 +531,12 @@ __device__ __forceinline__ void producer_warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-template <int PASS, int FMT, int BN, int NU>
+// TR: transposed tiles (M <= 128 output channels as the MMA's N, BN = 128
+// GEMM columns as its M); otherwise 128 output channels x BN columns.
+template <int PASS, int FMT, int BN, int NU, bool TR>
 __global__ void __launch_bounds__(kV2Threads, 1)
 conv_fd_kernel(const V2Args p) {
+  static_assert(!TR || BN == 128, "transposed tiles are 128 GEMM columns");
   using L = V2Smem<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -507,13 +552,17 @@ conv_fd_kernel(const V2Args p) {
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const int mt = tile / p.ntiles, nt = tile - mt * p.ntiles;
-      v2_epilogue<BN, true>(p, bars, acc, static_cast<int64_t>(mt) * 128,
-                            static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0, amax);
+      if (TR)
+        v2_epilogue_tr<BN>(p, bars, acc, static_cast<int64_t>(nt) * BN, amax);
+      else
+        v2_epilogue<BN, true>(p, bars, acc, static_cast<int64_t>(mt) * 128,
+                              static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0, amax);
     }
     epi_amax_flush(p.amax_out, amax);
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32_bmn(128, BN);
+      // TR: the gathered MN-major tile is the A operand, the weight rows B
+      const uint32_t idesc = TR ? idesc_f16_f32_amn(128, p.nc) : idesc_f16_f32_bmn(128, BN);
       int it = 0, kit = 0;
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
@@ -525,11 +574,15 @@ conv_fd_kernel(const V2Args p) {
           mbar_wait_bounded(&bars->full[s], (kit / kV2Stages) & 1, p.err, kErrWaitFull);
           tc_fence_after();
           const uint32_t a_tile = sbase + s * L::kStage;
-          const uint64_t adesc = smem_desc_sw128(a_tile);
-          const uint64_t bdesc = smem_desc_sw128_mn(a_tile + kATileBytes, 8192, 1024);
+          const uint64_t wdesc = smem_desc_sw128(a_tile);
+          const uint64_t gdesc = smem_desc_sw128_mn(a_tile + kATileBytes, 8192, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ss(dt, adesc + 2 * kk, bdesc + 128 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            if (TR)
+              mma_f16_ss(dt, gdesc + 128 * kk, wdesc + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_f16_ss(dt, wdesc + 2 * kk, gdesc + 128 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&bars->empty[s]);
         }
         mma_commit(&bars->acc_full[acc]);
@@ -541,12 +594,14 @@ conv_fd_kernel(const V2Args p) {
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
         const int mt = tile / p.ntiles;
         const uint8_t* src = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
+        // TR: only the first nc rows (128 B each) of a weight tile are used
+        const uint32_t bytes = TR ? static_cast<uint32_t>(p.nc) * 128u : kATileBytes;
         for (int kt = 0; kt < p.ktiles; ++kt, ++kit) {
           const int s = kit % kV2Stages;
           mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
-          mbar_arrive_expect_tx(&bars->full[s], kATileBytes);
-          bulk_copy_g2s(sbase + s * L::kStage, src + static_cast<int64_t>(kt) * kATileBytes,
-                        kATileBytes, &bars->full[s]);
+          mbar_arrive_expect_tx(&bars->full[s], bytes);
+          bulk_copy_g2s(sbase + s * L::kStage, src + static_cast<int64_t>(kt) * kATileBytes, bytes,
+                        &bars->full[s]);
         }
       }
     }

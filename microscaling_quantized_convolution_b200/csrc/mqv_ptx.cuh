@@ -255,6 +255,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// Instruction descriptor: kind::f16, A = B = fp16, D = fp32, A MN-major
+// (bit 15), B K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_amn(int M, int N) {
+  return (1u << 4) | (1u << 15) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Instruction descriptor: kind::f16, A = B = fp16, D = fp32, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
