@@ -389,11 +389,14 @@ cudaError_t set_smem(K kern, int bytes, bool (&done)[kMaxDevices]) {
 
 template <int PASS, int FMT, int BN, int NU, bool TR>
 cudaError_t launch_fd(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_fd_kernel<PASS, FMT, BN, NU, TR>;
+  // two producer groups where the register budget allows it (transposed
+  // tiles with 8-item units)
+  constexpr int kGr = TR && NU == 8 ? 2 : 1;
+  auto kern = conv_fd_kernel<PASS, FMT, BN, NU, TR, kGr>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, V2Smem<BN>::kBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<pl.grid, kV2Threads, V2Smem<BN>::kBytes, st>>>(pl.a);
+  kern<<<pl.grid, fd_threads(kGr), V2Smem<BN>::kBytes, st>>>(pl.a);
   return cudaGetLastError();
 }
 

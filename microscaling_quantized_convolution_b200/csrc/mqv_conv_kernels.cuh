@@ -531,10 +531,16 @@ __device__ __forceinline__ void producer_warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// Threads of conv_fd_kernel with GR producer groups.
+__host__ __device__ constexpr int fd_threads(int gr) { return kV2ProdWarp0 * 32 + gr * kV2ProdThreads; }
+
 // TR: transposed tiles (M <= 128 output channels as the MMA's N, BN = 128
 // GEMM columns as its M); otherwise 128 output channels x BN columns.
-template <int PASS, int FMT, int BN, int NU, bool TR>
-__global__ void __launch_bounds__(kV2Threads, 1)
+// GR producer groups of 8 warps take turns: group g fills the K iterations
+// g, g + GR, ... so that GR times as many gathers are in flight (GR = 2
+// needs at most 88 registers a thread).
+template <int PASS, int FMT, int BN, int NU, bool TR, int GR>
+__global__ void __launch_bounds__(fd_threads(GR), 1)
 conv_fd_kernel(const V2Args p) {
   static_assert(!TR || BN == 128, "transposed tiles are 128 GEMM columns");
   using L = V2Smem<BN>;
@@ -610,7 +616,9 @@ conv_fd_kernel(const V2Args p) {
     // stage i is stored, so each load has kLookahead stages of work (and of
     // waiting for free stages) to arrive in.  The ring of raw registers is
     // indexed at compile time (unrolled by kLookahead).
-    const int t = threadIdx.x - kV2ProdWarp0 * 32;
+    const int tg = threadIdx.x - kV2ProdWarp0 * 32;
+    const int grp = tg / kV2ProdThreads;      // producer group
+    const int t = tg - grp * kV2ProdThreads;
     const int total = p.ktiles * ((p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                                   static_cast<int>(gridDim.x));
     using Prod = FdProducer<PASS, FMT, BN, NU>;
@@ -620,31 +628,39 @@ conv_fd_kernel(const V2Args p) {
     uint32_t* ktab = nullptr;
     if (p.ktiles * 16 <= kKtabEntries) {
       ktab = reinterpret_cast<uint32_t*>(smem + L::kKtabOffset);
-      for (int e = t; e < p.ktiles * 16; e += kV2ProdThreads) ktab[e] = ktab_entry<PASS>(p, e >> 4, e & 15);
-      asm volatile("bar.sync 1, %0;" ::"n"(kV2ProdThreads) : "memory");
+      for (int e = tg; e < p.ktiles * 16; e += GR * kV2ProdThreads) ktab[e] = ktab_entry<PASS>(p, e >> 4, e & 15);
+      asm volatile("bar.sync 1, %0;" ::"n"(GR * kV2ProdThreads) : "memory");
     }
-    int ltile = blockIdx.x, lkt = 0;          // load cursor
+    // load cursor at this group's first K iteration (p.ktiles >= 1)
+    int ltile = blockIdx.x, lkt = grp;
+    while (lkt >= p.ktiles) {
+      lkt -= p.ktiles;
+      ltile += gridDim.x;
+    }
     TileCol tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
     auto load_next = [&](Prod& pr) {
       pr.load(p, tc, lkt, t, ktab);
-      if (++lkt == p.ktiles) {
-        lkt = 0;
+      lkt += GR;
+      bool moved = false;
+      while (lkt >= p.ktiles) {
+        lkt -= p.ktiles;
         ltile += gridDim.x;
-        tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
+        moved = true;
       }
+      if (moved) tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
     };
 #pragma unroll
     for (int r = 0; r < kLookahead; ++r)
-      if (r < total) load_next(ring[r]);
-    for (int kit = 0; kit < total;) {
+      if (grp + r * GR < total) load_next(ring[r]);
+    for (int kit = grp; kit < total;) {
 #pragma unroll
-      for (int r = 0; r < kLookahead; ++r, ++kit) {
+      for (int r = 0; r < kLookahead; ++r, kit += GR) {
         if (kit >= total) break;
         const int s = kit % kV2Stages;
         mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
         ring[r].store(sbase + s * L::kStage + kATileBytes, t);
         producer_warp_arrive(&bars->full[s]);
-        if (kit + kLookahead < total) load_next(ring[r]);
+        if (kit + kLookahead * GR < total) load_next(ring[r]);
       }
     }
   }
