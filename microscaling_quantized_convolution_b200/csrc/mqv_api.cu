@@ -4,6 +4,7 @@
 // arguments and enqueues launches on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -291,6 +292,49 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   auto waves = [&](int bn) { return ((a.Ncols + bn - 1) / bn * a.mtiles + kSMs - 1) / kSMs; };
   pl->bn = pl->tr ? 128 : (waves(256) * 256 <= waves(128) * 128 ? 256 : 128);
   a.ntiles = (int)((a.Ncols + pl->bn - 1) / pl->bn);
+  a.phases = 1;
+  a.ph_tile0[0] = 0;
+  a.ph_tile0[1] = a.ntiles;
+  a.ph_cols[0] = a.Ncols;
+  a.ph_nlive[0] = a.ktiles;
+  if (op == MQV_OP_DGRAD && d->stride == 2 && a.ktiles <= kMaxLiveWords * 32 && a.Cred >= 32) {
+    // Stride-2 input gradient: group the columns by (hi mod 2, wi mod 2); a
+    // K tile is live for a phase when one of its taps (kh, kw) satisfies
+    // hi + pad - kh = 0 and wi + pad - kw = 0 (mod 2).  With fewer than 32
+    // reduction channels a K tile spans four or more taps, most stay live,
+    // and the grouping measured slower (16 channels: 0.52 -> 0.71 ms on the
+    // 640 px stem), so it is kept to 32 and more.
+    a.phases = kMaxPhases;
+    int t0 = 0;
+    for (int q = 0; q < kMaxPhases; ++q) {
+      const int ph = q >> 1, pw = q & 1;
+      const int hp = a.H > ph ? (a.H - ph + 1) / 2 : 0;
+      const int wp = a.W > pw ? (a.W - pw + 1) / 2 : 0;
+      a.ph_h0[q] = ph;
+      a.ph_w0[q] = pw;
+      a.ph_wp[q] = wp;
+      a.ph_dwp[q] = make_fastdiv(wp > 0 ? wp : 1);
+      a.ph_cols[q] = (int64_t)hp * wp * a.N;
+      a.ph_tile0[q] = t0;
+      t0 += (int)((a.ph_cols[q] + pl->bn - 1) / pl->bn);
+      int nlive = 0;
+      for (int kt = 0; kt < a.ktiles; ++kt) {
+        const int64_t k0 = (int64_t)kt * 64, k1 = std::min<int64_t>(k0 + 63, a.Kdim - 1);
+        bool live = false;
+        for (int64_t tap = k0 / a.Cred; tap <= k1 / a.Cred && !live; ++tap) {
+          const int kh = (int)(tap / a.Kw), kw = (int)(tap % a.Kw);
+          live = ((ph + a.pad - kh) & 1) == 0 && ((pw + a.pad - kw) & 1) == 0;
+        }
+        if (live) {
+          a.ph_live[q][kt >> 5] |= 1u << (kt & 31);
+          ++nlive;
+        }
+      }
+      a.ph_nlive[q] = nlive;
+    }
+    a.ph_tile0[kMaxPhases] = t0;
+    a.ntiles = t0;
+  }
   const int64_t tiles_mn = (int64_t)a.ntiles * a.mtiles;
   int splits = 1;
   if (op == MQV_OP_WGRAD) {
@@ -387,17 +431,24 @@ cudaError_t set_smem(K kern, int bytes, bool (&done)[kMaxDevices]) {
   return cudaSuccess;
 }
 
-template <int PASS, int FMT, int BN, int NU, bool TR>
-cudaError_t launch_fd(const ConvPlan& pl, cudaStream_t st) {
+template <int PASS, int FMT, int BN, int NU, bool TR, bool PH>
+cudaError_t launch_fd_ph(const ConvPlan& pl, cudaStream_t st) {
   // two producer groups where the register budget allows it (transposed
   // tiles with 8-item units)
   constexpr int kGr = TR && NU == 8 ? 2 : 1;
-  auto kern = conv_fd_kernel<PASS, FMT, BN, NU, TR, kGr>;
+  auto kern = conv_fd_kernel<PASS, FMT, BN, NU, TR, kGr, PH>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, V2Smem<BN>::kBytes, done);
   if (e != cudaSuccess) return e;
   kern<<<pl.grid, fd_threads(kGr), V2Smem<BN>::kBytes, st>>>(pl.a);
   return cudaGetLastError();
+}
+
+// Stride-2 input gradients run with their columns grouped by phase.
+template <int PASS, int FMT, int BN, int NU, bool TR>
+cudaError_t launch_fd(const ConvPlan& pl, cudaStream_t st) {
+  if (PASS == kDgrad && pl.a.phases > 1) return launch_fd_ph<kDgrad, FMT, BN, NU, TR, true>(pl, st);
+  return launch_fd_ph<PASS, FMT, BN, NU, TR, false>(pl, st);
 }
 
 template <int FMT, int BN, int NU>

@@ -46,6 +46,8 @@ constexpr int kV2ProdThreads = 256;
 constexpr int kV2Threads = (kV2ProdWarp0 + kV2ProdThreads / 32) * 32;   // 448
 constexpr int kV2Stages = 4;
 constexpr uint32_t kATileBytes = 128 * 64 * 2;                             // 16 KB
+constexpr int kMaxPhases = 4;             // stride-2 input gradient: (hi mod 2, wi mod 2)
+constexpr int kMaxLiveWords = 8;          // live-K-tile masks cover up to 256 K tiles
 
 struct V2Args {
   const uint8_t* image;   // fwd/dgrad: A image [mtiles][ktiles] x 16 KB
@@ -76,7 +78,57 @@ struct V2Args {
   // columns are the output channels.
   int nc;
   FastDiv dN, dWo, dW, dCred, dKw, dCin, dS;
+  // Input gradient with stride 2 on the generic kernel: the GEMM columns are
+  // grouped by phase (hi mod 2, wi mod 2) so that the columns of a tile
+  // share one phase, and a tile gathers and multiplies only the K tiles that
+  // hold a tap of its phase (the other taps never reach its pixels).  With
+  // phases = 1 column tile nt covers GEMM columns nt·BN.. of the whole pass.
+  int phases;                             // 4, or 1 (no phase grouping)
+  int ph_tile0[kMaxPhases + 1];           // first column tile of each phase
+  int ph_h0[kMaxPhases], ph_w0[kMaxPhases];
+  int ph_wp[kMaxPhases];                  // pixels per row of the phase's grid
+  FastDiv ph_dwp[kMaxPhases];
+  int64_t ph_cols[kMaxPhases];            // GEMM columns of the phase (phase 0: all when phases = 1)
+  int ph_nlive[kMaxPhases];               // live K tiles of the phase
+  uint32_t ph_live[kMaxPhases][kMaxLiveWords];
 };
+
+// The kernels take the phase grouping as a template flag PH; without it
+// (phases = 1) these reduce to the plain column mapping at no cost.
+// Phase of column tile nt, and whether K tile kt holds a tap of phase q.
+template <bool PH>
+__device__ __forceinline__ int phase_of(const V2Args& p, int nt) {
+  int q = 0;
+  if (PH) {
+#pragma unroll
+    for (int i = 1; i < kMaxPhases; ++i)
+      if (nt >= p.ph_tile0[i]) q = i;
+  }
+  return q;
+}
+
+template <bool PH>
+__device__ __forceinline__ bool kt_live(const V2Args& p, int q, int kt) {
+  return !PH || ((p.ph_live[q][kt >> 5] >> (kt & 31)) & 1u);
+}
+
+// Output pixel and batch item of phase-local GEMM column lcol of phase q;
+// false past the phase's columns.
+template <bool PH>
+__device__ __forceinline__ bool col_pixel(const V2Args& p, int q, int64_t lcol, int& pix, int& n) {
+  const bool ok = lcol < (PH ? p.ph_cols[q] : p.Ncols);
+  const int c32 = ok ? static_cast<int>(lcol) : 0;     // GEMM columns stay below 2^31
+  const int pp = fdiv(c32, p.dN);
+  n = c32 - pp * p.N;
+  if (!PH) {
+    pix = pp;
+  } else {
+    const int i = fdiv(pp, p.ph_dwp[q]);
+    const int j = pp - i * p.ph_wp[q];
+    pix = (p.ph_h0[q] + 2 * i) * p.W + p.ph_w0[q] + 2 * j;
+  }
+  return ok;
+}
 
 // Entries of the per-CTA K-tile table of the forward / input-gradient
 // producers (16 per K tile): larger contractions decode on the fly.
@@ -89,7 +141,8 @@ struct V2Smem {
   static constexpr int kStage = kATileBytes + kBTile;
   static constexpr int kBarOffset = kV2Stages * kStage;
   static constexpr int kKtabOffset = kBarOffset + 256;
-  static constexpr int kBytes = kKtabOffset + kKtabEntries * 4 + 1024;
+  static constexpr int kLiveOffset = kKtabOffset + kKtabEntries * 4;     // kMaxPhases x 256 K tiles
+  static constexpr int kBytes = kLiveOffset + kMaxPhases * 256 + 1024;
 };
 
 // MN-major 128B-swizzled fp16 tile of BN rows (MN) x 64 K: atoms of 64 MN x
@@ -313,9 +366,10 @@ __device__ __forceinline__ void epi_amax_flush(uint32_t* amax_out, float m) {
   if ((threadIdx.x & 31) == 0) atomicMax(amax_out, __float_as_uint(m));
 }
 
-template <int BN, bool FD>
+// FD: col0 is the tile's first column local to phase q (see col_pixel).
+template <int BN, bool FD, bool PH = false>
 __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int acc, int64_t m0,
-                                            int64_t col0, int split, bool has_k, float& amax) {
+                                            int64_t col0, int split, bool has_k, float& amax, int q = 0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t m = m0 + warp * 32 + lane;
   const float scale = p.scale_out ? __fmul_rn(*p.ta, *p.tb) : 1.0f;
@@ -331,7 +385,7 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int64_t col = col0 + c + 4 * j;
-        if (col >= p.Ncols) continue;
+        if (col >= (FD && PH ? p.ph_cols[q] : p.Ncols)) continue;
         float4 o;
         o.x = has_k ? __uint_as_float(r[4 * j + 0]) * scale : 0.f;
         o.y = has_k ? __uint_as_float(r[4 * j + 1]) * scale : 0.f;
@@ -341,9 +395,9 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
         if (FD) {
           if (p.relu) o = epi_relu(o);
           amax = epi_absmax(amax, o);
-          const int c32 = static_cast<int>(col);           // GEMM columns stay below 2^31
-          const int pix = fdiv(c32, p.dN);
-          idx = (static_cast<int64_t>(pix) * p.M + m) * p.N + (c32 - pix * p.N);
+          int pix, n;
+          col_pixel<PH>(p, q, col, pix, n);
+          idx = (static_cast<int64_t>(pix) * p.M + m) * p.N + n;
         } else {
           idx = (static_cast<int64_t>(split) * p.M + m) * p.Ncols + col;
         }
@@ -359,17 +413,14 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
 // column = output channel.  Each lane stores its column's channels one by
 // one; for one channel the 32 lanes of a warp write consecutive batch items,
 // so every store of a warp covers runs of N contiguous floats.
-template <int BN>
-__device__ __forceinline__ void v2_epilogue_tr(const V2Args& p, V2Bars* bars, int acc, int64_t col0,
-                                               float& amax) {
+template <int BN, bool PH>
+__device__ __forceinline__ void v2_epilogue_tr(const V2Args& p, V2Bars* bars, int acc, int64_t col0, int q,
+                                               bool has_k, float& amax) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t col = col0 + warp * 32 + lane;
-  const bool ok = col < p.Ncols;
-  const int c32 = ok ? static_cast<int>(col) : 0;     // GEMM columns stay below 2^31
-  const int pix = fdiv(c32, p.dN);
-  float* out = p.out + static_cast<int64_t>(pix) * p.M * p.N + (c32 - pix * p.N);
+  int pix, n;
+  const bool ok = col_pixel<PH>(p, q, col0 + warp * 32 + lane, pix, n);
+  float* out = p.out + static_cast<int64_t>(pix) * p.M * p.N + n;
   const float scale = __fmul_rn(*p.ta, *p.tb);
-  const bool has_k = p.ktiles > 0;
   const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * BN;
 #pragma unroll 1
   for (int c = 0; c < p.nc; c += 16) {
@@ -458,9 +509,19 @@ struct TileCol {
   bool ok;
 };
 
-template <int PASS>
-__device__ __forceinline__ TileCol tile_col(const V2Args& p, int64_t col) {
+// Column `off` of column tile nt (off < BN).
+template <int PASS, int BN, bool PH>
+__device__ __forceinline__ TileCol tile_col(const V2Args& p, int nt, int off) {
   TileCol c;
+  if (PH) {
+    const int q = phase_of<PH>(p, nt);
+    int pix;
+    c.ok = col_pixel<PH>(p, q, static_cast<int64_t>(nt - p.ph_tile0[q]) * BN + off, pix, c.n);
+    c.h = fdiv(pix, p.dW);
+    c.w = pix - c.h * p.W;
+    return c;
+  }
+  const int64_t col = static_cast<int64_t>(nt) * BN + off;
   c.ok = col < p.Ncols;
   const int c32 = c.ok ? static_cast<int>(col) : 0;
   const int pix = fdiv(c32, p.dN);
@@ -539,9 +600,10 @@ __host__ __device__ constexpr int fd_threads(int gr) { return kV2ProdWarp0 * 32 
 // GR producer groups of 8 warps take turns: group g fills the K iterations
 // g, g + GR, ... so that GR times as many gathers are in flight (GR = 2
 // needs at most 88 registers a thread).
-template <int PASS, int FMT, int BN, int NU, bool TR, int GR>
+template <int PASS, int FMT, int BN, int NU, bool TR, int GR, bool PH>
 __global__ void __launch_bounds__(fd_threads(GR), 1)
-conv_fd_kernel(const V2Args p) {
+conv_fd_kernel(const __grid_constant__ V2Args p) {
+  static_assert(!PH || PASS == kDgrad, "phase grouping is for the input gradient");
   static_assert(!TR || BN == 128, "transposed tiles are 128 GEMM columns");
   using L = V2Smem<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -558,11 +620,13 @@ conv_fd_kernel(const V2Args p) {
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const int mt = tile / p.ntiles, nt = tile - mt * p.ntiles;
+      const int q = phase_of<PH>(p, nt);
+      const int64_t lcol0 = static_cast<int64_t>(nt - (PH ? p.ph_tile0[q] : 0)) * BN;
+      const bool has_k = PH ? p.ph_nlive[q] > 0 : p.ktiles > 0;
       if (TR)
-        v2_epilogue_tr<BN>(p, bars, acc, static_cast<int64_t>(nt) * BN, amax);
+        v2_epilogue_tr<BN, PH>(p, bars, acc, lcol0, q, has_k, amax);
       else
-        v2_epilogue<BN, true>(p, bars, acc, static_cast<int64_t>(mt) * 128,
-                              static_cast<int64_t>(nt) * BN, 0, p.ktiles > 0, amax);
+        v2_epilogue<BN, true, PH>(p, bars, acc, static_cast<int64_t>(mt) * 128, lcol0, 0, has_k, amax, q);
     }
     epi_amax_flush(p.amax_out, amax);
   } else if (warp == kV2MmaWarp) {
@@ -575,7 +639,10 @@ conv_fd_kernel(const V2Args p) {
         mbar_wait_bounded(&bars->acc_empty[acc], ((it >> 1) & 1) ^ 1, p.err, kErrWaitEmpty);
         tc_fence_after();
         const uint32_t dt = bars->tmem + acc * BN;
-        for (int kt = 0; kt < p.ktiles; ++kt, ++kit) {
+        const int q = phase_of<PH>(p, tile % p.ntiles);
+        uint32_t accum = 0;                    // 0 until the tile's first live K tile
+        for (int kt = 0; kt < p.ktiles; ++kt) {
+          if (!kt_live<PH>(p, q, kt)) continue;
           const int s = kit % kV2Stages;
           mbar_wait_bounded(&bars->full[s], (kit / kV2Stages) & 1, p.err, kErrWaitFull);
           tc_fence_after();
@@ -585,11 +652,13 @@ conv_fd_kernel(const V2Args p) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             if (TR)
-              mma_f16_ss(dt, gdesc + 128 * kk, wdesc + 2 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+              mma_f16_ss(dt, gdesc + 128 * kk, wdesc + 2 * kk, idesc, (accum | kk) ? 1u : 0u);
             else
-              mma_f16_ss(dt, wdesc + 2 * kk, gdesc + 128 * kk, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+              mma_f16_ss(dt, wdesc + 2 * kk, gdesc + 128 * kk, idesc, (accum | kk) ? 1u : 0u);
           }
+          accum = 1;
           mma_commit(&bars->empty[s]);
+          ++kit;
         }
         mma_commit(&bars->acc_full[acc]);
       }
@@ -602,12 +671,15 @@ conv_fd_kernel(const V2Args p) {
         const uint8_t* src = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
         // TR: only the first nc rows (128 B each) of a weight tile are used
         const uint32_t bytes = TR ? static_cast<uint32_t>(p.nc) * 128u : kATileBytes;
-        for (int kt = 0; kt < p.ktiles; ++kt, ++kit) {
+        const int q = phase_of<PH>(p, tile % p.ntiles);
+        for (int kt = 0; kt < p.ktiles; ++kt) {
+          if (!kt_live<PH>(p, q, kt)) continue;
           const int s = kit % kV2Stages;
           mbar_wait_bounded(&bars->empty[s], ((kit / kV2Stages) & 1) ^ 1, p.err, kErrWaitEmpty);
           mbar_arrive_expect_tx(&bars->full[s], bytes);
           bulk_copy_g2s(sbase + s * L::kStage, src + static_cast<int64_t>(kt) * kATileBytes, bytes,
                         &bars->full[s]);
+          ++kit;
         }
       }
     }
@@ -619,35 +691,65 @@ conv_fd_kernel(const V2Args p) {
     const int tg = threadIdx.x - kV2ProdWarp0 * 32;
     const int grp = tg / kV2ProdThreads;      // producer group
     const int t = tg - grp * kV2ProdThreads;
-    const int total = p.ktiles * ((p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                                  static_cast<int>(gridDim.x));
+    // the CTA's K iterations: each of its tiles contributes its phase's live K tiles
+    int total = p.ktiles * ((p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                            static_cast<int>(gridDim.x));
+    if (PH) {
+      total = 0;
+      for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) total += p.ph_nlive[phase_of<PH>(p, tile % p.ntiles)];
+    }
     using Prod = FdProducer<PASS, FMT, BN, NU>;
     constexpr int kLookahead = Prod::PER >= 4 ? 2 : 3;      // keep the ring in registers
     Prod ring[kLookahead];
     // the CTA's K-tile table, built once by the producer warps
     uint32_t* ktab = nullptr;
+    // phase grouping: the live K tiles of each phase, in order (built with the table)
+    uint8_t* live = smem + L::kLiveOffset;
     if (p.ktiles * 16 <= kKtabEntries) {
       ktab = reinterpret_cast<uint32_t*>(smem + L::kKtabOffset);
       for (int e = tg; e < p.ktiles * 16; e += GR * kV2ProdThreads) ktab[e] = ktab_entry<PASS>(p, e >> 4, e & 15);
-      asm volatile("bar.sync 1, %0;" ::"n"(GR * kV2ProdThreads) : "memory");
     }
-    // load cursor at this group's first K iteration (p.ktiles >= 1)
-    int ltile = blockIdx.x, lkt = grp;
-    while (lkt >= p.ktiles) {
-      lkt -= p.ktiles;
+    if (PH && tg < kMaxPhases) {
+      int i = 0;
+      for (int kt = 0; kt < p.ktiles; ++kt)
+        if (kt_live<PH>(p, tg, kt)) live[tg * 256 + i++] = static_cast<uint8_t>(kt);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(GR * kV2ProdThreads) : "memory");
+    // load cursor: tile ltile, K tile lkt; with phases, lkt is entry li of
+    // the phase's live list (tiles whose phase has none are passed over).
+    int ltile = blockIdx.x, lkt = 0, li = 0, lq = 0;
+    const int toff = (t % Prod::G) * NU;
+    auto next_tile = [&]() {
       ltile += gridDim.x;
+      if (PH) {
+        while (ltile < p.tiles && p.ph_nlive[lq = phase_of<PH>(p, ltile % p.ntiles)] == 0) ltile += gridDim.x;
+      }
+    };
+    if (PH) {
+      lq = phase_of<PH>(p, ltile % p.ntiles);
+      if (ltile < p.tiles && p.ph_nlive[lq] == 0) next_tile();
+      lkt = live[lq * 256];
     }
-    TileCol tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
+    TileCol tc = tile_col<PASS, BN, PH>(p, ltile % p.ntiles, toff);
+    auto step = [&]() {                        // one K iteration forward
+      if (PH) {
+        if (++li == p.ph_nlive[lq]) {
+          li = 0;
+          next_tile();
+          tc = tile_col<PASS, BN, PH>(p, ltile % p.ntiles, toff);
+        }
+        lkt = live[lq * 256 + li];
+      } else if (++lkt == p.ktiles) {
+        lkt = 0;
+        ltile += gridDim.x;
+        tc = tile_col<PASS, BN, PH>(p, ltile % p.ntiles, toff);
+      }
+    };
+    for (int g = 0; g < grp; ++g) step();     // this group's first K iteration
     auto load_next = [&](Prod& pr) {
       pr.load(p, tc, lkt, t, ktab);
-      lkt += GR;
-      bool moved = false;
-      while (lkt >= p.ktiles) {
-        lkt -= p.ktiles;
-        ltile += gridDim.x;
-        moved = true;
-      }
-      if (moved) tc = tile_col<PASS>(p, static_cast<int64_t>(ltile % p.ntiles) * BN + (t % Prod::G) * NU);
+#pragma unroll
+      for (int g = 0; g < GR; ++g) step();
     };
 #pragma unroll
     for (int r = 0; r < kLookahead; ++r)

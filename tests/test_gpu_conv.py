@@ -49,6 +49,12 @@ SMALL = [
     ("two_m_tiles", O.ConvShape(4, 16, 136, 6, 6, 3, 3, 1, 1), "nvfp4"),
     ("n12_c8", O.ConvShape(12, 8, 8, 5, 5, 3, 3, 1, 1), "nvfp6"),
     ("wide_k_s2_p2", O.ConvShape(4, 72, 68, 11, 11, 5, 5, 2, 2), "nvfp4"),
+    # stride 2 with 32+ output channels: input-gradient tiles grouped by
+    # pixel parity, some parities reached by no tap at all (1 x 1), a
+    # one-row input, two channel tiles
+    ("s2_1x1_empty_phases", O.ConvShape(4, 8, 32, 7, 7, 1, 1, 2, 0), "nvfp4"),
+    ("s2_one_row", O.ConvShape(4, 8, 36, 1, 7, 3, 3, 2, 1), "nvfp6"),
+    ("s2_m160_two_m_tiles", O.ConvShape(8, 160, 64, 9, 8, 3, 3, 2, 1), "nvfp4"),
     ("deep_cin", O.ConvShape(8, 256, 32, 4, 4, 3, 3, 1, 1), "nvfp4"),
     # stride-1 shapes of the kernel-row halo path (N | 256, N % 8 == 0, 64-channel chunks)
     ("halo_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp4"),
