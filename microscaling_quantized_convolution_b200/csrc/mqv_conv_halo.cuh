@@ -147,6 +147,61 @@ struct HaloCursor {
   }
 };
 
+// Epilogue of one tile for the warp on TMEM lane quarter `quarter`: the
+// 32-column chunks first, first + stride, ... of the accumulator.  Each lane
+// reads one accumulator row from TMEM; a swizzled 32 x 32 transpose in the
+// warp's 4 KB of shared memory (wbuf) turns that into stores of 128-byte runs
+// of one (pixel, channel) row's batch items.  Columns past bw·N hold no
+// output (j >= bw below).
+__device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGeom& g, uint32_t tmem, int acc,
+                                                   int tile, int quarter, uint32_t wbuf, int first, int stride,
+                                                   float& amax) {
+  const int lane = threadIdx.x & 31;
+  const int rsub = lane >> 3, q = lane & 7;
+  const int mt = tile / (g.out_h * g.tpr);
+  const int rest = tile - mt * g.out_h * g.tpr;
+  const int oh = rest / g.tpr;
+  const int ow0 = (rest - oh * g.tpr) * g.bw;
+  const float scale = __fmul_rn(*p.ta, *p.tb);
+  const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kHaloBN;
+#pragma unroll 1
+  for (int c = 32 * first; c < g.bn; c += 32 * stride) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(tbase + c + 16 * hf, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
+                     __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
+    }
+    __syncwarp();
+    const int lc = c + 4 * q;
+    const int j = fdiv(lc, p.dN);
+    const int n = lc - j * p.N;
+    const int ow = ow0 + j;
+    if (j < g.bw && ow < g.out_w) {
+      const int64_t pix = static_cast<int64_t>(oh) * g.out_w + ow;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = 4 * i + rsub;
+        const int64_t mrow = static_cast<int64_t>(mt) * 128 + quarter * 32 + row;
+        float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+        if (mrow < p.M) {
+          if (p.relu) o = epi_relu(o);
+          amax = epi_absmax(amax, o);
+          *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
 template <int PASS>
 __global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
@@ -183,61 +238,18 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
 
   if (warp < kV2EpiWarps) {
     // epilogue: column lc of the tile = (pixel j, batch item n) -> output
-    // pixel (oh, ow0 + j), skipped past the end of the output row.
+    // pixel (oh, ow0 + j), skipped past the end of the output row.  The
+    // CTA's last tile is shared with the producer warps (which are done by
+    // then): warp `warp` takes the 32-column chunks 0, 4, 8, ... of it.
     int it = 0;
     float amax = 0.f;
     const uint32_t wbuf = sbase + L::kEpiOffset + warp * 4096;
-    const int rsub = lane >> 3, q = lane & 7;
     for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
-      const int mt = tile / (g.out_h * g.tpr);
-      const int rest = tile - mt * g.out_h * g.tpr;
-      const int oh = rest / g.tpr;
-      const int ow0 = (rest - oh * g.tpr) * g.bw;
-      const float scale = __fmul_rn(*p.ta, *p.tb);
-      const uint32_t tbase = bars->tmem + (static_cast<uint32_t>(warp * 32) << 16) + acc * kHaloBN;
-      // columns past bw·N hold no output (j >= bw below)
-      // Each lane reads one accumulator row from TMEM; a swizzled 32 x 32
-      // transpose in shared memory turns that into stores of 128-byte runs of
-      // one (pixel, channel) row's batch items.
-#pragma unroll 1
-      for (int c = 0; c < g.bn; c += 32) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(tbase + c + 16 * hf, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_shared_v4(wbuf + lane * 128 + (((4 * hf + j) ^ (lane & 7)) << 4),
-                         __float_as_uint(__uint_as_float(r[4 * j + 0]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
-                         __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
-        }
-        __syncwarp();
-        const int lc = c + 4 * q;
-        const int j = fdiv(lc, p.dN);
-        const int n = lc - j * p.N;
-        const int ow = ow0 + j;
-        if (j < g.bw && ow < g.out_w) {
-          const int64_t pix = static_cast<int64_t>(oh) * g.out_w + ow;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int row = 4 * i + rsub;
-            const int64_t mrow = static_cast<int64_t>(mt) * 128 + warp * 32 + row;
-            float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
-            if (mrow < p.M) {
-              if (p.relu) o = epi_relu(o);
-              amax = epi_absmax(amax, o);
-              *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
-            }
-          }
-        }
-        __syncwarp();
-      }
+      const bool last = tile + static_cast<int>(gridDim.x) >= p.tiles;
+      halo_epilogue_tile(p, g, bars->tmem, acc, tile, warp & 3, wbuf, 0, last ? 4 : 1, amax);
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
     }
@@ -353,6 +365,20 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         producer_warp_arrive(&bars->bfull[sb]);
         if (kit + kHaloLookahead < total) load_next(ring[r]);
       }
+    }
+    // The CTA's last tile: once its accumulator is complete (so the B ring
+    // is no longer read), producer warp w takes chunks 1, 2 or 3 (of every 4)
+    // on TMEM lane quarter w % 4, staging through 4 KB of the B ring.
+    if (ntile_cta > 0) {
+      const int lit = ntile_cta - 1;
+      const int ltile_last = static_cast<int>(blockIdx.x) + lit * static_cast<int>(gridDim.x);
+      const int pw = warp - kV2ProdWarp0;
+      float amax = 0.f;
+      mbar_wait_bounded(&bars->acc_full[lit & 1], (lit >> 1) & 1, p.err, kErrWaitDone);
+      tc_fence_after();
+      halo_epilogue_tile(p, g, bars->tmem, lit & 1, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
+                         1 + pw / 4, 4, amax);
+      epi_amax_flush(p.amax_out, amax);
     }
   }
   tc_fence_before();
