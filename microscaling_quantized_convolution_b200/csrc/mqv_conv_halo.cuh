@@ -162,6 +162,7 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
   const int rest = tile - mt * g.out_h * g.tpr;
   const int oh = rest / g.tpr;
   const int ow0 = (rest - oh * g.tpr) * g.bw;
+  if (mt * 128 + quarter * 32 >= p.M) return;   // all 32 rows of this quarter past the M channels
   const float scale = __fmul_rn(*p.ta, *p.tb);
   const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kHaloBN;
 #pragma unroll 1
