@@ -194,7 +194,7 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
         float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
         if (mrow < p.M) {
           if (p.relu) o = epi_relu(o);
-          amax = epi_absmax(amax, o);
+          if (p.amax_out) amax = epi_absmax(amax, o);
           *reinterpret_cast<float4*>(p.out + (pix * p.M + mrow) * p.N + n) = o;
         }
       }

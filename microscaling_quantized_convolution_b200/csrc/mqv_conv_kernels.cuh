@@ -394,7 +394,7 @@ __device__ __forceinline__ void v2_epilogue(const V2Args& p, V2Bars* bars, int a
         int64_t idx;
         if (FD) {
           if (p.relu) o = epi_relu(o);
-          amax = epi_absmax(amax, o);
+          if (p.amax_out) amax = epi_absmax(amax, o);
           int pix, n;
           col_pixel<PH>(p, q, col, pix, n);
           idx = (static_cast<int64_t>(pix) * p.M + m) * p.N + n;
@@ -434,7 +434,7 @@ __device__ __forceinline__ void v2_epilogue_tr(const V2Args& p, V2Bars* bars, in
         if (m < p.M) {
           float v = has_k ? __uint_as_float(r[j]) * scale : 0.f;
           if (p.relu) v = v > 0.f ? v : 0.f;
-          amax = fmaxf(amax, fabsf(v));
+          if (p.amax_out) amax = fmaxf(amax, fabsf(v));
           out[static_cast<int64_t>(m) * p.N] = v;
         }
       }
