@@ -118,10 +118,12 @@ def run_gpu(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
+    # one process per GPU; ranks beyond the visible GPUs (a functional check
+    # of the multi-rank path on fewer GPUs, host collectives only) share them
+    torch.cuda.set_device(local % torch.cuda.device_count())
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.init_process_group(os.environ.get("MQV_DIST_BACKEND", "nccl"), timeout=timedelta(seconds=120))
     mqv.lib()
 
     layer = pick_layer(args.workload)
@@ -131,7 +133,7 @@ def run_gpu(args):
     xr, xc = layer.H * layer.W * layer.Cin, layer.N
     wr, wc = layer.Cout, layer.K * layer.K * layer.Cin
     gr, gc = Ho * Wo * layer.Cout, layer.N
-    dev = torch.device("cuda", local)
+    dev = torch.device("cuda", local % torch.cuda.device_count())
 
     # Inputs resident in HBM, rotated over enough sets to exceed the 126 MB L2
     quant_b, conv_b, (nx, nw, ng) = layer_bytes(layer)
@@ -337,7 +339,7 @@ def run_gpu(args):
     # Each kernel alone (one stream): the per-kernel durations and the
     # roofline.  Then the step as it is run: on one GPU the three passes
     # concurrently; that loop gives the reported throughput.
-    clocks = Clocks(local)
+    clocks = Clocks(local % torch.cuda.device_count())
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.15)
