@@ -106,3 +106,25 @@ def test_full_size_layer_fused_forward_and_next_quantization():
     assert torch.equal(y, torch.relu(y_plain))
     assert amax.item() == y.max().item()
     _same_codes(y, s.Ho * s.Wo * s.Cout, s.N, layer.fmt, mqv.RNE, 0, amax)
+
+
+@pytest.mark.parametrize("idx", [1, 3])
+def test_full_size_yolo_layers_fused_passes(idx):
+    """NVFP6 stride-2 layers of the YOLOv8n-shaped mix (the generic kernel on
+    transposed tiles, the input gradient grouped by pixel parity): fused
+    forward with ReLU and fused input gradient against the plain passes."""
+    layer = workloads.yolov8n_mix()[idx]
+    s = O.ConvShape(layer.N, layer.Cin, layer.Cout, layer.H, layer.W, layer.K, layer.K, layer.stride, layer.pad)
+    X, Wt, G = workloads.make_layer_inputs(layer)
+    d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+    qx = mqv.quantize(X.cuda().view(-1), *s.x_view(), layer.fmt, mqv.RNE)
+    qw = mqv.quantize(Wt.cuda().view(-1), *s.w_view(), layer.fmt, mqv.RNE)
+    qg = mqv.quantize(G.cuda().view(-1), *s.gy_view(), layer.fmt, mqv.SR, workloads.sr_seed(layer))
+    y_plain = mqv.conv_fwd(d, qw, qx)
+    y, ya = mqv.conv_fwd_fused(d, qw, qx, relu=True)
+    gx_plain = mqv.conv_dgrad(d, qw, qg)
+    gx, ga = mqv.conv_dgrad_fused(d, qw, qg)
+    torch.cuda.synchronize()
+    assert torch.equal(y, torch.relu(y_plain)) and ya.item() == y.max().item()
+    assert torch.equal(gx, gx_plain) and ga.item() == gx.abs().max().item()
+    assert mqv.device_errors() == 0

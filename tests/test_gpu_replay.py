@@ -116,3 +116,32 @@ def test_replay_buffer_full_size_sampled(C, H, N):
         assert np.array_equal(vals[band * cols:(band + 4) * cols].cpu().numpy(), want), band
     del codes_dev, packed, back, vals
     torch.cuda.empty_cache()
+
+
+def test_replay_buffer_e2m3_sampled():
+    """A 6.4 M-element NVFP6 buffer (5-bit magnitudes): whole-tensor negative
+    count, then packed bytes and values read back of 4 row bands."""
+    C, H, N = 512, 7, 256
+    rows, cols = H * H * C, N
+    g = torch.Generator(device="cuda").manual_seed(77)
+    codes_dev = torch.randint(0, 256, (rows * cols * 3 // 4,), dtype=torch.uint8, device="cuda", generator=g)
+    scales_dev = torch.randint(0, 0x7F, (rows // 4 * cols // 4,), dtype=torch.uint8, device="cuda", generator=g)
+    T = torch.tensor([2.0 ** -9], dtype=torch.float32, device="cuda")
+    q = mqv.QTensor(codes_dev, scales_dev, T, rows, cols, mqv.NVFP6)
+    neg = torch.zeros(1, dtype=torch.int32, device="cuda")
+    packed = mqv.replay_pack(q, negatives=neg)
+    vals = mqv.replay_dequantize(packed, scales_dev, T, rows, cols, "nvfp6")
+    torch.cuda.synchronize()
+    allc = O.unpack_codes(codes_dev.cpu().numpy(), rows, cols, O.FP6)
+    assert int(neg.item()) == int(np.count_nonzero((allc >= 32) & ((allc & 31) != 0)))
+    rng = np.random.default_rng(4)
+    pb, cb = 5 * cols // 8, 3 * cols // 4
+    for band in [0, rows - 4] + list(4 * rng.integers(0, rows // 4 - 1, 2)):
+        band = int(band)
+        c = allc[band:band + 4]
+        ref, _ = O.pack_unsigned(c, O.FP6)
+        assert np.array_equal(packed[band * pb:(band + 4) * pb].cpu().numpy(), ref), band
+        s = scales_dev[band // 4 * (cols // 4):(band // 4 + 1) * (cols // 4)].cpu().numpy().reshape(1, -1)
+        oq = O.QTensor(O.unpack_unsigned(ref, 4, cols, O.FP6), s, np.float32(2.0 ** -9), O.FP6)
+        assert np.array_equal(vals[band * cols:(band + 4) * cols].cpu().numpy(),
+                              O.dequantize(oq).astype(np.float32).reshape(-1)), band
