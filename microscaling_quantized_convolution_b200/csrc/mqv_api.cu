@@ -350,9 +350,9 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   }
   a.splits = splits;
   a.tiles = (int)(tiles_mn * splits);
-  // Stride-1 fwd/dgrad on NVFP4 with N | 256, N % 8 == 0, a halo of at most
+  // Stride-1 fwd/dgrad (NVFP4 or NVFP6) with N | 256, N % 8 == 0, a halo of at most
   // 384 rows and whole 64-channel chunks: the kernel-row halo path.
-  pl->halo = op != MQV_OP_WGRAD && d->fmt == MQV_NVFP4 && d->stride == 1 && d->N % 8 == 0 &&
+  pl->halo = op != MQV_OP_WGRAD && d->stride == 1 && d->N % 8 == 0 &&
              256 % d->N == 0 && (d->Kw - 1) * d->N <= 128 && a.Cred % 64 == 0 && d->Kw <= kHaloAStages;
   if (pl->halo) {
     HaloGeom& g = pl->g;
@@ -474,9 +474,9 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
   return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, false>(pl, st) : launch_fd<P, FMT, 128, 4, false>(pl, st);
 }
 
-template <int PASS>
+template <int PASS, int FMT>
 cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_halo_kernel<PASS>;
+  auto kern = conv_halo_kernel<PASS, FMT>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
   if (e != cudaSuccess) return e;
@@ -508,7 +508,9 @@ cudaError_t launch_wgk_kw(const ConvPlan& pl, cudaStream_t st) {
 
 template <int PASS>
 cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
-  if (PASS != kWgrad && pl.halo) return launch_halo<PASS == kWgrad ? kFwd : PASS>(pl, st);
+  if (PASS != kWgrad && pl.halo)
+    return fmt == MQV_NVFP4 ? launch_halo<PASS == kWgrad ? kFwd : PASS, 0>(pl, st)
+                            : launch_halo<PASS == kWgrad ? kFwd : PASS, 1>(pl, st);
   if (PASS == kWgrad && pl.wgk) return fmt == MQV_NVFP4 ? launch_wgk_kw<0>(pl, st) : launch_wgk_kw<1>(pl, st);
   return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
 }

@@ -74,7 +74,8 @@ struct HaloGeom {
 
 // Raw codes of one halo unit: 8 batch items (rows) x 8 channels (K).
 struct HaloUnit {
-  uint32_t w[8];      // codes of channel c0 + j for the 8 batch items
+  uint32_t w[8];      // codes of channel c0 + j for the 8 batch items (NVFP6: bytes 0-3)
+  uint32_t wh[8];     // NVFP6: bytes 4-5 of the 6-byte run
   uint32_t s[2];      // scales of channel blocks 0/1 (low byte: batch block 0)
   bool ok;
 };
@@ -83,9 +84,27 @@ struct HaloUnit {
 // the 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
 // channel words is interleaved nibble-wise first, so one cvt.e2m1x2 per
 // byte yields the (channel 2i, channel 2i+1) pair of one batch item.
+template <int FMT>
 __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile, uint32_t row0, uint32_t kg) {
   uint32_t out[8][4];
-  if (u.ok) {
+  if (u.ok && FMT == 1) {
+    // NVFP6: batch item r of channel c is bits [6r, 6r+6) of the 48-bit run;
+    // the two channels of a pair go to the low and high byte of one
+    // cvt.e2m3x2 input, giving the (2i, 2i+1) fp16 pair directly.
+    const uint32_t sc[2][2] = {{scale2(u.s[0] & 0xFF), scale2(u.s[0] >> 8)},
+                               {scale2(u.s[1] & 0xFF), scale2(u.s[1] >> 8)}};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t a = u.w[2 * i] | (static_cast<uint64_t>(u.wh[2 * i]) << 32);
+      const uint64_t b = u.w[2 * i + 1] | (static_cast<uint64_t>(u.wh[2 * i + 1]) << 32);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const uint32_t v = static_cast<uint32_t>((a >> (6 * r)) & 0x3F) |
+                           (static_cast<uint32_t>((b >> (6 * r)) & 0x3F) << 8);
+        out[r][i] = hmul2_u32(e2m3x2_to_f16x2(v), sc[i >> 1][r >> 2]);
+      }
+    }
+  } else if (u.ok) {
     const uint32_t sc[2][2] = {{scale2(u.s[0] & 0xFF), scale2(u.s[0] >> 8)},    // [channel block][batch block]
                                {scale2(u.s[1] & 0xFF), scale2(u.s[1] >> 8)}};
 #pragma unroll
@@ -115,7 +134,7 @@ __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile
 // Producer thread t owns unit t of every stage: K chunk kg = t % 8 (8
 // channels), rows 8(t/8)..8(t/8)+7 of the halo.  Lanes of an 8-lane phase
 // differ in kg, so their 16-byte stores hit 8 different swizzled chunks.
-template <int PASS>
+template <int PASS, int FMT>
 struct HaloCursor {
   int sc, n0;         // halo pixel column in the source, first batch item
   bool cok;           // unit inside the halo and its column inside the source
@@ -138,9 +157,20 @@ struct HaloCursor {
     u.ok = cok && sr >= 0 && sr < g.src_h;
     if (!u.ok) return;
     const int64_t row0 = (static_cast<int64_t>(sr) * g.src_w + sc) * p.Cred + 64 * c + 8 * (t & 7);
-    const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + (n0 >> 1);
+    if (FMT == 0) {
+      const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + (n0 >> 1);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u.w[j] = __ldg(reinterpret_cast<const uint32_t*>(cp + j * p.b.row_bytes));
+      for (int j = 0; j < 8; ++j) u.w[j] = __ldg(reinterpret_cast<const uint32_t*>(cp + j * p.b.row_bytes));
+    } else {
+      // 6 bytes at a 2-byte aligned offset (n0 is a multiple of 8)
+      const uint8_t* cp = p.b.codes + row0 * p.b.row_bytes + ((n0 * 3) >> 2);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const unsigned short* q = reinterpret_cast<const unsigned short*>(cp + j * p.b.row_bytes);
+        u.w[j] = static_cast<uint32_t>(__ldg(q)) | (static_cast<uint32_t>(__ldg(q + 1)) << 16);
+        u.wh[j] = __ldg(q + 2);
+      }
+    }
     const uint8_t* sp = p.b.scales + (row0 >> 2) * p.b.scale_cols + (n0 >> 2);
     u.s[0] = __ldg(reinterpret_cast<const unsigned short*>(sp));
     u.s[1] = __ldg(reinterpret_cast<const unsigned short*>(sp + p.b.scale_cols));
@@ -203,7 +233,7 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
   }
 }
 
-template <int PASS>
+template <int PASS, int FMT>
 __global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
   using L = HaloSmem;
@@ -336,7 +366,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
                           static_cast<int>(gridDim.x);
     const int total = ntile_cta * stages_per_tile;
     const int spatial = g.out_h * g.tpr;
-    HaloCursor<PASS> cursor;
+    HaloCursor<PASS, FMT> cursor;
     HaloUnit ring[kHaloLookahead];
     int ltile = blockIdx.x, lkh = 0, lc = 0;
     if (total > 0) cursor.begin_tile(p, g, ltile % spatial, t);
@@ -361,7 +391,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         const int sb = kit % kHaloBStages;
         mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
         if (t < g.rows)
-          halo_store_unit(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
+          halo_store_unit<FMT>(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
                           static_cast<uint32_t>(t & 7));
         producer_warp_arrive(&bars->bfull[sb]);
         if (kit + kHaloLookahead < total) load_next(ring[r]);

@@ -62,6 +62,10 @@ SMALL = [
     ("halo_n16_pad0", O.ConvShape(16, 64, 64, 7, 7, 3, 3, 1, 0), "nvfp4"),
     ("halo_n8_5x5", O.ConvShape(8, 64, 128, 9, 9, 5, 5, 1, 2), "nvfp4"),
     ("halo_1x1_n64", O.ConvShape(64, 128, 64, 5, 5, 1, 1, 1, 0), "nvfp4"),
+    # the same path on NVFP6 codes (6-byte runs of 8 batch items)
+    ("halo_fp6_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp6"),
+    ("halo_fp6_n16_1x1", O.ConvShape(16, 128, 64, 7, 7, 1, 1, 1, 0), "nvfp6"),
+    ("halo_fp6_n8_5x5", O.ConvShape(8, 64, 128, 9, 9, 5, 5, 1, 2), "nvfp6"),
     # stride-1 weight-gradient shapes whose kernel-row taps share operands
     # (N % 16 == 0): ragged rows and channels, split ranges that end inside a
     # row, several channel tiles, a 2 x 2 kernel
