@@ -12,7 +12,9 @@ all ranks / device time of the timed steps, max over ranks).
 Under torchrun (N > 1) each rank runs its own batch of the same layer (weak
 scaling, data parallel): the per-tensor max|x| of X and G_Y is MAX-all-reduced
 before quantizing (so every rank uses the global tensor scale) and G_W is
-SUM-all-reduced after the weight-gradient pass, both over NCCL.
+SUM-all-reduced after the weight-gradient pass, both over NCCL.  With
+MQV_DIST_BACKEND=gloo and more ranks than GPUs, ranks share the visible GPUs
+(a functional check of this path; its timing is not a measurement).
 """
 from __future__ import annotations
 
