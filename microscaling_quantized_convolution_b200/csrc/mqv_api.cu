@@ -70,14 +70,19 @@ mqv_status device_error_word(uint32_t** out) {
 
 // ------------------------------------------------------------ quantize geometry
 
-constexpr int64_t kMaxAmaxCtas = 148 * 8;
+constexpr int64_t kMaxAmaxCtas = 148 * 2;
 constexpr int64_t kMaxQuantCtas = 148 * 16;
 
+// One partial maximum per amax CTA; every quantize CTA reduces them before it
+// can scale anything, so keep them few (at most two CTAs per SM, which still
+// holds 64 KB of loads in flight per SM) and give every CTA the same number
+// of kAmaxThreads x 8-float4 chunks.
 int64_t amax_ctas(int64_t rows, int64_t cols) {
   const int64_t n4 = rows * cols / 4;
-  int64_t g = (n4 + kAmaxThreads * 4 - 1) / (kAmaxThreads * 4);
-  if (g < 1) g = 1;
-  return g < kMaxAmaxCtas ? g : kMaxAmaxCtas;
+  const int64_t chunk = kAmaxThreads * 8;
+  const int64_t nchunks = n4 > 0 ? (n4 + chunk - 1) / chunk : 1;
+  const int64_t passes = (nchunks + kMaxAmaxCtas - 1) / kMaxAmaxCtas;
+  return (nchunks + passes - 1) / passes;
 }
 
 int64_t quant_ctas(int64_t rows, int64_t cols) {

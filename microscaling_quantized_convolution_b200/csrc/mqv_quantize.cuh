@@ -29,9 +29,10 @@ struct PhiloxKeys {
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& k) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k.k0[r], lo1, hi0 ^ c.w ^ k.k1[r], lo0);
+    const uint64_t p0 = static_cast<uint64_t>(c.x) * 0xD2511F53u;
+    const uint64_t p1 = static_cast<uint64_t>(c.z) * 0xCD9E8D57u;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k.k0[r], static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k.k1[r], static_cast<uint32_t>(p0));
   }
   return c;
 }
@@ -39,31 +40,24 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& k) {
 // ------------------------------------------------- element rounding (a >= 0)
 // Round-to-nearest-even onto the element grid is the hardware conversion
 // (cvt.rn.satfinite.e2m1x2 / e2m3x2, see mqv_ptx.cuh).  For stochastic
-// rounding each grid is used as piecewise uniform: E2M1 steps 0.5 on [0,2),
-// 1 on [2,4), 2 on [4,6]; E2M3 steps 1/8 on [0,2), 1/4 on [2,4), 1/2 on
-// [4,7.5]; within a piece, code = piece base + (a - start)/step, where the
-// subtraction and the power-of-two scaling are exact.
-// Stochastic rounding: q = position in units of the local step, round up
-// iff u < frac(q) (frac is exact: q is an exact rescaling of a).  Selects
-// instead of branches, since neighbouring lanes land in different pieces.
+// rounding the grid is read as a binary format: with E = floor(log2(max(a, 1)))
+// the step on [2^E, 2^(E+1)) (and on [0, 1) for E = 0) is 2^(E-1) for E2M1
+// (0.5, 1, 2) and 2^(E-3) for E2M3 (1/8, 1/4, 1/2), and the magnitude code
+// below a is floor(a / step) + 2E (E2M1) or + 8E (E2M3).  q = a / step is a
+// power-of-two scaling and frac(q) = q - floor(q) is exact, so "round up
+// iff u < frac(q)" is decided exactly.  floor(q) comes from one add rounded
+// toward -inf onto 2^23 (the integer lands in the low mantissa bits), which
+// keeps the conversion pipe free; codes past the largest saturate.
 template <int FMT>
 __device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
-  float q;
-  uint32_t base;
-  if (FMT == 0) {
-    const bool p0 = a < 2.0f, p1 = a < 4.0f;
-    q = p0 ? a * 2.0f : (p1 ? a - 2.0f : (a - 4.0f) * 0.5f);
-    base = p0 ? 0u : (p1 ? 4u : 6u);
-  } else {
-    const bool p0 = a < 2.0f, p1 = a < 4.0f;
-    q = p0 ? a * 8.0f : (p1 ? (a - 2.0f) * 4.0f : (a - 4.0f) * 2.0f);
-    base = p0 ? 0u : (p1 ? 16u : 24u);
-  }
-  const float fl = floorf(q);
-  const float f = q - fl;
-  const uint32_t mag = base + static_cast<uint32_t>(fl) + (u < f ? 1u : 0u);
-  const float top = FMT == 0 ? 6.0f : 7.5f;
-  return a < top ? mag : (FMT == 0 ? 7u : 31u);
+  const uint32_t eb = __float_as_uint(fmaxf(a, 1.0f)) & 0x7F800000u;             // (127 + E) << 23
+  const float inv = __uint_as_float((FMT == 0 ? 0x7F800000u : 0x80800000u) - eb);  // 1 / step
+  const float q = __fmul_rn(a, inv);
+  const float t = __fadd_rd(q, 8388608.0f);                                        // 2^23 + floor(q)
+  const float f = __fsub_rn(q, __fsub_rn(t, 8388608.0f));
+  const uint32_t piece = FMT == 0 ? (eb >> 22) - 254u : (eb >> 20) - 1016u;      // 2E or 8E
+  const uint32_t mag = (__float_as_uint(t) - 0x4B000000u) + piece + (u < f ? 1u : 0u);
+  return min(mag, FMT == 0 ? 7u : 31u);
 }
 
 // Correctly rounded a / d for the elements of a block, which share d, by
@@ -135,6 +129,7 @@ amax_partial_kernel(const float4* __restrict__ src, int64_t n4, float* __restric
 __device__ __forceinline__ float block_max_of(const float* __restrict__ v, int count,
                                               float* red /* >= 32 floats smem */) {
   float m = 0.0f;
+#pragma unroll 2
   for (int i = threadIdx.x; i < count; i += blockDim.x) m = fmaxf(m, v[i]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -287,13 +282,19 @@ struct QuantArgs {
   FastDiv dcu;          // division by the work units per block row (unit count < 2^31)
 };
 
+template <int QB>
+__device__ __forceinline__ void load_unit(float4 (&x)[QB][4], const float* __restrict__ src, int64_t cols, int br,
+                                          int64_t bc0) {
+  const float* p = src + (static_cast<int64_t>(br) * 4) * cols + bc0 * 4;
+#pragma unroll
+  for (int q = 0; q < QB; ++q)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
+}
+
 template <int FMT, int RND, int QB>
 __device__ __forceinline__ void quantize_body(const QuantArgs& qa, const float* __restrict__ amax_src, int amax_count,
                                               int cta, int nctas) {
-  __shared__ float red[32];
-  const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
-  if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
-
   const int64_t cols = qa.cols;
   const int64_t cb = cols >> 2;                       // column blocks per block row
   const int cu = static_cast<int>(cb / QB);           // work units per block row
@@ -301,17 +302,28 @@ __device__ __forceinline__ void quantize_body(const QuantArgs& qa, const float* 
   const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
   const int stride = nctas * kQuantThreads;
 
-  for (int w = cta * kQuantThreads + static_cast<int>(threadIdx.x); w < nunits; w += stride) {
+  // The first unit's loads do not depend on the tensor scale: issue them
+  // before the reduction of the amax partials, so the two latencies overlap.
+  int w = cta * kQuantThreads + static_cast<int>(threadIdx.x);
+  float4 x[QB][4];
+  if (w < nunits) {
+    const int br = fdiv(w, qa.dcu);
+    load_unit<QB>(x, qa.src, cols, br, static_cast<int64_t>(w - br * cu) * QB);
+  }
+  __shared__ float red[32];
+  const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
+  if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
+
+  for (; w < nunits; w += stride) {
     const int br = fdiv(w, qa.dcu);
     const int64_t bc0 = static_cast<int64_t>(w - br * cu) * QB;
-    const float* p = qa.src + (static_cast<int64_t>(br) * 4) * cols + bc0 * 4;
-    float4 x[QB][4];
-#pragma unroll
-    for (int q = 0; q < QB; ++q)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
     quantize_unit<FMT, RND, QB>(x, ts, br, bc0, cb, row_bytes, qa.keys, qa.sr_cols, qa.sr_col0, qa.codes,
                                 qa.scales);
+    const int wn = w + stride;
+    if (wn < nunits) {
+      const int bn = fdiv(wn, qa.dcu);
+      load_unit<QB>(x, qa.src, cols, bn, static_cast<int64_t>(wn - bn * cu) * QB);
+    }
   }
 }
 
