@@ -66,8 +66,16 @@ __device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
 // Muller et al., Handbook of Floating-Point Arithmetic, 2nd ed., 2018,
 // sec. 4.9): with y = RN(1/d) and q0 = RN(a·y) within one ulp of a/d, the
 // remainder r = a - d·q0 is exact (one FMA) and RN(q0 + r·y) = RN(a/d).
-// The theorem assumes no underflow, so tiny nonzero quotients take the IEEE
-// divide (a = 0 gives q1 = 0 exactly and stays on the fast path).
+// The theorem needs r to be representable.  For block divisors d >= 2^-64
+// (kMarksteinMinDivisor) r is a multiple of at least 2^-140 for every
+// quotient >= 2^-30, so the result is exact there; y <= 2^64 stays finite
+// and, since d <= FLT_MAX / 6, normal.  Below 2^-30 only whether the
+// quotient is zero decides a code (stochastic rounding compares 24-bit u
+// against frac(q)): quotients below 1e-30 take the IEEE divide.  Blocks with
+// smaller divisors (tensors with max|x| below about 1e-13) divide exactly
+// throughout.
+constexpr float kMarksteinMinDivisor = 5.42101086242752217e-20f;   // 2^-64
+
 __device__ __forceinline__ float div_shared_divisor(float a, float d, float y) {
   const float q0 = __fmul_rn(a, y);
   const float r = __fmaf_rn(-d, q0, a);
@@ -75,12 +83,14 @@ __device__ __forceinline__ float div_shared_divisor(float a, float d, float y) {
   return (q0 >= 1.0e-30f || a == 0.0f) ? q1 : __fdiv_rn(a, d);
 }
 
-// The same for a signed a (d > 0), keeping the sign of a zero a.
-__device__ __forceinline__ float div_shared_divisor_signed(float a, float d, float y) {
+// Round-to-nearest-even codes need the quotient only where it can reach a
+// grid midpoint (>= 1/16), so the tiny-quotient check is dropped; the sign
+// is the sign of a in every case (also for y = 0, the zero-scale block,
+// where the magnitude comes out 0).
+__device__ __forceinline__ float div_shared_divisor_rne(float a, float d, float y) {
   const float q0 = __fmul_rn(a, y);
   const float r = __fmaf_rn(-d, q0, a);
-  const float q1 = __fmaf_rn(r, y, q0);
-  return fabsf(q0) >= 1.0e-30f ? q1 : (a == 0.0f ? a : __fdiv_rn(a, d));
+  return copysignf(__fmaf_rn(r, y, q0), a);
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
@@ -166,13 +176,20 @@ amax_finish_kernel(const float* __restrict__ partial, int count, float* __restri
 // batch shard) draws the words the whole view would (sr_cols = cols,
 // sr_col0 = 0 for an unsharded tensor).
 template <int FMT, int RND>
-__device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d, float y, const float (&u)[4]) {
+__device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d, float y, bool exact,
+                                                  const float (&u)[4]) {
   if (RND == 0) {
     // RNE: the conversion of the signed quotient gives sign bit and
-    // magnitude together (the sign of x, also for a zero quotient)
+    // magnitude together (the sign of x, also for a zero quotient; a block
+    // whose scale is 0 has y = 0 and gets magnitude 0)
     float v[4];
+    if (exact) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = d > 0.0f ? div_shared_divisor_signed(xv[j], d, y) : xv[j];
+      for (int j = 0; j < 4; ++j) v[j] = __fdiv_rn(xv[j], d);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = div_shared_divisor_rne(xv[j], d, y);
+    }
     if (FMT == 0) return f32x2_to_e2m1x2(v[0], v[1]) | (f32x2_to_e2m1x2(v[2], v[3]) << 8);
     const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
     return (b01 & 0x3F) | ((b01 >> 2) & 0xFC0) | ((b23 & 0x3F) << 12) | ((b23 & 0x3F00) << 10);
@@ -180,7 +197,7 @@ __device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d,
   uint32_t packed = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float v = d > 0.0f ? div_shared_divisor(fabsf(xv[j]), d, y) : 0.0f;
+    const float v = d > 0.0f ? (exact ? __fdiv_rn(fabsf(xv[j]), d) : div_shared_divisor(fabsf(xv[j]), d, y)) : 0.0f;
     const uint32_t mag = round_sr_mag<FMT>(v, u[j]);
     const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
     const uint32_t code = FMT == 0 ? (mag | (sgn << 3)) : (mag | (sgn << 5));
@@ -211,6 +228,7 @@ __device__ __forceinline__ void quantize_unit(const float4 (&x)[QB][4], const Te
   const float T = ts.T;
   uint32_t scode[QB];
   float d[QB], y[QB];
+  bool exact[QB];
 #pragma unroll
   for (int q = 0; q < QB; ++q) {
     float bmax = 0.0f;
@@ -224,8 +242,9 @@ __device__ __forceinline__ void quantize_unit(const float4 (&x)[QB][4], const Te
     if (T > 0.0f) {
       scode[q] = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
       d[q] = __fmul_rn(e4m3_to_f32(scode[q]), T);
-      y[q] = d[q] > 0.0f ? __frcp_rn(d[q]) : 0.0f;
+      y[q] = d[q] >= kMarksteinMinDivisor ? __frcp_rn(d[q]) : 0.0f;
     }
+    exact[q] = d[q] > 0.0f && d[q] < kMarksteinMinDivisor;
   }
   const int64_t b = br * cb + bc0;
   if (QB == 2) *reinterpret_cast<uint16_t*>(scales + b) = static_cast<uint16_t>(scode[0] | (scode[1] << 8));
@@ -248,7 +267,7 @@ __device__ __forceinline__ void quantize_unit(const float4 (&x)[QB][4], const Te
         u[2] = __uint2float_rn(wd.z >> 8) * s24;
         u[3] = __uint2float_rn(wd.w >> 8) * s24;
       }
-      packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], u);
+      packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], exact[q], u);
     }
     uint8_t* out = codes + (br * 4 + r) * row_bytes;
     if (FMT == 0) {

@@ -91,16 +91,19 @@ def test_rounding_ties_bit_exact(fmt, rnd):
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
 @pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
-def test_division_near_grid_points_with_arbitrary_scales(fmt, rnd):
+@pytest.mark.parametrize("amax", [3.7, 4e-17, 3.7e-18, 3.7e-33, 3.7e-37])
+def test_division_near_grid_points_with_arbitrary_scales(fmt, rnd, amax):
     """Elements within a few ulps of RN(m·d) for every grid value and grid
     midpoint m, with block divisors d = B·T that are not powers of two, so
-    the quotient x/d must be correctly rounded for the code to match."""
+    the quotient x/d must be correctly rounded for the code to match.  The
+    tensor maxima put the divisors in the normal range, just above and below
+    2^-64, near the bottom of the normal range and among the subnormals."""
     rng = np.random.default_rng(11 if fmt == "nvfp4" else 12)
     f = FMT[fmt]
     emax = np.float32(O.element_max(f))
     grid = O.element_grid(f)
     targets = np.concatenate([(grid[:-1] + grid[1:]) / 2, grid[1:]])
-    amax = np.float32(3.7)
+    amax = np.float32(amax)
     T = np.float32(amax / np.float32(448.0 * O.element_max(f)))
     nblocks = 4096
     x = np.zeros((4 * nblocks, 4), np.float32)
@@ -120,6 +123,34 @@ def test_division_near_grid_points_with_arbitrary_scales(fmt, rnd):
     rows, cols = x.shape
     q, c, sc, Tg = gpu_quantize(torch.from_numpy(x), rows, cols, fmt, rnd, seed=5)
     assert_quant_equal(x, rows, cols, fmt, rnd, 5, (c, sc, Tg))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+@pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
+@pytest.mark.parametrize("scale", [1e-13, 1e-20, 1e-36, 1e-40])
+def test_tiny_tensors_bit_exact(fmt, rnd, scale):
+    """Tensors of tiny magnitude, down to subnormal elements: block divisors
+    below 2^-64 or subnormal, where the quantizer divides exactly."""
+    rows, cols = 64, 32
+    x = _rand((rows, cols), 21, scale=scale, outliers=True)
+    q, c, s, T = gpu_quantize(x, rows, cols, fmt, rnd, seed=17)
+    assert_quant_equal(x.numpy(), rows, cols, fmt, rnd, 17, (c, s, T))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "nvfp6"])
+@pytest.mark.parametrize("rnd", [mqv.RNE, mqv.SR])
+def test_zero_scale_blocks_of_a_large_tensor(fmt, rnd):
+    """max|x| = 1e6 makes every block whose maximum is below 2^-10·T·emax
+    (about 2.2) round its E4M3 scale to 0: those elements, up to 2 in
+    magnitude, must get code 0 with their sign, not the code of x itself."""
+    rows, cols = 64, 32
+    rng = np.random.default_rng(8)
+    x = rng.uniform(-2.0, 2.0, (rows, cols)).astype(np.float32)
+    x[0, 0] = 1e6
+    q, c, s, T = gpu_quantize(torch.from_numpy(x), rows, cols, fmt, rnd, seed=4)
+    assert_quant_equal(x, rows, cols, fmt, rnd, 4, (c, s, T))
+    oq = O.quantize(x, FMT[fmt], O.RNE)
+    assert np.count_nonzero(oq.scales == 0) == oq.scales.size - 1
 
 
 def test_zero_tensor_and_negative_zero():
