@@ -4,7 +4,10 @@ One step = one pass of the whole path for one conv layer: quantize X and W
 (round-to-nearest-even) and G_Y (Philox stochastic rounding) into square-block
 NVFP4/NVFP6 form, then the implicit-GEMM forward, weight-gradient and
 input-gradient passes.  `value` is conv TFLOP/s (fwd + wgrad + dgrad FLOPs of
-all ranks / device time of the timed steps, max over ranks).
+all ranks / device time of the timed steps, max over ranks).  On one GPU the
+step is one CUDA graph replay: G_Y's quantization beside X's and W's, the
+forward pass after X and W, the two gradient passes after all three, each
+pass on its own stream.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, bounded sample
