@@ -70,13 +70,14 @@ mqv_status device_error_word(uint32_t** out) {
 
 // ------------------------------------------------------------ quantize geometry
 
-constexpr int64_t kMaxAmaxCtas = 148 * 2;
+constexpr int64_t kMaxAmaxCtas = 148 * 4;
 constexpr int64_t kMaxQuantCtas = 148 * 16;
 
 // One partial maximum per amax CTA; every quantize CTA reduces them before it
-// can scale anything, so keep them few (at most two CTAs per SM, which still
-// holds 64 KB of loads in flight per SM) and give every CTA the same number
-// of kAmaxThreads x 8-float4 chunks.
+// can scale anything, so keep them few (at most four CTAs per SM, 128 KB of
+// loads in flight per SM: two per SM leave large tensors about 5% short of
+// the copy rate) and give every CTA the same number of kAmaxThreads x
+// 8-float4 chunks.
 int64_t amax_ctas(int64_t rows, int64_t cols) {
   const int64_t n4 = rows * cols / 4;
   const int64_t chunk = kAmaxThreads * 8;
