@@ -122,6 +122,27 @@ def test_zero_tensor_and_zero_block():
     assert q.scales[1, 1] == 0 and q.codes[5, 5] == 0x8 and q.codes[4, 4] == 0
 
 
+@pytest.mark.parametrize("rounding", [O.RNE, O.SR])
+def test_zero_scale_block_of_nonzero_elements(rounding):
+    """T = 1 (max|x| = 2688, FP4).  A block whose max is 6·2^-10 has
+    bmax/(T·emax) = 2^-10, the E4M3 tie between 0 and 2^-9, which goes to
+    the even code 0: its elements, though nonzero, get magnitude 0 and keep
+    their sign.  A block max one ulp above rounds the scale up to 2^-9
+    (code 1), and that element becomes 3·(1 + 2^-23) in units of B·T, which
+    rounds to the grid value 3 (code 5) under RNE and to 3 or 4 under SR."""
+    x = np.zeros((8, 8), np.float32)
+    x[0, 0] = 2688.0
+    m = np.float32(6 * 2.0 ** -10)
+    x[4, 4], x[5, 6], x[6, 5] = m, -m / 2, np.float32(0.004)
+    x[4, 0] = np.nextafter(m, np.float32(1))
+    q = O.quantize(x, O.FP4, rounding, seed=3)
+    assert q.T == np.float32(1.0)
+    assert q.scales[1, 1] == 0
+    assert (q.codes[4, 4], q.codes[5, 6], q.codes[6, 5]) == (0, 0x8, 0)
+    assert q.scales[1, 0] == 1
+    assert q.codes[4, 0] == 5 if rounding == O.RNE else q.codes[4, 0] in (5, 6)
+
+
 # ------------------------------------- P3 exactness of representable blocks
 
 @pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
