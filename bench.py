@@ -519,6 +519,38 @@ def run_gpu(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                "pipeline": "inputs in, compute, outputs out on three streams, two device slots"}
 
+        # The link bound of that pipeline: one step's copies alone in each
+        # direction and both directions at once, on the same streams and
+        # pinned buffers (no compute).
+        def copies_ms(up, down, reps=5):
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            done = [torch.cuda.Event(), torch.cuda.Event()]
+            torch.cuda.synchronize()
+            t0.record(cur)
+            for j, (on, st) in enumerate(((up, s_in), (down, s_out))):
+                st.wait_event(t0)
+                with torch.cuda.stream(st):
+                    for _ in range(reps if on else 0):
+                        if st is s_in:
+                            for n, h in (("X", hX), ("W", hW), ("G", hG)):
+                                sets[0][n].copy_(h, non_blocking=True)
+                        else:
+                            for n in ("y", "gw", "gx"):
+                                hout[0][n].copy_(sets[0][n], non_blocking=True)
+                    done[j].record(st)
+                cur.wait_event(done[j])
+            t1.record(cur)
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / reps
+
+        up_ms, down_ms, both_ms = copies_ms(True, False), copies_ms(False, True), copies_ms(True, True)
+        e2e["link"] = {"h2d_gbs": round(h2d / (up_ms * 1e-3) / 1e9, 1),
+                       "d2h_gbs": round(d2h / (down_ms * 1e-3) / 1e9, 1),
+                       "both_ms": round(both_ms, 4),
+                       "frac": round(both_ms / e2e_ms, 4),
+                       "note": "one step's copies in both directions at once, no compute; frac = that "
+                               "time / the pipelined step time"}
+
     del graphs, step_graphs
     torch.cuda.synchronize()
     if world > 1:
