@@ -99,6 +99,25 @@ def test_sr_uniforms_use_counter_i_div_4_and_word_i_mod_4():
     assert np.all((u >= 0) & (u < 1))
 
 
+def test_sr_decisions_by_hand_from_the_known_answer_words():
+    """Seed 0 is Philox key (0, 0), and the first row of a 4-column view is
+    counter (0, 0, 0, 0), whose words the first known-answer vector gives:
+    u = (w >> 8)·2^-24 = 0x6627e8, 0xe169c5, 0xbc57ac, 0x9b00db over 2^24
+    (0.399, 0.8805, 0.7357, 0.6055).  With max|x| = 2688 (T = 1, B = 448)
+    the row 2688, 196, 616, -2240 sits at 6, 0.4375, 1.375, -5 in units of
+    B·T: fractional positions 0, 0.875 (step 0.5), 0.75 (step 0.5), 0.5
+    (step 2).  Round up iff u < f: 6 stays, 0.4375 goes down to 0, 1.375 up
+    to 1.5, -5 down to -4 (codes 7, 0, 3, 0xE).  Round to nearest gives
+    7, 1, 3, 0xE."""
+    x = np.zeros((4, 4), np.float32)
+    x[0] = [2688.0, 196.0, 616.0, -2240.0]
+    q = O.quantize(x, O.FP4, O.SR, seed=0)
+    assert q.T == np.float32(1.0) and q.scales[0, 0] == O.cast_e4m3(np.array([448.0], np.float32))[0]
+    assert [int(c) for c in q.codes[0]] == [7, 0, 3, 0xE]
+    r = O.quantize(x, O.FP4, O.RNE)
+    assert [int(c) for c in r.codes[0]] == [7, 1, 3, 0xE]
+
+
 # ------------------------------------------------ tensor/block scale formula
 
 def test_tensor_scale_formula():
