@@ -116,6 +116,15 @@ def test_sr_decisions_by_hand_from_the_known_answer_words():
     assert [int(c) for c in q.codes[0]] == [7, 0, 3, 0xE]
     r = O.quantize(x, O.FP4, O.RNE)
     assert [int(c) for c in r.codes[0]] == [7, 1, 3, 0xE]
+    # E2M3 (max|x| = 3360, T = 1): 7.5, 0.109375 (f 0.875, step 1/8),
+    # 2.1875 (f 0.75, step 1/4), -4.25 (f 0.5, step 1/2) -> 31, 0, 17, 0x38;
+    # RNE: 31, 1, 17, 0x38 (-4.25 is a tie, to the even code 24)
+    x[0] = [3360.0, 49.0, 980.0, -1904.0]
+    q = O.quantize(x, O.FP6, O.SR, seed=0)
+    assert q.T == np.float32(1.0)
+    assert [int(c) for c in q.codes[0]] == [31, 0, 17, 0x38]
+    r = O.quantize(x, O.FP6, O.RNE)
+    assert [int(c) for c in r.codes[0]] == [31, 1, 17, 0x38]
 
 
 # ------------------------------------------------ tensor/block scale formula
