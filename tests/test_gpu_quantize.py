@@ -153,6 +153,22 @@ def test_zero_scale_blocks_of_a_large_tensor(fmt, rnd):
     assert np.count_nonzero(oq.scales == 0) == oq.scales.size - 1
 
 
+@pytest.mark.parametrize("fmt,row,sr_bytes,rne_bytes", [
+    ("nvfp4", [2688.0, 196.0, 616.0, -2240.0], [0x07, 0xE3], [0x17, 0xE3]),
+    ("nvfp6", [3360.0, 49.0, 980.0, -1904.0], [0x1F, 0x10, 0xE1], [0x5F, 0x10, 0xE1])])
+def test_hand_derived_codes_of_the_known_answer_row(fmt, row, sr_bytes, rne_bytes):
+    """The row whose stochastic rounding is derived by hand from the first
+    Philox4x32-10 known-answer vector (seed 0, counter 0; T = 1, B = 448):
+    SR codes 7, 0, 3, 0xE (E2M1) and 31, 0, 17, 0x38 (E2M3), RNE codes
+    7, 1, 3, 0xE and 31, 1, 17, 0x38, packed by hand; the other rows are 0."""
+    x = torch.zeros(4, 4)
+    x[0] = torch.tensor(row)
+    for rnd, want in ((mqv.SR, sr_bytes), (mqv.RNE, rne_bytes)):
+        q, c, s, T = gpu_quantize(x, 4, 4, fmt, rnd, seed=0)
+        assert T == 1.0 and int(s[0]) == 0x7E            # E4M3 448
+        assert [int(b) for b in c[:len(want)]] == want and not c[len(want):].any()
+
+
 def test_zero_tensor_and_negative_zero():
     x = torch.zeros(16, 8)
     x[1, 1] = -0.0
