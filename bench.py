@@ -608,7 +608,7 @@ def run_gpu(args):
                    "storage": f"{layer.fmt} (4x4 blocks, e4m3 block scales, fp32 tensor scale)",
                    "step": "quantize X,W (RNE) and G_Y (SR); conv fwd, wgrad, dgrad",
                    "l2": f"inputs rotated over {nsets} resident sets ({nsets * per_set / 1e6:.0f} MB > 126 MB L2)",
-                   "launch": ("the whole step (both quantize launches pairs, the three passes on their "
+                   "launch": ("the whole step (both quantize launch pairs, the three passes on their "
                               "streams and the joins) replayed as one CUDA graph captured through the C ABI"
                               if concurrent else "each phase replayed as a CUDA graph captured through the C ABI"),
                    "schedule": ("quantize X,W beside quantize G_Y; fwd after X,W; wgrad and dgrad after "
