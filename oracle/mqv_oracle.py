@@ -54,6 +54,12 @@ Readings where the pages are silent (each also listed in the design notes):
   R21 replay form of a post-ReLU tensor: magnitudes only (3 or 5 bits),
       element i at bits [i·m, i·m + m) of a little-endian bit stream; the
       E4M3 block scales and T are kept as they are.
+  R22 depthwise layers, which the pages keep in BF16 outside the quantized
+      path (section "전제와 한계"): one Kh x Kw filter per channel (groups
+      = C, channel multiplier 1), weights [C][Kh][Kw], activations and
+      gradients in the same [H][W][C][N] layout; every operand rounded to
+      bfloat16 (round to nearest, ties to even), products summed exactly
+      (fp64 here), outputs fp32.
 """
 from __future__ import annotations
 
@@ -603,3 +609,85 @@ def naive_quantize_after_im2col(X: np.ndarray, s: ConvShape, fmt: str, along: st
 def bits_per_element(fmt: str) -> float:
     """Stored bits per element: the element code plus one E4M3 byte per 16."""
     return element_bits(fmt) + 8.0 / 16.0
+
+
+# ---------------------------------------------------------------------------
+# Depthwise layers in BF16 (reading R22).  Not part of quantize-once: the
+# pages keep these layers in BF16 (section "전제와 한계"), so their operands
+# are rounded to bfloat16 and nothing else.
+
+def to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> the nearest bfloat16 value (ties to even), returned as fp32.
+    bfloat16 is the top 16 bits of an fp32 encoding; rounding adds half of
+    the dropped field (0x7FFF, plus the kept field's last bit for ties to
+    even) before truncating.  Finite inputs only."""
+    b = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16 << 16
+    return b.astype(np.uint32).view(np.float32)
+
+
+def _dw_pad(X: np.ndarray, s: ConvShape) -> np.ndarray:
+    Xp = np.zeros((s.H + 2 * s.pad, s.W + 2 * s.pad) + X.shape[2:], dtype=np.float64)
+    Xp[s.pad:s.pad + s.H, s.pad:s.pad + s.W] = X
+    return Xp
+
+
+def _dw_window(Xp: np.ndarray, s: ConvShape, kh: int, kw: int) -> np.ndarray:
+    """The input pixels tap (kh, kw) meets: [Ho][Wo][C][N]."""
+    return Xp[kh:kh + s.stride * (s.Ho - 1) + 1:s.stride, kw:kw + s.stride * (s.Wo - 1) + 1:s.stride]
+
+
+def depthwise_fwd(Wd: np.ndarray, X: np.ndarray, s: ConvShape):
+    """Y[ho,wo,c,n] = sum_{kh,kw} W[c,kh,kw]·X[ho·s+kh-p, wo·s+kw-p, c, n]
+    (zero padding), fp64.  Wd [C][Kh][Kw], X [H][W][C][N] (s.Cin = s.Cout
+    = C).  Returns (Y [Ho][Wo][C][N], S = sum |W·X|)."""
+    Xp = _dw_pad(X, s)
+    Y = np.zeros((s.Ho, s.Wo, s.Cin, s.N))
+    S = np.zeros_like(Y)
+    for kh in range(s.Kh):
+        for kw in range(s.Kw):
+            w = Wd[:, kh, kw].astype(np.float64)[None, None, :, None]
+            x = _dw_window(Xp, s, kh, kw)
+            Y += w * x
+            S += np.abs(w) * np.abs(x)
+    return Y, S
+
+
+def depthwise_wgrad(G: np.ndarray, X: np.ndarray, s: ConvShape):
+    """G_W[c,kh,kw] = sum_{ho,wo,n} G_Y[ho,wo,c,n]·X[ho·s+kh-p, wo·s+kw-p, c, n],
+    fp64.  Returns (G_W [C][Kh][Kw], S)."""
+    Xp = _dw_pad(X, s)
+    G = G.astype(np.float64)
+    GW = np.zeros((s.Cin, s.Kh, s.Kw))
+    S = np.zeros_like(GW)
+    for kh in range(s.Kh):
+        for kw in range(s.Kw):
+            x = _dw_window(Xp, s, kh, kw)
+            GW[:, kh, kw] = (G * x).sum(axis=(0, 1, 3))
+            S[:, kh, kw] = (np.abs(G) * np.abs(x)).sum(axis=(0, 1, 3))
+    return GW, S
+
+
+def depthwise_dgrad(Wd: np.ndarray, G: np.ndarray, s: ConvShape):
+    """G_X, the adjoint of depthwise_fwd in X: every G_Y[ho,wo,c,n] adds
+    W[c,kh,kw]·G_Y to the input pixel tap (kh, kw) read; padding positions
+    are dropped.  Returns (G_X [H][W][C][N], S)."""
+    Gp = np.zeros((s.H + 2 * s.pad, s.W + 2 * s.pad, s.Cin, s.N))
+    Sp = np.zeros_like(Gp)
+    G = G.astype(np.float64)
+    for kh in range(s.Kh):
+        for kw in range(s.Kw):
+            w = Wd[:, kh, kw].astype(np.float64)[None, None, :, None]
+            _dw_window(Gp, s, kh, kw)[...] += w * G
+            _dw_window(Sp, s, kh, kw)[...] += np.abs(w) * np.abs(G)
+    return (Gp[s.pad:s.pad + s.H, s.pad:s.pad + s.W].copy(),
+            Sp[s.pad:s.pad + s.H, s.pad:s.pad + s.W].copy())
+
+
+def depthwise_layer_outputs(X: np.ndarray, Wd: np.ndarray, G: np.ndarray, s: ConvShape):
+    """The three passes of a BF16 depthwise layer from fp32 operands: each
+    operand rounded to bfloat16 first.  Returns {"y": (Y, S), "gw": ...,
+    "gx": ...}."""
+    Xb, Wb, Gb = to_bf16(X), to_bf16(Wd), to_bf16(G)
+    return {"y": depthwise_fwd(Wb, Xb, s), "gw": depthwise_wgrad(Gb, Xb, s),
+            "gx": depthwise_dgrad(Wb, Gb, s)}

@@ -511,3 +511,70 @@ def test_layer_outputs_apply_tensor_scales_and_roles():
     qg2 = O.quantize(G.reshape(s.gy_view()), O.FP4, O.SR, seed=6)
     assert not np.array_equal(qg.codes, qg2.codes)
     assert np.array_equal(qx.codes, O.quantize(X.reshape(s.x_view()), O.FP4, O.RNE).codes)
+
+
+# ----------------------------------- depthwise layers in BF16 (reading R22)
+
+def test_bf16_rounding_by_hand_and_against_torch():
+    """bfloat16 keeps 7 fraction bits.  By hand: 1 + 2^-8 lies halfway
+    between 1 and 1 + 2^-7 and goes to the even 1; 1 + 3·2^-8 lies halfway
+    between 1 + 2^-7 and 1 + 2^-6 and goes to the even 1 + 2^-6; one ulp
+    above a halfway point rounds up.  Then torch's own conversion on random,
+    tiny, subnormal and large values."""
+    half = np.float32(1 + 2.0 ** -8)
+    assert O.to_bf16(np.array([half]))[0] == 1.0
+    assert O.to_bf16(np.array([np.float32(1 + 3 * 2.0 ** -8)]))[0] == np.float32(1 + 2.0 ** -6)
+    assert O.to_bf16(np.array([np.nextafter(half, np.float32(2))]))[0] == np.float32(1 + 2.0 ** -7)
+    assert O.to_bf16(np.array([np.float32(-1 - 2.0 ** -8)]))[0] == -1.0
+    rng = np.random.default_rng(4)
+    x = np.concatenate([rng.standard_normal(100000), rng.standard_normal(1000) * 1e-39,
+                        rng.standard_normal(1000) * 1e37, [0.0, -0.0, 3.0e38]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(O.to_bf16(x).view(np.uint32), ref.view(np.uint32))
+
+
+DW_SHAPES = [O.ConvShape(4, 8, 8, 7, 9, 3, 3, 1, 1), O.ConvShape(4, 8, 8, 9, 7, 3, 3, 2, 1),
+             O.ConvShape(8, 4, 4, 10, 10, 5, 5, 2, 2), O.ConvShape(4, 12, 12, 6, 6, 3, 1, 1, 0)]
+
+
+@pytest.mark.parametrize("s", DW_SHAPES)
+def test_depthwise_passes_match_torch_grouped_conv_fp64(s):
+    """Depthwise fwd, weight and input gradients against torch's grouped
+    convolution (groups = C) in float64, stride and padding included."""
+    rng = np.random.default_rng(2)
+    C = s.Cin
+    X = rng.standard_normal((s.H, s.W, C, s.N))
+    Wd = rng.standard_normal((C, s.Kh, s.Kw))
+    G = rng.standard_normal((s.Ho, s.Wo, C, s.N))
+    Xt = torch.from_numpy(X).permute(3, 2, 0, 1)          # NCHW
+    Wt = torch.from_numpy(Wd).unsqueeze(1)               # C x 1 x Kh x Kw
+    Gt = torch.from_numpy(G).permute(3, 2, 0, 1)
+    Y, S = O.depthwise_fwd(Wd, X, s)
+    ref = torch.nn.functional.conv2d(Xt, Wt, stride=s.stride, padding=s.pad, groups=C)
+    assert np.allclose(Y, ref.permute(2, 3, 1, 0).numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(S >= np.abs(Y) - 1e-12)
+    GW, _ = O.depthwise_wgrad(G, X, s)
+    ref = torch.nn.grad.conv2d_weight(Xt, Wt.shape, Gt, stride=s.stride, padding=s.pad, groups=C)
+    assert np.allclose(GW, ref[:, 0].numpy(), rtol=1e-12, atol=1e-12)
+    GX, _ = O.depthwise_dgrad(Wd, G, s)
+    ref = torch.nn.grad.conv2d_input(Xt.shape, Wt, Gt, stride=s.stride, padding=s.pad, groups=C)
+    assert np.allclose(GX, ref.permute(2, 3, 1, 0).numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("s", DW_SHAPES)
+def test_depthwise_adjoint_identity_and_bf16_operands(s):
+    """<Y, G> = <X, G_X> = <W, G_W> for the three depthwise passes, and the
+    layer function rounds every operand to bfloat16 before the exact sums
+    (its outputs equal the passes on pre-rounded operands)."""
+    rng = np.random.default_rng(3)
+    C = s.Cin
+    X = rng.standard_normal((s.H, s.W, C, s.N)).astype(np.float32)
+    Wd = rng.standard_normal((C, s.Kh, s.Kw)).astype(np.float32)
+    G = rng.standard_normal((s.Ho, s.Wo, C, s.N)).astype(np.float32)
+    out = O.depthwise_layer_outputs(X, Wd, G, s)
+    Xb, Wb, Gb = (O.to_bf16(t).astype(np.float64) for t in (X, Wd, G))
+    a = np.sum(out["y"][0] * Gb)
+    assert math.isclose(a, np.sum(Xb * out["gx"][0]), rel_tol=1e-12, abs_tol=1e-9)
+    assert math.isclose(a, np.sum(Wb * out["gw"][0]), rel_tol=1e-12, abs_tol=1e-9)
+    assert np.array_equal(out["y"][0], O.depthwise_fwd(Wb, Xb, s)[0])
+    assert not np.array_equal(Xb, X.astype(np.float64))     # the rounding did something
