@@ -1,4 +1,4 @@
-"""The data-parallel exchange of the layer step on two CPU ranks (gloo).
+"""The data-parallel exchange of the layer step on two and four CPU ranks (gloo).
 
 Each rank runs its batch shard through `dp.data_parallel_step` with the
 oracle as the kernels: the sharded step must reproduce the single-process
@@ -95,8 +95,10 @@ def _rank_main(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_match_single_process(tmp_path):
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_match_single_process(tmp_path, world):
+    """Two ranks (8 batch items each) and four (4 each; the maxima of X and
+    G_Y then live on ranks 0 and 3)."""
     mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
                        start_method="spawn", join=True)
     X, W, G = _inputs()
