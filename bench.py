@@ -906,10 +906,28 @@ def cpu_baseline(layer: workloads.Layer, budget_s: float = 15.0):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = (time.perf_counter() - t0) / n
-    return {"value": round(3 * sample.flops() / dt / 1e12, 6), "unit": "TFLOP/s",
-            "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{sample.name}: quantize X,W,G_Y + fp64 im2col fwd/wgrad/dgrad with |ab| sums, "
-                      f"{3 * sample.flops() / 1e9:.3f} GFLOP per step, {n} steps in {n * dt:.1f} s"}
+    out = {"value": round(3 * sample.flops() / dt / 1e12, 6), "unit": "TFLOP/s",
+           "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{sample.name}: quantize X,W,G_Y + fp64 im2col fwd/wgrad/dgrad with |ab| sums, "
+                     f"{3 * sample.flops() / 1e9:.3f} GFLOP per step, {n} steps in {n * dt:.1f} s"}
+    # the same sample on one core (BLAS limited to one thread), a third of the budget
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        out["single_core"] = None
+        return out
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        m = 0
+        while True:
+            oracle_step(sample)
+            m += 1
+            if time.perf_counter() - t0 > budget_s / 3:
+                break
+        dt1 = (time.perf_counter() - t0) / m
+    out["single_core"] = {"value": round(3 * sample.flops() / dt1 / 1e12, 6), "cores": 1,
+                          "steps": m}
+    return out
 
 
 def run_reference(args):
