@@ -109,9 +109,10 @@ mqv_status mqv_quantize_workspace_size(int64_t rows, int64_t cols, size_t* bytes
  * round up iff (word>>8)·2^-24 < fractional position).  Two launches: a
  * |x| max reduction into `ws`, then the block quantizer (which finishes the
  * reduction itself).  src: rows x cols fp32, 16-byte aligned, finite (a NaN
- * or infinity gives unspecified codes, never a fault).  Tensors of any
- * finite magnitude, subnormals included, quantize exactly as defined.  out:
- * codes, scales and tscale written; out->rows/cols/fmt must match. */
+ * or infinity gives unspecified codes, never a fault).  Tiny tensors,
+ * subnormal elements included, quantize exactly as defined (blocks whose
+ * divisor B·T is below 2^-64 divide with the IEEE divide).  out: codes,
+ * scales and tscale written; out->rows/cols/fmt must match. */
 mqv_status mqv_quantize_cbf(const float* src, int64_t rows, int64_t cols, int32_t fmt,
                             int32_t rounding, uint64_t seed, const mqv_qtensor* out,
                             void* ws, size_t ws_bytes, void* stream);
