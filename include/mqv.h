@@ -278,6 +278,40 @@ mqv_status mqv_im2col(const mqv_conv_desc* d, const float* x, float* xc, void* s
  * (kh, kw) order.  gc: fp32 [Ho][Wo][Kh·Kw·Cin][N]; gx: fp32 [H][W][Cin][N]. */
 mqv_status mqv_col2im(const mqv_conv_desc* d, const float* gc, float* gx, void* stream);
 
+/* ---- Depthwise layers in BF16 (section "전제와 한계": the pages keep the
+ * depthwise convolutions in BF16, outside quantize-once).  One Kh x Kw
+ * filter per channel (groups = C), stride and zero padding as for
+ * mqv_conv_desc.  Operands are bfloat16 bit patterns (uint16, round to
+ * nearest even from fp32 is the caller's conversion): w [C][Kh][Kw], x and
+ * gx [H][W][C][N], y and gy [Ho][Wo][C][N]; outputs are fp32.  Products are
+ * summed with fp32 FMAs in a fixed order, so results repeat run to run.
+ * Validation: sizes positive, N % 4 == 0, stride >= 1, 0 <= pad < Kh, Kw,
+ * every tensor below 2^31 elements, pointers 16-byte aligned device
+ * memory the caller owns; failures return before anything is launched.
+ * Asynchronous on `stream`. */
+typedef struct {
+  int64_t N, C, H, W, Kh, Kw, stride, pad;
+  int32_t reserved; /* must be 0 */
+  int32_t reserved2; /* must be 0 */
+} mqv_dw_desc;
+
+/* y[ho][wo][c][n] = sum_{kh,kw} w[c][kh][kw]·x[ho·stride+kh-pad][wo·stride+kw-pad][c][n]. */
+mqv_status mqv_dw_fwd(const mqv_dw_desc* d, const void* w, const void* x, float* y, void* stream);
+
+/* gx, the adjoint of mqv_dw_fwd in x: gx[hi][wi][c][n] = sum over the taps
+ * whose output pixel exists of w[c][kh][kw]·gy[ho][wo][c][n]. */
+mqv_status mqv_dw_dgrad(const mqv_dw_desc* d, const void* w, const void* gy, float* gx, void* stream);
+
+/* Workspace bytes of mqv_dw_wgrad (the partial sums of its (ho, wo) parts).
+ * Host-only. */
+mqv_status mqv_dw_wgrad_workspace_size(const mqv_dw_desc* d, size_t* bytes);
+
+/* gw[c][kh][kw] = sum_{ho,wo,n} gy[ho][wo][c][n]·x[ho·stride+kh-pad][wo·stride+kw-pad][c][n]:
+ * partial sums over ranges of output pixels into ws, then added in range
+ * order.  ws: at least mqv_dw_wgrad_workspace_size bytes. */
+mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const void* x, float* gw, void* ws,
+                        size_t ws_bytes, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word that
  * bounded waits inside the conv kernels set when they give up
  * (*flags = 0: none).  Returns MQV_ERR_TIMEOUT if a flag was set. */

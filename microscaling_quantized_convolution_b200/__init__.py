@@ -55,6 +55,12 @@ class QuantJobC(ctypes.Structure):
                 ("out", QTensorC)]
 
 
+class DwDesc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("C", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64),
+                ("Kh", ctypes.c_int64), ("Kw", ctypes.c_int64), ("stride", ctypes.c_int64),
+                ("pad", ctypes.c_int64), ("reserved", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
+
+
 _lib = None
 
 _SIGS = {
@@ -108,6 +114,13 @@ _SIGS = {
                                          ctypes.c_void_p, ctypes.c_void_p]),
     "mqv_replay_dequantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
+    "mqv_dw_fwd": (ctypes.c_int, [ctypes.POINTER(DwDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_void_p]),
+    "mqv_dw_dgrad": (ctypes.c_int, [ctypes.POINTER(DwDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p]),
+    "mqv_dw_wgrad_workspace_size": (ctypes.c_int, [ctypes.POINTER(DwDesc), ctypes.POINTER(ctypes.c_size_t)]),
+    "mqv_dw_wgrad": (ctypes.c_int, [ctypes.POINTER(DwDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
 }
 
 
@@ -446,3 +459,55 @@ def device_errors(stream=None) -> int:
     if st not in (MQV_OK, 5):
         _check(st)
     return f.value
+
+
+# ------------------------------------------- depthwise layers in BF16
+
+def dw_desc(N, C, H, W, Kh, Kw, stride=1, pad=0) -> DwDesc:
+    """Descriptor of a BF16 depthwise layer (one filter per channel)."""
+    return DwDesc(N, C, H, W, Kh, Kw, stride, pad, 0, 0)
+
+
+def dw_out_hw(d: DwDesc) -> tuple[int, int]:
+    return (d.H + 2 * d.pad - d.Kh) // d.stride + 1, (d.W + 2 * d.pad - d.Kw) // d.stride + 1
+
+
+def dw_wgrad_workspace_bytes(d: DwDesc) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().mqv_dw_wgrad_workspace_size(ctypes.byref(d), ctypes.byref(b)))
+    return b.value
+
+
+def dw_fwd(d: DwDesc, w: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
+    """Y [Ho][Wo][C][N] fp32 from bfloat16 w [C][Kh][Kw] and x [H][W][C][N]."""
+    _require_cuda(w, "w", torch.bfloat16)
+    _require_cuda(x, "x", torch.bfloat16)
+    Ho, Wo = dw_out_hw(d)
+    y = y if y is not None else torch.empty((Ho, Wo, d.C, d.N), dtype=torch.float32, device=x.device)
+    _require_cuda(y, "y", torch.float32)
+    _check(lib().mqv_dw_fwd(ctypes.byref(d), w.data_ptr(), x.data_ptr(), y.data_ptr(), _stream(stream)))
+    return y
+
+
+def dw_dgrad(d: DwDesc, w: torch.Tensor, gy: torch.Tensor, gx: torch.Tensor | None = None, stream=None):
+    """G_X [H][W][C][N] fp32 from bfloat16 w and gy [Ho][Wo][C][N]."""
+    _require_cuda(w, "w", torch.bfloat16)
+    _require_cuda(gy, "gy", torch.bfloat16)
+    gx = gx if gx is not None else torch.empty((d.H, d.W, d.C, d.N), dtype=torch.float32, device=gy.device)
+    _require_cuda(gx, "gx", torch.float32)
+    _check(lib().mqv_dw_dgrad(ctypes.byref(d), w.data_ptr(), gy.data_ptr(), gx.data_ptr(), _stream(stream)))
+    return gx
+
+
+def dw_wgrad(d: DwDesc, gy: torch.Tensor, x: torch.Tensor, gw: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None):
+    """G_W [C][Kh][Kw] fp32 from bfloat16 gy and x."""
+    _require_cuda(gy, "gy", torch.bfloat16)
+    _require_cuda(x, "x", torch.bfloat16)
+    gw = gw if gw is not None else torch.empty((d.C, d.Kh, d.Kw), dtype=torch.float32, device=x.device)
+    _require_cuda(gw, "gw", torch.float32)
+    if ws is None:
+        ws = torch.empty(dw_wgrad_workspace_bytes(d), dtype=torch.uint8, device=x.device)
+    _check(lib().mqv_dw_wgrad(ctypes.byref(d), gy.data_ptr(), x.data_ptr(), gw.data_ptr(), ws.data_ptr(),
+                              ws.numel(), _stream(stream)))
+    return gw

@@ -16,6 +16,7 @@
 #include "mqv_conv_kernels.cuh"
 #include "mqv_conv_halo.cuh"
 #include "mqv_conv_wgk.cuh"
+#include "mqv_depthwise.cuh"
 #include "mqv_naive.cuh"
 #include "mqv_quantize.cuh"
 #include "mqv_replay.cuh"
@@ -1020,4 +1021,95 @@ extern "C" mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_q
   float* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch))) return st;
   return run_conv(MQV_OP_WGRAD, d, gy, "gy", x, "x", gw, scratch, kNoAllocScratchBytes, stream);
+}
+
+// ------------------------------------------------- depthwise layers in BF16
+
+namespace {
+
+// Checks a depthwise descriptor and fills the geometry (every tensor below
+// 2^31 elements, so thread indices fit one grid dimension of 2^31 - 1 CTAs).
+mqv_status plan_dw(const mqv_dw_desc* d, DwGeom* g) {
+  if (!d) return fail(MQV_ERR_INVALID_ARG, "null depthwise descriptor");
+  if (d->reserved || d->reserved2)
+    return fail(MQV_ERR_INVALID_ARG, "depthwise descriptor: reserved fields must be 0");
+  if (d->N <= 0 || d->C <= 0 || d->H <= 0 || d->W <= 0 || d->Kh <= 0 || d->Kw <= 0)
+    return fail(MQV_ERR_INVALID_ARG, "depthwise descriptor: sizes must be positive");
+  if (d->N % 4) return fail(MQV_ERR_INVALID_ARG, "depthwise descriptor: N = %lld is not a multiple of 4",
+                            (long long)d->N);
+  if (d->stride < 1 || d->pad < 0 || d->pad >= d->Kh || d->pad >= d->Kw)
+    return fail(MQV_ERR_INVALID_ARG, "depthwise descriptor: need stride >= 1 and 0 <= pad < Kh, Kw");
+  const int64_t ho = (d->H + 2 * d->pad - d->Kh) / d->stride + 1;
+  const int64_t wo = (d->W + 2 * d->pad - d->Kw) / d->stride + 1;
+  if (d->H + 2 * d->pad < d->Kh || d->W + 2 * d->pad < d->Kw || ho < 1 || wo < 1)
+    return fail(MQV_ERR_INVALID_ARG, "depthwise descriptor: the kernel is larger than the padded input");
+  const int64_t lim = int64_t(1) << 31;
+  if (d->H * d->W > lim / d->C / d->N || ho * wo > lim / d->C / d->N || d->Kh * d->Kw > lim / d->C)
+    return fail(MQV_ERR_UNSUPPORTED, "depthwise layer too large (a tensor of 2^31 elements or more)");
+  *g = dw_geom(d->N, d->C, d->H, d->W, d->Kh, d->Kw, d->stride, d->pad);
+  return MQV_OK;
+}
+
+unsigned dw_grid(int64_t total) { return static_cast<unsigned>((total + kDwThreads - 1) / kDwThreads); }
+
+}  // namespace
+
+extern "C" mqv_status mqv_dw_wgrad_workspace_size(const mqv_dw_desc* d, size_t* bytes) {
+  DwGeom g;
+  mqv_status st = plan_dw(d, &g);
+  if (st) return st;
+  if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
+  *bytes = (size_t)((dw_wgrad_threads(g) * (int64_t)sizeof(float) + 255) / 256 * 256);
+  return ok();
+}
+
+extern "C" mqv_status mqv_dw_fwd(const mqv_dw_desc* d, const void* w, const void* x, float* y, void* stream) {
+  DwGeom g;
+  mqv_status st = plan_dw(d, &g);
+  if (st) return st;
+  if (!w || !x || !y || !aligned16(w) || !aligned16(x) || !aligned16(y))
+    return fail(MQV_ERR_INVALID_ARG, "w, x and y must be 16-byte aligned device pointers");
+  const int64_t total = dw_fwd_threads(g);
+  dw_fwd_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(x), y);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "depthwise fwd launch");
+  return ok();
+}
+
+extern "C" mqv_status mqv_dw_dgrad(const mqv_dw_desc* d, const void* w, const void* gy, float* gx,
+                                   void* stream) {
+  DwGeom g;
+  mqv_status st = plan_dw(d, &g);
+  if (st) return st;
+  if (!w || !gy || !gx || !aligned16(w) || !aligned16(gy) || !aligned16(gx))
+    return fail(MQV_ERR_INVALID_ARG, "w, gy and gx must be 16-byte aligned device pointers");
+  const int64_t total = dw_dgrad_threads(g);
+  dw_dgrad_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(gy), gx);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "depthwise dgrad launch");
+  return ok();
+}
+
+extern "C" mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const void* x, float* gw, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  DwGeom g;
+  mqv_status st = plan_dw(d, &g);
+  if (st) return st;
+  if (!gy || !x || !gw || !aligned16(gy) || !aligned16(x) || !aligned16(gw))
+    return fail(MQV_ERR_INVALID_ARG, "gy, x and gw must be 16-byte aligned device pointers");
+  const int64_t total = dw_wgrad_threads(g);
+  const size_t need = (size_t)total * sizeof(float);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes required", need);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(ws);
+  dw_wgrad_kernel<<<dw_grid(total), kDwThreads, 0, s>>>(g, total, static_cast<const uint16_t*>(gy),
+                                                        static_cast<const uint16_t*>(x), part);
+  const int64_t nw = g.C * g.Kh * g.Kw;
+  dw_wgrad_reduce_kernel<<<dw_grid(nw), kDwThreads, 0, s>>>(g, nw, part, gw);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "depthwise wgrad launch");
+  return ok();
 }

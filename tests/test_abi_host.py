@@ -165,3 +165,24 @@ def test_cuda_path_has_no_cpu_fallback():
     x = torch.zeros(16)
     with pytest.raises(ValueError):
         mqv.quantize(x, 4, 4, "nvfp4")
+
+
+def test_depthwise_entry_points_validate_before_launching(lib):
+    """Workspace of the BF16 depthwise weight gradient (parts x C x Kh x Kw
+    floats, rounded up to 256 bytes) and descriptor or pointer errors
+    returned without a launch."""
+    d = mqv.dw_desc(16, 32, 20, 20, 3, 3, 1, 1)       # 400 pixels: 16 parts
+    assert mqv.dw_wgrad_workspace_bytes(d) == 16 * 32 * 9 * 4
+    d = mqv.dw_desc(32, 2, 56, 56, 3, 3, 1, 1)        # 3136 pixels x 8 lanes / 1024: 25 parts
+    assert mqv.dw_wgrad_workspace_bytes(d) == 2048    # 25 x 18 x 4 = 1800, rounded up
+    for bad in (mqv.dw_desc(6, 2, 4, 4, 3, 3, 1, 1), mqv.dw_desc(4, 2, 4, 4, 3, 3, 0, 1),
+                mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 3), mqv.dw_desc(4, 0, 4, 4, 3, 3, 1, 1),
+                mqv.dw_desc(4, 2, 2, 2, 5, 5, 1, 1)):
+        with pytest.raises(mqv.MqvError):
+            mqv.dw_wgrad_workspace_bytes(bad)
+    d = mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 1)
+    invalid = 1                                        # MQV_ERR_INVALID_ARG
+    assert lib.mqv_dw_fwd(ctypes.byref(d), None, None, None, None) == invalid
+    assert lib.mqv_dw_dgrad(ctypes.byref(d), None, None, None, None) == invalid
+    assert lib.mqv_dw_wgrad(ctypes.byref(d), None, None, None, None, 0, None) == invalid
+    assert lib.mqv_dw_fwd(None, None, None, None, None) == invalid
