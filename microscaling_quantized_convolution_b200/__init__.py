@@ -468,33 +468,51 @@ def dw_desc(N, C, H, W, Kh, Kw, stride=1, pad=0) -> DwDesc:
     return DwDesc(N, C, H, W, Kh, Kw, stride, pad, 0, 0)
 
 
-def dw_out_hw(d: DwDesc) -> tuple[int, int]:
-    return (d.H + 2 * d.pad - d.Kh) // d.stride + 1, (d.W + 2 * d.pad - d.Kw) // d.stride + 1
-
-
 def dw_wgrad_workspace_bytes(d: DwDesc) -> int:
+    """Workspace bytes of dw_wgrad; raises MqvError for an invalid descriptor
+    (the library's own check, which every dw_* call runs first)."""
     b = ctypes.c_size_t()
     _check(lib().mqv_dw_wgrad_workspace_size(ctypes.byref(d), ctypes.byref(b)))
     return b.value
 
 
+def dw_out_hw(d: DwDesc) -> tuple[int, int]:
+    """Output pixel grid (Ho, Wo) of a validated descriptor."""
+    dw_wgrad_workspace_bytes(d)
+    return (d.H + 2 * d.pad - d.Kh) // d.stride + 1, (d.W + 2 * d.pad - d.Kw) // d.stride + 1
+
+
+def _dw_numel(t: torch.Tensor, name: str, n: int):
+    # the C ABI takes no tensor sizes: a short tensor would be read or
+    # written out of bounds on the device, so the sizes are checked here
+    if t.numel() != n:
+        raise ValueError(f"{name}: {t.numel()} elements, the descriptor needs {n}")
+
+
 def dw_fwd(d: DwDesc, w: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None, stream=None):
     """Y [Ho][Wo][C][N] fp32 from bfloat16 w [C][Kh][Kw] and x [H][W][C][N]."""
+    Ho, Wo = dw_out_hw(d)
     _require_cuda(w, "w", torch.bfloat16)
     _require_cuda(x, "x", torch.bfloat16)
-    Ho, Wo = dw_out_hw(d)
     y = y if y is not None else torch.empty((Ho, Wo, d.C, d.N), dtype=torch.float32, device=x.device)
     _require_cuda(y, "y", torch.float32)
+    _dw_numel(w, "w", d.C * d.Kh * d.Kw)
+    _dw_numel(x, "x", d.H * d.W * d.C * d.N)
+    _dw_numel(y, "y", Ho * Wo * d.C * d.N)
     _check(lib().mqv_dw_fwd(ctypes.byref(d), w.data_ptr(), x.data_ptr(), y.data_ptr(), _stream(stream)))
     return y
 
 
 def dw_dgrad(d: DwDesc, w: torch.Tensor, gy: torch.Tensor, gx: torch.Tensor | None = None, stream=None):
     """G_X [H][W][C][N] fp32 from bfloat16 w and gy [Ho][Wo][C][N]."""
+    Ho, Wo = dw_out_hw(d)
     _require_cuda(w, "w", torch.bfloat16)
     _require_cuda(gy, "gy", torch.bfloat16)
     gx = gx if gx is not None else torch.empty((d.H, d.W, d.C, d.N), dtype=torch.float32, device=gy.device)
     _require_cuda(gx, "gx", torch.float32)
+    _dw_numel(w, "w", d.C * d.Kh * d.Kw)
+    _dw_numel(gy, "gy", Ho * Wo * d.C * d.N)
+    _dw_numel(gx, "gx", d.H * d.W * d.C * d.N)
     _check(lib().mqv_dw_dgrad(ctypes.byref(d), w.data_ptr(), gy.data_ptr(), gx.data_ptr(), _stream(stream)))
     return gx
 
@@ -502,10 +520,14 @@ def dw_dgrad(d: DwDesc, w: torch.Tensor, gy: torch.Tensor, gx: torch.Tensor | No
 def dw_wgrad(d: DwDesc, gy: torch.Tensor, x: torch.Tensor, gw: torch.Tensor | None = None,
              ws: torch.Tensor | None = None, stream=None):
     """G_W [C][Kh][Kw] fp32 from bfloat16 gy and x."""
+    Ho, Wo = dw_out_hw(d)
     _require_cuda(gy, "gy", torch.bfloat16)
     _require_cuda(x, "x", torch.bfloat16)
     gw = gw if gw is not None else torch.empty((d.C, d.Kh, d.Kw), dtype=torch.float32, device=x.device)
     _require_cuda(gw, "gw", torch.float32)
+    _dw_numel(gy, "gy", Ho * Wo * d.C * d.N)
+    _dw_numel(x, "x", d.H * d.W * d.C * d.N)
+    _dw_numel(gw, "gw", d.C * d.Kh * d.Kw)
     if ws is None:
         ws = torch.empty(dw_wgrad_workspace_bytes(d), dtype=torch.uint8, device=x.device)
     _check(lib().mqv_dw_wgrad(ctypes.byref(d), gy.data_ptr(), x.data_ptr(), gw.data_ptr(), ws.data_ptr(),

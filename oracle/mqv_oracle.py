@@ -197,14 +197,28 @@ def philox4x32_10(ctr: np.ndarray, key) -> np.ndarray:
 
 
 def sr_uniforms(seed: int, index: np.ndarray) -> np.ndarray:
-    """u = (w >> 8)·2^-24 for the element indices given (reading R8)."""
-    index = np.asarray(index, dtype=np.uint64)
+    """u = (w >> 8)·2^-24 for the element indices given (reading R8).
+
+    Element i uses word i & 3 of the Philox block of counter i >> 2.  When
+    the indices cover a compact range of counters (a whole view or a band of
+    one), each counter's block is computed once and its four words serve the
+    four elements that share it; otherwise one block per element."""
+    index = np.asarray(index, dtype=np.uint64).reshape(-1)
+    if index.size == 0:
+        return np.zeros(0, np.float64)
     group = index >> np.uint64(2)
-    ctr = np.zeros((index.size, 4), dtype=np.uint64)
-    ctr[:, 0] = group & np.uint64(0xFFFFFFFF)
-    ctr[:, 1] = group >> np.uint64(32)
+    g0 = int(group.min())
+    span = int(group.max()) - g0 + 1
+    if span <= index.size:
+        counters = np.arange(g0, g0 + span, dtype=np.uint64)
+        row = (group - np.uint64(g0)).astype(np.int64)
+    else:
+        counters, row = group, np.arange(index.size)
+    ctr = np.zeros((counters.size, 4), dtype=np.uint64)
+    ctr[:, 0] = counters & np.uint64(0xFFFFFFFF)
+    ctr[:, 1] = counters >> np.uint64(32)
     words = philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
-    w = words[np.arange(index.size), (index & np.uint64(3)).astype(np.int64)]
+    w = words[row, (index & np.uint64(3)).astype(np.int64)]
     return (w >> np.uint32(8)).astype(np.float64) * 2.0 ** -24
 
 

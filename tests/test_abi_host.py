@@ -186,3 +186,37 @@ def test_depthwise_entry_points_validate_before_launching(lib):
     assert lib.mqv_dw_dgrad(ctypes.byref(d), None, None, None, None) == invalid
     assert lib.mqv_dw_wgrad(ctypes.byref(d), None, None, None, None, 0, None) == invalid
     assert lib.mqv_dw_fwd(None, None, None, None, None) == invalid
+
+
+def test_depthwise_bindings_validate_before_shape_arithmetic(lib):
+    """The Python calls ask the library to check the descriptor before they
+    size anything, so a bad descriptor raises MqvError (a stride of 0 must
+    not become a Python ZeroDivisionError)."""
+    import torch
+    x = torch.zeros(16, dtype=torch.bfloat16)
+    y = torch.zeros(16, dtype=torch.float32)
+    for bad in (mqv.dw_desc(6, 2, 4, 4, 3, 3, 1, 1), mqv.dw_desc(4, 2, 4, 4, 3, 3, 0, 1),
+                mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 3)):
+        for call in (lambda: mqv.dw_fwd(bad, x, x, y), lambda: mqv.dw_dgrad(bad, x, x, y),
+                     lambda: mqv.dw_wgrad(bad, x, x, y), lambda: mqv.dw_out_hw(bad)):
+            with pytest.raises(mqv.MqvError):
+                call()
+
+
+def test_noalloc_scratch_covers_every_planned_layer(lib):
+    """The weight gradient's split planner keeps its partial sums under the
+    32 MiB array of mqv_conv_wgrad_noalloc for every shape (at most 148
+    tiles of 128 x 384 fp32), so no layer of the benchmarked workloads, nor
+    any shape of a wide sweep, is rejected by that entry point.  Sizing is a
+    host call: no GPU needed."""
+    import workloads
+    shapes = [l.dims() | {"fmt": l.fmt} for l in
+              [workloads.tiny_layer(), workloads.resnet18_layer2()] + workloads.resnet18_body()
+              + workloads.yolov8n_mix()]
+    for cin in (4, 16, 64, 128, 256, 512, 1024):
+        for cout in (16, 64, 128, 384, 512, 2048):
+            for k in (1, 3, 5):
+                shapes.append(dict(N=32, Cin=cin, Cout=cout, H=14, W=14, Kh=k, Kw=k, stride=1,
+                                   pad=k // 2, fmt="nvfp4"))
+    worst = max(mqv.conv_workspace_bytes(mqv.conv_desc(**s), mqv.OP_WGRAD) for s in shapes)
+    assert 0 < worst <= 148 * 128 * 384 * 4 < 32 << 20

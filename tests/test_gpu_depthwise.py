@@ -1,6 +1,6 @@
 """GPU parity of the BF16 depthwise passes (reading R22) against the oracle:
 fwd, input and weight gradients within the parity tolerance, the same bits
-on a second run.  Collected last: the newest kernels of the library."""
+on a second run; the bindings reject bad descriptors and short tensors."""
 import numpy as np
 import pytest
 import torch
@@ -43,4 +43,26 @@ def test_depthwise_rejects_bad_descriptors():
                 mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 3)):      # pad >= K
         with pytest.raises(mqv.MqvError):
             mqv.dw_fwd(bad, x, x, y)
+    assert mqv.device_errors() == 0
+
+
+def test_depthwise_rejects_short_tensors():
+    """The C ABI takes no tensor sizes; the bindings compare every operand's
+    element count with the descriptor before anything is launched."""
+    d = mqv.dw_desc(4, 8, 6, 6, 3, 3, 1, 1)
+    w = torch.zeros(8 * 9, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(6 * 6 * 8 * 4, dtype=torch.bfloat16, device="cuda")
+    short = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        mqv.dw_fwd(d, w, short)
+    with pytest.raises(ValueError):
+        mqv.dw_fwd(d, short, x)
+    with pytest.raises(ValueError):
+        mqv.dw_fwd(d, w, x, torch.zeros(16, device="cuda"))
+    with pytest.raises(ValueError):
+        mqv.dw_dgrad(d, w, short)
+    with pytest.raises(ValueError):
+        mqv.dw_wgrad(d, short, x)
+    with pytest.raises(ValueError):
+        mqv.dw_wgrad(d, x, x, torch.zeros(16, device="cuda"))
     assert mqv.device_errors() == 0

@@ -99,6 +99,21 @@ def test_sr_uniforms_use_counter_i_div_4_and_word_i_mod_4():
     assert np.all((u >= 0) & (u < 1))
 
 
+def test_sr_uniforms_sparse_and_compact_index_sets_agree():
+    """The words of an index do not depend on which other indices are asked
+    for: a scattered set (one Philox block per element) and each index on
+    its own (one block per counter) give the same u; so does a contiguous
+    range against its elements taken in reverse order."""
+    rng = np.random.default_rng(3)
+    idx = rng.choice(1 << 40, 64, replace=False).astype(np.uint64)
+    seed = 0xDEADBEEF12
+    together = O.sr_uniforms(seed, idx)
+    alone = np.array([O.sr_uniforms(seed, idx[i:i + 1])[0] for i in range(idx.size)])
+    assert np.array_equal(together, alone)
+    rng_idx = np.arange(1000, 1400, dtype=np.uint64)
+    assert np.array_equal(O.sr_uniforms(seed, rng_idx)[::-1], O.sr_uniforms(seed, rng_idx[::-1]))
+
+
 def test_sr_decisions_by_hand_from_the_known_answer_words():
     """Seed 0 is Philox key (0, 0), and the first row of a 4-column view is
     counter (0, 0, 0, 0), whose words the first known-answer vector gives:
@@ -279,6 +294,73 @@ def test_sr_depends_on_seed_only_through_codes():
 
 
 # ------------------------------------------------------- packing (R16)
+
+def _outlier_tensor(rows, cols, seed):
+    """Signed N(0,1) with 0.1 % of the entries x100 and the largest one
+    placed in the first rows, outside every band below."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    idx = rng.choice(x.size, max(1, x.size // 1000), replace=False)
+    x.reshape(-1)[idx] *= np.float32(100)
+    r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    x[[0, r]] = x[[r, 0]]
+    return x
+
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+@pytest.mark.parametrize("rounding", [O.RNE, O.SR])
+def test_band_with_global_amax_equals_rows_of_whole_view(fmt, rounding):
+    """Section "무엇과 다른가" takes T from max|X| of the whole tensor, and the
+    stochastic-rounding counter is the element's index in the whole view
+    (reading R8); so a band of rows quantized with the whole view's max|x|
+    and its row offset is exactly those rows of the whole-view result: codes,
+    scales and T.  The band below holds none of the largest elements."""
+    x = _outlier_tensor(64, 24, 11)
+    whole = O.quantize(x, fmt, rounding, seed=77)
+    amax = float(np.max(np.abs(x)))
+    assert np.max(np.abs(x[16:48])) < amax
+    for r0, r1 in ((16, 48), (4, 8), (60, 64), (0, 64)):
+        band = O.quantize(x[r0:r1], fmt, rounding, seed=77, amax=amax, row_offset=r0)
+        assert band.T == whole.T
+        assert np.array_equal(band.codes, whole.codes[r0:r1])
+        assert np.array_equal(band.scales, whole.scales[r0 // 4:r1 // 4])
+    if rounding == O.SR:
+        # the offset matters: numbering the band from row 0 draws other words
+        wrong = O.quantize(x[16:48], fmt, rounding, seed=77, amax=amax, row_offset=0)
+        assert not np.array_equal(wrong.codes, whole.codes[16:48])
+
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+@pytest.mark.parametrize("rounding", [O.RNE, O.SR])
+def test_column_window_equals_columns_of_whole_view(fmt, rounding):
+    """A batch shard: columns [c0, c0 + w) of the [rows][cols] view (batch
+    items c0.. of every (pixel, channel) row), quantized with the global
+    max|x|, its column offset and the whole view's column count, is exactly
+    those columns of the whole-view result (blocks never straddle a shard
+    since c0 and w are multiples of 4); a band of rows of a shard likewise."""
+    x = _outlier_tensor(32, 48, 12)
+    whole = O.quantize(x, fmt, rounding, seed=5)
+    amax = float(np.max(np.abs(x)))
+    for c0, w in ((0, 16), (16, 16), (32, 16), (8, 4), (44, 4)):
+        win = O.quantize(x[:, c0:c0 + w], fmt, rounding, seed=5, amax=amax, col_offset=c0, total_cols=48)
+        assert win.T == whole.T
+        assert np.array_equal(win.codes, whole.codes[:, c0:c0 + w])
+        assert np.array_equal(win.scales, whole.scales[:, c0 // 4:(c0 + w) // 4])
+    both = O.quantize(x[8:20, 20:28], fmt, rounding, seed=5, amax=amax, row_offset=8, col_offset=20,
+                      total_cols=48)
+    assert np.array_equal(both.codes, whole.codes[8:20, 20:28])
+    assert np.array_equal(both.scales, whole.scales[2:5, 5:7])
+
+
+def test_band_amax_sets_the_tensor_scale_formula():
+    """With amax given, T = fp32(amax / (448·emax)) exactly as for the whole
+    tensor (T depends on the band only through amax)."""
+    x = _outlier_tensor(16, 16, 13)
+    for fmt, emax in ((O.FP4, 6.0), (O.FP6, 7.5)):
+        for amax in (1.0, 3.0, 1234.5, 1e-20):
+            q = O.quantize(x[:8], fmt, O.RNE, amax=amax)
+            assert q.T == np.float32(np.float32(amax) / np.float32(448.0 * emax))
+
 
 def test_packing_bit_layout():
     assert list(O.pack_codes(np.array([[1, 2, 15, 0]]), O.FP4)) == [0x21, 0x0F]
