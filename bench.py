@@ -674,6 +674,8 @@ def run_sweeps(args, dev, peaks):
         buffers: pack and unpack (0.5 + 0.375 B moved per element) and
         values read straight back (0.375 + 1/16 B read, 4 B written),
         beside mqv_dequantize of the full codes;
+      - depthwise_bf16: the BF16 depthwise passes on YOLOv26n-style
+        3x3 layers, against bytes / copy rate;
       - resnet18_body and yolov8n_mix: every layer's step (quantize, fwd,
         wgrad, dgrad) timed phase by phase with L2 flushed before each
         phase; per-network sums against the sum of per-pass rooflines."""
@@ -733,6 +735,36 @@ def run_sweeps(args, dev, peaks):
         torch.cuda.empty_cache()
     res["replay_quantize"] = rq
     res["replay_form"] = rf
+
+    # depthwise 3x3 layers in BF16 (outside quantize-once): HBM-bound, so
+    # each pass against bytes / copy rate, algorithmic bytes = the two bf16
+    # operands read once (2 B/element) + the fp32 output written once
+    dw = []
+    for C, H, stv in workloads.DEPTHWISE_SHAPES:
+        N = workloads.DEPTHWISE_N
+        x, w, gy = (t.to(torch.bfloat16).contiguous()
+                    for t in workloads.make_depthwise_inputs(C, H, stv, N, seed=C + H, device=dev))
+        d = mqv.dw_desc(N, C, H, H, 3, 3, stv, 1)
+        ho, _ = mqv.dw_out_hw(d)
+        y = torch.empty(ho * ho * C * N, device=dev)
+        gx = torch.empty(H * H * C * N, device=dev)
+        gw = torch.empty(C * 9, device=dev)
+        wsd = torch.empty(max(16, mqv.dw_wgrad_workspace_bytes(d)), dtype=torch.uint8, device=dev)
+        nx, ny, nw = H * H * C * N, ho * ho * C * N, C * 9
+        calls = {"fwd": (lambda: mqv.dw_fwd(d, w, x, y), 2 * (nw + nx) + 4 * ny),
+                 "dgrad": (lambda: mqv.dw_dgrad(d, w, gy, gx), 2 * (nw + ny) + 4 * nx),
+                 "wgrad": (lambda: mqv.dw_wgrad(d, gy, x, gw, ws=wsd), 2 * (ny + nx) + 4 * nw)}
+        ent = {"C": C, "H": H, "stride": stv, "N": N}
+        for name, (fn, nbytes) in calls.items():
+            for _ in range(3):
+                fn()
+            ms = _timed(torch, fn, 10, flush)
+            launches += 13 * (2 if name == "wgrad" else 1)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            ent[name] = {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4)}
+        dw.append(ent)
+        del x, w, gy, y, gx, gw, wsd
+    res["depthwise_bf16"] = dw
 
     for net, layers in (("resnet18_body", workloads.resnet18_body()), ("yolov8n_mix", workloads.yolov8n_mix())):
         tot = {"quantize": 0.0, "fwd": 0.0, "wgrad": 0.0, "dgrad": 0.0}

@@ -89,7 +89,8 @@ int64_t amax_ctas(int64_t rows, int64_t cols) {
 
 int64_t quant_ctas(int64_t rows, int64_t cols) {
   const int64_t nb = rows * cols / 16;
-  int64_t g = (nb + kQuantThreads - 1) / kQuantThreads;
+  const int64_t per_cta = static_cast<int64_t>(kQuantThreads) * kQuantUnits;
+  int64_t g = (nb + per_cta - 1) / per_cta;
   if (g < 1) g = 1;
   return g < kMaxQuantCtas ? g : kMaxQuantCtas;
 }
@@ -145,7 +146,6 @@ PhiloxKeys philox_keys(uint64_t seed) {
   return k;
 }
 
-// One 4 x 4 block per work unit (QB = 1): the fewest registers per thread.
 QuantArgs make_quant_args(const float* src, int64_t rows, int64_t cols, uint64_t seed, int64_t sr_cols,
                           int64_t sr_col0, const mqv_qtensor* out) {
   QuantArgs qa;
@@ -158,14 +158,14 @@ QuantArgs make_quant_args(const float* src, int64_t rows, int64_t cols, uint64_t
   qa.keys = philox_keys(seed);
   qa.sr_cols = sr_cols;
   qa.sr_col0 = sr_col0;
-  qa.dcu = make_fastdiv(cols / 4);
+  qa.dcb = make_fastdiv(cols / 4);
   return qa;
 }
 
 template <int FMT, int RND>
 void launch_quantize(const QuantArgs& qa, const float* amax_src, int amax_count, cudaStream_t st) {
   const unsigned g = (unsigned)quant_ctas(qa.rows, qa.cols);
-  quantize_kernel<FMT, RND, 1><<<g, kQuantThreads, 0, st>>>(qa, amax_src, amax_count);
+  quantize_kernel<FMT, RND><<<g, kQuantThreads, 0, st>>>(qa, amax_src, amax_count);
 }
 
 mqv_status enqueue_quantize(const float* src, int64_t rows, int64_t cols, int32_t fmt,
@@ -637,7 +637,6 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
     qj.qa = make_quant_args(j.src, j.rows, j.cols, j.seed, j.cols, 0, &j.out);
     qj.fmt = j.fmt;
     qj.rounding = j.rounding;
-    qj.qb = 1;
     qj.amax_cta0 = a;
     qj.amax_ctas = (int)amax_ctas(j.rows, j.cols);
     qj.quant_cta0 = q;

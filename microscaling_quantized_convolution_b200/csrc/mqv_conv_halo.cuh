@@ -58,6 +58,7 @@ struct HaloBars {
   uint64_t bempty[kHaloBStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t last_full;   // the CTA's last tile accumulated (one phase; see the producers' last epilogue)
   uint32_t tmem;
 };
 
@@ -254,6 +255,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       mbar_init(&bars->acc_full[a], 1);
       mbar_init(&bars->acc_empty[a], kV2EpiWarps * 32);
     }
+    mbar_init(&bars->last_full, 1);
     fence_mbar_init();
   }
   if (warp == kV2MmaWarp) {
@@ -332,6 +334,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
           }
         }
         mma_commit(&bars->acc_full[acc]);
+        if (tile + static_cast<int>(gridDim.x) >= p.tiles) mma_commit(&bars->last_full);
       }
     }
   } else if (warp == kV2LoadWarp) {
@@ -405,7 +408,11 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       const int ltile_last = static_cast<int>(blockIdx.x) + lit * static_cast<int>(gridDim.x);
       const int pw = warp - kV2ProdWarp0;
       float amax = 0.f;
-      mbar_wait_bounded(&bars->acc_full[lit & 1], (lit >> 1) & 1, p.err, kErrWaitDone);
+      // The producers can finish their last stage more than one accumulator
+      // phase ahead of the MMAs (a 1 x 1 layer has one stage a tile), and a
+      // parity wait on acc_full would then alias an earlier phase: the last
+      // tile has its own single-phase barrier.
+      mbar_wait_bounded(&bars->last_full, 0, p.err, kErrWaitDone);
       tc_fence_after();
       halo_epilogue_tile(p, g, bars->tmem, lit & 1, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
                          1 + pw / 4, 4, amax);

@@ -37,27 +37,37 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& k) {
   return c;
 }
 
-// ------------------------------------------------- element rounding (a >= 0)
+// ------------------------------------------------- element rounding
 // Round-to-nearest-even onto the element grid is the hardware conversion
-// (cvt.rn.satfinite.e2m1x2 / e2m3x2, see mqv_ptx.cuh).  For stochastic
-// rounding the grid is read as a binary format: with E = floor(log2(max(a, 1)))
-// the step on [2^E, 2^(E+1)) (and on [0, 1) for E = 0) is 2^(E-1) for E2M1
-// (0.5, 1, 2) and 2^(E-3) for E2M3 (1/8, 1/4, 1/2), and the magnitude code
-// below a is floor(a / step) + 2E (E2M1) or + 8E (E2M3).  q = a / step is a
-// power-of-two scaling and frac(q) = q - floor(q) is exact, so "round up
-// iff u < frac(q)" is decided exactly.  floor(q) comes from one add rounded
-// toward -inf onto 2^23 (the integer lands in the low mantissa bits), which
-// keeps the conversion pipe free; codes past the largest saturate.
+// (cvt.rn.satfinite.e2m1x2 / e2m3x2, see mqv_ptx.cuh).
+//
+// Stochastic rounding reads the grid as a binary format: with
+// E = floor(log2(max(a, 1))) the step on [2^E, 2^(E+1)) (and on [0, 1) for
+// E = 0) is 2^(E-1) for E2M1 (0.5, 1, 2) and 2^(E-3) for E2M3 (1/8, 1/4,
+// 1/2), and the magnitude code of the grid point at or below a is
+// floor(q) + 2E (E2M1) or + 8E (E2M3), q = a / step (a power-of-two
+// scaling, exact).  "Round up iff u < frac(q)", u = (w >> 8)·2^-24, gives
+// floor(q) + [u < frac(q)] = ceil(q - u): q - u lies in (floor(q) - 1,
+// floor(q) + 1) and exceeds floor(q) exactly when u < frac(q); a value on the
+// grid (frac(q) = 0) stays.  ceil(q - u) takes two operations rounded toward
+// +inf: z = RU(q - u), one FMA of the integer w >> 8 with -2^-24 (rounding
+// upward never passes an integer, so ceil(z) = ceil(q - u)), then
+// RU(z + 1.5·2^23), whose ulp is 1, so its low mantissa bits are ceil(z)
+// for z in (-1, 2^22).  Codes past the largest saturate.
 template <int FMT>
-__device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
-  const uint32_t eb = __float_as_uint(fmaxf(a, 1.0f)) & 0x7F800000u;             // (127 + E) << 23
-  const float inv = __uint_as_float((FMT == 0 ? 0x7F800000u : 0x80800000u) - eb);  // 1 / step
-  const float q = __fmul_rn(a, inv);
-  const float t = __fadd_rd(q, 8388608.0f);                                        // 2^23 + floor(q)
-  const float f = __fsub_rn(q, __fsub_rn(t, 8388608.0f));
-  const uint32_t piece = FMT == 0 ? (eb >> 22) - 254u : (eb >> 20) - 1016u;      // 2E or 8E
-  const uint32_t mag = (__float_as_uint(t) - 0x4B000000u) + piece + (u < f ? 1u : 0u);
-  return min(mag, FMT == 0 ? 7u : 31u);
+__device__ __forceinline__ void round_sr_mag2(float2 a, uint32_t w0, uint32_t w1, uint32_t& m0, uint32_t& m1) {
+  constexpr uint32_t kInv = FMT == 0 ? 0x7F800000u : 0x80800000u;    // 1 / step = bits kInv - (127 + E) << 23
+  constexpr uint32_t kTop = FMT == 0 ? 7u : 31u;
+  const uint32_t e0 = max(__float_as_uint(a.x), 0x3F800000u) & 0x7F800000u;
+  const uint32_t e1 = max(__float_as_uint(a.y), 0x3F800000u) & 0x7F800000u;
+  const float2 q = __fmul2_rn(a, make_float2(__uint_as_float(kInv - e0), __uint_as_float(kInv - e1)));
+  const float2 u = make_float2(__uint2float_rn(w0 >> 8), __uint2float_rn(w1 >> 8));
+  const float2 z = __ffma2_ru(u, make_float2(-0x1p-24f, -0x1p-24f), q);
+  const float2 t = __fadd2_ru(z, make_float2(12582912.0f, 12582912.0f));      // 1.5·2^23
+  // ceil(q - u) + 2E (E2M1: (e >> 22) - 254) or + 8E (E2M3: (e >> 20) - 1016)
+  constexpr uint32_t kBase = FMT == 0 ? 0x4B400000u + 254u : 0x4B400000u + 1016u;
+  m0 = min(__float_as_uint(t.x) + (FMT == 0 ? e0 >> 22 : e0 >> 20) - kBase, kTop);
+  m1 = min(__float_as_uint(t.y) + (FMT == 0 ? e1 >> 22 : e1 >> 20) - kBase, kTop);
 }
 
 // Correctly rounded a / d for the elements of a block, which share d, by
@@ -73,28 +83,24 @@ __device__ __forceinline__ uint32_t round_sr_mag(float a, float u) {
 // quotient is zero decides a code (stochastic rounding compares 24-bit u
 // against frac(q)): quotients below 1e-30 take the IEEE divide.  Blocks with
 // smaller divisors (tensors with max|x| below about 1e-13) divide exactly
-// throughout.
+// throughout.  Two elements per step with the paired fp32 operations of
+// sm_100 (each lane rounds as its scalar counterpart).
 constexpr float kMarksteinMinDivisor = 5.42101086242752217e-20f;   // 2^-64
 
-__device__ __forceinline__ float div_shared_divisor(float a, float d, float y) {
-  const float q0 = __fmul_rn(a, y);
-  const float r = __fmaf_rn(-d, q0, a);
-  const float q1 = __fmaf_rn(r, y, q0);
-  return (q0 >= 1.0e-30f || a == 0.0f) ? q1 : __fdiv_rn(a, d);
-}
-
-// Round-to-nearest-even codes need the quotient only where it can reach a
-// grid midpoint (>= 1/16), so the tiny-quotient check is dropped; the sign
-// is the sign of a in every case (also for y = 0, the zero-scale block,
-// where the magnitude comes out 0).
-__device__ __forceinline__ float div_shared_divisor_rne(float a, float d, float y) {
-  const float q0 = __fmul_rn(a, y);
-  const float r = __fmaf_rn(-d, q0, a);
-  return copysignf(__fmaf_rn(r, y, q0), a);
+__device__ __forceinline__ float2 div2_shared_divisor(float2 a, float2 nd, float2 y, float2& q0) {
+  q0 = __fmul2_rn(a, y);
+  const float2 r = __ffma2_rn(nd, q0, a);
+  return __ffma2_rn(r, y, q0);
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return f16_lo_to_f32(e4m3x2_to_f16x2(code));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // ------------------------------------------------------------- amax
@@ -166,45 +172,14 @@ amax_finish_kernel(const float* __restrict__ partial, int count, float* __restri
 }
 
 // ----------------------------------------------------------- quantize
-// One thread per QB horizontally adjacent 4 x 4 blocks of the rows x cols
-// view (QB = 2 when the view has an even number of column blocks, so each
-// thread keeps eight float4 loads in flight and stores 32-bit code words);
-// consecutive threads take consecutive column blocks, so each of the 4 rows
-// is read as one coalesced run.  `amax_src` holds `amax_count` partial
-// maxima; every CTA reduces them.  Stochastic rounding numbers element
-// (r, c) as r·sr_cols + sr_col0 + c, so a column slice of a wider view (a
-// batch shard) draws the words the whole view would (sr_cols = cols,
-// sr_col0 = 0 for an unsharded tensor).
-template <int FMT, int RND>
-__device__ __forceinline__ uint32_t quantize_row4(const float (&xv)[4], float d, float y, bool exact,
-                                                  const float (&u)[4]) {
-  if (RND == 0) {
-    // RNE: the conversion of the signed quotient gives sign bit and
-    // magnitude together (the sign of x, also for a zero quotient; a block
-    // whose scale is 0 has y = 0 and gets magnitude 0)
-    float v[4];
-    if (exact) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = __fdiv_rn(xv[j], d);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = div_shared_divisor_rne(xv[j], d, y);
-    }
-    if (FMT == 0) return f32x2_to_e2m1x2(v[0], v[1]) | (f32x2_to_e2m1x2(v[2], v[3]) << 8);
-    const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
-    return (b01 & 0x3F) | ((b01 >> 2) & 0xFC0) | ((b23 & 0x3F) << 12) | ((b23 & 0x3F00) << 10);
-  }
-  uint32_t packed = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float v = d > 0.0f ? (exact ? __fdiv_rn(fabsf(xv[j]), d) : div_shared_divisor(fabsf(xv[j]), d, y)) : 0.0f;
-    const uint32_t mag = round_sr_mag<FMT>(v, u[j]);
-    const uint32_t sgn = __float_as_uint(xv[j]) >> 31;
-    const uint32_t code = FMT == 0 ? (mag | (sgn << 3)) : (mag | (sgn << 5));
-    packed |= code << (j * (FMT == 0 ? 4 : 6));
-  }
-  return packed;
-}
+// Each thread quantizes kQuantUnits 4 x 4 blocks (grid-stride, the next
+// block's loads issued as soon as a block is done); consecutive threads take
+// consecutive column blocks, so each of the 4 rows is read as one coalesced
+// run.  `amax_src` holds `amax_count` partial maxima; every CTA reduces them.
+// Stochastic rounding numbers element (r, c) as r·sr_cols + sr_col0 + c, so a
+// column slice of a wider view (a batch shard) draws the words the whole
+// view would (sr_cols = cols, sr_col0 = 0 for an unsharded tensor).
+constexpr int kQuantUnits = 1;
 
 // Scale constants of a tensor from its amax (every scale step one IEEE fp32
 // operation in the formula's order).
@@ -218,75 +193,54 @@ struct TensorScale {
   }
 };
 
-// Quantize QB horizontally adjacent 4 x 4 blocks (block row br, first column
-// block bc0) whose 4 rows are x[q][r], and store their scales and codes.
-template <int FMT, int RND, int QB>
-__device__ __forceinline__ void quantize_unit(const float4 (&x)[QB][4], const TensorScale<FMT>& ts, int64_t br,
-                                              int64_t bc0, int64_t cb, int64_t row_bytes, const PhiloxKeys& keys,
-                                              int64_t sr_cols, int64_t sr_col0,
-                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  const float T = ts.T;
-  uint32_t scode[QB];
-  float d[QB], y[QB];
-  bool exact[QB];
-#pragma unroll
-  for (int q = 0; q < QB; ++q) {
-    float bmax = 0.0f;
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-      bmax = fmaxf(bmax, fmaxf(fmaxf(fabsf(x[q][r].x), fabsf(x[q][r].y)),
-                               fmaxf(fabsf(x[q][r].z), fabsf(x[q][r].w))));
-    scode[q] = 0;
-    d[q] = 0.0f;
-    y[q] = 0.0f;
-    if (T > 0.0f) {
-      scode[q] = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
-      d[q] = __fmul_rn(e4m3_to_f32(scode[q]), T);
-      y[q] = d[q] >= kMarksteinMinDivisor ? __frcp_rn(d[q]) : 0.0f;
-    }
-    exact[q] = d[q] > 0.0f && d[q] < kMarksteinMinDivisor;
-  }
-  const int64_t b = br * cb + bc0;
-  if (QB == 2) *reinterpret_cast<uint16_t*>(scales + b) = static_cast<uint16_t>(scode[0] | (scode[1] << 8));
-  else scales[b] = static_cast<uint8_t>(scode[0]);
-
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    uint32_t packed[QB];
-#pragma unroll
-    for (int q = 0; q < QB; ++q) {
-      const float xv[4] = {x[q][r].x, x[q][r].y, x[q][r].z, x[q][r].w};
-      float u[4] = {0.f, 0.f, 0.f, 0.f};
-      if (RND == 1) {
-        // element index in the (possibly wider) view the SR stream is defined on
-        const uint64_t g = static_cast<uint64_t>((br * 4 + r) * sr_cols + sr_col0 + (bc0 + q) * 4) >> 2;
-        const uint4 wd = philox4x32_10(make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), keys);
-        const float s24 = 5.9604644775390625e-08f;   // 2^-24
-        u[0] = __uint2float_rn(wd.x >> 8) * s24;
-        u[1] = __uint2float_rn(wd.y >> 8) * s24;
-        u[2] = __uint2float_rn(wd.z >> 8) * s24;
-        u[3] = __uint2float_rn(wd.w >> 8) * s24;
-      }
-      packed[q] = quantize_row4<FMT, RND>(xv, d[q], y[q], exact[q], u);
-    }
-    uint8_t* out = codes + (br * 4 + r) * row_bytes;
-    if (FMT == 0) {
-      if (QB == 2) *reinterpret_cast<uint32_t*>(out + bc0 * 2) = packed[0] | (packed[1] << 16);
-      else *reinterpret_cast<uint16_t*>(out + bc0 * 2) = static_cast<uint16_t>(packed[0]);
+// Codes of one 4-element row of a block (element j at bits [j·b, j·b + b),
+// b = 4 or 6), given the block divisor d = B·T, y = RN(1/d) (0 for a block
+// whose scale is 0) and, for stochastic rounding, the row's Philox words.
+template <int FMT, int RND>
+__device__ __forceinline__ uint32_t quantize_row4(float4 x, float d, float y, bool exact, uint4 w) {
+  const float2 nd = make_float2(-d, -d), y2 = make_float2(y, y);
+  constexpr int kB = FMT == 0 ? 4 : 6;
+  if (RND == 0) {
+    // RNE: the conversion of the signed quotient gives sign bit and
+    // magnitude together.  The quotient's sign is copied from x so that
+    // zeros keep it (a block whose scale is 0 has y = 0: magnitude 0).
+    float v[4];
+    if (exact) {
+      v[0] = __fdiv_rn(x.x, d); v[1] = __fdiv_rn(x.y, d); v[2] = __fdiv_rn(x.z, d); v[3] = __fdiv_rn(x.w, d);
     } else {
-      if (QB == 2) {   // 48 bits at a 6-byte (2-aligned) offset
-        uint16_t* o16 = reinterpret_cast<uint16_t*>(out + bc0 * 3);
-        o16[0] = static_cast<uint16_t>(packed[0]);
-        o16[1] = static_cast<uint16_t>((packed[0] >> 16) | (packed[1] << 8));
-        o16[2] = static_cast<uint16_t>(packed[1] >> 8);
-      } else {
-        out += bc0 * 3;
-        out[0] = static_cast<uint8_t>(packed[0]);
-        out[1] = static_cast<uint8_t>(packed[0] >> 8);
-        out[2] = static_cast<uint8_t>(packed[0] >> 16);
-      }
+      float2 q0;
+      const float2 v01 = div2_shared_divisor(make_float2(x.x, x.y), nd, y2, q0);
+      const float2 v23 = div2_shared_divisor(make_float2(x.z, x.w), nd, y2, q0);
+      v[0] = copysignf(v01.x, x.x); v[1] = copysignf(v01.y, x.y);
+      v[2] = copysignf(v23.x, x.z); v[3] = copysignf(v23.y, x.w);
+    }
+    if (FMT == 0) return f32x2_to_e2m1x2(v[0], v[1]) | (f32x2_to_e2m1x2(v[2], v[3]) << 8);
+    const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
+    return (b01 & 0x3F) | ((b01 >> 2) & 0xFC0) | ((b23 & 0x3F) << 12) | ((b23 & 0x3F00) << 10);
+  }
+  const float2 a01 = make_float2(fabsf(x.x), fabsf(x.y)), a23 = make_float2(fabsf(x.z), fabsf(x.w));
+  float2 v01, v23;
+  if (exact) {
+    v01 = make_float2(__fdiv_rn(a01.x, d), __fdiv_rn(a01.y, d));
+    v23 = make_float2(__fdiv_rn(a23.x, d), __fdiv_rn(a23.y, d));
+  } else {
+    float2 q01, q23;
+    v01 = div2_shared_divisor(a01, nd, y2, q01);
+    v23 = div2_shared_divisor(a23, nd, y2, q23);
+    if (fminf(fminf(q01.x, q01.y), fminf(q23.x, q23.y)) < 1.0e-30f && d > 0.0f) {
+      // a quotient below 1e-30 (or a zero): the IEEE divide where it matters
+      if (q01.x < 1.0e-30f && a01.x != 0.0f) v01.x = __fdiv_rn(a01.x, d);
+      if (q01.y < 1.0e-30f && a01.y != 0.0f) v01.y = __fdiv_rn(a01.y, d);
+      if (q23.x < 1.0e-30f && a23.x != 0.0f) v23.x = __fdiv_rn(a23.x, d);
+      if (q23.y < 1.0e-30f && a23.y != 0.0f) v23.y = __fdiv_rn(a23.y, d);
     }
   }
+  uint32_t m[4];
+  round_sr_mag2<FMT>(v01, w.x, w.y, m[0], m[1]);
+  round_sr_mag2<FMT>(v23, w.z, w.w, m[2], m[3]);
+  const uint32_t sgn = (__float_as_uint(x.x) >> 31) | ((__float_as_uint(x.y) >> 31) << kB) |
+                       ((__float_as_uint(x.z) >> 31) << (2 * kB)) | ((__float_as_uint(x.w) >> 31) << (3 * kB));
+  return (m[0] | (m[1] << kB) | (m[2] << (2 * kB)) | (m[3] << (3 * kB))) | (sgn << (kB - 1));
 }
 
 // Per-tensor parameters of the quantize pass.
@@ -298,58 +252,110 @@ struct QuantArgs {
   float* tscale;
   PhiloxKeys keys;
   int64_t sr_cols, sr_col0;
-  FastDiv dcu;          // division by the work units per block row (unit count < 2^31)
+  FastDiv dcb;          // division by the column blocks of a block row (block count < 2^31)
 };
 
-template <int QB>
-__device__ __forceinline__ void load_unit(float4 (&x)[QB][4], const float* __restrict__ src, int64_t cols, int br,
-                                          int64_t bc0) {
-  const float* p = src + (static_cast<int64_t>(br) * 4) * cols + bc0 * 4;
+// Quantize the 4 x 4 block (br, bc) whose 4 rows are x[r], and store its
+// scale and codes.
+template <int FMT, int RND>
+__device__ __forceinline__ void quantize_block(const float4 (&x)[4], const TensorScale<FMT>& ts, const QuantArgs& qa,
+                                               int64_t br, int64_t bc, int64_t cb, int64_t row_bytes) {
+  const float T = ts.T;
+  float bmax = max3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[0].z));
+  bmax = max3f(bmax, fabsf(x[0].w), fabsf(x[1].x));
+  bmax = max3f(bmax, fabsf(x[1].y), fabsf(x[1].z));
+  float b2 = max3f(fabsf(x[1].w), fabsf(x[2].x), fabsf(x[2].y));
+  b2 = max3f(b2, fabsf(x[2].z), fabsf(x[2].w));
+  float b3 = max3f(fabsf(x[3].x), fabsf(x[3].y), fabsf(x[3].z));
+  bmax = max3f(bmax, b2, fmaxf(b3, fabsf(x[3].w)));
+  uint32_t scode = 0;
+  float d = 0.0f, y = 0.0f;
+  if (T > 0.0f) {
+    scode = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
+    d = __fmul_rn(e4m3_to_f32(scode), T);
+    y = d >= kMarksteinMinDivisor ? __frcp_rn(d) : 0.0f;
+  }
+  const bool exact = d > 0.0f && d < kMarksteinMinDivisor;
+  qa.scales[br * cb + bc] = static_cast<uint8_t>(scode);
+  // Philox counter of row r: (element index of its first element) / 4
+  uint64_t g = 0, gstep = 0;
+  if (RND == 1) {
+    g = static_cast<uint64_t>(br * 4 * qa.sr_cols + qa.sr_col0 + bc * 4) >> 2;
+    gstep = static_cast<uint64_t>(qa.sr_cols) >> 2;
+  }
 #pragma unroll
-  for (int q = 0; q < QB; ++q)
-#pragma unroll
-    for (int r = 0; r < 4; ++r) x[q][r] = __ldg(reinterpret_cast<const float4*>(p + r * cols + 4 * q));
+  for (int r = 0; r < 4; ++r) {
+    uint4 wd = make_uint4(0u, 0u, 0u, 0u);
+    if (RND == 1) {
+      wd = philox4x32_10(make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), qa.keys);
+      g += gstep;
+    }
+    const uint32_t packed = quantize_row4<FMT, RND>(x[r], d, y, exact, wd);
+    uint8_t* out = qa.codes + (br * 4 + r) * row_bytes;
+    if (FMT == 0) {
+      *reinterpret_cast<uint16_t*>(out + bc * 2) = static_cast<uint16_t>(packed);
+    } else {
+      out += bc * 3;
+      out[0] = static_cast<uint8_t>(packed);
+      out[1] = static_cast<uint8_t>(packed >> 8);
+      out[2] = static_cast<uint8_t>(packed >> 16);
+    }
+  }
 }
 
-template <int FMT, int RND, int QB>
+__device__ __forceinline__ void load_block(float4 (&x)[4], const float* __restrict__ src, int64_t cols, int64_t br,
+                                           int64_t bc) {
+  const float* p = src + br * 4 * cols + bc * 4;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) x[r] = __ldg(reinterpret_cast<const float4*>(p + r * cols));
+}
+
+template <int FMT, int RND>
 __device__ __forceinline__ void quantize_body(const QuantArgs& qa, const float* __restrict__ amax_src, int amax_count,
                                               int cta, int nctas) {
   const int64_t cols = qa.cols;
   const int64_t cb = cols >> 2;                       // column blocks per block row
-  const int cu = static_cast<int>(cb / QB);           // work units per block row
-  const int nunits = static_cast<int>((qa.rows >> 2) * cu);
+  const int nunits = static_cast<int>((qa.rows >> 2) * cb);
   const int64_t row_bytes = FMT == 0 ? (cols >> 1) : (cols * 3) >> 2;
-  const int stride = nctas * kQuantThreads;
+  const int nthr = nctas * kQuantThreads;
+  const int w0 = cta * kQuantThreads + static_cast<int>(threadIdx.x);
 
-  // The first unit's loads do not depend on the tensor scale: issue them
+  // The first blocks' loads do not depend on the tensor scale: issue them
   // before the reduction of the amax partials, so the two latencies overlap.
-  int w = cta * kQuantThreads + static_cast<int>(threadIdx.x);
-  float4 x[QB][4];
-  if (w < nunits) {
-    const int br = fdiv(w, qa.dcu);
-    load_unit<QB>(x, qa.src, cols, br, static_cast<int64_t>(w - br * cu) * QB);
+  float4 x[kQuantUnits][4];
+#pragma unroll
+  for (int i = 0; i < kQuantUnits; ++i) {
+    const int w = w0 + i * nthr;
+    if (w < nunits) {
+      const int br = fdiv(w, qa.dcb);
+      load_block(x[i], qa.src, cols, br, w - static_cast<int64_t>(br) * cb);
+    }
   }
   __shared__ float red[32];
   const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
   if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
 
-  for (; w < nunits; w += stride) {
-    const int br = fdiv(w, qa.dcu);
-    const int64_t bc0 = static_cast<int64_t>(w - br * cu) * QB;
-    quantize_unit<FMT, RND, QB>(x, ts, br, bc0, cb, row_bytes, qa.keys, qa.sr_cols, qa.sr_col0, qa.codes,
-                                qa.scales);
-    const int wn = w + stride;
-    if (wn < nunits) {
-      const int bn = fdiv(wn, qa.dcu);
-      load_unit<QB>(x, qa.src, cols, bn, static_cast<int64_t>(wn - bn * cu) * QB);
+  for (int w = w0; w < nunits; w += kQuantUnits * nthr) {
+#pragma unroll
+    for (int i = 0; i < kQuantUnits; ++i) {
+      const int wi = w + i * nthr;
+      if (wi < nunits) {
+        const int br = fdiv(wi, qa.dcb);
+        quantize_block<FMT, RND>(x[i], ts, qa, br, wi - static_cast<int64_t>(br) * cb, cb, row_bytes);
+        const int wn = wi + kQuantUnits * nthr;
+        if (wn < nunits) {
+          const int bn = fdiv(wn, qa.dcb);
+          load_block(x[i], qa.src, cols, bn, wn - static_cast<int64_t>(bn) * cb);
+        }
+      }
     }
   }
 }
 
-template <int FMT, int RND, int QB>
+template <int FMT, int RND>
 __global__ void __launch_bounds__(kQuantThreads)
 quantize_kernel(const __grid_constant__ QuantArgs qa, const float* __restrict__ amax_src, int amax_count) {
-  quantize_body<FMT, RND, QB>(qa, amax_src, amax_count, blockIdx.x, gridDim.x);
+  quantize_body<FMT, RND>(qa, amax_src, amax_count, blockIdx.x, gridDim.x);
 }
 
 // ------------------------------------------------ several tensors at once
@@ -362,7 +368,7 @@ constexpr int kMaxQuantJobs = 8;
 
 struct QuantJob {
   QuantArgs qa;
-  int32_t fmt, rounding, qb;
+  int32_t fmt, rounding;
   int32_t amax_cta0, amax_ctas;     // this job's range of amax CTAs (= its partials)
   int32_t quant_cta0, quant_ctas;   // this job's range of quantize CTAs
 };
@@ -391,12 +397,12 @@ quantize_many_kernel(const __grid_constant__ QuantJobs jobs, const float* __rest
   const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, true)];
   const int cta = blockIdx.x - jb.quant_cta0;
   const float* amax = partial + jb.amax_cta0;
-#define MQV_QUANT_CASE(F, R, Q)                                                                   \
-  if (jb.fmt == F && jb.rounding == R && jb.qb == Q) {                                            \
-    quantize_body<F, R, Q>(jb.qa, amax, jb.amax_ctas, cta, jb.quant_ctas);                         \
+#define MQV_QUANT_CASE(F, R)                                                                      \
+  if (jb.fmt == F && jb.rounding == R) {                                                          \
+    quantize_body<F, R>(jb.qa, amax, jb.amax_ctas, cta, jb.quant_ctas);                            \
     return;                                                                                       \
   }
-  MQV_QUANT_CASE(0, 0, 1) MQV_QUANT_CASE(0, 1, 1) MQV_QUANT_CASE(1, 0, 1) MQV_QUANT_CASE(1, 1, 1)
+  MQV_QUANT_CASE(0, 0) MQV_QUANT_CASE(0, 1) MQV_QUANT_CASE(1, 0) MQV_QUANT_CASE(1, 1)
 #undef MQV_QUANT_CASE
 }
 

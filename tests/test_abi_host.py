@@ -80,8 +80,12 @@ def test_conv_workspace_sizes(lib):
     d = _desc()
     # fwd/dgrad: one 128 x 64 fp16 tile of the dequantized weight image per
     # (row tile, K tile): 1 x 18 tiles of 16 KB for 128 -> 128 channels, 3x3
+    # (row-major tiles for the stride-1 halo kernel, swizzled otherwise)
     assert mqv.conv_workspace_bytes(d, mqv.OP_FWD) == 18 * 16384
     assert mqv.conv_workspace_bytes(d, mqv.OP_DGRAD) == 18 * 16384
+    d2 = _desc(stride=2)
+    assert mqv.conv_workspace_bytes(d2, mqv.OP_FWD) == 18 * 16384
+    assert mqv.conv_workspace_bytes(d2, mqv.OP_DGRAD) == 18 * 16384
     ws = mqv.conv_workspace_bytes(d, mqv.OP_WGRAD)
     assert ws > 0 and ws % (128 * 1152 * 4) == 0          # whole split partial tiles
 

@@ -66,6 +66,11 @@ SMALL = [
     ("halo_fp6_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp6"),
     ("halo_fp6_n16_1x1", O.ConvShape(16, 128, 64, 7, 7, 1, 1, 1, 0), "nvfp6"),
     ("halo_fp6_n8_5x5", O.ConvShape(8, 64, 128, 9, 9, 5, 5, 1, 2), "nvfp6"),
+    # more than two tiles per persistent CTA, so the weight loaders and the
+    # producers finish well before the MMAs (a 1 x 1 layer has one stage a
+    # tile) and share the epilogue of the CTA's last tile
+    ("halo_multitile_1x1_fp6", O.ConvShape(16, 64, 64, 64, 64, 1, 1, 1, 0), "nvfp6"),
+    ("halo_multitile_3x3_n32", O.ConvShape(32, 64, 64, 48, 48, 3, 3, 1, 1), "nvfp4"),
     # stride-1 weight-gradient shapes whose kernel-row taps share operands
     # (N % 16 == 0): ragged rows and channels, split ranges that end inside a
     # row, several channel tiles, a 2 x 2 kernel

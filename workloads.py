@@ -103,6 +103,24 @@ REPLAY_SHAPES = [(256, 7, 84), (512, 7, 256), (256, 14, 256), (512, 14, 256),
                  (512, 14, 2560), (512, 14, 10240)]
 
 
+# Depthwise 3x3 layers kept in BF16 (the YOLOv26n-style stages at 640 px
+# input, batch 16): (C, H = W, stride); stride-2 layers halve the pixels.
+DEPTHWISE_SHAPES = [(32, 160, 1), (64, 160, 2), (64, 80, 1), (128, 80, 2), (128, 40, 1),
+                    (256, 40, 2), (256, 20, 1)]
+DEPTHWISE_N = 16
+
+
+def make_depthwise_inputs(C: int, H: int, stride: int, N: int = DEPTHWISE_N, seed: int = 0, device="cpu"):
+    """(x [H][H][C][N], w [C][3][3], gy [Ho][Ho][C][N]) fp32: x = SiLU(N(0,1)),
+    w ~ N(0, 2/9) (one 3x3 filter per channel), gy ~ N(0, 1e-4)."""
+    g = _gen(seed, device)
+    ho = (H + 2 - 3) // stride + 1
+    x = torch.nn.functional.silu(torch.randn((H, H, C, N), generator=g, device=device))
+    w = torch.randn((C, 3, 3), generator=g, device=device) * math.sqrt(2.0 / 9.0)
+    gy = torch.randn((ho, ho, C, N), generator=g, device=device) * 1e-4
+    return x, w, gy
+
+
 def _gen(seed: int, device="cpu") -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(seed)
