@@ -639,6 +639,8 @@ def run_gpu(args):
         naive_res["step_time_ratio"] = round(naive_res["ms_per_step"] / (serial_ms / args.steps), 3)
         naive_res["quantize_time_ratio"] = round(naive_res["phase_ms"]["quant"] / mean["quantize"], 3)
         out["naive_baseline"] = naive_res
+    if world == 1:
+        out["mma_form"] = run_mma_form(dev, layer, peaks)
     if world == 1 and not args.no_sweeps:
         out["fused_epilogue"] = run_fused(dev, layer, peaks)
         out["sweeps"] = run_sweeps(args, dev, peaks)
@@ -823,6 +825,42 @@ def run_sweeps(args, dev, peaks):
     if flags:
         raise SystemExit(f"device wait timeout flags {flags:#x} in the sweeps")
     res["launches"] = launches
+    return res
+
+
+def run_mma_form(dev, layer, peaks):
+    """The forward pass of the layer in the two MMA forms the square blocks
+    allow: fp16 products of dequantized codes (kind::f16, the default) and
+    the native block-scaled MMA with each 4-element block row padded to a
+    16-element scale group (kind::mxf4nvf4, mqv_conv_fwd_blockscaled).  Each
+    call includes its weight image; L2 flushed before each call."""
+    import torch
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+    try:
+        mqv.conv_workspace_bytes(d, mqv.OP_FWD_BLOCKSCALED)
+    except mqv.MqvError as e:
+        return {"unsupported": str(e)}
+    X, Wt, _ = (t.view(-1) for t in workloads.make_layer_inputs(layer, device=dev))
+    xr, wr, wc = layer.H * layer.W * layer.Cin, layer.Cout, layer.K * layer.K * layer.Cin
+    qx = mqv.quantize(X, xr, layer.N, layer.fmt, mqv.RNE)
+    qw = mqv.quantize(Wt, wr, wc, layer.fmt, mqv.RNE)
+    y = torch.empty(layer.Ho * layer.Wo * layer.Cout * layer.N, device=dev)
+    ws_f = torch.empty(max(16, mqv.conv_workspace_bytes(d, mqv.OP_FWD)), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(mqv.conv_workspace_bytes(d, mqv.OP_FWD_BLOCKSCALED), dtype=torch.uint8, device=dev)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    tc = peaks["bf16_tflops"]
+    res = {"layer": layer.name, "note": "same layer, same quantized operands, weight image included, L2 flushed"}
+    for name, fn in (("f16_dequantized", lambda: mqv.conv_fwd(d, qw, qx, y=y, ws=ws_f)),
+                     ("mxf4nvf4_padded", lambda: mqv.conv_fwd_blockscaled(d, qw, qx, y=y, ws=ws_b))):
+        for _ in range(3):
+            fn()
+        ms = _timed(torch, fn, 20, flush)
+        tfl = layer.flops() / (ms * 1e-3) / 1e12
+        res[name] = {"ms": round(ms, 5), "tflops": round(tfl, 2), "frac_of_dense_peak": round(tfl / tc, 4)}
+    res["winner"] = min(("f16_dequantized", "mxf4nvf4_padded"), key=lambda k: res[k]["ms"])
     return res
 
 

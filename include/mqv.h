@@ -63,7 +63,7 @@ typedef enum {
 
 typedef enum { MQV_NVFP4 = 0 /* E2M1 elements */, MQV_NVFP6 = 1 /* E2M3 */ } mqv_format;
 typedef enum { MQV_RNE = 0, MQV_SR = 1 } mqv_rounding;
-typedef enum { MQV_OP_FWD = 1, MQV_OP_WGRAD = 2, MQV_OP_DGRAD = 3 } mqv_op;
+typedef enum { MQV_OP_FWD = 1, MQV_OP_WGRAD = 2, MQV_OP_DGRAD = 3, MQV_OP_FWD_BLOCKSCALED = 4 } mqv_op;
 
 /* Shape of one convolution layer (the pages' N, Cin, Cout, H, W, Kh, Kw,
  * stride, pad, format).  Requirements: all > 0 (pad >= 0), Cin, Cout and N
@@ -202,6 +202,24 @@ mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* b
  * w: view Cout x Kh·Kw·Cin; x: view H·W·Cin x N; y fp32 [Ho][Wo][Cout][N]. */
 mqv_status mqv_conv_fwd(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
                         float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* The forward pass of mqv_conv_fwd on the other MMA form sm_100a offers for
+ * these operands: the native block-scaled MMA (tcgen05.mma kind::mxf4nvf4,
+ * E2M1 operands with one UE4M3 scale per 16 consecutive K elements).  Section
+ * "무엇과 다른가" gives each 4 x 4 square block one E4M3 scale, i.e. 4 K
+ * elements per scale in every row, so the only exact mapping pads each
+ * 4-element block row with 12 zero codes: the codes enter the MMA without
+ * dequantization, the block scales travel in tensor memory, and 3/4 of the
+ * MMA's K is zeros.  Kept beside mqv_conv_fwd (fp16 products of dequantized
+ * operands, exact) so the two forms can be measured on the same layer; the
+ * outputs agree within the parity tolerance (both accumulate exact products
+ * in fp32, in different orders).  Supported: NVFP4, stride 1, N = 64 or
+ * 128 with (128/N + Kw - 1)·N <= 256, Kw <= 3, Cin a multiple of 64; other
+ * layers return MQV_ERR_UNSUPPORTED before any launch.  ws:
+ * mqv_conv_workspace_size(d, MQV_OP_FWD_BLOCKSCALED) bytes (the padded
+ * weight image and its scales); other arguments as mqv_conv_fwd. */
+mqv_status mqv_conv_fwd_blockscaled(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
+                                    float* y, void* ws, size_t ws_bytes, void* stream);
 
 /* Weight-gradient GEMM G_W = G_Y·X'^T: contraction over (ho, wo, n), split
  * across CTAs and summed in a fixed order (deterministic) through `ws`.

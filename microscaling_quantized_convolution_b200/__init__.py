@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmqv.so")
 
 NVFP4, NVFP6 = 0, 1
 RNE, SR = 0, 1
-OP_FWD, OP_WGRAD, OP_DGRAD = 1, 2, 3
+OP_FWD, OP_WGRAD, OP_DGRAD, OP_FWD_BLOCKSCALED = 1, 2, 3, 4
 FORMATS = {"nvfp4": NVFP4, "nvfp6": NVFP6, NVFP4: NVFP4, NVFP6: NVFP6}
 
 
@@ -85,6 +85,9 @@ _SIGS = {
     "mqv_conv_fwd": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                     ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_fwd_blockscaled": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                                ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_conv_wgrad": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                       ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]),
@@ -380,6 +383,19 @@ def conv_fwd(d: ConvDesc, w: QTensor, x: QTensor, y: torch.Tensor | None = None,
     wc, xc = w.c(), x.c()
     _check(lib().mqv_conv_fwd(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), y.data_ptr(),
                               _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return y
+
+
+def conv_fwd_blockscaled(d: ConvDesc, w: QTensor, x: QTensor, y: torch.Tensor | None = None,
+                         ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y as conv_fwd, on the native block-scaled MMA with each 4-element
+    block row padded to a 16-element scale group (see mqv_conv_fwd_blockscaled)."""
+    Ho, Wo = out_hw(d)
+    y = y if y is not None else torch.empty((Ho, Wo, d.Cout, d.N), dtype=torch.float32, device=x.codes.device)
+    ws = _ws(d, OP_FWD_BLOCKSCALED, ws, x.codes.device)
+    wc, xc = w.c(), x.c()
+    _check(lib().mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), y.data_ptr(),
+                                          _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return y
 
 

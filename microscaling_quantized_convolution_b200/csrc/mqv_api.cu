@@ -15,6 +15,7 @@
 #include "mqv_conv_common.cuh"
 #include "mqv_conv_kernels.cuh"
 #include "mqv_conv_halo.cuh"
+#include "mqv_conv_nvf4.cuh"
 #include "mqv_conv_wgk.cuh"
 #include "mqv_depthwise.cuh"
 #include "mqv_naive.cuh"
@@ -538,6 +539,39 @@ cudaError_t launch_prep(int op, int fmt, const ConvPlan& pl, const QView& w, uin
   return cudaGetLastError();
 }
 
+// Geometry of the block-scaled forward pass (conv_fwd_nvf4_kernel): halo
+// tiles of 128 GEMM columns (128 / N pixels of one output row x N batch
+// items) x 128 output channels.
+mqv_status plan_blockscaled(const mqv_conv_desc* d, ConvPlan* pl) {
+  // N % 64 == 0: a tap shifts the halo rows by N, the scale columns by
+  // N / 32, and a scale-factor address in tensor memory must be an even
+  // column (an odd one, N = 32, faulted with a misaligned address)
+  if (d->fmt != MQV_NVFP4 || d->stride != 1 || d->N % 64 || 128 % d->N || d->Kw > 3 || d->Cin % 64 ||
+      (128 / d->N + d->Kw - 1) * d->N > kNvf4MaxRows)
+    return fail(MQV_ERR_UNSUPPORTED,
+                "block-scaled forward pass: NVFP4, stride 1, N = 64 or 128 with a halo of at most %d rows, "
+                "Kw <= 3, Cin a multiple of 64",
+                kNvf4MaxRows);
+  plan_conv(d, MQV_OP_FWD, pl);
+  V2Args& a = pl->a;
+  HaloGeom& g = pl->g;
+  g.out_h = a.Ho;
+  g.out_w = a.Wo;
+  g.src_h = a.H;
+  g.src_w = a.W;
+  g.cchunks = a.Cin / 64;
+  g.bw = kNvf4BN / a.N;
+  g.bn = kNvf4BN;
+  g.rows = (g.bw + a.Kw - 1) * a.N;
+  g.tpr = (g.out_w + g.bw - 1) / g.bw;
+  a.tiles = a.mtiles * g.out_h * g.tpr;
+  pl->grid = a.tiles < kSMs ? a.tiles : kSMs;
+  pl->image_bytes = (size_t)a.mtiles * a.ktiles * kNvf4ATile;
+  pl->partial_bytes = 0;
+  pl->ws_bytes = pl->image_bytes;
+  return MQV_OK;
+}
+
 mqv_status check_operand(const mqv_qtensor* q, const char* name, int64_t rows, int64_t cols, int32_t fmt) {
   mqv_status st = check_qtensor(q, name);
   if (st) return st;
@@ -639,11 +673,16 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
     qj.rounding = j.rounding;
     qj.amax_cta0 = a;
     qj.amax_ctas = (int)amax_ctas(j.rows, j.cols);
-    qj.quant_cta0 = q;
     qj.quant_ctas = (int)quant_ctas(j.rows, j.cols);
     a += qj.amax_ctas;
-    q += qj.quant_ctas;
   }
+  // quantize CTA ranges: stochastic-rounding jobs first (see quantize_many_kernel)
+  for (int pass = 0; pass < 2; ++pass)
+    for (int i = 0; i < count; ++i)
+      if ((plan->job[i].rounding == MQV_SR) == (pass == 0)) {
+        plan->job[i].quant_cta0 = q;
+        q += plan->job[i].quant_ctas;
+      }
   *amax_total = a;
   *quant_total = q;
   return MQV_OK;
@@ -856,12 +895,53 @@ mqv_status mqv_replay_dequantize(const void* packed, const uint8_t* scales, cons
 mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* bytes) {
   mqv_status st = check_desc(d);
   if (st) return st;
-  if (op != MQV_OP_FWD && op != MQV_OP_WGRAD && op != MQV_OP_DGRAD)
+  if (op != MQV_OP_FWD && op != MQV_OP_WGRAD && op != MQV_OP_DGRAD && op != MQV_OP_FWD_BLOCKSCALED)
     return fail(MQV_ERR_INVALID_ARG, "unknown op %d", op);
   if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
   ConvPlan pl;
-  plan_conv(d, op, &pl);
+  if (op == MQV_OP_FWD_BLOCKSCALED) {
+    if ((st = plan_blockscaled(d, &pl))) return st;
+  } else {
+    plan_conv(d, op, &pl);
+  }
   *bytes = pl.ws_bytes;
+  return ok();
+}
+
+mqv_status mqv_conv_fwd_blockscaled(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x, float* y,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  mqv_status st = check_desc(d);
+  if (st) return st;
+  ConvPlan pl;
+  if ((st = plan_blockscaled(d, &pl))) return st;
+  if ((st = check_operand(w, "w", d->Cout, d->Kh * d->Kw * d->Cin, d->fmt)) ||
+      (st = check_operand(x, "x", d->H * d->W * d->Cin, d->N, d->fmt)))
+    return st;
+  if (!y || !aligned16(y)) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
+  if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))
+    return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required, got %zu", pl.ws_bytes,
+                ws ? ws_bytes : (size_t)0);
+  uint32_t* err = nullptr;
+  if ((st = device_error_word(&err))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* image = static_cast<uint8_t*>(ws);
+  const V2Args& a = pl.a;
+  const int chunks = a.mtiles * 128 * a.ktiles * 8;
+  prep_nvf4_image_kernel<<<(unsigned)((chunks + kPrepThreads - 1) / kPrepThreads), kPrepThreads, 0, s>>>(
+      make_view(w), a.M, a.ktiles, a.mtiles, make_fastdiv((int64_t)a.ktiles * 8), image);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block-scaled weight image launch");
+  pl.a.err = err;
+  pl.a.image = image;
+  pl.a.b = make_view(x);
+  pl.a.ta = w->tscale;
+  pl.a.tb = x->tscale;
+  pl.a.out = y;
+  static bool done[kMaxDevices] = {};
+  if ((e = set_smem(conv_fwd_nvf4_kernel, Nvf4Smem::kBytes, done)) != cudaSuccess) return cuda_fail(e, "smem attribute");
+  conv_fwd_nvf4_kernel<<<pl.grid, kNvf4Threads, Nvf4Smem::kBytes, s>>>(pl.a, pl.g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "block-scaled conv launch");
   return ok();
 }
 

@@ -178,13 +178,14 @@ struct HaloCursor {
   }
 };
 
-// Epilogue of one tile for the warp on TMEM lane quarter `quarter`: the
-// 32-column chunks first, first + stride, ... of the accumulator.  Each lane
+// Epilogue of one tile (accumulator at TMEM column acc_col) for the warp on
+// TMEM lane quarter `quarter`: the 32-column chunks first, first + stride,
+// ... of the accumulator.  Each lane
 // reads one accumulator row from TMEM; a swizzled 32 x 32 transpose in the
 // warp's 4 KB of shared memory (wbuf) turns that into stores of 128-byte runs
 // of one (pixel, channel) row's batch items.  Columns past bw·N hold no
 // output (j >= bw below).
-__device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGeom& g, uint32_t tmem, int acc,
+__device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGeom& g, uint32_t tmem, int acc_col,
                                                    int tile, int quarter, uint32_t wbuf, int first, int stride,
                                                    float& amax) {
   const int lane = threadIdx.x & 31;
@@ -195,7 +196,7 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
   const int ow0 = (rest - oh * g.tpr) * g.bw;
   if (mt * 128 + quarter * 32 >= p.M) return;   // all 32 rows of this quarter past the M channels
   const float scale = __fmul_rn(*p.ta, *p.tb);
-  const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kHaloBN;
+  const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc_col;
 #pragma unroll 1
   for (int c = 32 * first; c < g.bn; c += 32 * stride) {
 #pragma unroll
@@ -282,7 +283,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const bool last = tile + static_cast<int>(gridDim.x) >= p.tiles;
-      halo_epilogue_tile(p, g, bars->tmem, acc, tile, warp & 3, wbuf, 0, last ? 4 : 1, amax);
+      halo_epilogue_tile(p, g, bars->tmem, acc * kHaloBN, tile, warp & 3, wbuf, 0, last ? 4 : 1, amax);
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
     }
@@ -414,7 +415,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       // tile has its own single-phase barrier.
       mbar_wait_bounded(&bars->last_full, 0, p.err, kErrWaitDone);
       tc_fence_after();
-      halo_epilogue_tile(p, g, bars->tmem, lit & 1, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
+      halo_epilogue_tile(p, g, bars->tmem, (lit & 1) * kHaloBN, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
                          1 + pw / 4, 4, amax);
       epi_amax_flush(p.amax_out, amax);
     }

@@ -361,9 +361,11 @@ quantize_kernel(const __grid_constant__ QuantArgs qa, const float* __restrict__ 
 // ------------------------------------------------ several tensors at once
 // The quantize-once step of a layer (X, W, G_Y) in two launches instead of
 // six: every CTA of a launch serves one tensor ("job"), CTAs are assigned to
-// jobs in contiguous ranges.  Results are bit-identical to one
-// amax_partial_kernel + quantize_kernel pair per tensor with the same CTA
-// counts.
+// jobs in contiguous ranges.  In the quantize launch the stochastic-rounding
+// jobs take the first ranges: their CTAs are bound by arithmetic and start
+// first, while the memory-bound round-to-nearest CTAs fill the SMs around
+// them.  Results are bit-identical to one amax_partial_kernel +
+// quantize_kernel pair per tensor with the same CTA counts.
 constexpr int kMaxQuantJobs = 8;
 
 struct QuantJob {
@@ -380,8 +382,11 @@ struct QuantJobs {
 
 __device__ __forceinline__ int job_of(const QuantJobs& jobs, int cta, bool quant) {
   int j = 0;
-  for (int i = 1; i < jobs.count; ++i)
-    if (cta >= (quant ? jobs.job[i].quant_cta0 : jobs.job[i].amax_cta0)) j = i;
+  for (int i = 0; i < jobs.count; ++i) {
+    const int c0 = quant ? jobs.job[i].quant_cta0 : jobs.job[i].amax_cta0;
+    const int n = quant ? jobs.job[i].quant_ctas : jobs.job[i].amax_ctas;
+    if (cta >= c0 && cta < c0 + n) j = i;
+  }
   return j;
 }
 

@@ -224,3 +224,20 @@ def test_noalloc_scratch_covers_every_planned_layer(lib):
                                    pad=k // 2, fmt="nvfp4"))
     worst = max(mqv.conv_workspace_bytes(mqv.conv_desc(**s), mqv.OP_WGRAD) for s in shapes)
     assert 0 < worst <= 148 * 128 * 384 * 4 < 32 << 20
+
+
+def test_blockscaled_forward_workspace_and_rejections(lib):
+    """The block-scaled forward pass: its weight image is 18 KB per (row tile,
+    K tile) (16 KB of padded codes and 2 KB of scale atoms); layers outside
+    its range (NVFP6, stride 2, N other than 64 or 128, Cin not a multiple
+    of 64, Kw > 3) are rejected as unsupported before any launch."""
+    d = _desc()
+    assert mqv.conv_workspace_bytes(d, mqv.OP_FWD_BLOCKSCALED) == 18 * 18432
+    for kw in (dict(fmt=mqv.NVFP6), dict(stride=2), dict(N=16), dict(N=32), dict(N=256), dict(Cin=96),
+               dict(Kh=5, Kw=5, pad=2)):
+        with pytest.raises(mqv.MqvError) as e:
+            mqv.conv_workspace_bytes(_desc(**kw), mqv.OP_FWD_BLOCKSCALED)
+        assert e.value.status == 2
+    w = mqv.QTensorC(16, 16, 16, 128, 1152, 0, 0)
+    x = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, 0)
+    assert lib.mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, None, 0, None) == 3
