@@ -642,7 +642,10 @@ def run_gpu(args):
     if world == 1:
         out["mma_form"] = run_mma_form(dev, layer, peaks)
     if world == 1 and not args.no_sweeps:
-        out["fused_epilogue"] = run_fused(dev, layer, peaks)
+        # the benchmarked (tensor-bound) layer and an HBM-bound 1 x 1 layer,
+        # where the fp32 output is most of the pass's bytes
+        hbm_layer = {l.name: l for l in workloads.yolov8n_mix()}["yolov8n_l12_1x1_128_40px"]
+        out["fused_epilogue"] = [run_fused(dev, layer, peaks), run_fused(dev, hbm_layer, peaks)]
         out["sweeps"] = run_sweeps(args, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(layer, budget_s=args.cpu_budget)
@@ -928,6 +931,32 @@ def run_fused(dev, layer, peaks):
                                         "max, the quantizer reads it once")
     res["fwd_relu_quantize"]["bytes_removed"] = 12 * ne
     res["dgrad_quantize"]["bytes_removed"] = 4 * xr * xc
+    # quantized producer output: the epilogue writes the next operand's codes
+    # and scales with T from a given max (here the previous call's), so no
+    # fp32 output goes through HBM at all
+    tq = torch.empty(1, device=dev)
+    mqv.conv_fwd_fused(d, qw, qx, relu=True, y=y, y_amax=tq, ws=wsf)
+    tg = gx.abs().max().reshape(1)
+
+    def fwd_quantized():
+        mqv.conv_fwd_quantized(d, qw, qx, tq, relu=1, y_q=qy, y_amax=amax, ws=wsf)
+
+    def dgrad_quantized():
+        mqv.conv_dgrad_quantized(d, qw, qg, tg, 4, gx_q=qgx, gx_amax=amax, ws=wsd)
+
+    for name, fn, base in (("fwd_relu_quantize", fwd_quantized, "fused_ms"),
+                           ("dgrad_quantize", dgrad_quantized, "fused_ms")):
+        try:
+            for _ in range(3):
+                fn()
+        except mqv.MqvError as e:
+            res[name]["quantized_output"] = {"unsupported": str(e)}
+            continue
+        tq_ms = _timed(torch, fn, 50, flush)
+        res[name]["quantized_output"] = {
+            "ms": round(tq_ms, 5), "speedup_vs_plain": round(res[name]["plain_ms"] / tq_ms, 3),
+            "speedup_vs_fused": round(res[name][base] / tq_ms, 3),
+            "note": "one pass: the epilogue writes codes and scales (T from a given max, delayed scaling)"}
     flags = mqv.device_errors()
     if flags:
         raise SystemExit(f"device wait timeout flags {flags:#x} in the fused chains")

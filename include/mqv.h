@@ -280,6 +280,37 @@ mqv_status mqv_conv_fwd_fused(const mqv_conv_desc* d, const mqv_qtensor* w, cons
 mqv_status mqv_conv_dgrad_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy, float* gx,
                                 float* gx_amax, void* ws, size_t ws_bytes, void* stream);
 
+/* The forward pass writing the next layer's quantized input instead of
+ * fp32 Y (section "어떻게 동작하나": Y comes out in the channel-batch-first
+ * layout the next layer consumes, so the epilogue can quantize it in place
+ * and the fp32 round trip through HBM disappears).  Quantize-once needs T
+ * before any block can be scaled, and a tile's epilogue runs before the
+ * whole output exists, so T comes from a given max |x|: t_amax, a device
+ * fp32, for example max|Y| of the previous step (delayed scaling; the call
+ * reports this step's max in y_amax).  With t_amax equal to max|Y| of this
+ * output the codes, scales and T are exactly those of mqv_quantize_cbf on
+ * the fp32 Y (after ReLU when relu = 1) that mqv_conv_fwd_fused stores;
+ * with another value they are those of mqv_quantize_with_amax given it
+ * (values above it saturate).  Round to nearest (the activations' rule).
+ *   y_q    the next layer's X: a view of Ho·Wo·Cout rows x N, d->fmt;
+ *          codes, scales and tscale written (nothing in fp32).
+ *   relu, y_amax  as mqv_conv_fwd_fused (y_amax NULL or a device fp32).
+ * Stride-1 layers of the kernel-row path (N divides 256, N % 8 == 0, Cin a
+ * multiple of 64); other layers return MQV_ERR_UNSUPPORTED. */
+mqv_status mqv_conv_fwd_quantized(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
+                                  int32_t relu, const float* t_amax, const mqv_qtensor* y_q, float* y_amax,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* The input-gradient pass writing G_X quantized as the next (earlier)
+ * layer's G_Y, with Philox stochastic rounding (the gradients' rule; element
+ * (r, c) of the H·W·Cin x N view draws word (r·N + c) & 3 of counter
+ * (r·N + c) >> 2 with key `seed`, as mqv_quantize_cbf) and T from t_amax as
+ * above; gx_amax NULL or a device fp32 that receives max|G_X|.  Stride-1
+ * layers of the kernel-row path (Cout a multiple of 64). */
+mqv_status mqv_conv_dgrad_quantized(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
+                                    const float* t_amax, uint64_t seed, const mqv_qtensor* gx_q, float* gx_amax,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* The baseline the method removes (section "무엇인가": quantize after the
  * im2col expansion, once per GEMM direction), for measuring it on the same
  * kernels.  Explicit im2col of fp32 X [H][W][Cin][N] into

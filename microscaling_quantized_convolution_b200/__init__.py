@@ -88,6 +88,14 @@ _SIGS = {
     "mqv_conv_fwd_blockscaled": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                                 ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_fwd_quantized": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                              ctypes.POINTER(QTensorC), ctypes.c_int32, ctypes.c_void_p,
+                                              ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_size_t, ctypes.c_void_p]),
+    "mqv_conv_dgrad_quantized": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
+                                                ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_uint64,
+                                                ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_conv_wgrad": (ctypes.c_int, [ctypes.POINTER(ConvDesc), ctypes.POINTER(QTensorC),
                                       ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]),
@@ -397,6 +405,35 @@ def conv_fwd_blockscaled(d: ConvDesc, w: QTensor, x: QTensor, y: torch.Tensor | 
     _check(lib().mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), y.data_ptr(),
                                           _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return y
+
+
+def conv_fwd_quantized(d: ConvDesc, w: QTensor, x: QTensor, t_amax: torch.Tensor, relu: int = 1,
+                       y_q: QTensor | None = None, y_amax: torch.Tensor | None = None,
+                       ws: torch.Tensor | None = None, stream=None) -> QTensor:
+    """The next layer's X quantized straight from the forward epilogue, T from
+    the device max |x| t_amax (see mqv_conv_fwd_quantized)."""
+    Ho, Wo = out_hw(d)
+    y_q = y_q or QTensor.empty(Ho * Wo * d.Cout, d.N, d.fmt, x.codes.device)
+    ws = _ws(d, OP_FWD, ws, x.codes.device)
+    wc, xc, yc = w.c(), x.c(), y_q.c()
+    _check(lib().mqv_conv_fwd_quantized(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(xc), relu,
+                                        t_amax.data_ptr(), ctypes.byref(yc), _ptr(y_amax), _ptr(ws),
+                                        0 if ws is None else ws.numel(), _stream(stream)))
+    return y_q
+
+
+def conv_dgrad_quantized(d: ConvDesc, w: QTensor, gy: QTensor, t_amax: torch.Tensor, seed: int,
+                         gx_q: QTensor | None = None, gx_amax: torch.Tensor | None = None,
+                         ws: torch.Tensor | None = None, stream=None) -> QTensor:
+    """G_X quantized (stochastic rounding) straight from the input-gradient
+    epilogue, T from t_amax (see mqv_conv_dgrad_quantized)."""
+    gx_q = gx_q or QTensor.empty(d.H * d.W * d.Cin, d.N, d.fmt, gy.codes.device)
+    ws = _ws(d, OP_DGRAD, ws, gy.codes.device)
+    wc, gc, xc = w.c(), gy.c(), gx_q.c()
+    _check(lib().mqv_conv_dgrad_quantized(ctypes.byref(d), ctypes.byref(wc), ctypes.byref(gc), t_amax.data_ptr(),
+                                          seed, ctypes.byref(xc), _ptr(gx_amax), _ptr(ws),
+                                          0 if ws is None else ws.numel(), _stream(stream)))
+    return gx_q
 
 
 def conv_wgrad(d: ConvDesc, gy: QTensor, x: QTensor, gw: torch.Tensor | None = None,

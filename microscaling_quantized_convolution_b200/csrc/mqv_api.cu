@@ -482,14 +482,19 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
   return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, false>(pl, st) : launch_fd<P, FMT, 128, 4, false>(pl, st);
 }
 
-template <int PASS, int FMT>
-cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_halo_kernel<PASS, FMT>;
+template <int PASS, int FMT, bool QOUT>
+cudaError_t launch_halo_q(const ConvPlan& pl, cudaStream_t st) {
+  auto kern = conv_halo_kernel<PASS, FMT, QOUT>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
   if (e != cudaSuccess) return e;
   kern<<<pl.grid, kHaloThreads, HaloSmem::kBytes, st>>>(pl.a, pl.g);
   return cudaGetLastError();
+}
+
+template <int PASS, int FMT>
+cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
+  return pl.a.q_codes ? launch_halo_q<PASS, FMT, true>(pl, st) : launch_halo_q<PASS, FMT, false>(pl, st);
 }
 
 template <int FMT, int KW, bool PAIR>
@@ -581,9 +586,16 @@ mqv_status check_operand(const mqv_qtensor* q, const char* name, int64_t rows, i
   return MQV_OK;
 }
 
+// Quantized output of a fwd/dgrad pass (see V2Args::q_codes).
+struct QuantOut {
+  const mqv_qtensor* q;
+  const float* t_amax;
+  uint64_t seed;
+};
+
 mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const char* na,
                     const mqv_qtensor* qb, const char* nb, float* out, void* ws, size_t ws_bytes,
-                    void* stream, int32_t relu = 0, float* amax = nullptr) {
+                    void* stream, int32_t relu = 0, float* amax = nullptr, const QuantOut* qo = nullptr) {
   mqv_status st = check_desc(d);
   if (st) return st;
   const int64_t Ho = (d->H + 2 * d->pad - d->Kh) / d->stride + 1;
@@ -597,12 +609,26 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
   } else {
     if ((st = check_operand(qa, na, wr, wc, d->fmt)) || (st = check_operand(qb, nb, gr, d->N, d->fmt))) return st;
   }
-  if (!out || !aligned16(out)) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
+  if (!qo && (!out || !aligned16(out))) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
   if (relu != 0 && relu != 1) return fail(MQV_ERR_INVALID_ARG, "relu must be 0 or 1");
   if (amax && (reinterpret_cast<uintptr_t>(amax) & 3u))
     return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
   ConvPlan pl;
   plan_conv(d, op, &pl);
+  if (qo) {
+    if (!pl.halo)
+      return fail(MQV_ERR_UNSUPPORTED, "quantized output: stride-1 layers of the kernel-row path only "
+                                       "(N | 256, N %% 8 == 0, reduction channels a multiple of 64)");
+    const int64_t rows = op == MQV_OP_FWD ? Ho * Wo * d->Cout : d->H * d->W * d->Cin;
+    if ((st = check_operand(qo->q, "quantized output", rows, d->N, d->fmt))) return st;
+    if (!qo->t_amax || (reinterpret_cast<uintptr_t>(qo->t_amax) & 3u))
+      return fail(MQV_ERR_INVALID_ARG, "t_amax must be a 4-byte aligned device pointer");
+    pl.a.q_codes = static_cast<uint8_t*>(qo->q->codes);
+    pl.a.q_scales = qo->q->scales;
+    pl.a.q_tscale = qo->q->tscale;
+    pl.a.q_amax = qo->t_amax;
+    pl.a.q_keys = philox_keys(qo->seed);
+  }
   if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws)))
     return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required, got %zu",
                 pl.ws_bytes, ws ? ws_bytes : (size_t)0);
@@ -968,6 +994,20 @@ mqv_status mqv_conv_fwd_fused(const mqv_conv_desc* d, const mqv_qtensor* w, cons
 mqv_status mqv_conv_dgrad_fused(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy, float* gx,
                                 float* gx_amax, void* ws, size_t ws_bytes, void* stream) {
   return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", gx, ws, ws_bytes, stream, 0, gx_amax);
+}
+
+mqv_status mqv_conv_fwd_quantized(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x, int32_t relu,
+                                  const float* t_amax, const mqv_qtensor* y_q, float* y_amax, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  const QuantOut qo{y_q, t_amax, 0};
+  return run_conv(MQV_OP_FWD, d, w, "w", x, "x", nullptr, ws, ws_bytes, stream, relu, y_amax, &qo);
+}
+
+mqv_status mqv_conv_dgrad_quantized(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
+                                    const float* t_amax, uint64_t seed, const mqv_qtensor* gx_q, float* gx_amax,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  const QuantOut qo{gx_q, t_amax, seed};
+  return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", nullptr, ws, ws_bytes, stream, 0, gx_amax, &qo);
 }
 
 mqv_status mqv_device_errors(uint32_t* flags, void* stream) {

@@ -185,6 +185,38 @@ struct HaloCursor {
 // warp's 4 KB of shared memory (wbuf) turns that into stores of 128-byte runs
 // of one (pixel, channel) row's batch items.  Columns past bw·N hold no
 // output (j >= bw below).
+// With p.q_codes set the values are quantized instead of stored: a 4 x 4
+// block of the next operand is 4 channel rows x 4 batch items at one pixel,
+// held by the lanes q, q + 8, q + 16, q + 24 (rows 4i .. 4i + 3), so two
+// shuffles give its max|x|, and each lane quantizes its row of the block
+// with the quantizer's own arithmetic (RND 0: round to nearest, 1:
+// stochastic with the element's Philox word).
+template <int FMT, int RND>
+__device__ __forceinline__ void halo_quantize_row(const V2Args& p, float4 o, bool ok, int64_t row, int n,
+                                                  const TensorScale<FMT>& ts, int rsub) {
+  float bm = ok ? absmax4(o) : 0.0f;
+  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+  if (!ok) return;
+  const BlockScale<FMT> bs(bm, ts);
+  uint4 w = make_uint4(0u, 0u, 0u, 0u);
+  if (RND == 1) {
+    const uint64_t gc = static_cast<uint64_t>(row * p.N + n) >> 2;
+    w = philox4x32_10(make_uint4(static_cast<uint32_t>(gc), static_cast<uint32_t>(gc >> 32), 0u, 0u), p.q_keys);
+  }
+  const uint32_t packed = quantize_row4<FMT, RND>(o, bs.d, bs.y, bs.exact, w);
+  if (FMT == 0) {
+    *reinterpret_cast<uint16_t*>(p.q_codes + row * (p.N >> 1) + (n >> 1)) = static_cast<uint16_t>(packed);
+  } else {
+    uint8_t* c = p.q_codes + row * ((p.N * 3) >> 2) + ((n * 3) >> 2);
+    c[0] = static_cast<uint8_t>(packed);
+    c[1] = static_cast<uint8_t>(packed >> 8);
+    c[2] = static_cast<uint8_t>(packed >> 16);
+  }
+  if (rsub == 0) p.q_scales[(row >> 2) * (p.N >> 2) + (n >> 2)] = static_cast<uint8_t>(bs.scode);
+}
+
+template <int FMT, int RND, bool QOUT>
 __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGeom& g, uint32_t tmem, int acc_col,
                                                    int tile, int quarter, uint32_t wbuf, int first, int stride,
                                                    float& amax) {
@@ -217,8 +249,22 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
     const int j = fdiv(lc, p.dN);
     const int n = lc - j * p.N;
     const int ow = ow0 + j;
-    if (j < g.bw && ow < g.out_w) {
-      const int64_t pix = static_cast<int64_t>(oh) * g.out_w + ow;
+    const bool colok = j < g.bw && ow < g.out_w;
+    const int64_t pix = static_cast<int64_t>(oh) * g.out_w + ow;
+    if (QOUT) {
+      // every lane takes part in the block-max shuffles
+      const TensorScale<FMT> ts(*p.q_amax);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = 4 * i + rsub;
+        const int64_t mrow = static_cast<int64_t>(mt) * 128 + quarter * 32 + row;
+        float4 o = ld_shared_v4_f32(wbuf + row * 128 + ((q ^ (row & 7)) << 4));
+        const bool ok = colok && mrow < p.M;
+        if (p.relu) o = epi_relu(o);
+        if (ok && p.amax_out) amax = epi_absmax(amax, o);
+        halo_quantize_row<FMT, RND>(p, o, ok, pix * p.M + mrow, n, ts, rsub);
+      }
+    } else if (colok) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int row = 4 * i + rsub;
@@ -235,7 +281,9 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
   }
 }
 
-template <int PASS, int FMT>
+// QOUT: the quantized-output epilogue (V2Args::q_codes), a separate
+// instance so that the plain passes keep their code and registers.
+template <int PASS, int FMT, bool QOUT>
 __global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
   using L = HaloSmem;
@@ -270,6 +318,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
   const int stages_per_tile = p.Kh * g.cchunks;
   const int na = kHaloAStages / p.Kw;     // weight stages in the ring (Kw <= kHaloAStages)
 
+  if (QOUT && blockIdx.x == 0 && threadIdx.x == 0) *p.q_tscale = TensorScale<FMT>(*p.q_amax).T;
   if (warp < kV2EpiWarps) {
     // epilogue: column lc of the tile = (pixel j, batch item n) -> output
     // pixel (oh, ow0 + j), skipped past the end of the output row.  The
@@ -283,7 +332,8 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const bool last = tile + static_cast<int>(gridDim.x) >= p.tiles;
-      halo_epilogue_tile(p, g, bars->tmem, acc * kHaloBN, tile, warp & 3, wbuf, 0, last ? 4 : 1, amax);
+      halo_epilogue_tile<FMT, PASS == kDgrad, QOUT>(p, g, bars->tmem, acc * kHaloBN, tile, warp & 3, wbuf, 0,
+                                                    last ? 4 : 1, amax);
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
     }
@@ -415,8 +465,8 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       // tile has its own single-phase barrier.
       mbar_wait_bounded(&bars->last_full, 0, p.err, kErrWaitDone);
       tc_fence_after();
-      halo_epilogue_tile(p, g, bars->tmem, (lit & 1) * kHaloBN, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
-                         1 + pw / 4, 4, amax);
+      halo_epilogue_tile<FMT, PASS == kDgrad, QOUT>(p, g, bars->tmem, (lit & 1) * kHaloBN, ltile_last, warp & 3,
+                                                    sbase + L::kBOffset + pw * 4096, 1 + pw / 4, 4, amax);
       epi_amax_flush(p.amax_out, amax);
     }
   }

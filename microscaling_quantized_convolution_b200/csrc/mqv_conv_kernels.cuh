@@ -35,6 +35,7 @@
 
 #include "mqv_conv_common.cuh"
 #include "mqv_ptx.cuh"
+#include "mqv_quantize.cuh"
 
 namespace mqv {
 
@@ -73,6 +74,16 @@ struct V2Args {
   // atomicMax (non-negative floats order like their bit patterns).
   uint32_t* amax_out;
   int relu;
+  // Quantized output (kernel-row halo kernel only): with q_codes set the
+  // output is not stored in fp32 but quantized as the next operand of the
+  // method, a (pixels·M) x N view in q_codes / q_scales, with the tensor
+  // scale T from the device max |x| *q_amax (written to *q_tscale); round to
+  // nearest for the forward pass, stochastic rounding (q_keys) for dgrad.
+  uint8_t* q_codes;
+  uint8_t* q_scales;
+  float* q_tscale;
+  const float* q_amax;
+  PhiloxKeys q_keys;
   // Transposed tiles of the generic fwd/dgrad kernel (TR): the MMA's 128
   // rows are GEMM columns (pixel, n) and its N = nc (M rounded up to 16)
   // columns are the output channels.

@@ -194,7 +194,7 @@ conv_fwd_nvf4_kernel(const V2Args p, const HaloGeom g) {
       mbar_wait_bounded(&bars->acc_full[acc], (it >> 1) & 1, p.err, kErrWaitDone);
       tc_fence_after();
       const bool last = tile + static_cast<int>(gridDim.x) >= p.tiles;
-      halo_epilogue_tile(p, g, bars->tmem, acc * kNvf4BN, tile, warp & 3, wbuf, 0, last ? 3 : 1, amax);
+      halo_epilogue_tile<0, 0, false>(p, g, bars->tmem, acc * kNvf4BN, tile, warp & 3, wbuf, 0, last ? 3 : 1, amax);
       tc_fence_before();
       mbar_arrive(&bars->acc_empty[acc]);
     }
@@ -325,7 +325,7 @@ conv_fwd_nvf4_kernel(const V2Args p, const HaloGeom g) {
       float amax = 0.f;
       mbar_wait_bounded(&bars->last_full, 0, p.err, kErrWaitDone);
       tc_fence_after();
-      halo_epilogue_tile(p, g, bars->tmem, (lit & 1) * kNvf4BN, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
+      halo_epilogue_tile<0, 0, false>(p, g, bars->tmem, (lit & 1) * kNvf4BN, ltile_last, warp & 3, sbase + L::kBOffset + pw * 4096,
                          1 + pw / 4, 3, amax);
       epi_amax_flush(p.amax_out, amax);
     }

@@ -255,12 +255,36 @@ struct QuantArgs {
   FastDiv dcb;          // division by the column blocks of a block row (block count < 2^31)
 };
 
+// Block scale of a block with max|x| = bmax: the E4M3 code, the divisor
+// d = B·T, y = RN(1/d) (0 where the Markstein quotient does not apply) and
+// whether the block divides with the IEEE divide.
+template <int FMT>
+struct BlockScale {
+  uint32_t scode;
+  float d, y;
+  bool exact;
+  __device__ __forceinline__ BlockScale(float bmax, const TensorScale<FMT>& ts) {
+    scode = 0;
+    d = 0.0f;
+    y = 0.0f;
+    if (ts.T > 0.0f) {
+      scode = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
+      d = __fmul_rn(e4m3_to_f32(scode), ts.T);
+      y = d >= kMarksteinMinDivisor ? __frcp_rn(d) : 0.0f;
+    }
+    exact = d > 0.0f && d < kMarksteinMinDivisor;
+  }
+};
+
+__device__ __forceinline__ float absmax4(float4 v) {
+  return fmaxf(max3f(fabsf(v.x), fabsf(v.y), fabsf(v.z)), fabsf(v.w));
+}
+
 // Quantize the 4 x 4 block (br, bc) whose 4 rows are x[r], and store its
 // scale and codes.
 template <int FMT, int RND>
 __device__ __forceinline__ void quantize_block(const float4 (&x)[4], const TensorScale<FMT>& ts, const QuantArgs& qa,
                                                int64_t br, int64_t bc, int64_t cb, int64_t row_bytes) {
-  const float T = ts.T;
   float bmax = max3f(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[0].z));
   bmax = max3f(bmax, fabsf(x[0].w), fabsf(x[1].x));
   bmax = max3f(bmax, fabsf(x[1].y), fabsf(x[1].z));
@@ -268,14 +292,10 @@ __device__ __forceinline__ void quantize_block(const float4 (&x)[4], const Tenso
   b2 = max3f(b2, fabsf(x[2].z), fabsf(x[2].w));
   float b3 = max3f(fabsf(x[3].x), fabsf(x[3].y), fabsf(x[3].z));
   bmax = max3f(bmax, b2, fmaxf(b3, fabsf(x[3].w)));
-  uint32_t scode = 0;
-  float d = 0.0f, y = 0.0f;
-  if (T > 0.0f) {
-    scode = f32_to_e4m3_satfinite(__fdiv_rn(bmax, ts.Temax));
-    d = __fmul_rn(e4m3_to_f32(scode), T);
-    y = d >= kMarksteinMinDivisor ? __frcp_rn(d) : 0.0f;
-  }
-  const bool exact = d > 0.0f && d < kMarksteinMinDivisor;
+  const BlockScale<FMT> bs(bmax, ts);
+  const uint32_t scode = bs.scode;
+  const float d = bs.d, y = bs.y;
+  const bool exact = bs.exact;
   qa.scales[br * cb + bc] = static_cast<uint8_t>(scode);
   // Philox counter of row r: (element index of its first element) / 4
   uint64_t g = 0, gstep = 0;

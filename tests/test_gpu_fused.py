@@ -128,3 +128,77 @@ def test_full_size_yolo_layers_fused_passes(idx):
     assert torch.equal(y, torch.relu(y_plain)) and ya.item() == y.max().item()
     assert torch.equal(gx, gx_plain) and ga.item() == gx.abs().max().item()
     assert mqv.device_errors() == 0
+
+
+# ----------------------------------------------- quantized producer output
+
+QCASES = [
+    ("halo_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp4"),
+    ("halo_n32_two_m_tiles_fp6", O.ConvShape(32, 128, 192, 5, 9, 3, 3, 1, 1), "nvfp6"),
+    ("halo_multitile_1x1", O.ConvShape(16, 64, 64, 40, 40, 1, 1, 1, 0), "nvfp4"),
+]
+
+
+def _oracle_codes(q: "mqv.QTensor", fmt):
+    return (O.unpack_codes(q.codes.cpu().numpy(), q.rows, q.cols, FMT[fmt]),
+            q.scales.cpu().numpy().reshape(q.rows // 4, q.cols // 4), np.float32(q.tscale.item()))
+
+
+def _assert_quantized(got: "mqv.QTensor", ref: O.QTensor, fmt, what):
+    codes, scales, T = _oracle_codes(got, fmt)
+    assert T == ref.T, what
+    assert np.array_equal(scales, ref.scales), f"{what}: scales"
+    assert np.array_equal(codes, ref.codes), f"{what}: {int(np.sum(codes != ref.codes))} codes differ"
+
+
+@pytest.mark.parametrize("name,s,fmt", QCASES, ids=[c[0] for c in QCASES])
+@pytest.mark.parametrize("amax_factor", [1.0, 0.5, 3.0])
+def test_forward_writes_next_layer_input_quantized(name, s, fmt, amax_factor):
+    """The forward epilogue quantizes ReLU(Y) into the next layer's X with T
+    from a given max |x|: codes, scales and T equal the oracle's quantizer on
+    the fp32 ReLU(Y) the fused pass stores, given that max (the true max,
+    half of it, so that blocks saturate, and three times it); the reported
+    max is this output's."""
+    (X, Wt, G), d, qx, qw, qg = _quantized(s, fmt, name)
+    y, amax = mqv.conv_fwd_fused(d, qw, qx, relu=True)
+    t_amax = amax * amax_factor
+    y_amax = torch.zeros(1, device="cuda")
+    yq = mqv.conv_fwd_quantized(d, qw, qx, t_amax, relu=1, y_amax=y_amax)
+    torch.cuda.synchronize()
+    assert mqv.device_errors() == 0
+    assert y_amax.item() == amax.item()
+    ref = O.quantize(y.cpu().numpy().reshape(s.Ho * s.Wo * s.Cout, s.N), FMT[fmt], O.RNE,
+                     amax=float(t_amax.item()))
+    _assert_quantized(yq, ref, fmt, f"{name} fwd x{amax_factor}")
+    if amax_factor == 1.0:      # the true max: the two-pass quantizer's codes
+        two = mqv.quantize(y.view(-1), s.Ho * s.Wo * s.Cout, s.N, fmt, mqv.RNE)
+        torch.cuda.synchronize()
+        for f in ("codes", "scales", "tscale"):
+            assert torch.equal(getattr(two, f), getattr(yq, f)), f
+
+
+@pytest.mark.parametrize("name,s,fmt", QCASES, ids=[c[0] for c in QCASES])
+def test_input_gradient_writes_quantized_with_stochastic_rounding(name, s, fmt):
+    """The input-gradient epilogue quantizes G_X with stochastic rounding
+    (the element's Philox word, the quantizer's numbering) and T from a given
+    max: equal to the oracle's quantizer on the fp32 G_X of the plain pass."""
+    (X, Wt, G), d, qx, qw, qg = _quantized(s, fmt, name)
+    gx = mqv.conv_dgrad(d, qw, qg)
+    t_amax = gx.abs().max().reshape(1) * 0.75
+    gx_amax = torch.zeros(1, device="cuda")
+    gq = mqv.conv_dgrad_quantized(d, qw, qg, t_amax, seed=1234, gx_amax=gx_amax)
+    torch.cuda.synchronize()
+    assert mqv.device_errors() == 0
+    assert gx_amax.item() == gx.abs().max().item()
+    ref = O.quantize(gx.cpu().numpy().reshape(s.H * s.W * s.Cin, s.N), FMT[fmt], O.SR, 1234,
+                     amax=float(t_amax.item()))
+    _assert_quantized(gq, ref, fmt, f"{name} dgrad")
+
+
+def test_quantized_output_rejects_other_layers():
+    s = O.ConvShape(8, 24, 40, 9, 9, 3, 3, 2, 1)          # stride 2: the generic kernel
+    (X, Wt, G), d, qx, qw, qg = _quantized(s, "nvfp4", "reject")
+    t = torch.ones(1, device="cuda")
+    with pytest.raises(mqv.MqvError) as e:
+        mqv.conv_fwd_quantized(d, qw, qx, t)
+    assert e.value.status == 2
