@@ -118,7 +118,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     import microscaling_quantized_convolution_b200 as mqv
-    from microscaling_quantized_convolution_b200 import naive
+    from microscaling_quantized_convolution_b200 import dp, naive
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -173,15 +173,10 @@ def run_gpu(args):
         dtype=torch.uint8, device=dev)
 
     def quantize_all(s, step):
-        if world == 1:
-            # X and W round to nearest, G_Y stochastically; one amax pass, one quantize pass
-            mqv.quantize_many([(s["X"], xr, xc, fmt, mqv.RNE, 0, s["qx"]),
-                               (s["W"], wr, wc, fmt, mqv.RNE, 0, s["qw"]),
-                               (s["G"], gr, gc, fmt, mqv.SR, seed + step, s["qg"])], ws=ws_many)
-        else:
-            amax_all(s)
-            dist.all_reduce(amax_buf, op=dist.ReduceOp.MAX)
-            quantize_with_global_amax(s, step)
+        # X and W round to nearest, G_Y stochastically; one amax pass, one quantize pass
+        mqv.quantize_many([(s["X"], xr, xc, fmt, mqv.RNE, 0, s["qx"]),
+                           (s["W"], wr, wc, fmt, mqv.RNE, 0, s["qw"]),
+                           (s["G"], gr, gc, fmt, mqv.SR, seed + step, s["qg"])], ws=ws_many)
 
     # the same quantization as two independent calls (X and W for fwd, G_Y
     # for the gradients), each with its own workspace, for the concurrent step
@@ -197,18 +192,6 @@ def run_gpu(args):
     def quantize_g(s, step):
         mqv.quantize_many([(s["G"], gr, gc, fmt, mqv.SR, seed + step, s["qg"])], ws=ws_g)
 
-    def amax_all(s):
-        mqv.amax(s["X"], xr, xc, out=amax_buf[0:1], ws=ws_q[0])
-        mqv.amax(s["G"], gr, gc, out=amax_buf[2:3], ws=ws_q[2])
-
-    def quantize_with_global_amax(s, step):
-        # this rank's batch is columns [rank·N, (rank+1)·N) of the global batch
-        mqv.quantize_with_amax(s["X"], xr, xc, fmt, mqv.RNE, 0, amax_buf[0:1], out=s["qx"],
-                               sr_col0=rank * xc, sr_cols=world * xc)
-        mqv.quantize(s["W"], wr, wc, fmt, mqv.RNE, 0, out=s["qw"], ws=ws_q[1])
-        mqv.quantize_with_amax(s["G"], gr, gc, fmt, mqv.SR, seed + step, amax_buf[2:3], out=s["qg"],
-                               sr_col0=rank * gc, sr_cols=world * gc)
-
     def fwd(s):
         mqv.conv_fwd(d, s["qw"], s["qx"], y=s["y"], ws=ws_fwd)
 
@@ -218,13 +201,70 @@ def run_gpu(args):
     def dgrad(s):
         mqv.conv_dgrad(d, s["qw"], s["qg"], gx=s["gx"], ws=ws_dgrad)
 
+    class ShardOps:
+        """The kernels of the data-parallel step (dp.data_parallel_step, the
+        one implementation of the exchange) on input set k's fixed buffers:
+        each call runs its library call, or replays the CUDA graph captured
+        from that call."""
+        RNE, SR = mqv.RNE, mqv.SR
+
+        def __init__(self, k, graphs=None, capture_into=None):
+            self.k, self.s, self.g, self.cap = k, sets[k], graphs, capture_into
+
+        def _run(self, name, fn):
+            if self.cap is not None:
+                self.cap[name] = capture(fn)
+            elif self.g is not None:
+                self.g[name].replay()
+            else:
+                fn()
+
+        def amax(self, t, rows, cols):
+            x = t is self.s["X"]
+            out = amax_buf[0:1] if x else amax_buf[2:3]
+            self._run("amax_x" if x else "amax_g", lambda: mqv.amax(t, rows, cols, out=out, ws=ws_q[0 if x else 2]))
+            return out
+
+        def quantize_with_amax(self, t, rows, cols, f, rnd, sd, a, c0, tc):
+            x = t is self.s["X"]
+            q = self.s["qx"] if x else self.s["qg"]
+            self._run("quant_x" if x else "quant_g",
+                      lambda: mqv.quantize_with_amax(t, rows, cols, f, rnd, sd, a, out=q, sr_col0=c0, sr_cols=tc))
+            return q
+
+        def quantize(self, t, rows, cols, f, rnd, sd):
+            self._run("quant_w", lambda: mqv.quantize(t, rows, cols, f, rnd, sd, out=self.s["qw"], ws=ws_q[1]))
+            return self.s["qw"]
+
+        def fwd(self, dims, qw, qx):
+            self._run("fwd", lambda: fwd(self.s))
+            return self.s["y"]
+
+        def wgrad(self, dims, qg, qx):
+            self._run("wgrad", lambda: wgrad(self.s))
+            return self.s["gw"]
+
+        def dgrad(self, dims, qw, qg):
+            self._run("dgrad", lambda: dgrad(self.s))
+            return self.s["gx"]
+
+    comm = dp.torch_comm() if world > 1 else None
+
+    def dp_step(k, ops, mark=None):
+        # this rank's batch is columns [rank·N, (rank+1)·N) of the global batch
+        s = sets[k]
+        dp.data_parallel_step(ops, comm, s["X"], s["W"], s["G"], layer.dims(), fmt, world * layer.N, rank, world,
+                              seed + k, mark=mark)
+
     def step(i, s=None):
-        s = sets[i % nsets] if s is None else s
+        k = i % nsets if s is None else next(j for j in range(nsets) if sets[j] is s)
+        if world > 1:
+            dp_step(k, ShardOps(k))
+            return
+        s = sets[k]
         quantize_all(s, i)
         fwd(s)
         wgrad(s)
-        if world > 1:
-            dist.all_reduce(s["gw"])
         dgrad(s)
 
     for i in range(args.warmup):
@@ -252,8 +292,9 @@ def run_gpu(args):
             gk["quant_xw"] = capture(lambda: quantize_xw(s))
             gk["quant_g"] = capture(lambda: quantize_g(s, k))
         else:
-            gk["amax"] = capture(lambda: amax_all(s))
-            gk["quant"] = capture(lambda: quantize_with_global_amax(s, k))
+            # every kernel call of the data-parallel step, captured as the
+            # step makes it (the collectives between them run eagerly)
+            dp_step(k, ShardOps(k, capture_into=gk))
         graphs.append(gk)
     torch.cuda.synchronize()
 
@@ -293,8 +334,12 @@ def run_gpu(args):
                 cur.wait_event(ev[3 + 2 * j])
             return
         if world > 1:
-            gk["amax"].replay()
-            dist.all_reduce(amax_buf, op=dist.ReduceOp.MAX)
+            # the data-parallel step replaying its captured calls; its phase
+            # boundaries record the events the serial step records below
+            marks = {"start": (), "quantized": (ev[1], ev[2]), "fwd": (ev[3], ev[4]), "wgrad": (ev[5], ev[6]),
+                     "dgrad": (ev[7],)}
+            dp_step(k, ShardOps(k, graphs=gk), mark=lambda nm: [e.record() for e in marks[nm]])
+            return
         gk["quant"].replay()
         ev[1].record()
         ev[2].record()
@@ -302,8 +347,6 @@ def run_gpu(args):
         ev[3].record()
         ev[4].record()
         gk["wgrad"].replay()
-        if world > 1:
-            dist.all_reduce(s["gw"])
         ev[5].record()
         ev[6].record()
         gk["dgrad"].replay()

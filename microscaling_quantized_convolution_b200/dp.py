@@ -46,7 +46,7 @@ def shard_columns(n_global: int, rank: int, world: int) -> tuple[int, int]:
 
 
 def data_parallel_step(ops, comm: Comm, X, W, G, dims: dict, fmt, n_global: int, rank: int,
-                       world: int, seed: int):
+                       world: int, seed: int, mark=None, quantized=None):
     """One layer: quantize X, W (RNE), G_Y (SR), then fwd, wgrad, dgrad.
 
     X [H][W][Cin][n_local], G [Ho][Wo][Cout][n_local]: this rank's shard.
@@ -55,7 +55,12 @@ def data_parallel_step(ops, comm: Comm, X, W, G, dims: dict, fmt, n_global: int,
     quantize_with_amax(t, rows, cols, fmt, rounding, seed, amax, sr_col0, sr_cols),
     quantize(t, rows, cols, fmt, rounding, seed), fwd(dims, qw, qx), wgrad(dims, qg, qx),
     dgrad(dims, qw, qg), and the rounding constants RNE and SR.
+    `mark(name)`, if given, is called at the phase boundaries "start",
+    "quantized", "fwd", "wgrad" (after the G_W sum) and "dgrad" (the
+    benchmark records timing events there); `quantized`, if a dict, receives
+    the quantized operands (qx, qw, qg).
     Returns (Y_local, G_W (summed over ranks), G_X_local)."""
+    mark = mark or (lambda name: None)
     col0, n_local = shard_columns(n_global, rank, world)
     assert dims["N"] == n_local
     Ho = (dims["H"] + 2 * dims["pad"] - dims["Kh"]) // dims["stride"] + 1
@@ -63,6 +68,7 @@ def data_parallel_step(ops, comm: Comm, X, W, G, dims: dict, fmt, n_global: int,
     xr = dims["H"] * dims["W"] * dims["Cin"]
     gr = Ho * Wo * dims["Cout"]
     wr, wc = dims["Cout"], dims["Kh"] * dims["Kw"] * dims["Cin"]
+    mark("start")
     ax = ops.amax(X, xr, n_local)
     ag = ops.amax(G, gr, n_local)
     comm.all_reduce_max(ax)
@@ -70,10 +76,16 @@ def data_parallel_step(ops, comm: Comm, X, W, G, dims: dict, fmt, n_global: int,
     qx = ops.quantize_with_amax(X, xr, n_local, fmt, ops.RNE, 0, ax, col0, n_global)
     qg = ops.quantize_with_amax(G, gr, n_local, fmt, ops.SR, seed, ag, col0, n_global)
     qw = ops.quantize(W, wr, wc, fmt, ops.RNE, 0)
+    if quantized is not None:
+        quantized.update(qx=qx, qw=qw, qg=qg)
+    mark("quantized")
     y = ops.fwd(dims, qw, qx)
+    mark("fwd")
     gw = ops.wgrad(dims, qg, qx)
     comm.all_reduce_sum(gw)
+    mark("wgrad")
     gx = ops.dgrad(dims, qw, qg)
+    mark("dgrad")
     return y, gw, gx
 
 
