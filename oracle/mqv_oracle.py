@@ -620,6 +620,111 @@ def naive_quantize_after_im2col(X: np.ndarray, s: ConvShape, fmt: str, along: st
     return xhat.T if along == "k" else xhat
 
 
+@dataclass
+class QTensor1D:
+    codes: np.ndarray    # int64 (rows, cols): sign bit | magnitude code
+    scales: np.ndarray   # uint8: (rows, cols/16) for blocks along a row, (rows/16, cols) down a column
+    T: np.float32
+    fmt: str
+    axis: int            # 1: 1 x 16 blocks along a row; 0: 16 x 1 blocks down a column
+
+
+def quantize_1d(x2d: np.ndarray, fmt: str, rounding: str, seed: int = 0, axis: int = 1) -> QTensor1D:
+    """Two-level quantization with plain 16-element blocks along one axis of
+    a 2D view: the NVFP4 formulas of section "무엇과 다른가" (T from max|X|,
+    B = CastE4M3(blockmax / (T·emax)), code = Round(x / (B·T))) on the
+    blocks the scheme of section "무엇인가" uses, 16 consecutive elements of
+    a GEMM operand along its contraction.  axis = 1: 1 x 16 blocks along each
+    row (cols a multiple of 16); axis = 0: 16 x 1 blocks down each column
+    (rows a multiple of 16).  Rounding as in `quantize` (RNE, or SR with the
+    row-major index of the element in the view)."""
+    x = np.ascontiguousarray(x2d, dtype=np.float32)
+    rows, cols = x.shape
+    assert (cols if axis == 1 else rows) % 16 == 0
+    emax = np.float32(element_max(fmt))
+    T = tensor_scale(x, fmt)
+    mbits = element_bits(fmt) - 1
+    sign = np.signbit(x).astype(np.int64) << mbits
+    shape = (rows, cols // 16) if axis == 1 else (rows // 16, cols)
+    if T == 0:
+        return QTensor1D(sign, np.zeros(shape, np.uint8), T, fmt, axis)
+    a = np.abs(x)
+    bmax = (a.reshape(rows, cols // 16, 16).max(axis=2) if axis == 1
+            else a.reshape(rows // 16, 16, cols).max(axis=1)).astype(np.float32)
+    scales = cast_e4m3((bmax / np.float32(T * emax)).astype(np.float32))
+    B = E4M3_GRID[scales].astype(np.float32)
+    d = (B * T).astype(np.float32)
+    d = np.repeat(d, 16, axis=1) if axis == 1 else np.repeat(d, 16, axis=0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = (a / d).astype(np.float32)
+    v = np.where(d == 0, np.float32(0), v)
+    if rounding == RNE:
+        mag = round_rne(v, fmt)
+    else:
+        idx = np.arange(rows * cols, dtype=np.uint64)
+        mag = round_sr(v, sr_uniforms(seed, idx).reshape(rows, cols), fmt)
+    mag = np.where(d == 0, 0, mag)
+    return QTensor1D(sign | mag, scales, T, fmt, axis)
+
+
+def code_values_1d(q: QTensor1D) -> np.ndarray:
+    """code·B of a 1-D-block quantized view, fp64 (exact)."""
+    mbits = element_bits(q.fmt) - 1
+    mag = element_grid(q.fmt)[q.codes & ((1 << mbits) - 1)]
+    val = np.where((q.codes >> mbits) & 1, -mag, mag)
+    B = E4M3_GRID[q.scales]
+    return val * (np.repeat(B, 16, axis=1) if q.axis == 1 else np.repeat(B, 16, axis=0))
+
+
+def expanded_view(X: np.ndarray, s: ConvShape) -> np.ndarray:
+    """X' of the naive scheme in the channel-batch-first layout of a 1 x 1
+    convolution with Kh·Kw·Cin input channels: rows (ho, wo, kh, kw, ci),
+    columns n (the im2col matrix with its column index (ho, wo, n) split)."""
+    K = s.Kh * s.Kw * s.Cin
+    return np.ascontiguousarray(im2col(X, s).reshape(K, s.Ho * s.Wo, s.N).transpose(1, 0, 2)).reshape(-1, s.N)
+
+
+def naive_layer(X: np.ndarray, Wt: np.ndarray, GY: np.ndarray, s: ConvShape, fmt: str, seed: int = 0):
+    """The layer step of the scheme section "무엇인가" describes: expand X
+    with im2col first, then quantize every GEMM operand with plain
+    16-element blocks along that GEMM's contraction, one copy per direction:
+      X'  along K for Y = W·X' (16 x 1 down the expanded view's rows) and
+          along P for G_W = G_Y·X'^T (1 x 16 along its batch columns);
+      W   along K for Y (1 x 16 along its rows), along Cout for G_X'
+          (16 x 1 down its columns);
+      G_Y along P for G_W (1 x 16), along Cout for G_X' (16 x 1);
+    RNE for X' and W, stochastic rounding for G_Y (the same element
+    numbering and seed for both of its copies).  The GEMMs are 1 x 1
+    convolutions over the Kh·Kw·Cin expanded channels, and G_X = col2im(G_X').
+    Returns the six copies and the outputs (values, |product| sums), in fp64
+    with the tensor scales applied."""
+    K = s.Kh * s.Kw * s.Cin
+    xv = expanded_view(X.astype(np.float32), s)
+    wv = Wt.reshape(s.Cout, K).astype(np.float32)
+    gv = GY.reshape(s.Ho * s.Wo * s.Cout, s.N).astype(np.float32)
+    q = {"x_fwd": quantize_1d(xv, fmt, RNE, axis=0), "x_wgrad": quantize_1d(xv, fmt, RNE, axis=1),
+         "w_fwd": quantize_1d(wv, fmt, RNE, axis=1), "w_dgrad": quantize_1d(wv, fmt, RNE, axis=0),
+         "g_wgrad": quantize_1d(gv, fmt, SR, seed, axis=1), "g_dgrad": quantize_1d(gv, fmt, SR, seed, axis=0)}
+    s1 = ConvShape(s.N, K, s.Cout, s.Ho, s.Wo, 1, 1, 1, 0)
+    val = {k: code_values_1d(v) for k, v in q.items()}
+    T = {k: np.float64(v.T) for k, v in q.items()}
+    xf = val["x_fwd"].reshape(s.Ho, s.Wo, K, s.N)
+    xw = val["x_wgrad"].reshape(s.Ho, s.Wo, K, s.N)
+    wf = val["w_fwd"].reshape(s.Cout, 1, 1, K)
+    wd = val["w_dgrad"].reshape(s.Cout, 1, 1, K)
+    gw_ = val["g_wgrad"].reshape(s.Ho, s.Wo, s.Cout, s.N)
+    gd = val["g_dgrad"].reshape(s.Ho, s.Wo, s.Cout, s.N)
+    Y, SY = conv_fwd(wf, xf, s1)
+    GW, SW = conv_wgrad(gw_, xw, s1)
+    GXe, SXe = conv_dgrad(wd, gd, s1)                      # [Ho][Wo][K][N], the expanded gradient
+    unexp = lambda t: col2im(t.reshape(s.Ho * s.Wo, K, s.N).transpose(1, 0, 2).reshape(K, -1), s)
+    tf, tw, td = T["w_fwd"] * T["x_fwd"], T["g_wgrad"] * T["x_wgrad"], T["w_dgrad"] * T["g_dgrad"]
+    out = {"y": (Y * tf, SY * tf), "gw": (GW.reshape(s.Cout, s.Kh, s.Kw, s.Cin) * tw,
+                                           SW.reshape(s.Cout, s.Kh, s.Kw, s.Cin) * tw),
+           "gx": (unexp(GXe) * td, unexp(SXe) * td)}
+    return q, out
+
+
 def bits_per_element(fmt: str) -> float:
     """Stored bits per element: the element code plus one E4M3 byte per 16."""
     return element_bits(fmt) + 8.0 / 16.0

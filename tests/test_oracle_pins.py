@@ -553,6 +553,141 @@ def test_quantize_once_gives_one_value_per_pixel_naive_does_not(cin, along):
     assert sum(len(v) > 1 for v in naive.values()) > 0
 
 
+# ------------------------------------------ 16-element blocks (the naive scheme)
+
+def test_1d_blocks_are_the_naive_im2col_quantization():
+    """quantize_1d on the explicit im2col matrix (K rows x P columns) with
+    blocks down its columns (along K) or along its rows (along P) dequantizes
+    to the values of naive_quantize_after_im2col, the scheme of section
+    "무엇인가" pinned above (P5): the same codes and scales, the values equal
+    up to the fp32 rounding of B·T that function multiplies by (relative
+    2^-24; a different code or scale would differ by 1/8 or more)."""
+    s = O.ConvShape(4, 16, 8, 6, 6, 3, 3, 1, 1)
+    rng = np.random.default_rng(21)
+    X = rng.standard_normal((s.H, s.W, s.Cin, s.N)).astype(np.float32)
+    Xc = O.im2col(X, s).astype(np.float32)                  # (Kh·Kw·Cin) x (Ho·Wo·N)
+    for axis, along in ((0, "k"), (1, "p")):
+        q = O.quantize_1d(Xc, O.FP4, O.RNE, axis=axis)
+        got = O.code_values_1d(q) * np.float64(q.T)
+        ref = O.naive_quantize_after_im2col(X, s, O.FP4, along)
+        assert np.all(np.abs(got - ref) <= 2.0 ** -23 * np.abs(ref))
+        assert np.count_nonzero(got) > 0.5 * got.size
+
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+@pytest.mark.parametrize("rounding", [O.RNE, O.SR])
+@pytest.mark.parametrize("axis", [0, 1])
+def test_1d_representable_blocks_are_recovered_exactly(fmt, rounding, axis):
+    """x = c·s·T with T a power of two and s an E4M3 value whose block
+    holds the code emax: every step of the formula is exact, so the codes
+    and scales come back unchanged (stochastic rounding leaves grid values
+    where they are)."""
+    rng = np.random.default_rng(22 + axis)
+    grid = O.element_grid(fmt)
+    nb, emax = 6, grid[-1]
+    T = np.float32(2.0 ** -3)
+    amax_block = 0
+    s_codes = rng.integers(0x18, 0x60, nb).astype(np.uint8)
+    s_codes[0] = 0x7E                                          # 448: the tensor max
+    c = rng.integers(0, len(grid), (nb, 16))
+    c[:, 0] = len(grid) - 1                                    # emax in every block
+    sign = rng.integers(0, 2, (nb, 16))
+    vals = np.where(sign == 1, -grid[c], grid[c]) * O.E4M3_GRID[s_codes][:, None] * np.float64(T)
+    x = vals.astype(np.float32)                                # one block per row
+    if axis == 0:
+        x = x.T.copy()                                         # one block per column
+    q = O.quantize_1d(x, fmt, rounding, seed=9, axis=axis)
+    assert q.T == T
+    want_codes = c | (sign << (O.element_bits(fmt) - 1))
+    got_codes = q.codes if axis == 1 else q.codes.T
+    got_scales = q.scales.reshape(-1)
+    assert np.array_equal(got_scales, s_codes)
+    assert np.array_equal(got_codes, want_codes)
+
+
+@pytest.mark.parametrize("fmt", [O.FP4, O.FP6])
+def test_1d_transposed_view_and_global_max(fmt):
+    """Blocks down the columns of X are blocks along the rows of X^T (round
+    to nearest: same codes and scales, transposed), and the element of
+    largest magnitude gets scale 448 and the top code."""
+    rng = np.random.default_rng(23)
+    x = (rng.standard_normal((32, 48)) * np.exp(rng.standard_normal((32, 48)))).astype(np.float32)
+    a = O.quantize_1d(x, fmt, O.RNE, axis=0)
+    b = O.quantize_1d(np.ascontiguousarray(x.T), fmt, O.RNE, axis=1)
+    assert a.T == b.T
+    assert np.array_equal(a.codes, b.codes.T) and np.array_equal(a.scales, b.scales.T)
+    r, cidx = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    top = len(O.element_grid(fmt)) - 1
+    assert a.scales[r // 16, cidx] == O.cast_e4m3(np.array([448.0], np.float32))[0]
+    assert a.codes[r, cidx] & top == top
+
+
+def test_1d_stochastic_rounding_brackets_and_keeps_grid_values():
+    """SR codes are always one of the two grid neighbours of x/(B·T), and
+    values already on the grid never move (any seed)."""
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((16, 64)).astype(np.float32)
+    rn = O.quantize_1d(x, O.FP4, O.RNE, axis=1)
+    grid = O.element_grid(O.FP4)
+    d = np.repeat(O.E4M3_GRID[rn.scales], 16, axis=1) * np.float64(rn.T)
+    v = np.abs(x) / d
+    for seed in (1, 2, 3):
+        q = O.quantize_1d(x, O.FP4, O.SR, seed, axis=1)
+        assert np.array_equal(q.scales, rn.scales)
+        mag = grid[q.codes & 7]
+        lo = grid[np.clip(np.searchsorted(grid, v, side="right") - 1, 0, 7)]
+        hi = grid[np.clip(np.searchsorted(grid, v, side="left"), 0, 7)]
+        assert np.all((mag == lo) | (mag == hi))
+        on_grid = np.isin(v, grid)
+        assert np.array_equal(mag[on_grid], v[on_grid])
+
+
+def test_expanded_view_by_brute_force():
+    """The naive scheme's expanded X' in the channel-batch-first layout of a
+    1 x 1 convolution: row (ho, wo, kh, kw, ci), column n, value
+    X[ho·s + kh - p][wo·s + kw - p][ci][n] or 0 outside (stride 2, pad 1)."""
+    s = O.ConvShape(4, 3, 2, 5, 6, 3, 2, 2, 1)
+    X = np.random.default_rng(25).standard_normal((s.H, s.W, s.Cin, s.N)).astype(np.float32)
+    v = O.expanded_view(X, s).reshape(s.Ho, s.Wo, s.Kh, s.Kw, s.Cin, s.N)
+    for ho in range(s.Ho):
+        for wo in range(s.Wo):
+            for kh in range(s.Kh):
+                for kw in range(s.Kw):
+                    hi, wi = ho * s.stride + kh - s.pad, wo * s.stride + kw - s.pad
+                    want = X[hi, wi] if 0 <= hi < s.H and 0 <= wi < s.W else 0 * X[0, 0]
+                    assert np.array_equal(v[ho, wo, kh, kw], want)
+
+
+def test_naive_layer_gemms_against_torch():
+    """The naive step's three GEMMs on its own quantized copies equal torch's
+    fp64 contractions of the dequantized copies (einsum for Y and G_W, and
+    conv2d_input for G_X = col2im(W^T·G_Y)), and each copy is the 1-D block
+    quantization of its operand along the stated direction."""
+    s = O.ConvShape(16, 16, 16, 5, 5, 3, 3, 1, 1)
+    rng = np.random.default_rng(26)
+    X = np.maximum(rng.standard_normal((s.H, s.W, s.Cin, s.N)), 0).astype(np.float32)
+    Wt = (rng.standard_normal((s.Cout, s.Kh, s.Kw, s.Cin)) * 0.1).astype(np.float32)
+    G = (rng.standard_normal((s.Ho, s.Wo, s.Cout, s.N)) * 1e-3).astype(np.float32)
+    q, out = O.naive_layer(X, Wt, G, s, O.FP4, seed=3)
+    K = s.Kh * s.Kw * s.Cin
+    assert q["x_fwd"].axis == 0 and q["x_wgrad"].axis == 1 and q["w_fwd"].axis == 1
+    assert q["w_dgrad"].axis == 0 and q["g_wgrad"].axis == 1 and q["g_dgrad"].axis == 0
+    deq = {k: torch.from_numpy(O.code_values_1d(v) * np.float64(v.T)) for k, v in q.items()}
+    xf = deq["x_fwd"].reshape(s.Ho * s.Wo, K, s.N)
+    xw = deq["x_wgrad"].reshape(s.Ho * s.Wo, K, s.N)
+    y = torch.einsum("ck,pkn->pcn", deq["w_fwd"], xf)
+    gw = torch.einsum("pcn,pkn->ck", deq["g_wgrad"].reshape(s.Ho * s.Wo, s.Cout, s.N), xw)
+    wd = deq["w_dgrad"].reshape(s.Cout, s.Kh, s.Kw, s.Cin).permute(0, 3, 1, 2)
+    gd = deq["g_dgrad"].reshape(s.Ho, s.Wo, s.Cout, s.N).permute(3, 2, 0, 1)
+    gx = torch.nn.grad.conv2d_input((s.N, s.Cin, s.H, s.W), wd, gd, stride=s.stride, padding=s.pad)
+    np.testing.assert_allclose(out["y"][0].reshape(-1), y.numpy().reshape(-1), rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(out["gw"][0].reshape(-1), gw.numpy().reshape(-1), rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(out["gx"][0], gx.permute(2, 3, 1, 0).numpy(), rtol=1e-12, atol=1e-18)
+    # the two directions give different copies of the same operand
+    for a, b in (("x_fwd", "x_wgrad"), ("w_fwd", "w_dgrad"), ("g_wgrad", "g_dgrad")):
+        assert not np.array_equal(O.code_values_1d(q[a]), O.code_values_1d(q[b]))
+
+
 def test_naive_needs_two_copies():
     """The two GEMM directions quantize the same X' differently."""
     s = O.ConvShape(4, 16, 16, 6, 6, 3, 3, 1, 0)
