@@ -445,9 +445,8 @@ def run_gpu(args):
 
     # The baseline the method removes (expand with im2col first, quantize each
     # operand once per GEMM direction), timed the same way on one GPU.
-    naive_res = None
-    if world == 1 and args.naive_steps > 0:
-        nb = naive.plan(d, dev)
+    def run_naive(blocks):
+        nb = naive.plan(d, dev, blocks)
         nout = {"y": torch.empty_like(sets[0]["y"]), "gw": torch.empty_like(sets[0]["gw"]),
                 "gx": torch.empty_like(sets[0]["gx"])}
 
@@ -498,9 +497,18 @@ def run_gpu(args):
                      "algorithmic_bytes_ratio": round(sum(nbytes.values()) / once_bytes, 3),
                      "quantized_elements_ratio": round((2 * ex + 2 * nw + 2 * ng) / (nx + nw + ng), 3),
                      "expanded_x_ratio": round(ex / nx, 3),
-                     "flow": "im2col, every operand quantized once per GEMM direction, 1x1 GEMMs, col2im"}
-        del ngraphs
+                     "flow": "im2col, every operand quantized once per GEMM direction, 1x1 GEMMs, col2im",
+                     "blocks": ("16-element lines along each GEMM's contraction (x' 16x1 and 1x16, w 1x16 "
+                                "and 16x1, g_y 1x16 and 16x1)" if blocks == "line" else
+                                "4x4 squares over (kh*kw*ci, n) of the expanded tensor")}
+        del ngraphs, nb
         torch.cuda.synchronize()
+        return naive_res
+
+    naive_res = naive_sq = None
+    if world == 1 and args.naive_steps > 0:
+        naive_res = run_naive("line")
+        naive_sq = run_naive("square")
 
     # End to end through the public API with pinned host buffers, pipelined
     # as a training loop would be: step i copies its inputs in on one stream,
@@ -677,11 +685,12 @@ def run_gpu(args):
                                        "waits between them; the concurrent phase durations come from this loop"}
     if e2e:
         out["e2e"] = e2e
-    if naive_res:
-        # against the quantize-once step on one stream, as the baseline runs
-        naive_res["step_time_ratio"] = round(naive_res["ms_per_step"] / (serial_ms / args.steps), 3)
-        naive_res["quantize_time_ratio"] = round(naive_res["phase_ms"]["quant"] / mean["quantize"], 3)
-        out["naive_baseline"] = naive_res
+    # against the quantize-once step on one stream, as the baseline runs
+    for key, nr in (("naive_baseline", naive_res), ("naive_square_blocks", naive_sq)):
+        if nr:
+            nr["step_time_ratio"] = round(nr["ms_per_step"] / (serial_ms / args.steps), 3)
+            nr["quantize_time_ratio"] = round(nr["phase_ms"]["quant"] / mean["quantize"], 3)
+            out[key] = nr
     if world == 1:
         out["mma_form"] = run_mma_form(dev, layer, peaks)
     if world == 1 and not args.no_sweeps:

@@ -74,6 +74,22 @@ typedef struct {
   int32_t reserved; /* must be 0 */
 } mqv_conv_desc;
 
+/* Block shape of a quantized view's scale plane.  MicroQonv's own blocks are
+ * the 4 x 4 squares.  The two 16-element line shapes are the plain blocks of
+ * the scheme the MicroQonv summary (section "무엇인가") sets it against:
+ * after im2col, each GEMM operand is quantized in 16 consecutive elements
+ * along that GEMM's contraction, once per direction.
+ *   MQV_BLOCKS_4X4   scales [rows/4][cols/4]
+ *   MQV_BLOCKS_1X16  16 consecutive columns of one row: scales [rows][cols/16]
+ *                    (cols a multiple of 16)
+ *   MQV_BLOCKS_16X1  16 consecutive rows of one column: scales [rows/16][cols]
+ *                    (rows a multiple of 16)
+ * The code plane is the same for all three.  Every entry point takes the
+ * square blocks.  mqv_quantize_many and mqv_dequantize take all three.  The
+ * conv passes take the line shapes only on the kernels the naive scheme
+ * runs on: a stride-1 1 x 1 layer, with the shapes listed at each pass. */
+typedef enum { MQV_BLOCKS_4X4 = 0, MQV_BLOCKS_1X16 = 1, MQV_BLOCKS_16X1 = 2 } mqv_blocks;
+
 /* A quantized rows x cols view (see the layout notes above).  codes and
  * scales must be 16-byte aligned device pointers. */
 typedef struct {
@@ -82,7 +98,7 @@ typedef struct {
   float* tscale;
   int64_t rows, cols;
   int32_t fmt;
-  int32_t reserved; /* must be 0 */
+  int32_t blocks;   /* mqv_blocks; 0 (the 4 x 4 squares) unless stated */
 } mqv_qtensor;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -199,7 +215,10 @@ mqv_status mqv_conv_workspace_size(const mqv_conv_desc* d, int32_t op, size_t* b
  * X' are gathered from the quantized X on chip, never stored.
  * y[ho][wo][co][n] = T_w·T_x·sum_{kh,kw,ci} Wq[co][kh][kw][ci]·Xq[hi][wi][ci][n]
  * with hi = ho·stride + kh - pad, wi = wo·stride + kw - pad, zero outside.
- * w: view Cout x Kh·Kw·Cin; x: view H·W·Cin x N; y fp32 [Ho][Wo][Cout][N]. */
+ * w: view Cout x Kh·Kw·Cin; x: view H·W·Cin x N; y fp32 [Ho][Wo][Cout][N].
+ * Block shapes: both operands 4 x 4, or, on a stride-1 1 x 1 layer with
+ * N a multiple of 16, w in MQV_BLOCKS_1X16 and x in MQV_BLOCKS_16X1 (the
+ * naive scheme's blocks along the contraction K). */
 mqv_status mqv_conv_fwd(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* x,
                         float* y, void* ws, size_t ws_bytes, void* stream);
 
@@ -223,7 +242,9 @@ mqv_status mqv_conv_fwd_blockscaled(const mqv_conv_desc* d, const mqv_qtensor* w
 
 /* Weight-gradient GEMM G_W = G_Y·X'^T: contraction over (ho, wo, n), split
  * across CTAs and summed in a fixed order (deterministic) through `ws`.
- * gy: view Ho·Wo·Cout x N; x: view H·W·Cin x N; gw fp32 [Cout][Kh][Kw][Cin]. */
+ * gy: view Ho·Wo·Cout x N; x: view H·W·Cin x N; gw fp32 [Cout][Kh][Kw][Cin].
+ * Block shapes: both 4 x 4, or, on a stride-1 1 x 1 layer, both
+ * MQV_BLOCKS_1X16 (blocks along the contraction over (ho, wo, n)). */
 mqv_status mqv_conv_wgrad(const mqv_conv_desc* d, const mqv_qtensor* gy, const mqv_qtensor* x,
                           float* gw, void* ws, size_t ws_bytes, void* stream);
 
@@ -253,7 +274,10 @@ mqv_status mqv_conv_wgrad_noalloc(const mqv_conv_desc* d, const mqv_qtensor* gy,
 /* Input-gradient G_X = col2im(W^T·G_Y), computed directly as an implicit
  * transposed convolution: gx[hi][wi][ci][n] = T_w·T_g·sum over (kh, kw, co)
  * and every (ho, wo) with ho·stride + kh - pad = hi, wo·stride + kw - pad = wi.
- * w: view Cout x Kh·Kw·Cin; gy: view Ho·Wo·Cout x N; gx fp32 [H][W][Cin][N]. */
+ * w: view Cout x Kh·Kw·Cin; gy: view Ho·Wo·Cout x N; gx fp32 [H][W][Cin][N].
+ * Block shapes: both 4 x 4, or, on a stride-1 1 x 1 layer with N a
+ * multiple of 16, both MQV_BLOCKS_16X1 (blocks along the contraction over
+ * Cout). */
 mqv_status mqv_conv_dgrad(const mqv_conv_desc* d, const mqv_qtensor* w, const mqv_qtensor* gy,
                           float* gx, void* ws, size_t ws_bytes, void* stream);
 

@@ -46,7 +46,7 @@ class ConvDesc(ctypes.Structure):
 class QTensorC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("tscale", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("fmt", ctypes.c_int32), ("blocks", ctypes.c_int32)]
 
 
 class QuantJobC(ctypes.Structure):
@@ -182,27 +182,33 @@ def qtensor_bytes(rows: int, cols: int, fmt) -> tuple[int, int]:
     return cb.value, sb.value
 
 
+BLOCKS_4X4, BLOCKS_1X16, BLOCKS_16X1 = 0, 1, 2
+
+
 @dataclass
 class QTensor:
-    """A quantized rows x cols view: packed codes, E4M3 scale plane, fp32 T."""
+    """A quantized rows x cols view: packed codes, E4M3 scale plane, fp32 T.
+    blocks: the scale blocks (mqv_blocks): 4 x 4 squares, or the 16-element
+    lines of 1 x 16 along a row / 16 x 1 down a column."""
     codes: torch.Tensor
     scales: torch.Tensor
     tscale: torch.Tensor
     rows: int
     cols: int
     fmt: int
+    blocks: int = BLOCKS_4X4
 
     @classmethod
-    def empty(cls, rows: int, cols: int, fmt, device="cuda") -> "QTensor":
+    def empty(cls, rows: int, cols: int, fmt, device="cuda", blocks: int = BLOCKS_4X4) -> "QTensor":
         fmt = _fmt(fmt)
         cb, sb = qtensor_bytes(rows, cols, fmt)
         return cls(torch.empty(cb, dtype=torch.uint8, device=device),
                    torch.empty(sb, dtype=torch.uint8, device=device),
-                   torch.empty(1, dtype=torch.float32, device=device), rows, cols, fmt)
+                   torch.empty(1, dtype=torch.float32, device=device), rows, cols, fmt, blocks)
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(), self.tscale.data_ptr(),
-                        self.rows, self.cols, self.fmt, 0)
+                        self.rows, self.cols, self.fmt, self.blocks)
 
 
 def quantize_workspace_bytes(rows: int, cols: int) -> int:
@@ -228,7 +234,8 @@ def quantize(src: torch.Tensor, rows: int, cols: int, fmt, rounding: int = RNE, 
 
 def quantize_many(jobs, ws: torch.Tensor | None = None, stream=None) -> list[QTensor]:
     """Quantize several tensors in two launches (see mqv_quantize_many).
-    jobs: (src, rows, cols, fmt, rounding, seed[, out QTensor]) tuples."""
+    jobs: (src, rows, cols, fmt, rounding, seed[, out QTensor]) tuples; the
+    block shape is the out QTensor's (4 x 4 when no out is given)."""
     outs, cjobs = [], []
     for j in jobs:
         src, rows, cols, fmt, rnd, seed = j[:6]

@@ -88,8 +88,9 @@ int64_t amax_ctas(int64_t rows, int64_t cols) {
   return (nchunks + passes - 1) / passes;
 }
 
-int64_t quant_ctas(int64_t rows, int64_t cols) {
-  const int64_t nb = rows * cols / 16;
+int64_t quant_ctas(int64_t rows, int64_t cols, int32_t blocks = MQV_BLOCKS_4X4) {
+  // one thread per 16 elements; 16 x 1 line blocks take four blocks a thread
+  const int64_t nb = rows * cols / (blocks == MQV_BLOCKS_16X1 ? 64 : 16);
   const int64_t per_cta = static_cast<int64_t>(kQuantThreads) * kQuantUnits;
   int64_t g = (nb + per_cta - 1) / per_cta;
   if (g < 1) g = 1;
@@ -125,7 +126,12 @@ mqv_status check_qtensor(const mqv_qtensor* q, const char* name) {
   mqv_status st = check_view(q->rows, q->cols);
   if (st) return st;
   if ((st = check_fmt(q->fmt))) return st;
-  if (q->reserved) return fail(MQV_ERR_INVALID_ARG, "%s: reserved field must be 0", name);
+  if (q->blocks != MQV_BLOCKS_4X4 && q->blocks != MQV_BLOCKS_1X16 && q->blocks != MQV_BLOCKS_16X1)
+    return fail(MQV_ERR_INVALID_ARG, "%s: unknown block shape %d", name, q->blocks);
+  if (q->blocks == MQV_BLOCKS_1X16 && q->cols % 16)
+    return fail(MQV_ERR_INVALID_ARG, "%s: 1 x 16 blocks need cols a multiple of 16", name);
+  if (q->blocks == MQV_BLOCKS_16X1 && q->rows % 16)
+    return fail(MQV_ERR_INVALID_ARG, "%s: 16 x 1 blocks need rows a multiple of 16", name);
   if (!q->codes || !q->scales || !q->tscale) return fail(MQV_ERR_INVALID_ARG, "%s: null pointer", name);
   if (!aligned16(q->codes) || !aligned16(q->scales))
     return fail(MQV_ERR_INVALID_ARG, "%s: codes and scales must be 16-byte aligned", name);
@@ -160,6 +166,7 @@ QuantArgs make_quant_args(const float* src, int64_t rows, int64_t cols, uint64_t
   qa.sr_cols = sr_cols;
   qa.sr_col0 = sr_col0;
   qa.dcb = make_fastdiv(cols / 4);
+  qa.blocks = out->blocks;
   return qa;
 }
 
@@ -186,7 +193,7 @@ mqv_status enqueue_quantize(const float* src, int64_t rows, int64_t cols, int32_
 }
 
 mqv_status check_quantize_args(const float* src, int64_t rows, int64_t cols, int32_t fmt,
-                               int32_t rounding, const mqv_qtensor* out) {
+                               int32_t rounding, const mqv_qtensor* out, bool line_blocks = false) {
   mqv_status st = check_view(rows, cols);
   if (st) return st;
   if ((st = check_fmt(fmt))) return st;
@@ -198,6 +205,8 @@ mqv_status check_quantize_args(const float* src, int64_t rows, int64_t cols, int
     return fail(MQV_ERR_INVALID_ARG, "out describes a %lld x %lld fmt %d view, expected %lld x %lld fmt %d",
                 (long long)out->rows, (long long)out->cols, out->fmt, (long long)rows,
                 (long long)cols, fmt);
+  if (!line_blocks && out->blocks != MQV_BLOCKS_4X4)
+    return fail(MQV_ERR_UNSUPPORTED, "out: this entry point writes 4 x 4 blocks only");
   return MQV_OK;
 }
 
@@ -251,7 +260,8 @@ QView make_view(const mqv_qtensor* q) {
   v.scales = q->scales;
   v.tscale = q->tscale;
   v.row_bytes = q->fmt == MQV_NVFP4 ? q->cols / 2 : q->cols * 3 / 4;
-  v.scale_cols = q->cols / 4;
+  v.blocks = q->blocks;
+  v.scale_cols = q->blocks == MQV_BLOCKS_1X16 ? q->cols / 16 : q->blocks == MQV_BLOCKS_16X1 ? q->cols : q->cols / 4;
   return v;
 }
 
@@ -482,9 +492,9 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
   return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, false>(pl, st) : launch_fd<P, FMT, 128, 4, false>(pl, st);
 }
 
-template <int PASS, int FMT, bool QOUT>
+template <int PASS, int FMT, bool QOUT, bool LINE = false>
 cudaError_t launch_halo_q(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_halo_kernel<PASS, FMT, QOUT>;
+  auto kern = conv_halo_kernel<PASS, FMT, QOUT, LINE>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
   if (e != cudaSuccess) return e;
@@ -494,12 +504,13 @@ cudaError_t launch_halo_q(const ConvPlan& pl, cudaStream_t st) {
 
 template <int PASS, int FMT>
 cudaError_t launch_halo(const ConvPlan& pl, cudaStream_t st) {
+  if (pl.a.b.blocks != MQV_BLOCKS_4X4) return launch_halo_q<PASS, FMT, false, true>(pl, st);
   return pl.a.q_codes ? launch_halo_q<PASS, FMT, true>(pl, st) : launch_halo_q<PASS, FMT, false>(pl, st);
 }
 
-template <int FMT, int KW, bool PAIR>
+template <int FMT, int KW, bool PAIR, bool LINE = false>
 cudaError_t launch_wgk(const ConvPlan& pl, cudaStream_t st) {
-  auto kern = conv_wgk_kernel<FMT, KW, PAIR>;
+  auto kern = conv_wgk_kernel<FMT, KW, PAIR, LINE>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, WgkSmem::kBytes, done);
   if (e != cudaSuccess) return e;
@@ -512,6 +523,7 @@ cudaError_t launch_wgk(const ConvPlan& pl, cudaStream_t st) {
 template <int FMT>
 cudaError_t launch_wgk_kw(const ConvPlan& pl, cudaStream_t st) {
   const bool pair = pl.a.N == 64;
+  if (pl.a.b.blocks != MQV_BLOCKS_4X4) return launch_wgk<FMT, 1, false, true>(pl, st);   // 1 x 1 layers only
   switch (pl.a.Kw) {
     case 1: return launch_wgk<FMT, 1, false>(pl, st);
     case 2: return pair ? launch_wgk<FMT, 2, true>(pl, st) : launch_wgk<FMT, 2, false>(pl, st);
@@ -615,6 +627,19 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
     return fail(MQV_ERR_INVALID_ARG, "amax must be a 4-byte aligned pointer");
   ConvPlan pl;
   plan_conv(d, op, &pl);
+  if (qa->blocks != MQV_BLOCKS_4X4 || qb->blocks != MQV_BLOCKS_4X4) {
+    // the naive scheme's line blocks, on the kernels that run its 1 x 1 GEMMs
+    const bool one = d->Kh == 1 && d->Kw == 1 && d->stride == 1 && d->pad == 0;
+    const int want_a = op == MQV_OP_DGRAD ? MQV_BLOCKS_16X1 : MQV_BLOCKS_1X16;
+    const int want_b = op == MQV_OP_WGRAD ? MQV_BLOCKS_1X16 : MQV_BLOCKS_16X1;
+    const bool kern = op == MQV_OP_WGRAD ? pl.wgk : pl.halo;
+    if (!one || qa->blocks != want_a || qb->blocks != want_b || !kern || qo)
+      return fail(MQV_ERR_UNSUPPORTED,
+                  "line blocks: a stride-1 1 x 1 layer of the kernel-row path with %s %s and %s %s, no quantized "
+                  "output (got %d and %d)",
+                  na, want_a == MQV_BLOCKS_1X16 ? "1 x 16" : "16 x 1", nb, want_b == MQV_BLOCKS_1X16 ? "1 x 16" : "16 x 1",
+                  qa->blocks, qb->blocks);
+  }
   if (qo) {
     if (!pl.halo)
       return fail(MQV_ERR_UNSUPPORTED, "quantized output: stride-1 layers of the kernel-row path only "
@@ -687,7 +712,9 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
     const mqv_quantize_job& j = jobs[i];
     mqv_status st = MQV_OK;
     if (check_pointers) {
-      st = check_quantize_args(j.src, j.rows, j.cols, j.fmt, j.rounding, &j.out);
+      st = check_quantize_args(j.src, j.rows, j.cols, j.fmt, j.rounding, &j.out, true);
+      if (!st && (j.out.blocks == MQV_BLOCKS_4X4) != (jobs[0].out.blocks == MQV_BLOCKS_4X4))
+        st = fail(MQV_ERR_UNSUPPORTED, "4 x 4 and line blocks mixed in one call");
     } else if (!(st = check_view(j.rows, j.cols)) && !(st = check_fmt(j.fmt)) &&
                j.rounding != MQV_RNE && j.rounding != MQV_SR) {
       st = fail(MQV_ERR_INVALID_ARG, "unknown rounding %d", j.rounding);
@@ -699,7 +726,7 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
     qj.rounding = j.rounding;
     qj.amax_cta0 = a;
     qj.amax_ctas = (int)amax_ctas(j.rows, j.cols);
-    qj.quant_ctas = (int)quant_ctas(j.rows, j.cols);
+    qj.quant_ctas = (int)quant_ctas(j.rows, j.cols, j.out.blocks);
     a += qj.amax_ctas;
   }
   // quantize CTA ranges: stochastic-rounding jobs first (see quantize_many_kernel)
@@ -812,7 +839,8 @@ mqv_status mqv_quantize_many(const mqv_quantize_job* jobs, int32_t count, void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(ws);
   amax_many_kernel<<<a, kAmaxThreads, 0, s>>>(plan, part);
-  quantize_many_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
+  if (plan.job[0].qa.blocks == MQV_BLOCKS_4X4) quantize_many_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
+  else quantize_many_line_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize_many launch");
   return ok();
@@ -826,9 +854,9 @@ mqv_status mqv_dequantize(const mqv_qtensor* q, float* dst, void* stream) {
   const unsigned g = (unsigned)quant_ctas(q->rows, q->cols);
   const uint8_t* c = static_cast<const uint8_t*>(q->codes);
   if (q->fmt == MQV_NVFP4)
-    dequantize_kernel<0><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, dst);
+    dequantize_kernel<0><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, q->blocks, dst);
   else
-    dequantize_kernel<1><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, dst);
+    dequantize_kernel<1><<<g, kQuantThreads, 0, s>>>(c, q->scales, q->tscale, q->rows, q->cols, q->blocks, dst);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
@@ -943,6 +971,8 @@ mqv_status mqv_conv_fwd_blockscaled(const mqv_conv_desc* d, const mqv_qtensor* w
   if ((st = check_operand(w, "w", d->Cout, d->Kh * d->Kw * d->Cin, d->fmt)) ||
       (st = check_operand(x, "x", d->H * d->W * d->Cin, d->N, d->fmt)))
     return st;
+  if (w->blocks != MQV_BLOCKS_4X4 || x->blocks != MQV_BLOCKS_4X4)
+    return fail(MQV_ERR_UNSUPPORTED, "block-scaled forward pass: 4 x 4 blocks only");
   if (!y || !aligned16(y)) return fail(MQV_ERR_INVALID_ARG, "output must be a 16-byte aligned pointer");
   if (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))
     return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required, got %zu", pl.ws_bytes,

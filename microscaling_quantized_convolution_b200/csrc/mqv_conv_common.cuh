@@ -20,8 +20,16 @@ struct QView {
   const uint8_t* scales;
   const float* tscale;
   int64_t row_bytes;    // bytes per row of packed codes
-  int64_t scale_cols;   // blocks per row of the scale plane (= cols / 4)
+  int64_t scale_cols;   // entries per row of the scale plane (cols / 4, cols / 16 or cols by `blocks`)
+  int32_t blocks;       // scale blocks: 0 4 x 4, 1 1 x 16 along a row, 2 16 x 1 down a column
 };
+
+// Scale-plane index of element (row, col) of a view.
+__device__ __forceinline__ int64_t scale_index(const QView& v, int64_t row, int64_t col) {
+  if (v.blocks == 1) return row * v.scale_cols + (col >> 4);
+  if (v.blocks == 2) return (row >> 4) * v.scale_cols + col;
+  return (row >> 2) * v.scale_cols + (col >> 2);
+}
 
 // Byte offset of (row, k) inside a K-major, 128-byte-swizzled fp16 tile.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t k) {

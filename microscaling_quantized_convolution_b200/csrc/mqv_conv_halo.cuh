@@ -77,7 +77,8 @@ struct HaloGeom {
 struct HaloUnit {
   uint32_t w[8];      // codes of channel c0 + j for the 8 batch items (NVFP6: bytes 0-3)
   uint32_t wh[8];     // NVFP6: bytes 4-5 of the 6-byte run
-  uint32_t s[2];      // scales of channel blocks 0/1 (low byte: batch block 0)
+  uint32_t s[2];      // scales of channel blocks 0/1 (low byte: batch block 0);
+                      // 16 x 1 line blocks: byte j of s[0], s[1] = batch item j, 4 + j
   bool ok;
 };
 
@@ -85,9 +86,16 @@ struct HaloUnit {
 // the 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
 // channel words is interleaved nibble-wise first, so one cvt.e2m1x2 per
 // byte yields the (channel 2i, channel 2i+1) pair of one batch item.
-template <int FMT>
+// LINE: the operand has 16 x 1 line blocks down its (pixel, channel) rows, so
+// the unit's 8 channels share one scale per batch item.
+template <int FMT, bool LINE>
 __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile, uint32_t row0, uint32_t kg) {
   uint32_t out[8][4];
+  uint32_t sl[8];
+  if (LINE) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) sl[r] = scale2((u.s[r >> 2] >> (8 * (r & 3))) & 0xFF);
+  }
   if (u.ok && FMT == 1) {
     // NVFP6: batch item r of channel c is bits [6r, 6r+6) of the 48-bit run;
     // the two channels of a pair go to the low and high byte of one
@@ -102,7 +110,7 @@ __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile
       for (int r = 0; r < 8; ++r) {
         const uint32_t v = static_cast<uint32_t>((a >> (6 * r)) & 0x3F) |
                            (static_cast<uint32_t>((b >> (6 * r)) & 0x3F) << 8);
-        out[r][i] = hmul2_u32(e2m3x2_to_f16x2(v), sc[i >> 1][r >> 2]);
+        out[r][i] = hmul2_u32(e2m3x2_to_f16x2(v), LINE ? sl[r] : sc[i >> 1][r >> 2]);
       }
     }
   } else if (u.ok) {
@@ -119,8 +127,8 @@ __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const uint32_t s2 = sc[i >> 1][q >> 1];             // batch items 2q, 2q+1: block q/2
-        out[2 * q][i] = hmul2_u32(he[q], s2);
-        out[2 * q + 1][i] = hmul2_u32(ho[q], s2);
+        out[2 * q][i] = hmul2_u32(he[q], LINE ? sl[2 * q] : s2);
+        out[2 * q + 1][i] = hmul2_u32(ho[q], LINE ? sl[2 * q + 1] : s2);
       }
     }
   } else {
@@ -135,7 +143,7 @@ __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile
 // Producer thread t owns unit t of every stage: K chunk kg = t % 8 (8
 // channels), rows 8(t/8)..8(t/8)+7 of the halo.  Lanes of an 8-lane phase
 // differ in kg, so their 16-byte stores hit 8 different swizzled chunks.
-template <int PASS, int FMT>
+template <int PASS, int FMT, bool LINE = false>
 struct HaloCursor {
   int sc, n0;         // halo pixel column in the source, first batch item
   bool cok;           // unit inside the halo and its column inside the source
@@ -171,6 +179,13 @@ struct HaloCursor {
         u.w[j] = static_cast<uint32_t>(__ldg(q)) | (static_cast<uint32_t>(__ldg(q + 1)) << 16);
         u.wh[j] = __ldg(q + 2);
       }
+    }
+    if (LINE) {
+      // rows row0 .. row0 + 7 lie in one 16-row block (row0 % 8 == 0)
+      const uint2 sv = __ldg(reinterpret_cast<const uint2*>(p.b.scales + (row0 >> 4) * p.b.scale_cols + n0));
+      u.s[0] = sv.x;
+      u.s[1] = sv.y;
+      return;
     }
     const uint8_t* sp = p.b.scales + (row0 >> 2) * p.b.scale_cols + (n0 >> 2);
     u.s[0] = __ldg(reinterpret_cast<const unsigned short*>(sp));
@@ -282,8 +297,9 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
 }
 
 // QOUT: the quantized-output epilogue (V2Args::q_codes), a separate
-// instance so that the plain passes keep their code and registers.
-template <int PASS, int FMT, bool QOUT>
+// instance so that the plain passes keep their code and registers.  LINE:
+// the B operand has 16 x 1 line blocks (see halo_store_unit).
+template <int PASS, int FMT, bool QOUT, bool LINE = false>
 __global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
   using L = HaloSmem;
@@ -420,7 +436,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
                           static_cast<int>(gridDim.x);
     const int total = ntile_cta * stages_per_tile;
     const int spatial = g.out_h * g.tpr;
-    HaloCursor<PASS, FMT> cursor;
+    HaloCursor<PASS, FMT, LINE> cursor;
     HaloUnit ring[kHaloLookahead];
     int ltile = blockIdx.x, lkh = 0, lc = 0;
     if (total > 0) cursor.begin_tile(p, g, ltile % spatial, t);
@@ -445,7 +461,7 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         const int sb = kit % kHaloBStages;
         mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
         if (t < g.rows)
-          halo_store_unit<FMT>(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
+          halo_store_unit<FMT, LINE>(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
                           static_cast<uint32_t>(t & 7));
         producer_warp_arrive(&bars->bfull[sb]);
         if (kit + kHaloLookahead < total) load_next(ring[r]);

@@ -258,7 +258,7 @@ prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int
   }
   uint32_t h[4] = {0u, 0u, 0u, 0u};
   if (m < M) {
-    if (!TRANS && k0 + 8 <= Kdim && (FMT == 0 ? (w.row_bytes & 3) == 0 : (w.row_bytes & 1) == 0)) {
+    if (!TRANS && w.blocks == 0 && k0 + 8 <= Kdim && (FMT == 0 ? (w.row_bytes & 3) == 0 : (w.row_bytes & 1) == 0)) {
       // eight consecutive codes of one weight row: one word (FP4) or three
       // half-words (FP6) and the two block scales
       uint32_t hi = 0;
@@ -279,16 +279,19 @@ prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int
           row = co;
           col = tap * Cin + m;
         }
-        const uint32_t s = __ldg(w.scales + (row >> 2) * w.scale_cols + (col >> 2));
         uint32_t c0, c1;
         const uint8_t* p = w.codes + static_cast<int64_t>(row) * w.row_bytes;
         const int row2 = TRANS ? row + 1 : row;       // second element: next co (dgrad)
         const int col2 = TRANS ? col : col + 1;
+        // the pair's two scales (4 x 4 blocks: one block holds both, as
+        // row (dgrad) or col (forward) is even)
+        const uint32_t s0 = __ldg(w.scales + scale_index(w, row, col));
+        const uint32_t s = s0 | ((w.blocks ? __ldg(w.scales + scale_index(w, row2, col2)) : s0) << 8);
         const uint8_t* p2 = w.codes + static_cast<int64_t>(row2) * w.row_bytes;
         if (FMT == 0) {
           c0 = (__ldg(p + (col >> 1)) >> ((col & 1) * 4)) & 0xF;
           c1 = (__ldg(p2 + (col2 >> 1)) >> ((col2 & 1) * 4)) & 0xF;
-          h[e >> 1] = hmul2_u32(e2m1x2_to_f16x2(c0 | (c1 << 4)), scale2(s));
+          h[e >> 1] = hmul2_u32(e2m1x2_to_f16x2(c0 | (c1 << 4)), e4m3x2_to_f16x2(s));
         } else {
           auto code6 = [](const uint8_t* base, int c) -> uint32_t {
             const uint8_t* q = base + (c >> 2) * 3;
@@ -298,7 +301,7 @@ prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int
           };
           c0 = code6(p, col);
           c1 = code6(p2, col2);
-          h[e >> 1] = hmul2_u32(e2m3x2_to_f16x2(c0 | (c1 << 8)), scale2(s));
+          h[e >> 1] = hmul2_u32(e2m3x2_to_f16x2(c0 | (c1 << 8)), e4m3x2_to_f16x2(s));
         }
       }
     }

@@ -130,7 +130,9 @@ struct WgkCursor {
 
 // X producer: one unit (4 channels x 8 consecutive (pixel, n) elements) per
 // thread per stage; 256 units fill a 128-channel x 64-element chunk.
-template <int FMT>
+// LINE: both operands carry 1 x 16 line blocks along their batch columns, so
+// every row of a unit or piece has one scale for its 8 or 16 elements.
+template <int FMT, bool LINE>
 __device__ __forceinline__ void wgk_x_load(const V2Args& p, const WgkTile& w, const WgkCursor& c, int tid,
                                            UnitRaw<FMT, 8>& r) {
   const int hi = c.ho + w.kh - p.pad;
@@ -141,20 +143,35 @@ __device__ __forceinline__ void wgk_x_load(const V2Args& p, const WgkTile& w, co
   const int ci = w.ct * 128 + 4 * rq;
   const int wi = pix - p.pad;
   const bool ok = ci < p.Cin && hi >= 0 && hi < p.H && wi >= 0 && wi < p.W;
-  load_unit<FMT, 8>(p.b, (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci, n, ok, r);
+  const int64_t row = (static_cast<int64_t>(hi) * p.W + wi) * p.Cin + ci;
+  if (!LINE) {
+    load_unit<FMT, 8>(p.b, row, n, ok, r);
+    return;
+  }
+  r.ok = ok;
+  if (!ok) return;
+  r.ss = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    r.lo[j] = load_codes<FMT, 8>(p.b, row + j, n, r.hi[j]);
+    r.ss |= static_cast<uint32_t>(__ldg(p.b.scales + (row + j) * p.b.scale_cols + (n >> 4))) << (8 * j);
+  }
 }
 
 // Dequantize the unit into X slot `slot` and, when `mirror` is nonzero, into
 // that second slot as well.
-template <int FMT>
+template <int FMT, bool LINE>
 __device__ __forceinline__ void wgk_x_store(const UnitRaw<FMT, 8>& un, uint32_t slot, uint32_t mirror, int tid) {
   const uint32_t row0 = static_cast<uint32_t>(4 * (tid >> 3)), kl = static_cast<uint32_t>(8 * (tid & 7));
-  const uint32_t s2lo = un.ok ? scale2(un.ss & 0xFF) : 0u;
-  const uint32_t s2hi = un.ok ? scale2(un.ss >> 8) : 0u;
+  const uint32_t s2lo = un.ok && !LINE ? scale2(un.ss & 0xFF) : 0u;
+  const uint32_t s2hi = un.ok && !LINE ? scale2(un.ss >> 8) : 0u;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t h[4] = {0u, 0u, 0u, 0u};
-    if (un.ok) dequant_run<FMT, 8>(un.lo[j], un.hi[j], s2lo, s2hi, h);
+    if (un.ok) {
+      const uint32_t sj = LINE ? scale2((un.ss >> (8 * j)) & 0xFF) : 0u;
+      dequant_run<FMT, 8>(un.lo[j], un.hi[j], LINE ? sj : s2lo, LINE ? sj : s2hi, h);
+    }
     const uint32_t off = sw128_offset(row0 + j, kl);
     st_shared_v4(slot + off, h[0], h[1], h[2], h[3]);
     if (mirror) st_shared_v4(mirror + off, h[0], h[1], h[2], h[3]);
@@ -170,7 +187,7 @@ struct WgkGRaw {
   uint32_t ok;          // bit per piece
 };
 
-template <int FMT>
+template <int FMT, bool LINE>
 __device__ __forceinline__ void wgk_g_load(const V2Args& p, const WgkTile& w, const WgkCursor& c, int row, int half,
                                            WgkGRaw& r) {
   const int co = w.mt * 128 + row;
@@ -194,7 +211,8 @@ __device__ __forceinline__ void wgk_g_load(const V2Args& p, const WgkTile& w, co
         r.c[pc][1] = __ldg(q + 1);
         r.c[pc][2] = __ldg(q + 2);
       }
-      r.s[pc] = __ldg(reinterpret_cast<const uint32_t*>(p.a.scales + (vrow >> 2) * p.a.scale_cols + (n >> 2)));
+      if (LINE) r.s[pc] = static_cast<uint32_t>(__ldg(p.a.scales + vrow * p.a.scale_cols + (n >> 4))) * 0x01010101u;
+      else r.s[pc] = __ldg(reinterpret_cast<const uint32_t*>(p.a.scales + (vrow >> 2) * p.a.scale_cols + (n >> 2)));
     }
   }
 }
@@ -278,7 +296,7 @@ __device__ __forceinline__ void wgk_epilogue(const V2Args& e, const WgkTile& w, 
   }
 }
 
-template <int FMT, int KW, bool PAIR>
+template <int FMT, int KW, bool PAIR, bool LINE = false>
 __global__ void __launch_bounds__(kWgkThreads, 1)
 conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   using L = WgkSmem;
@@ -321,7 +339,7 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
 #pragma unroll
     for (int r = 0; r < kWgkLookahead; ++r)
       if (ld.valid) {
-        wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
+        wgk_x_load<FMT, LINE>(p, w, ld, tid, ring[r]);
         ld.advance(g, g.sx);
       }
     int n = 0;
@@ -332,10 +350,10 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
         const int s = n % kWgkXSlots;
         if (n >= kWgkXSlots) wait_done(n - kWgkXSlots + g.sx);
         const uint32_t mirror = (PAIR && s < kWgkXMirrors) ? sbase + (kWgkXSlots + s) * L::kXSlot : 0u;
-        wgk_x_store<FMT>(ring[r], sbase + s * L::kXSlot, mirror, tid);
+        wgk_x_store<FMT, LINE>(ring[r], sbase + s * L::kXSlot, mirror, tid);
         producer_warp_arrive(&bars->full[s]);
         if (ld.valid) {
-          wgk_x_load<FMT>(p, w, ld, tid, ring[r]);
+          wgk_x_load<FMT, LINE>(p, w, ld, tid, ring[r]);
           ld.advance(g, g.sx);
         }
         cur.advance(g, g.sx);
@@ -357,7 +375,7 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
 #pragma unroll
     for (int r = 0; r < kWgkLookahead; ++r)
       if (ld.valid) {
-        wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
+        wgk_g_load<FMT, LINE>(p, w, ld, row, half, ring[r]);
         ld.advance(g, 0);
       }
     int n = 0, a = 0;
@@ -381,7 +399,7 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full[n % kWgkXSlots]);
         if (ld.valid) {
-          wgk_g_load<FMT>(p, w, ld, row, half, ring[r]);
+          wgk_g_load<FMT, LINE>(p, w, ld, row, half, ring[r]);
           ld.advance(g, 0);
         }
         cur.advance(g, g.sx);

@@ -253,6 +253,7 @@ struct QuantArgs {
   PhiloxKeys keys;
   int64_t sr_cols, sr_col0;
   FastDiv dcb;          // division by the column blocks of a block row (block count < 2^31)
+  int32_t blocks;       // 0: 4 x 4 squares; 1: 1 x 16 along a row; 2: 16 x 1 down a column
 };
 
 // Block scale of a block with max|x| = bmax: the E4M3 code, the divisor
@@ -378,6 +379,141 @@ quantize_kernel(const __grid_constant__ QuantArgs qa, const float* __restrict__ 
   quantize_body<FMT, RND>(qa, amax_src, amax_count, blockIdx.x, gridDim.x);
 }
 
+// ------------------------------------------- 16-element line blocks
+// The plain blocks of the scheme MicroQonv is set against (MicroQonv
+// summary, section "무엇인가"): 16 consecutive elements along one axis of
+// the view.  Every per-element step is the square quantizer's (T, the E4M3
+// block scale, the divisor B·T, the division, both roundings and the
+// element numbering of stochastic rounding); only the grouping differs.
+//   1 x 16: one unit is one block, 16 consecutive columns of a row, scale
+//           plane [rows][cols/16];
+//   16 x 1: one unit is 16 rows x 4 columns, four blocks side by side (so
+//           that each row's 4 codes are one packed store), scale plane
+//           [rows/16][cols].
+
+// Codes of 4 consecutive elements of a row that lie in 4 different blocks
+// (divisors d.x .. d.w): quantize_row4 with a divisor per element.
+template <int FMT, int RND>
+__device__ __forceinline__ uint32_t quantize_row4_cols(float4 x, float4 d, float4 y, uint4 w) {
+  constexpr int kB = FMT == 0 ? 4 : 6;
+  const float xs[4] = {x.x, x.y, x.z, x.w}, ds[4] = {d.x, d.y, d.z, d.w};
+  const float2 nd01 = make_float2(-d.x, -d.y), nd23 = make_float2(-d.z, -d.w);
+  const float2 y01 = make_float2(y.x, y.y), y23 = make_float2(y.z, y.w);
+  float a[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a[j] = fabsf(xs[j]);
+  float2 q01, q23;
+  const float2 v01 = div2_shared_divisor(make_float2(a[0], a[1]), nd01, y01, q01);
+  const float2 v23 = div2_shared_divisor(make_float2(a[2], a[3]), nd23, y23, q23);
+  float v[4] = {v01.x, v01.y, v23.x, v23.y};
+  const float q0[4] = {q01.x, q01.y, q23.x, q23.y};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // the IEEE divide for blocks below the Markstein range, and (stochastic
+    // rounding) for quotients below 1e-30, exactly as the square blocks
+    const bool exact = ds[j] > 0.0f && ds[j] < kMarksteinMinDivisor;
+    const bool tiny = RND == 1 && ds[j] > 0.0f && q0[j] < 1.0e-30f && a[j] != 0.0f;
+    if (exact || tiny) v[j] = __fdiv_rn(a[j], ds[j]);
+    if (ds[j] == 0.0f) v[j] = 0.0f;
+  }
+  if (RND == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = copysignf(v[j], xs[j]);
+    if (FMT == 0) return f32x2_to_e2m1x2(v[0], v[1]) | (f32x2_to_e2m1x2(v[2], v[3]) << 8);
+    const uint32_t b01 = f32x2_to_e2m3x2(v[0], v[1]), b23 = f32x2_to_e2m3x2(v[2], v[3]);
+    return (b01 & 0x3F) | ((b01 >> 2) & 0xFC0) | ((b23 & 0x3F) << 12) | ((b23 & 0x3F00) << 10);
+  }
+  uint32_t m[4];
+  round_sr_mag2<FMT>(make_float2(v[0], v[1]), w.x, w.y, m[0], m[1]);
+  round_sr_mag2<FMT>(make_float2(v[2], v[3]), w.z, w.w, m[2], m[3]);
+  uint32_t out = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) out |= (m[j] | ((__float_as_uint(xs[j]) >> 31) << (kB - 1))) << (j * kB);
+  return out;
+}
+
+__device__ __forceinline__ uint4 philox_at(const QuantArgs& qa, uint64_t g) {
+  return philox4x32_10(make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u), qa.keys);
+}
+
+template <int FMT, int RND>
+__device__ __forceinline__ void quantize_unit_1x16(const QuantArgs& qa, const TensorScale<FMT>& ts, int64_t r,
+                                                   int64_t c16, int64_t row_bytes) {
+  const float* src = qa.src + r * qa.cols + c16 * 16;
+  float4 x[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x[j] = __ldg(reinterpret_cast<const float4*>(src) + j);
+  const float bmax = fmaxf(fmaxf(absmax4(x[0]), absmax4(x[1])), fmaxf(absmax4(x[2]), absmax4(x[3])));
+  const BlockScale<FMT> bs(bmax, ts);
+  qa.scales[r * (qa.cols >> 4) + c16] = static_cast<uint8_t>(bs.scode);
+  const uint64_t g = static_cast<uint64_t>(r * qa.sr_cols + qa.sr_col0 + c16 * 16) >> 2;
+  uint32_t pk[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    pk[j] = quantize_row4<FMT, RND>(x[j], bs.d, bs.y, bs.exact, RND == 1 ? philox_at(qa, g + j) : make_uint4(0, 0, 0, 0));
+  uint8_t* out = qa.codes + r * row_bytes;
+  if (FMT == 0) {
+    *reinterpret_cast<uint2*>(out + c16 * 8) = make_uint2(pk[0] | (pk[1] << 16), pk[2] | (pk[3] << 16));
+  } else {
+    uint32_t* o = reinterpret_cast<uint32_t*>(out + c16 * 12);
+    o[0] = pk[0] | (pk[1] << 24);
+    o[1] = (pk[1] >> 8) | (pk[2] << 16);
+    o[2] = (pk[2] >> 16) | (pk[3] << 8);
+  }
+}
+
+template <int FMT, int RND>
+__device__ __forceinline__ void quantize_unit_16x1(const QuantArgs& qa, const TensorScale<FMT>& ts, int64_t rb,
+                                                   int64_t cq, int64_t row_bytes) {
+  const float* src = qa.src + rb * 16 * qa.cols + cq * 4;
+  float4 x[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) x[r] = __ldg(reinterpret_cast<const float4*>(src + r * qa.cols));
+  float4 m = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    m.x = fmaxf(m.x, fabsf(x[r].x)); m.y = fmaxf(m.y, fabsf(x[r].y));
+    m.z = fmaxf(m.z, fabsf(x[r].z)); m.w = fmaxf(m.w, fabsf(x[r].w));
+  }
+  const BlockScale<FMT> b0(m.x, ts), b1(m.y, ts), b2(m.z, ts), b3(m.w, ts);
+  *reinterpret_cast<uint32_t*>(qa.scales + rb * qa.cols + cq * 4) =
+      b0.scode | (b1.scode << 8) | (b2.scode << 16) | (b3.scode << 24);
+  const float4 d = make_float4(b0.d, b1.d, b2.d, b3.d), y = make_float4(b0.y, b1.y, b2.y, b3.y);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int64_t row = rb * 16 + r;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (RND == 1) w = philox_at(qa, static_cast<uint64_t>(row * qa.sr_cols + qa.sr_col0 + cq * 4) >> 2);
+    const uint32_t packed = quantize_row4_cols<FMT, RND>(x[r], d, y, w);
+    uint8_t* out = qa.codes + row * row_bytes;
+    if (FMT == 0) {
+      *reinterpret_cast<uint16_t*>(out + cq * 2) = static_cast<uint16_t>(packed);
+    } else {
+      out += cq * 3;
+      out[0] = static_cast<uint8_t>(packed);
+      out[1] = static_cast<uint8_t>(packed >> 8);
+      out[2] = static_cast<uint8_t>(packed >> 16);
+    }
+  }
+}
+
+template <int FMT, int RND>
+__device__ __forceinline__ void quantize_line_body(const QuantArgs& qa, const float* __restrict__ amax_src,
+                                                   int amax_count, int cta, int nctas) {
+  __shared__ float red[32];
+  const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
+  if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
+  const int64_t row_bytes = FMT == 0 ? (qa.cols >> 1) : (qa.cols * 3) >> 2;
+  const int64_t per_row = qa.blocks == 1 ? qa.cols >> 4 : qa.cols >> 2;
+  const int64_t units = qa.blocks == 1 ? qa.rows * per_row : (qa.rows >> 4) * per_row;
+  const int64_t nthr = static_cast<int64_t>(nctas) * kQuantThreads;
+  for (int64_t u = static_cast<int64_t>(cta) * kQuantThreads + threadIdx.x; u < units; u += nthr) {
+    const int64_t a = u / per_row, b = u - a * per_row;
+    if (qa.blocks == 1) quantize_unit_1x16<FMT, RND>(qa, ts, a, b, row_bytes);
+    else quantize_unit_16x1<FMT, RND>(qa, ts, a, b, row_bytes);
+  }
+}
+
 // ------------------------------------------------ several tensors at once
 // The quantize-once step of a layer (X, W, G_Y) in two launches instead of
 // six: every CTA of a launch serves one tensor ("job"), CTAs are assigned to
@@ -431,12 +567,30 @@ quantize_many_kernel(const __grid_constant__ QuantJobs jobs, const float* __rest
 #undef MQV_QUANT_CASE
 }
 
+// The same for calls whose jobs all use line blocks (a separate kernel, so
+// the square quantizer keeps its own register budget).
+__global__ void __launch_bounds__(kQuantThreads)
+quantize_many_line_kernel(const __grid_constant__ QuantJobs jobs, const float* __restrict__ partial) {
+  const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, true)];
+  const int cta = blockIdx.x - jb.quant_cta0;
+  const float* amax = partial + jb.amax_cta0;
+#define MQV_QUANT_CASE(F, R)                                                     \
+  if (jb.fmt == F && jb.rounding == R) {                                         \
+    quantize_line_body<F, R>(jb.qa, amax, jb.amax_ctas, cta, jb.quant_ctas);     \
+    return;                                                                      \
+  }
+  MQV_QUANT_CASE(0, 0) MQV_QUANT_CASE(0, 1) MQV_QUANT_CASE(1, 0) MQV_QUANT_CASE(1, 1)
+#undef MQV_QUANT_CASE
+}
+
 // ---------------------------------------------------------- dequantize
-// dst = (code·B in fp16, exact) · T, one thread per 4 x 4 block.
+// dst = (code·B in fp16, exact) · T, one thread per 4 x 4 piece of the
+// view; `blocks` as QuantArgs::blocks (each piece lies in one square, in
+// 4 line blocks of 1 x 16, one per row, or in 4 of 16 x 1, one per column).
 template <int FMT>
 __global__ void __launch_bounds__(kQuantThreads)
 dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                  const float* __restrict__ tscale, int64_t rows, int64_t cols,
+                  const float* __restrict__ tscale, int64_t rows, int64_t cols, int blocks,
                   float* __restrict__ dst) {
   const float T = *tscale;
   const int64_t cb = cols >> 2;
@@ -446,10 +600,21 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
   for (int64_t b = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x; b < nblocks;
        b += stride) {
     const int64_t br = b / cb, bc = b - br * cb;
-    const uint32_t s = scales[b];
-    const uint32_t s2 = e4m3x2_to_f16x2(s | (s << 8));
+    uint32_t s01 = 0, s23 = 0;
+    if (blocks == 0) {
+      const uint32_t s = scales[b];
+      s01 = s23 = e4m3x2_to_f16x2(s | (s << 8));
+    } else if (blocks == 2) {
+      const uint32_t s = *reinterpret_cast<const uint32_t*>(scales + (br >> 2) * cols + bc * 4);
+      s01 = e4m3x2_to_f16x2(s & 0xFFFF);
+      s23 = e4m3x2_to_f16x2(s >> 16);
+    }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
+      if (blocks == 1) {
+        const uint32_t s = scales[(br * 4 + r) * (cols >> 4) + (bc >> 2)];
+        s01 = s23 = e4m3x2_to_f16x2(s | (s << 8));
+      }
       const uint8_t* in = codes + (br * 4 + r) * row_bytes;
       uint32_t h01, h23;
       if (FMT == 0) {
@@ -462,8 +627,8 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
         h01 = e2m3x2_to_f16x2((q & 0x3F) | ((q << 2) & 0x3F00));
         h23 = e2m3x2_to_f16x2(((q >> 12) & 0x3F) | ((q >> 10) & 0x3F00));
       }
-      h01 = hmul2_u32(h01, s2);
-      h23 = hmul2_u32(h23, s2);
+      h01 = hmul2_u32(h01, s01);
+      h23 = hmul2_u32(h23, s23);
       float4 o;
       o.x = __fmul_rn(f16_lo_to_f32(h01), T);
       o.y = __fmul_rn(f16_hi_to_f32(h01), T);

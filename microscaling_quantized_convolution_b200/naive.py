@@ -1,15 +1,29 @@
 """The baseline MicroQonv removes, run on the same kernels for measurement.
 
 Section "무엇인가" of the MicroQonv summary (onedev.kr/papers/182) describes
-the usual low-precision training flow: expand X with im2col first, quantize
-the expanded matrix, and quantize every operand once per GEMM direction
-(W for the forward and the input gradient, G_Y for the two gradients, the
-expanded X for the forward and the weight gradient).  This module composes
-that flow from the library's entry points: `mqv_im2col`, the quantizer on the
-expanded tensor (4 x 4 blocks over (kh·kw·ci, n), which for the
-channel-batch-first layout gives every duplicate of a pixel the same codes,
-so the results match the quantize-once path up to summation order), 1 x 1
-convolutions as the three GEMMs, and `mqv_col2im` for the input gradient.
+the usual low-precision training flow: expand X with im2col first, then
+quantize every GEMM operand with plain 16-element blocks along that GEMM's
+contraction, once per direction (W for the forward and the input gradient,
+G_Y for the two gradients, the expanded X' for the forward and the weight
+gradient).  This module composes that flow from the library's entry points:
+`mqv_im2col`; one `mqv_quantize_many` call writing the six copies
+
+    X'  16 x 1 down its (pixel, K) rows for Y = W·X' (contraction K),
+        1 x 16 along its batch columns for G_W = G_Y·X'^T (contraction P);
+    W   1 x 16 along its K rows for Y, 16 x 1 down its Cout column for G_X';
+    G_Y 1 x 16 along its batch columns for G_W, 16 x 1 down its (pixel,
+        Cout) rows for G_X' (stochastic rounding, one seed and element
+        numbering for both copies);
+
+1 x 1 convolutions over the Kh·Kw·Cin expanded channels as the three GEMMs;
+and `mqv_col2im` for the input gradient.  One pixel's duplicates in X' land
+in different blocks and take different codes, and each operand's two copies
+differ: the numerics of the scheme, not only its memory traffic.
+
+`blocks="square"` keeps a second variant under its own name: the same flow
+with 4 x 4 blocks over (kh·kw·ci, n) of the expanded tensor, whose
+duplicates all get equal codes (its six copies are three identical pairs);
+it isolates the cost of the expansion from the change of numerics.
 Every step runs on the GPU; nothing here computes on the host."""
 from __future__ import annotations
 
@@ -17,9 +31,13 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (NVFP4, RNE, SR, ConvDesc, QTensor, col2im, conv_desc, conv_dgrad, conv_fwd,
-               conv_wgrad, conv_workspace_bytes, im2col, out_hw, quantize_many,
+from . import (NVFP4, RNE, SR, BLOCKS_1X16, BLOCKS_16X1, BLOCKS_4X4, ConvDesc, QTensor, col2im, conv_desc,
+               conv_dgrad, conv_fwd, conv_wgrad, conv_workspace_bytes, im2col, out_hw, quantize_many,
                quantize_many_workspace_bytes, OP_FWD, OP_WGRAD, OP_DGRAD)
+
+# block shape of each copy: along the contraction of the GEMM it feeds
+LINE_BLOCKS = {"x_fwd": BLOCKS_16X1, "x_wgrad": BLOCKS_1X16, "w_fwd": BLOCKS_1X16, "w_dgrad": BLOCKS_16X1,
+               "g_wgrad": BLOCKS_1X16, "g_dgrad": BLOCKS_16X1}
 
 
 @dataclass
@@ -33,16 +51,20 @@ class NaivePlan:
     ws: dict             # workspaces
 
 
-def plan(d: ConvDesc, device="cuda") -> NaivePlan:
+def plan(d: ConvDesc, device="cuda", blocks: str = "line") -> NaivePlan:
+    """blocks: "line" (the scheme's 16-element blocks) or "square"."""
+    if blocks not in ("line", "square"):
+        raise ValueError(f"blocks must be 'line' or 'square', got {blocks!r}")
     Ho, Wo = out_hw(d)
     K = d.Kh * d.Kw * d.Cin
     d1 = conv_desc(d.N, K, d.Cout, Ho, Wo, 1, 1, 1, 0, d.fmt)
     xc = torch.empty((Ho, Wo, K, d.N), dtype=torch.float32, device=device)
     gxc = torch.empty_like(xc)
     rows_x, rows_g = Ho * Wo * K, Ho * Wo * d.Cout
-    q = {"x_fwd": QTensor.empty(rows_x, d.N, d.fmt, device), "x_wgrad": QTensor.empty(rows_x, d.N, d.fmt, device),
-         "w_fwd": QTensor.empty(d.Cout, K, d.fmt, device), "w_dgrad": QTensor.empty(d.Cout, K, d.fmt, device),
-         "g_wgrad": QTensor.empty(rows_g, d.N, d.fmt, device), "g_dgrad": QTensor.empty(rows_g, d.N, d.fmt, device)}
+    shape = {"x_fwd": (rows_x, d.N), "x_wgrad": (rows_x, d.N), "w_fwd": (d.Cout, K), "w_dgrad": (d.Cout, K),
+             "g_wgrad": (rows_g, d.N), "g_dgrad": (rows_g, d.N)}
+    q = {k: QTensor.empty(r, c, d.fmt, device, LINE_BLOCKS[k] if blocks == "line" else BLOCKS_4X4)
+         for k, (r, c) in shape.items()}
     jobs = [(None, rows_x, d.N, d.fmt, RNE, 0), (None, rows_x, d.N, d.fmt, RNE, 0),
             (None, d.Cout, K, d.fmt, RNE, 0), (None, d.Cout, K, d.fmt, RNE, 0),
             (None, rows_g, d.N, d.fmt, SR, 0), (None, rows_g, d.N, d.fmt, SR, 0)]
@@ -55,7 +77,7 @@ def plan(d: ConvDesc, device="cuda") -> NaivePlan:
 
 def quantize_all(p: NaivePlan, X: torch.Tensor, W: torch.Tensor, G: torch.Tensor, seed: int):
     """im2col, then every operand once per GEMM direction (six quantized
-    tensors in one two-launch call)."""
+    tensors in one two-launch call, each in its copy's block shape)."""
     d, d1 = p.d, p.d1
     im2col(d, X, p.xc)
     rows_x = d1.H * d1.W * d1.Cin

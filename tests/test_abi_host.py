@@ -241,3 +241,41 @@ def test_blockscaled_forward_workspace_and_rejections(lib):
     w = mqv.QTensorC(16, 16, 16, 128, 1152, 0, 0)
     x = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, 0)
     assert lib.mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, None, 0, None) == 3
+
+
+def test_block_shapes_are_validated(lib):
+    """The 16-element line blocks of the naive scheme: accepted by the
+    many-tensor quantizer (not mixed with squares in one call), refused by
+    the single-tensor quantizer, by shapes that do not split into lines, and
+    by conv passes other than the stride-1 1 x 1 GEMMs in the stated shapes.
+    Every refusal comes before any CUDA call."""
+    def job(rows, cols, blocks):
+        return mqv.QuantJobC(16, rows, cols, 0, 0, 0, mqv.QTensorC(16, 16, 16, rows, cols, 0, blocks))
+
+    def many(*jobs):
+        arr = (mqv.QuantJobC * len(jobs))(*jobs)
+        return lib.mqv_quantize_many(arr, len(jobs), 16, 1 << 20, None)
+
+    assert many(job(64, 64, 3)) == 1                             # unknown shape
+    assert many(job(64, 8, mqv.BLOCKS_1X16)) == 1                # cols not a multiple of 16
+    assert many(job(8, 64, mqv.BLOCKS_16X1)) == 1                # rows not a multiple of 16
+    assert many(job(64, 64, mqv.BLOCKS_4X4), job(64, 64, mqv.BLOCKS_1X16)) == 2   # mixed in one call
+    q = mqv.QTensorC(16, 16, 16, 64, 64, 0, mqv.BLOCKS_1X16)
+    assert lib.mqv_quantize_cbf(16, 64, 64, 0, 0, 0, ctypes.byref(q), 16, 256, None) == 2
+    # conv passes: a 3 x 3 layer refuses line blocks
+    d = _desc()
+    w = mqv.QTensorC(16, 16, 16, 128, 1152, 0, mqv.BLOCKS_1X16)
+    x = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, mqv.BLOCKS_16X1)
+    assert lib.mqv_conv_fwd(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 16, 1 << 24, None) == 2
+    assert b"line blocks" in lib.mqv_last_error()
+    # a 1 x 1 layer: only the stated shape per operand
+    d1 = _desc(Cin=1152, Kh=1, Kw=1, pad=0)
+    w1 = mqv.QTensorC(16, 16, 16, 128, 1152, 0, mqv.BLOCKS_16X1)          # fwd wants 1 x 16
+    x1 = mqv.QTensorC(16, 16, 16, 28 * 28 * 1152, 64, 0, mqv.BLOCKS_16X1)
+    assert lib.mqv_conv_fwd(ctypes.byref(d1), ctypes.byref(w1), ctypes.byref(x1), 16, 16, 1 << 24, None) == 2
+    gy = mqv.QTensorC(16, 16, 16, 28 * 28 * 128, 64, 0, mqv.BLOCKS_16X1)  # wgrad wants 1 x 16
+    xw = mqv.QTensorC(16, 16, 16, 28 * 28 * 1152, 64, 0, mqv.BLOCKS_1X16)
+    assert lib.mqv_conv_wgrad(ctypes.byref(d1), ctypes.byref(gy), ctypes.byref(xw), 16, 16, 1 << 28, None) == 2
+    # the block-scaled forward pass takes squares only
+    assert lib.mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 16, 1 << 24,
+                                        None) == 2
