@@ -1109,6 +1109,42 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_probe(args):
+    """A small fixed case for single-kernel ncu captures: the layer's step
+    (quantize X, W, G_Y in one call; fwd in both MMA forms, wgrad, dgrad)
+    `args.probe` times through the public API, then a device-error check.
+    Prints one line; no timing (numbers taken under a profiler are not
+    bench values)."""
+    import torch
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    layer = pick_layer(args.workload)
+    dev = torch.device("cuda", 0)
+    X, Wt, G = (t.view(-1) for t in workloads.make_layer_inputs(layer, device=dev))
+    d = mqv.conv_desc(**layer.dims(), fmt=layer.fmt)
+    xr, wr, wc = layer.H * layer.W * layer.Cin, layer.Cout, layer.K * layer.K * layer.Cin
+    gr = layer.Ho * layer.Wo * layer.Cout
+    try:
+        mqv.conv_workspace_bytes(d, mqv.OP_FWD_BLOCKSCALED)
+        blockscaled = True
+    except mqv.MqvError:
+        blockscaled = False
+    for i in range(args.probe):
+        qx, qw, qg = mqv.quantize_many([(X, xr, layer.N, layer.fmt, mqv.RNE, 0), (Wt, wr, wc, layer.fmt, mqv.RNE, 0),
+                                        (G, gr, layer.N, layer.fmt, mqv.SR, 7 + i)])
+        mqv.conv_fwd(d, qw, qx)
+        if blockscaled:
+            mqv.conv_fwd_blockscaled(d, qw, qx)
+        mqv.conv_wgrad(d, qg, qx)
+        mqv.conv_dgrad(d, qw, qg)
+    torch.cuda.synchronize()
+    flags = mqv.device_errors()
+    print(json.dumps({"probe": layer.name, "iterations": args.probe, "device_error_flags": flags}))
+    if flags:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1126,13 +1162,17 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    ap.add_argument("--probe", type=int, default=0,
+                    help="run the layer's step this many times for a profiler capture and exit (no timing)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.traffic = None
     if os.path.exists(args.traffic_json):
         with open(args.traffic_json) as f:
             args.traffic = json.load(f).get(args.workload)
-    if args.impl == "reference":
+    if args.probe > 0:
+        run_probe(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
