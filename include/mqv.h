@@ -387,8 +387,20 @@ mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const void* x, flo
 
 /* Synchronizes `stream`, then reports and clears the device error word that
  * bounded waits inside the conv kernels set when they give up
- * (*flags = 0: none).  Returns MQV_ERR_TIMEOUT if a flag was set. */
+ * (*flags = 0: none).  Returns MQV_ERR_TIMEOUT if a flag was set.  Bits:
+ * 1 a wait for a free pipeline stage, 2 a wait for a filled stage, 4 a wait
+ * for a finished accumulator, 8 the wait of mqv_selftest_wait_timeout.
+ * Every such wait polls its mbarrier for about 2^32 SM cycles (about two
+ * seconds) before it gives up; the kernel then returns without faulting, so
+ * the CUDA context stays usable. */
 mqv_status mqv_device_errors(uint32_t* flags, void* stream);
+
+/* Test hook for the timeout path: one CTA waits, with the conv kernels'
+ * bounded wait, on an mbarrier that nothing ever arrives at, for at most
+ * limit_cycles SM cycles (1 .. 2^32), then sets bit 8 of the device error
+ * word and returns.  Nothing else is touched; mqv_device_errors then returns
+ * MQV_ERR_TIMEOUT with that bit.  Not part of the method. */
+mqv_status mqv_selftest_wait_timeout(int64_t limit_cycles, void* stream);
 
 #ifdef __cplusplus
 }

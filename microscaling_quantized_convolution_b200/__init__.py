@@ -103,6 +103,7 @@ _SIGS = {
                                       ctypes.POINTER(QTensorC), ctypes.c_void_p, ctypes.c_void_p,
                                       ctypes.c_size_t, ctypes.c_void_p]),
     "mqv_device_errors": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_void_p]),
+    "mqv_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
     "mqv_quantize_many_workspace_size": (ctypes.c_int, [ctypes.POINTER(QuantJobC), ctypes.c_int32,
                                                         ctypes.POINTER(ctypes.c_size_t)]),
     "mqv_quantize_many": (ctypes.c_int, [ctypes.POINTER(QuantJobC), ctypes.c_int32, ctypes.c_void_p,
@@ -519,6 +520,13 @@ def device_errors(stream=None) -> int:
     if st not in (MQV_OK, 5):
         _check(st)
     return f.value
+
+
+def selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Test hook: a one-CTA kernel whose bounded wait runs out after
+    limit_cycles SM cycles and sets bit 8 of the device error word (see
+    mqv_selftest_wait_timeout); read it with device_errors()."""
+    _check(lib().mqv_selftest_wait_timeout(limit_cycles, _stream(stream)))
 
 
 # ------------------------------------------- depthwise layers in BF16

@@ -741,6 +741,19 @@ static mqv_status plan_quantize_many(const mqv_quantize_job* jobs, int32_t count
   return MQV_OK;
 }
 
+// The timeout path of the bounded waits, on its own: an mbarrier that
+// nothing arrives at (a fresh barrier's phase 0 never completes), waited for
+// with mbar_wait_bounded and a caller-given limit.
+__global__ void wait_selftest_kernel(uint32_t* err, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, err, kErrWaitSelfTest, limit);
+}
+
 }  // namespace
 
 extern "C" {
@@ -1038,6 +1051,18 @@ mqv_status mqv_conv_dgrad_quantized(const mqv_conv_desc* d, const mqv_qtensor* w
                                     void* ws, size_t ws_bytes, void* stream) {
   const QuantOut qo{gx_q, t_amax, seed};
   return run_conv(MQV_OP_DGRAD, d, w, "w", gy, "gy", nullptr, ws, ws_bytes, stream, 0, gx_amax, &qo);
+}
+
+mqv_status mqv_selftest_wait_timeout(int64_t limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 32))
+    return fail(MQV_ERR_INVALID_ARG, "limit_cycles %lld outside 1 .. 2^32", (long long)limit_cycles);
+  uint32_t* err = nullptr;
+  mqv_status st = device_error_word(&err);
+  if (st) return st;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_cycles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return ok();
 }
 
 mqv_status mqv_device_errors(uint32_t* flags, void* stream) {

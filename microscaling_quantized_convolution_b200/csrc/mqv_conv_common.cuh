@@ -13,7 +13,7 @@ namespace mqv {
 enum ConvPass { kFwd = 0, kWgrad = 1, kDgrad = 2 };
 
 // Device error bits set by bounded waits.
-constexpr uint32_t kErrWaitEmpty = 1u, kErrWaitFull = 2u, kErrWaitDone = 4u;
+constexpr uint32_t kErrWaitEmpty = 1u, kErrWaitFull = 2u, kErrWaitDone = 4u, kErrWaitSelfTest = 8u;
 
 struct QView {
   const uint8_t* codes;

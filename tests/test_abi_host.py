@@ -279,3 +279,9 @@ def test_block_shapes_are_validated(lib):
     # the block-scaled forward pass takes squares only
     assert lib.mqv_conv_fwd_blockscaled(ctypes.byref(d), ctypes.byref(w), ctypes.byref(x), 16, 16, 1 << 24,
                                         None) == 2
+
+
+def test_selftest_wait_limit_is_validated(lib):
+    for bad in (0, -5, (1 << 32) + 1):
+        assert lib.mqv_selftest_wait_timeout(bad, None) == 1
+    assert b"limit_cycles" in lib.mqv_last_error()
