@@ -398,9 +398,48 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return t0.elapsed_time(t1)
 
+    # The serial step on one GPU: one graph per step with the phase
+    # boundaries recorded as event nodes inside it (external events), so the
+    # per-phase device times carry no graph launch between phases.  Each of
+    # the nk graphs keeps its own events: after the timed loop they hold the
+    # last nk steps' phase times, which give the per-kernel durations.
+    nk = 4 * nsets
+    kev, kgraphs = [], []
+    if world == 1:
+        kev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(nk)]
+
+        def serial_marked(j):
+            k = j % nsets
+            s, e = sets[k], kev[j]
+            e[0].record()
+            quantize_all(s, k)
+            e[1].record()
+            fwd(s)
+            e[2].record()
+            wgrad(s)
+            e[3].record()
+            dgrad(s)
+            e[4].record()
+
+        kgraphs = [capture(lambda j=j: serial_marked(j)) for j in range(nk)]
+        torch.cuda.synchronize()
+
     def timed_loop(conc):
         """K steps between a barrier + synchronize on both sides; returns the
         whole-loop time and each phase's mean duration (max over ranks)."""
+        if world == 1 and not conc:
+            for i in range(nk):
+                kgraphs[i].replay()
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for i in range(args.steps):
+                kgraphs[i % nk].replay()
+            t1.record()
+            torch.cuda.synchronize()
+            names = ("quantize", "fwd", "wgrad", "dgrad")
+            parts = {ph: [e[j].elapsed_time(e[j + 1]) for e in kev] for j, ph in enumerate(names)}
+            return t0.elapsed_time(t1), {k: sum(v) / len(v) for k, v in parts.items()}
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
         for i in range(3):
             graph_step(i, evs[0], conc)
@@ -602,7 +641,7 @@ def run_gpu(args):
                        "note": "one step's copies in both directions at once, no compute; frac = that "
                                "time / the pipelined step time"}
 
-    del graphs, step_graphs
+    del graphs, step_graphs, kgraphs
     torch.cuda.synchronize()
     if world > 1:
         dist.destroy_process_group()
@@ -661,7 +700,9 @@ def run_gpu(args):
                    "l2": f"inputs rotated over {nsets} resident sets ({nsets * per_set / 1e6:.0f} MB > 126 MB L2)",
                    "launch": ("the whole step (both quantize launch pairs, the three passes on their "
                               "streams and the joins) replayed as one CUDA graph captured through the C ABI"
-                              if concurrent else "each phase replayed as a CUDA graph captured through the C ABI"),
+                              if concurrent else ("the serial step replayed as one CUDA graph captured through "
+                                                  "the C ABI" if world == 1 else
+                                                  "each phase replayed as a CUDA graph captured through the C ABI")),
                    "schedule": ("quantize X,W beside quantize G_Y; fwd after X,W; wgrad and dgrad after "
                                 "all three; the passes on separate streams" if concurrent
                                 else "quantize, fwd, wgrad, dgrad on one stream"),
@@ -675,8 +716,11 @@ def run_gpu(args):
     }
     out["serial"] = {"ms_per_step": round(serial_ms / args.steps, 5),
                      "value": round(3 * flops * world / (serial_ms / args.steps * 1e-3) / 1e12, 3),
-                     "note": "the same step with fwd, wgrad, dgrad one after another; the per-kernel "
-                             "durations and the roofline come from this loop"}
+                     "note": ("the same step with quantize, fwd, wgrad, dgrad one after another, one graph per "
+                              "step; the per-kernel durations and the roofline come from event nodes inside "
+                              f"those graphs (the last {nk} steps of this loop)" if world == 1 else
+                              "the same step with fwd, wgrad, dgrad one after another; the per-kernel "
+                              "durations and the roofline come from this loop")}
     if concurrent:
         out["kernels_concurrent_ms"] = {k: round(v, 5) for k, v in conc_mean.items()}
         out["phase_graphs"] = {"ms_per_step": round(phase_ms / args.steps, 5),

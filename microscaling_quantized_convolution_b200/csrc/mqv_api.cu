@@ -492,13 +492,28 @@ cudaError_t launch_pass(const ConvPlan& pl, cudaStream_t st) {
   return pl.nu == 8 ? launch_fd<P, FMT, 128, 8, false>(pl, st) : launch_fd<P, FMT, 128, 4, false>(pl, st);
 }
 
+// The halo kernel follows its weight-image kernel with programmatic
+// dependent launch: its barrier setup, tensor-memory allocation and first
+// activation loads overlap the image kernel, and only its weight loader
+// waits for the image (pdl_wait_prerequisite).
 template <int PASS, int FMT, bool QOUT, bool LINE = false>
 cudaError_t launch_halo_q(const ConvPlan& pl, cudaStream_t st) {
   auto kern = conv_halo_kernel<PASS, FMT, QOUT, LINE>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, HaloSmem::kBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<pl.grid, kHaloThreads, HaloSmem::kBytes, st>>>(pl.a, pl.g);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+  cfg.blockDim = dim3(kHaloThreads);
+  cfg.dynamicSmemBytes = HaloSmem::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, pl.a, pl.g);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

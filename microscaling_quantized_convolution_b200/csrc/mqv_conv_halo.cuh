@@ -37,10 +37,10 @@ constexpr int kHaloBN = 256;                  // most GEMM columns per tile (TME
 constexpr int kHaloMaxRows = 384;             // halo rows: 256 + (Kw - 1)·N <= 384
 constexpr int kHaloBStages = 2;
 constexpr int kHaloAStages = 6;
+constexpr int kHaloLookahead = 2;                        // stages of codes in flight per producer (block-scaled kernel)
 constexpr int kHaloProdWarps = 12;                       // one 8 x 8 unit per thread per stage
 constexpr int kHaloProdThreads = kHaloProdWarps * 32;    // 384 = the largest halo
 constexpr int kHaloThreads = (kV2ProdWarp0 + kHaloProdWarps) * 32;
-constexpr int kHaloLookahead = 2;                        // stages of codes in flight per thread
 constexpr uint32_t kHaloBTile = kHaloMaxRows * 128;   // 48 KB
 
 struct HaloSmem {
@@ -82,15 +82,15 @@ struct HaloUnit {
   bool ok;
 };
 
-// Transposed dequantize + store of one unit: row row0 + r of the tile gets
-// the 8 channels (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
+// Transposed dequantize of one unit (halo_dequant_unit, into registers) and
+// its store (halo_st_unit): row row0 + r of the tile gets the 8 channels
+// (c0..c0+7) of batch item n0 + r at K chunk kg.  Each pair of
 // channel words is interleaved nibble-wise first, so one cvt.e2m1x2 per
 // byte yields the (channel 2i, channel 2i+1) pair of one batch item.
 // LINE: the operand has 16 x 1 line blocks down its (pixel, channel) rows, so
 // the unit's 8 channels share one scale per batch item.
 template <int FMT, bool LINE>
-__device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile, uint32_t row0, uint32_t kg) {
-  uint32_t out[8][4];
+__device__ __forceinline__ void halo_dequant_unit(const HaloUnit& u, uint32_t (&out)[8][4]) {
   uint32_t sl[8];
   if (LINE) {
 #pragma unroll
@@ -135,6 +135,9 @@ __device__ __forceinline__ void halo_store_unit(const HaloUnit& u, uint32_t tile
 #pragma unroll
     for (int r = 0; r < 8; ++r) out[r][0] = out[r][1] = out[r][2] = out[r][3] = 0u;
   }
+}
+
+__device__ __forceinline__ void halo_st_unit(const uint32_t (&out)[8][4], uint32_t tile, uint32_t row0, uint32_t kg) {
 #pragma unroll
   for (int r = 0; r < 8; ++r)
     st_shared_v4(tile + sw128_offset(row0 + r, 8 * kg), out[r][0], out[r][1], out[r][2], out[r][3]);
@@ -298,7 +301,7 @@ __device__ __forceinline__ void halo_epilogue_tile(const V2Args& p, const HaloGe
 
 // QOUT: the quantized-output epilogue (V2Args::q_codes), a separate
 // instance so that the plain passes keep their code and registers.  LINE:
-// the B operand has 16 x 1 line blocks (see halo_store_unit).
+// the B operand has 16 x 1 line blocks (see halo_dequant_unit).
 template <int PASS, int FMT, bool QOUT, bool LINE = false>
 __global__ void __launch_bounds__(kHaloThreads, 1)
 conv_halo_kernel(const V2Args p, const HaloGeom g) {
@@ -408,6 +411,9 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
     if (lane == 0) {
       int sa = 0;
       uint32_t pa = 1;                 // first pass: the empty slots count as released
+      // the weight image comes from the kernel before this one, which this
+      // kernel may overlap (programmatic dependent launch): wait for it
+      pdl_wait_prerequisite();
       for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x) {
         const int mt = tile / (g.out_h * g.tpr);
         const uint8_t* img = p.image + static_cast<int64_t>(mt) * p.ktiles * kATileBytes;
@@ -429,15 +435,18 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
       }
     }
   } else {
-    // producers: kHaloLookahead stages of codes in flight per thread (a ring
-    // of registers indexed at compile time)
+    // producers: the next stage's unit is dequantized into registers while
+    // the MMAs read the current one, so between a slot's release (bempty)
+    // and its refill signal (bfull) a producer only stores; the unit after
+    // that is loaded one stage ahead.
     const int t = threadIdx.x - kV2ProdWarp0 * 32;
     const int ntile_cta = (p.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                           static_cast<int>(gridDim.x);
     const int total = ntile_cta * stages_per_tile;
     const int spatial = g.out_h * g.tpr;
     HaloCursor<PASS, FMT, LINE> cursor;
-    HaloUnit ring[kHaloLookahead];
+    HaloUnit raw;
+    uint32_t out[8][4];
     int ltile = blockIdx.x, lkh = 0, lc = 0;
     if (total > 0) cursor.begin_tile(p, g, ltile % spatial, t);
     auto load_next = [&](HaloUnit& u) {
@@ -451,23 +460,23 @@ conv_halo_kernel(const V2Args p, const HaloGeom g) {
         }
       }
     };
-#pragma unroll
-    for (int r = 0; r < kHaloLookahead; ++r)
-      if (r < total) load_next(ring[r]);
-    for (int kit = 0; kit < total;) {
-#pragma unroll
-      for (int r = 0; r < kHaloLookahead; ++r, ++kit) {
-        if (kit >= total) break;
-        const int sb = kit % kHaloBStages;
-        mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
-        if (t < g.rows)
-          halo_store_unit<FMT, LINE>(ring[r], sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
-                          static_cast<uint32_t>(t & 7));
-        producer_warp_arrive(&bars->bfull[sb]);
-        if (kit + kHaloLookahead < total) load_next(ring[r]);
-      }
+    if (total > 0) {
+      load_next(raw);
+      halo_dequant_unit<FMT, LINE>(raw, out);
+      if (total > 1) load_next(raw);
     }
-    // The CTA's last tile: once its accumulator is complete (so the B ring
+    for (int kit = 0; kit < total; ++kit) {
+      const int sb = kit % kHaloBStages;
+      mbar_wait_bounded(&bars->bempty[sb], ((kit / kHaloBStages) & 1) ^ 1, p.err, kErrWaitEmpty);
+      if (t < g.rows)
+        halo_st_unit(out, sbase + L::kBOffset + sb * kHaloBTile, static_cast<uint32_t>(8 * (t >> 3)),
+                     static_cast<uint32_t>(t & 7));
+      producer_warp_arrive(&bars->bfull[sb]);
+      if (kit + 1 < total) {
+        halo_dequant_unit<FMT, LINE>(raw, out);
+        if (kit + 2 < total) load_next(raw);
+      }
+    }    // The CTA's last tile: once its accumulator is complete (so the B ring
     // is no longer read), producer warp w takes chunks 1, 2 or 3 (of every 4)
     // on TMEM lane quarter w % 4, staging through 4 KB of the B ring.
     if (ntile_cta > 0) {

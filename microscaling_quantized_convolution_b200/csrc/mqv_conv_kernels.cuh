@@ -240,6 +240,9 @@ template <int FMT, bool TRANS>
 __global__ void __launch_bounds__(kPrepThreads)
 prep_image_kernel(QView w, int M, int Kdim, int ktiles, int mtiles, int Cin, int Cout, FastDiv dkt8,
                   FastDiv dcout, uint8_t* __restrict__ image) {
+  // the conv kernel after this one may start its own setup now (it waits
+  // for this kernel's completion before it reads the image)
+  pdl_launch_dependents();
   const int chunks = mtiles * 128 * ktiles * 8;
   const int id = blockIdx.x * kPrepThreads + threadIdx.x;
   if (id >= chunks) return;

@@ -158,23 +158,30 @@ __device__ __forceinline__ void wgk_x_load(const V2Args& p, const WgkTile& w, co
   }
 }
 
-// Dequantize the unit into X slot `slot` and, when `mirror` is nonzero, into
-// that second slot as well.
+// Dequantize the unit into registers (wgk_x_dequant), then store it into X
+// slot `slot` and, when `mirror` is nonzero, into that second slot as well
+// (wgk_x_st).
 template <int FMT, bool LINE>
-__device__ __forceinline__ void wgk_x_store(const UnitRaw<FMT, 8>& un, uint32_t slot, uint32_t mirror, int tid) {
-  const uint32_t row0 = static_cast<uint32_t>(4 * (tid >> 3)), kl = static_cast<uint32_t>(8 * (tid & 7));
+__device__ __forceinline__ void wgk_x_dequant(const UnitRaw<FMT, 8>& un, uint32_t (&h)[4][4]) {
   const uint32_t s2lo = un.ok && !LINE ? scale2(un.ss & 0xFF) : 0u;
   const uint32_t s2hi = un.ok && !LINE ? scale2(un.ss >> 8) : 0u;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint32_t h[4] = {0u, 0u, 0u, 0u};
+    h[j][0] = h[j][1] = h[j][2] = h[j][3] = 0u;
     if (un.ok) {
       const uint32_t sj = LINE ? scale2((un.ss >> (8 * j)) & 0xFF) : 0u;
-      dequant_run<FMT, 8>(un.lo[j], un.hi[j], LINE ? sj : s2lo, LINE ? sj : s2hi, h);
+      dequant_run<FMT, 8>(un.lo[j], un.hi[j], LINE ? sj : s2lo, LINE ? sj : s2hi, h[j]);
     }
+  }
+}
+
+__device__ __forceinline__ void wgk_x_st(const uint32_t (&h)[4][4], uint32_t slot, uint32_t mirror, int tid) {
+  const uint32_t row0 = static_cast<uint32_t>(4 * (tid >> 3)), kl = static_cast<uint32_t>(8 * (tid & 7));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
     const uint32_t off = sw128_offset(row0 + j, kl);
-    st_shared_v4(slot + off, h[0], h[1], h[2], h[3]);
-    if (mirror) st_shared_v4(mirror + off, h[0], h[1], h[2], h[3]);
+    st_shared_v4(slot + off, h[j][0], h[j][1], h[j][2], h[j][3]);
+    if (mirror) st_shared_v4(mirror + off, h[j][0], h[j][1], h[j][2], h[j][3]);
   }
 }
 
@@ -329,35 +336,38 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
     mbar_wait_bounded(&bars->done[m % kWgkXSlots], (m / kWgkXSlots) & 1, p.err, kErrWaitEmpty);
   };
   if (xi >= 0) {
-    // X producer: kWgkLookahead stages of codes in flight (a ring of
-    // registers indexed at compile time)
+    // X producer: the next stage's unit is dequantized into registers
+    // before the slot is free, so the wait is followed only by stores; the
+    // unit after that is loaded one stage ahead.
     const int tid = xi * 32 + lane;
     WgkCursor cur, ld;
     cur.begin(p, g, w);
     ld = cur;
-    UnitRaw<FMT, 8> ring[kWgkLookahead];
-#pragma unroll
-    for (int r = 0; r < kWgkLookahead; ++r)
+    UnitRaw<FMT, 8> raw;
+    uint32_t hx[4][4];
+    auto load_next = [&]() {
       if (ld.valid) {
-        wgk_x_load<FMT, LINE>(p, w, ld, tid, ring[r]);
+        wgk_x_load<FMT, LINE>(p, w, ld, tid, raw);
         ld.advance(g, g.sx);
       }
+    };
+    load_next();
+    if (cur.valid) {
+      wgk_x_dequant<FMT, LINE>(raw, hx);
+      load_next();
+    }
     int n = 0;
     while (cur.valid) {
-#pragma unroll
-      for (int r = 0; r < kWgkLookahead; ++r) {
-        if (!cur.valid) break;
-        const int s = n % kWgkXSlots;
-        if (n >= kWgkXSlots) wait_done(n - kWgkXSlots + g.sx);
-        const uint32_t mirror = (PAIR && s < kWgkXMirrors) ? sbase + (kWgkXSlots + s) * L::kXSlot : 0u;
-        wgk_x_store<FMT, LINE>(ring[r], sbase + s * L::kXSlot, mirror, tid);
-        producer_warp_arrive(&bars->full[s]);
-        if (ld.valid) {
-          wgk_x_load<FMT, LINE>(p, w, ld, tid, ring[r]);
-          ld.advance(g, g.sx);
-        }
-        cur.advance(g, g.sx);
-        ++n;
+      const int s = n % kWgkXSlots;
+      if (n >= kWgkXSlots) wait_done(n - kWgkXSlots + g.sx);
+      const uint32_t mirror = (PAIR && s < kWgkXMirrors) ? sbase + (kWgkXSlots + s) * L::kXSlot : 0u;
+      wgk_x_st(hx, sbase + s * L::kXSlot, mirror, tid);
+      producer_warp_arrive(&bars->full[s]);
+      cur.advance(g, g.sx);
+      ++n;
+      if (cur.valid) {
+        wgk_x_dequant<FMT, LINE>(raw, hx);
+        load_next();
       }
     }
   } else if (warp < 4 || (warp >= 8 && warp < 12)) {

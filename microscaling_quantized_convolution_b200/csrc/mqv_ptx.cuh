@@ -72,6 +72,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Programmatic dependent launch (PTX griddepcontrol): a kernel launched with
+// programmatic stream serialization may start while the kernel before it in
+// the stream still runs, once every CTA of that kernel has executed
+// launch_dependents (or exited); wait_prerequisite then blocks until that
+// kernel has completed and its memory operations are visible.  Both are
+// no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prerequisite() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Arrive once on `bar` and add `bytes` to the transaction count it waits for.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
