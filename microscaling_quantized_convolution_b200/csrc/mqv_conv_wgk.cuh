@@ -39,11 +39,10 @@ constexpr int kWgkXMirrors = 2;         // copies of slots 0 and 1 after the rin
 constexpr int kWgkASlots = 4;           // G_Y chunks in tensor memory
 constexpr int kWgkMaxTaps = 3;
 constexpr int kWgkACol = kWgkMaxTaps * 128;     // first TMEM column of the G_Y ring
-constexpr int kWgkLookahead = 2;        // stages of codes in flight per producer thread
-// Roles: warps 0-3 produce the first half of each G_Y chunk, warps 8-11 the
-// second (each G_Y warp owns its TMEM lane quarter, warp % 4); warps 6, 7 and
-// 12-17 produce X; warp 4 issues the MMAs; warp 5 has no role.  All 16
-// producer warps then run the epilogue.
+// Roles: warps 0-3 produce the even G_Y chunks, warps 8-11 the odd ones
+// (each G_Y warp owns its TMEM lane quarter, warp % 4); warps 6, 7 and 12-17
+// produce X; warp 4 issues the MMAs; warp 5 has no role.  All 16 producer
+// warps then run the epilogue.
 constexpr int kWgkWarps = 18;
 constexpr int kWgkThreads = kWgkWarps * 32;
 constexpr int kWgkXWarps = 8;
@@ -69,9 +68,11 @@ struct WgkSmem {
   static constexpr int kBytes = kBarOffset + 256 + 1024;
 };
 
-// One full and one done barrier per stage of the X ring: both producers
-// arrive on full[n % 8] for every stage n (the G_Y warps with the A chunk
-// of an MMA stage, immediately otherwise), and the MMA thread commits
+// One full and one done barrier per stage of the X ring: the 8 X warps and
+// 4 G_Y warps (the chunk's owners, one per lane quarter) arrive on
+// full[n % 8] for every stage n (the G_Y warps with the A chunk of an MMA
+// stage; warps 0-3 alone, once stage n - 8 is done, otherwise), and the MMA
+// thread commits
 // done[n % 8] after every stage, so it waits once and commits once a stage.
 // X stage n reuses its slot once stage n - 8 + SX (the last that reads the
 // previous X chunk in it) is done; G_Y chunk a reuses A slot a % 4 once the
@@ -185,23 +186,22 @@ __device__ __forceinline__ void wgk_x_st(const uint32_t (&h)[4][4], uint32_t slo
   }
 }
 
-// G_Y producer: 32 of the 64 codes of one output-channel row of an output
-// chunk (half h: elements 32h..32h+31), as two 16-element pieces, each inside
-// one pixel since N % 16 == 0.
-struct WgkGRaw {
-  uint32_t c[2][3];     // FP4: 8 bytes in c[.][0..1]; FP6: 12 bytes
-  uint32_t s[2];        // the four E4M3 block scales of a piece
+// G_Y producer: the 64 codes of one output-channel row of an output chunk,
+// as four 16-element pieces, each inside one pixel since N % 16 == 0.
+struct WgkGRow {
+  uint32_t c[4][3];     // FP4: 8 bytes in c[.][0..1]; FP6: 12 bytes
+  uint32_t s[4];        // the four E4M3 block scales of a piece
   uint32_t ok;          // bit per piece
 };
 
 template <int FMT, bool LINE>
-__device__ __forceinline__ void wgk_g_load(const V2Args& p, const WgkTile& w, const WgkCursor& c, int row, int half,
-                                           WgkGRaw& r) {
+__device__ __forceinline__ void wgk_g_load_row(const V2Args& p, const WgkTile& w, const WgkCursor& c, int row,
+                                               WgkGRow& r) {
   const int co = w.mt * 128 + row;
   r.ok = 0;
 #pragma unroll
-  for (int pc = 0; pc < 2; ++pc) {
-    const int e = c.t * 64 + 32 * half + 16 * pc;
+  for (int pc = 0; pc < 4; ++pc) {
+    const int e = c.t * 64 + 16 * pc;
     const int pix = fdiv(e, p.dN);
     const int n = e - pix * p.N;
     if (co < p.Cout && pix < p.Wo) {
@@ -225,9 +225,9 @@ __device__ __forceinline__ void wgk_g_load(const V2Args& p, const WgkTile& w, co
 }
 
 template <int FMT>
-__device__ __forceinline__ void wgk_g_dequant(const WgkGRaw& r, uint32_t (&h)[16]) {
+__device__ __forceinline__ void wgk_g_dequant_row(const WgkGRow& r, uint32_t (&h)[32]) {
 #pragma unroll
-  for (int pc = 0; pc < 2; ++pc) {
+  for (int pc = 0; pc < 4; ++pc) {
     uint32_t* o = h + 8 * pc;
     if (!((r.ok >> pc) & 1u)) {
 #pragma unroll
@@ -313,7 +313,7 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kWgkXSlots; ++s) {
-      mbar_init(&bars->full[s], kWgkXWarps + kWgkGWarps);
+      mbar_init(&bars->full[s], kWgkXWarps + kWgkGWarps / 2);   // X warps and one G_Y warp per lane quarter
       mbar_init(&bars->done[s], 1);
     }
     mbar_init(&bars->tile_done, 1);
@@ -372,50 +372,58 @@ conv_wgk_kernel(const V2Args p, const WgkGeom g) {
     }
   } else if (warp < 4 || (warp >= 8 && warp < 12)) {
     // G_Y producer: thread = output-channel row (this warp's TMEM lane
-    // quarter); warps 0-3 write columns 0-15 of a slot, warps 8-11 columns
-    // 16-31.  It walks the X stages, loading ahead along the output chunks.
-    // All producer warps run the epilogue afterwards.
-    const int quarter = warp & 3, half = warp < 4 ? 0 : 1;
+    // quarter).  Warps 0-3 take the even G_Y chunks, warps 8-11 the odd
+    // ones, a whole 64-element row each, so each warp has two stages' time
+    // for its loads and its dequantization; the next owned chunk is
+    // dequantized while the MMAs run, and the one after it is loaded.
+    // Stages with no G_Y chunk are signalled by warps 0-3.  All producer
+    // warps run the epilogue afterwards.
+    const int quarter = warp & 3, par = warp < 4 ? 0 : 1;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     WgkCursor cur, ld;
     cur.begin(p, g, w);
     ld = cur;
-    WgkGRaw ring[kWgkLookahead];
-#pragma unroll
-    for (int r = 0; r < kWgkLookahead; ++r)
+    if (par == 1 && ld.valid) ld.advance(g, 0);
+    WgkGRow raw;
+    uint32_t h[32];
+    auto load_owned = [&]() {          // the chunk at ld, then ld moves two chunks on
+      raw.ok = 0;
       if (ld.valid) {
-        wgk_g_load<FMT, LINE>(p, w, ld, row, half, ring[r]);
+        wgk_g_load_row<FMT, LINE>(p, w, ld, row, raw);
         ld.advance(g, 0);
+        if (ld.valid) ld.advance(g, 0);
       }
+    };
+    load_owned();
+    wgk_g_dequant_row<FMT>(raw, h);
+    load_owned();
     int n = 0, a = 0;
     while (cur.valid) {
-#pragma unroll
-      for (int r = 0; r < kWgkLookahead; ++r) {
-        while (cur.valid && !cur.mma_stage(g)) {    // stages with no G_Y chunk
+      if (!cur.mma_stage(g)) {           // a stage with no G_Y chunk
+        if (par == 0) {
+          if (n >= kWgkXSlots) wait_done(n - kWgkXSlots);
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->full[n % kWgkXSlots]);
-          cur.advance(g, g.sx);
-          ++n;
         }
-        if (!cur.valid) break;
-        uint32_t h[16];
-        wgk_g_dequant<FMT>(ring[r], h);
+        cur.advance(g, g.sx);
+        ++n;
+        continue;
+      }
+      if ((a & 1) == par) {
         if (n >= kWgkASlots) wait_done(n - kWgkASlots);
         tc_fence_after();
-        tmem_st_32x32b_x16(tmem + lane_base + kWgkACol + (a % kWgkASlots) * 32 + 16 * half, h);
+        tmem_st_32x32b_x32(tmem + lane_base + kWgkACol + (a % kWgkASlots) * 32, h);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full[n % kWgkXSlots]);
-        if (ld.valid) {
-          wgk_g_load<FMT, LINE>(p, w, ld, row, half, ring[r]);
-          ld.advance(g, 0);
-        }
-        cur.advance(g, g.sx);
-        ++n;
-        ++a;
+        wgk_g_dequant_row<FMT>(raw, h);
+        load_owned();
       }
+      cur.advance(g, g.sx);
+      ++n;
+      ++a;
     }
   } else if (warp == kV2MmaWarp) {
     if (lane == 0) {
