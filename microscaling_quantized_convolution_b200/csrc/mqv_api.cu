@@ -689,8 +689,11 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
     if (pl.a.splits > 1) {
       const int64_t n4 = (int64_t)pl.a.M * pl.a.Ncols / 4;
       const int64_t g = (n4 + kReduceCols - 1) / kReduceCols;
+      // whole 128-byte lines of partials can be dropped from L2 once read
+      const int discard = (reinterpret_cast<uintptr_t>(wsb) & 127u) == 0 && n4 % 8 == 0;
       wgrad_reduce_kernel<<<(unsigned)g, kReduceCols * kReduceGroups, 0, s>>>(reinterpret_cast<const float4*>(wsb), pl.a.splits, n4,
-                                                       qa->tscale, qb->tscale, reinterpret_cast<float4*>(out));
+                                                       qa->tscale, qb->tscale, reinterpret_cast<float4*>(out),
+                                                       discard);
       e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(e, "wgrad reduce launch");
     }

@@ -40,12 +40,16 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t k) {
 // float4 columns; four thread groups each add a contiguous quarter of the
 // splits in split order, and the four group sums are added in group order, so
 // the result is the same on every run.  Sixteen independent loads per thread
-// keep enough bytes in flight to run at memory speed.
+// keep enough bytes in flight to run at memory speed.  The partials are
+// scratch: with `discard` set (128-byte aligned lines, checked on the host)
+// each 128-byte line, once the block has read it, is dropped from L2 without
+// being written back (PTX discard.global.L2), so the partials cost no DRAM
+// writes when they never left L2.
 constexpr int kReduceCols = 64, kReduceGroups = 4;
 __global__ void __launch_bounds__(kReduceCols * kReduceGroups)
 wgrad_reduce_kernel(const float4* __restrict__ partial, int splits, int64_t n4,
                     const float* __restrict__ ta, const float* __restrict__ tb,
-                    float4* __restrict__ out) {
+                    float4* __restrict__ out, int discard) {
   __shared__ float4 part[kReduceGroups][kReduceCols];
   const int col = threadIdx.x % kReduceCols, grp = threadIdx.x / kReduceCols;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * kReduceCols + col;
@@ -78,6 +82,12 @@ wgrad_reduce_kernel(const float4* __restrict__ partial, int splits, int64_t n4,
   }
   part[grp][col] = acc;
   __syncthreads();
+  // every partial of this block's columns has been read and added: drop
+  // their lines (one 128-byte line per 8 columns and split)
+  if (discard && (col & 7) == 0 && i + 7 < n4) {
+    for (int s = s0; s < s1; ++s)
+      asm volatile("discard.global.L2 [%0], 128;" ::"l"(partial + static_cast<int64_t>(s) * n4 + i) : "memory");
+  }
   if (grp == 0 && i < n4) {
     float4 t = part[0][col];
 #pragma unroll
