@@ -81,7 +81,7 @@ def test_host_build_of_depthwise_kernels_matches_oracle(harness, tmp_path, dims)
 
 def test_host_build_of_depthwise_weight_gradient_long_reduction(harness, tmp_path):
     """A 56x56, N = 32 layer: 100,352 terms per weight, split into parts of
-    about 1024 terms per running sum, still within the tolerance."""
+    about 512 terms per running sum, still within the tolerance."""
     dims = (32, 2, 56, 56, 3, 3, 1, 1)
     N, C, H, W, Kh, Kw, st, pad = dims
     s = O.ConvShape(N, C, C, H, W, Kh, Kw, st, pad)
