@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmqv.so")
 SOURCES = ["mqv_api.cu"]
-HEADERS = ["mqv_ptx.cuh", "mqv_quantize.cuh", "mqv_conv_common.cuh", "mqv_conv_kernels.cuh", "mqv_conv_halo.cuh", "mqv_conv_nvf4.cuh", "mqv_conv_wgk.cuh", "mqv_naive.cuh", "mqv_replay.cuh", "mqv_depthwise.cuh", "mqv_depthwise_core.h"]
+HEADERS = ["mqv_ptx.cuh", "mqv_quantize.cuh", "mqv_conv_common.cuh", "mqv_conv_kernels.cuh", "mqv_conv_halo.cuh", "mqv_conv_nvf4.cuh", "mqv_conv_wgk.cuh", "mqv_conv_narrow.cuh", "mqv_naive.cuh", "mqv_replay.cuh", "mqv_depthwise.cuh", "mqv_depthwise_core.h"]
 
 
 def nvcc_cmd(out=LIB, extra=()):

@@ -17,6 +17,7 @@
 #include "mqv_conv_halo.cuh"
 #include "mqv_conv_nvf4.cuh"
 #include "mqv_conv_wgk.cuh"
+#include "mqv_conv_narrow.cuh"
 #include "mqv_depthwise.cuh"
 #include "mqv_naive.cuh"
 #include "mqv_quantize.cuh"
@@ -218,6 +219,7 @@ struct ConvPlan {
   HaloGeom g;
   bool wgk;             // stride-1 wgrad with the taps of a kernel row sharing operands
   WgkGeom wg;
+  bool narrow;          // dgrad of a narrow layer on CUDA cores (conv_narrow_dgrad_kernel)
   bool tr;              // generic fwd/dgrad on transposed tiles (M <= 128)
   int bn;               // 128 or 256 columns per tile
   int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0
@@ -428,7 +430,17 @@ void plan_conv(const mqv_conv_desc* d, int op, ConvPlan* pl) {
   // persistent kernels: one CTA per SM at most; the kernel-row weight
   // gradient runs one tile per CTA
   pl->grid = pl->wgk ? a.tiles : (a.tiles < kSMs ? a.tiles : kSMs);
-  pl->image_bytes = op == MQV_OP_WGRAD ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
+  // Input gradient of a 4-input-channel layer (a stem) with N % 16 == 0:
+  // bound by memory (Cout products per element and tap), so it runs on CUDA
+  // cores without a weight image (conv_narrow_dgrad_kernel).
+  pl->narrow = op == MQV_OP_DGRAD && !pl->halo && d->Cin == 4 && d->N % 16 == 0 &&
+               d->Cout * d->Kh * d->Kw * 4 * (int64_t)sizeof(float) <= kNarrowMaxWeightBytes;
+  if (pl->narrow) {
+    const int64_t units = d->H * d->W * (d->N / 16);
+    const int64_t g = (units + kNarrowThreads - 1) / kNarrowThreads;
+    pl->grid = (int)(g < 8 * kSMs ? g : 8 * kSMs);
+  }
+  pl->image_bytes = op == MQV_OP_WGRAD || pl->narrow ? 0 : (size_t)a.mtiles * a.ktiles * kATileBytes;
   pl->partial_bytes = splits > 1 ? (size_t)splits * a.M * a.Ncols * sizeof(float) : 0;
   pl->ws_bytes = pl->image_bytes + pl->partial_bytes;
 }
@@ -553,6 +565,13 @@ cudaError_t launch_pass_fmt(int fmt, const ConvPlan& pl, cudaStream_t st) {
                             : launch_halo<PASS == kWgrad ? kFwd : PASS, 1>(pl, st);
   if (PASS == kWgrad && pl.wgk) return fmt == MQV_NVFP4 ? launch_wgk_kw<0>(pl, st) : launch_wgk_kw<1>(pl, st);
   return fmt == MQV_NVFP4 ? launch_pass<PASS, 0>(pl, st) : launch_pass<PASS, 1>(pl, st);
+}
+
+cudaError_t launch_narrow_dgrad(int fmt, const ConvPlan& pl, const QView& w, cudaStream_t st) {
+  const int smem = pl.a.Cout * pl.a.Kh * pl.a.Kw * 4 * (int)sizeof(float);
+  if (fmt == MQV_NVFP4) conv_narrow_dgrad_kernel<0><<<pl.grid, kNarrowThreads, smem, st>>>(pl.a, w);
+  else conv_narrow_dgrad_kernel<1><<<pl.grid, kNarrowThreads, smem, st>>>(pl.a, w);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_prep(int op, int fmt, const ConvPlan& pl, const QView& w, uint8_t* image, cudaStream_t st) {
@@ -706,6 +725,15 @@ mqv_status run_conv(int op, const mqv_conv_desc* d, const mqv_qtensor* qa, const
   }
   pl.a.relu = relu;
   pl.a.amax_out = reinterpret_cast<uint32_t*>(amax);
+  if (pl.narrow) {
+    pl.a.b = make_view(qb);
+    pl.a.ta = qa->tscale;
+    pl.a.tb = qb->tscale;
+    pl.a.out = out;
+    e = launch_narrow_dgrad(d->fmt, pl, make_view(qa), s);
+    if (e != cudaSuccess) return cuda_fail(e, "narrow dgrad launch");
+    return ok();
+  }
   e = launch_prep(op, d->fmt, pl, make_view(qa), wsb, s);
   if (e != cudaSuccess) return cuda_fail(e, "operand image launch");
   pl.a.image = wsb;

@@ -175,10 +175,10 @@ def test_depthwise_entry_points_validate_before_launching(lib):
     """Workspace of the BF16 depthwise weight gradient (parts x C x Kh x Kw
     floats, rounded up to 256 bytes) and descriptor or pointer errors
     returned without a launch."""
-    d = mqv.dw_desc(16, 32, 20, 20, 3, 3, 1, 1)       # 400 pixels: 16 parts
-    assert mqv.dw_wgrad_workspace_bytes(d) == 16 * 32 * 9 * 4
-    d = mqv.dw_desc(32, 2, 56, 56, 3, 3, 1, 1)        # 3136 pixels x 8 lanes / 1024: 25 parts
-    assert mqv.dw_wgrad_workspace_bytes(d) == 2048    # 25 x 18 x 4 = 1800, rounded up
+    d = mqv.dw_desc(16, 32, 20, 20, 3, 3, 1, 1)       # 400 pixels: 64 parts
+    assert mqv.dw_wgrad_workspace_bytes(d) == 64 * 32 * 9 * 4
+    d = mqv.dw_desc(32, 2, 56, 56, 3, 3, 1, 1)        # 3136 pixels x 8 lanes / 512 needs 49; 64 spread the threads
+    assert mqv.dw_wgrad_workspace_bytes(d) == 4608    # 64 x 18 x 4
     for bad in (mqv.dw_desc(6, 2, 4, 4, 3, 3, 1, 1), mqv.dw_desc(4, 2, 4, 4, 3, 3, 0, 1),
                 mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 3), mqv.dw_desc(4, 0, 4, 4, 3, 3, 1, 1),
                 mqv.dw_desc(4, 2, 2, 2, 5, 5, 1, 1)):

@@ -56,6 +56,11 @@ SMALL = [
     ("s2_one_row", O.ConvShape(4, 8, 36, 1, 7, 3, 3, 2, 1), "nvfp6"),
     ("s2_m160_two_m_tiles", O.ConvShape(8, 160, 64, 9, 8, 3, 3, 2, 1), "nvfp4"),
     ("deep_cin", O.ConvShape(8, 256, 32, 4, 4, 3, 3, 1, 1), "nvfp4"),
+    # 4-input-channel stems with N % 16 == 0: the input gradient runs on CUDA
+    # cores (conv_narrow_dgrad_kernel), stride 2 and 1, both formats
+    ("stem_cin4_n16_s2_fp6", O.ConvShape(16, 4, 16, 12, 12, 3, 3, 2, 1), "nvfp6"),
+    ("stem_cin4_n32_s2", O.ConvShape(32, 4, 32, 9, 10, 3, 3, 2, 1), "nvfp4"),
+    ("stem_cin4_n16_5x5_s1", O.ConvShape(16, 4, 8, 7, 7, 5, 5, 1, 2), "nvfp4"),
     # stride-1 shapes of the kernel-row halo path (N | 256, N % 8 == 0, 64-channel chunks)
     ("halo_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp4"),
     ("halo_n32_two_m_tiles", O.ConvShape(32, 128, 192, 5, 9, 3, 3, 1, 1), "nvfp4"),

@@ -23,6 +23,7 @@ CASES = [
     ("tiny_3x3_s1_p0", O.ConvShape(4, 16, 16, 8, 8, 3, 3, 1, 0), "nvfp4"),       # generic kernel
     ("ragged_3x3_s2_p1", O.ConvShape(8, 24, 40, 9, 9, 3, 3, 2, 1), "nvfp4"),     # strided
     ("cin4_3x3_s2_fp6", O.ConvShape(4, 4, 16, 12, 12, 3, 3, 2, 1), "nvfp6"),
+    ("stem_cin4_n16_s2_fp6", O.ConvShape(16, 4, 16, 12, 12, 3, 3, 2, 1), "nvfp6"),   # CUDA-core dgrad
     ("halo_n64_ragged_row", O.ConvShape(64, 64, 64, 6, 10, 3, 3, 1, 1), "nvfp4"),  # halo kernel
     ("halo_n32_two_m_tiles", O.ConvShape(32, 128, 192, 5, 9, 3, 3, 1, 1), "nvfp6"),
 ]
