@@ -190,11 +190,18 @@ def sampled_check(layer: workloads.Layer, nsamp=96, full_wgrad=False):
         got.append(gx[hi, wi, ci, n]); ref.append(acc * Tw * Tg); S.append(sacc * Tw * Tg)
     assert_close(np.array(got), np.array(ref), np.array(S), f"{layer.name} dgrad sampled")
     if full_wgrad:                                          # weight-gradient samples
-        Xcv = O.code_values(O.quantize(X.numpy().reshape(s.x_view()), of, O.RNE)).reshape(X.shape)
-        Gcv = O.code_values(O.quantize(G.numpy().reshape(s.gy_view()), of, O.SR, seed)).reshape(G.shape)
+        oqx = O.quantize(X.numpy().reshape(s.x_view()), of, O.RNE)
+        oqg = O.quantize(G.numpy().reshape(s.gy_view()), of, O.SR, seed)
+        # the whole quantized X and G_Y, byte for byte, at full size
+        for what, q, oq in (("X", qx, oqx), ("G_Y", qg, oqg)):
+            assert np.float32(q.tscale.item()) == np.float32(oq.T), what
+            assert np.array_equal(q.scales.cpu().numpy(), oq.scales.reshape(-1)), f"{layer.name} {what} scales"
+            assert np.array_equal(q.codes.cpu().numpy(), O.pack_codes(oq.codes, of)), f"{layer.name} {what} codes"
+        Xcv = O.code_values(oqx).reshape(X.shape)
+        Gcv = O.code_values(oqg).reshape(G.shape)
         gw = gw.reshape(s.Cout, s.Kh, s.Kw, s.Cin)
         got, ref, S = [], [], []
-        for _ in range(max(16, nsamp // 4)):
+        for _ in range(max(32, nsamp // 2)):
             co, kh, kw, ci = (int(rng.integers(d)) for d in (s.Cout, s.Kh, s.Kw, s.Cin))
             v, sa = O.wgrad_at(Gcv, Xcv, s, co, kh, kw, ci)
             got.append(gw[co, kh, kw, ci]); ref.append(v * Tg * Tx); S.append(sa * Tg * Tx)
@@ -210,7 +217,8 @@ BODY = workloads.resnet18_body()
 
 @pytest.mark.parametrize("layer", BODY, ids=[l.name for l in BODY])
 def test_resnet18_body_full_size_sampled(layer):
-    sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (4, 8, 15))
+    # the weight gradient and the whole quantized operands on every layer
+    sampled_check(layer, nsamp=48, full_wgrad=True)
 
 
 YOLO = workloads.yolov8n_mix()
@@ -218,7 +226,9 @@ YOLO = workloads.yolov8n_mix()
 
 @pytest.mark.parametrize("layer", YOLO, ids=[l.name for l in YOLO])
 def test_yolov8n_full_size_sampled(layer):
-    sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (3, 6, 17))
+    # NVFP6 at 640²: the weight gradient and the whole quantized operands on
+    # the stem, the narrow early layers and one layer per later stage
+    sampled_check(layer, nsamp=48, full_wgrad=layer.seed in (0, 1, 3, 7, 17))
 
 
 def test_concurrent_passes_match_serial():
