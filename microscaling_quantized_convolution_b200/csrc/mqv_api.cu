@@ -219,7 +219,7 @@ struct ConvPlan {
   HaloGeom g;
   bool wgk;             // stride-1 wgrad with the taps of a kernel row sharing operands
   WgkGeom wg;
-  bool narrow;          // dgrad of a narrow layer on CUDA cores (conv_narrow_dgrad_kernel)
+  bool narrow;          // dgrad of a 4-channel stem on CUDA cores (conv_narrow_dgrad_kernel)
   bool tr;              // generic fwd/dgrad on transposed tiles (M <= 128)
   int bn;               // 128 or 256 columns per tile
   int nu;               // batch items per producer unit: 8, or 4 when N % 8 != 0

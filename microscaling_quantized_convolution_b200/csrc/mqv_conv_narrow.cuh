@@ -1,4 +1,4 @@
-// Input gradient of narrow layers on CUDA cores (MicroQonv summary,
+// Input gradient of 4-channel stems on CUDA cores (MicroQonv summary,
 // onedev.kr/papers/182, section "무엇과 다른가": G_X' = W^T·G_Y, then
 // col2im, here gathered directly).
 //
