@@ -1272,6 +1272,100 @@ mqv_status plan_dw(const mqv_dw_desc* d, DwGeom* g) {
 
 unsigned dw_grid(int64_t total) { return static_cast<unsigned>((total + kDwThreads - 1) / kDwThreads); }
 
+// Tiles of dw_tile_kernel.  The staged window plus the weights stay within
+// 56 KB of shared memory (four CTAs per SM, as the kernel's register bound
+// allows); the first tile shape from 8 x 8 down, and the most channels per
+// tile (a divisor of C, at most 32), that give at least four CTAs per SM win;
+// if none does, the fitting choice with the most CTAs.  3x3 filters (forward
+// at stride 1 or 2, input gradient at stride 1) take the row path, whose
+// tiles are 8 wide.  N > 1024 (more than 256 batch quads per channel) has no
+// tile.
+constexpr int kDwTileSmem = 56 * 1024;
+constexpr int64_t kDwTileMinCtas = 4 * 148;
+
+void dw_tile_window(const DwGeom& g, bool dgrad, int th, int tw, int* ih, int* iw) {
+  const int s = (int)g.stride, Kh = (int)g.Kh, Kw = (int)g.Kw;
+  if (dgrad) {
+    // G_Y rows r0 .. r0 + (th + Kh + s - 3) / s: see dw_tile_kernel
+    *ih = (th + Kh + s - 3) / s + 1;
+    *iw = (tw + Kw + s - 3) / s + 1;
+  } else {
+    *ih = (th - 1) * s + Kh;
+    *iw = (tw - 1) * s + Kw;
+  }
+}
+
+int64_t dw_tile_smem(const DwGeom& g, int ih, int iw, int cg) {
+  return ((cg * g.Kh * g.Kw * 4 + 15) & ~int64_t{15}) + (int64_t)ih * iw * cg * g.N * 2;
+}
+
+bool plan_dw_tile(const DwGeom& g, bool dgrad, DwTile* t) {
+  static const int shapes[][2] = {{8, 8}, {4, 8}, {4, 4}, {2, 4}, {2, 2}, {1, 2}, {1, 1}};
+  static const int rows3_shapes[][2] = {{8, 8}, {4, 8}, {2, 8}, {1, 8}};
+  t->rows3 = g.Kh == 3 && g.Kw == 3 && (dgrad ? g.stride == 1 : g.stride <= 2);
+  const int nq = (int)(g.N / 4);
+  if (nq > kDwThreads) return false;
+  const int out_h = (int)(dgrad ? g.H : g.Ho), out_w = (int)(dgrad ? g.W : g.Wo);
+  int64_t best_ctas = 0;
+  bool found = false;
+  const int nshapes = t->rows3 ? 4 : 7;
+  for (int si = 0; si < nshapes; ++si) {
+    const int th = t->rows3 ? rows3_shapes[si][0] : shapes[si][0];
+    const int tw = t->rows3 ? rows3_shapes[si][1] : shapes[si][1];
+    int ih, iw;
+    dw_tile_window(g, dgrad, th, tw, &ih, &iw);
+    const int64_t tiles = (int64_t)((out_h + th - 1) / th) * ((out_w + tw - 1) / tw);
+    for (int c = 32; c >= 1; --c) {
+      if (g.C % c || c * nq > kDwThreads || dw_tile_smem(g, ih, iw, c) > kDwTileSmem) continue;
+      const int64_t ctas = tiles * (g.C / c);
+      if (ctas > best_ctas) {
+        best_ctas = ctas;
+        found = true;
+        t->th = th;
+        t->tw = tw;
+        t->cg = c;
+        t->ih = ih;
+        t->iw = iw;
+      }
+      if (ctas >= kDwTileMinCtas) goto chosen;
+    }
+  }
+  if (!found) return false;
+chosen:
+  t->src_h = (int)(dgrad ? g.Ho : g.H);
+  t->src_w = (int)(dgrad ? g.Wo : g.W);
+  t->out_h = out_h;
+  t->out_w = out_w;
+  t->tiles_w = (out_w + t->tw - 1) / t->tw;
+  t->tiles_h = (out_h + t->th - 1) / t->th;
+  t->vec16 = (g.C * g.N) % 8 == 0 && ((int64_t)t->cg * g.N) % 8 == 0;
+  return (int64_t)t->tiles_w * t->tiles_h * (g.C / t->cg) < (int64_t{1} << 31);
+}
+
+template <bool DGRAD, int S, bool ROWS3>
+cudaError_t launch_dw_tile_s(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
+                             cudaStream_t st) {
+  auto kern = dw_tile_kernel<DGRAD, S, ROWS3>;
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(kern, kDwTileSmem, done);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (int64_t)t.tiles_w * t.tiles_h * (g.C / t.cg);
+  kern<<<(unsigned)blocks, kDwThreads, (size_t)dw_tile_smem(g, t.ih, t.iw, t.cg), st>>>(g, t, w, src, out);
+  return cudaGetLastError();
+}
+
+template <bool DGRAD>
+cudaError_t launch_dw_tile(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
+                           cudaStream_t st) {
+  if (t.rows3) {
+    if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, true>(g, t, w, src, out, st);
+    if (!DGRAD) return launch_dw_tile_s<DGRAD, 2, !DGRAD>(g, t, w, src, out, st);
+  }
+  if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, false>(g, t, w, src, out, st);
+  if (g.stride == 2) return launch_dw_tile_s<DGRAD, 2, false>(g, t, w, src, out, st);
+  return launch_dw_tile_s<DGRAD, 0, false>(g, t, w, src, out, st);
+}
+
 }  // namespace
 
 extern "C" mqv_status mqv_dw_wgrad_workspace_size(const mqv_dw_desc* d, size_t* bytes) {
@@ -1289,10 +1383,17 @@ extern "C" mqv_status mqv_dw_fwd(const mqv_dw_desc* d, const void* w, const void
   if (st) return st;
   if (!w || !x || !y || !aligned16(w) || !aligned16(x) || !aligned16(y))
     return fail(MQV_ERR_INVALID_ARG, "w, x and y must be 16-byte aligned device pointers");
-  const int64_t total = dw_fwd_threads(g);
-  dw_fwd_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(x), y);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  DwTile t;
+  if (plan_dw_tile(g, false, &t)) {
+    e = launch_dw_tile<false>(g, t, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(x), y,
+                              static_cast<cudaStream_t>(stream));
+  } else {
+    const int64_t total = dw_fwd_threads(g);
+    dw_fwd_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(x), y);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return cuda_fail(e, "depthwise fwd launch");
   return ok();
 }
@@ -1304,10 +1405,17 @@ extern "C" mqv_status mqv_dw_dgrad(const mqv_dw_desc* d, const void* w, const vo
   if (st) return st;
   if (!w || !gy || !gx || !aligned16(w) || !aligned16(gy) || !aligned16(gx))
     return fail(MQV_ERR_INVALID_ARG, "w, gy and gx must be 16-byte aligned device pointers");
-  const int64_t total = dw_dgrad_threads(g);
-  dw_dgrad_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(gy), gx);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  DwTile t;
+  if (plan_dw_tile(g, true, &t)) {
+    e = launch_dw_tile<true>(g, t, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(gy), gx,
+                             static_cast<cudaStream_t>(stream));
+  } else {
+    const int64_t total = dw_dgrad_threads(g);
+    dw_dgrad_kernel<<<dw_grid(total), kDwThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        g, total, static_cast<const uint16_t*>(w), static_cast<const uint16_t*>(gy), gx);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return cuda_fail(e, "depthwise dgrad launch");
   return ok();
 }

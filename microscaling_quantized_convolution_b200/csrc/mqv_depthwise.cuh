@@ -40,4 +40,181 @@ dw_wgrad_reduce_kernel(const DwGeom g, int64_t total, const float* __restrict__ 
   if (t < total) dw_wgrad_reduce_thread(g, t, partial, gw);
 }
 
+// Spatial tiles.  A CTA takes TH x TW output pixels of CG channels (all N
+// batch items) and stages in shared memory the window of its source tensor
+// those pixels read, IH x IW pixels of CG·N bf16 each (zeros outside the
+// tensor), with asynchronous 8- or 16-byte copies that zero-fill out of
+// range, so every thread has all its copies in flight at once.  Each source
+// pixel then comes from memory once per tile instead of once per tap.
+//   forward:  source x, window origin (ho0·s - p, wo0·s - p), tap (kh, kw) of
+//             output (ho, wo) at window row (ho - ho0)·s + kh;
+//   DGRAD:    source G_Y, the adjoint gathered: G_X pixel (hi, wi) takes tap
+//             (kh, kw) where hi + p - kh is a multiple of s, from G_Y row
+//             (hi + p - kh) / s; window origin r0 = floor((hi0 + p - Kh + 1) / s).
+// Taps run in (kh, kw) order, as in dw_fwd_thread and dw_dgrad_thread; a tap
+// that lands outside the source reads a staged zero (adds +0·w).  Results go
+// out as float4 stores.  S: the stride when it is 1 or 2 (cheap index
+// arithmetic), 0 for any other.  ROWS3: 3x3 filters in tiles 8 wide, one
+// output row per thread (dw_tile_rows3); otherwise a thread takes one output
+// pixel of one (channel, batch quad) lane at a time, taps in runtime loops.
+struct DwTile {
+  int th, tw, cg;          // output pixels per tile (rows, columns), channels per tile
+  int ih, iw;              // staged window, pixels (rows, columns)
+  int src_h, src_w;        // extent of the source (x, or G_Y for the input gradient)
+  int out_h, out_w;        // extent of the output
+  int tiles_w, tiles_h;    // tiles along the output width and height
+  int vec16;               // 1: 16-byte copies (C·N and CG·N multiples of 8), else 8-byte
+  int rows3;               // 1: the 3x3 row path (tw = 8)
+};
+
+__device__ __forceinline__ int dw_floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// 3x3 filters, the forward pass at stride S and the input gradient at stride
+// 1, tiles 8 pixels wide: a thread takes one output row of the tile for one
+// (channel, batch quad) lane, keeps its nine weights and the row's 8 x 4
+// sums in registers, and streams the staged source columns of each kernel
+// row once (7·S + 3 of them), adding each into every output that reads it.
+// An output still sees its taps in (kh, kw) order: the forward pass walks
+// the columns left to right, the input gradient (a correlation with the
+// flipped filter) right to left.
+template <bool DGRAD, int S>
+__device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int oh0, int ow0, const float* wsh,
+                                              const uint16_t* xs, float* out, int64_t out_pix_stride,
+                                              int pix_elems) {
+  constexpr int TW = 8, NC = 7 * S + 3;
+  const int nq = N >> 2, lanes = t.cg * nq;
+  for (int u = threadIdx.x; u < t.th * lanes; u += kDwThreads) {
+    const int oy = u / lanes, lane = u - oy * lanes;
+    const int c = lane / nq, q = lane - c * nq;
+    const int oh = oh0 + oy;
+    if (oh >= t.out_h) continue;
+    float wr[9];
+#pragma unroll
+    for (int k = 0; k < 9; ++k) wr[k] = wsh[c * 9 + k];
+    float acc[TW][4];
+#pragma unroll
+    for (int o = 0; o < TW; ++o)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[o][j] = 0.0f;
+    const uint16_t* xl = xs + c * N + 4 * q;
+#pragma unroll
+    for (int kh = 0; kh < 3; ++kh) {
+      const int row = DGRAD ? oy + 2 - kh : oy * S + kh;
+      const uint16_t* rp = xl + row * t.iw * pix_elems;
+#pragma unroll
+      for (int jj = 0; jj < NC; ++jj) {
+        const int j = DGRAD ? NC - 1 - jj : jj;
+        const uint2 v = *reinterpret_cast<const uint2*>(rp + j * pix_elems);
+        const float x[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                            __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u)};
+#pragma unroll
+        for (int kw = 0; kw < 3; ++kw) {
+          // the output that reads column j through tap kw
+          const int o = DGRAD ? j + kw - 2 : (j - kw) / S;
+          if (DGRAD ? (o < 0 || o >= TW) : (j < kw || (j - kw) % S || o >= TW)) continue;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[o][e] = __fmaf_rn(wr[kh * 3 + kw], x[e], acc[o][e]);
+        }
+      }
+    }
+    float* orow = out + (static_cast<int64_t>(oh) * t.out_w + ow0) * out_pix_stride + c * N + 4 * q;
+#pragma unroll
+    for (int o = 0; o < TW; ++o)
+      if (ow0 + o < t.out_w)
+        *reinterpret_cast<float4*>(orow + o * out_pix_stride) = make_float4(acc[o][0], acc[o][1], acc[o][2], acc[o][3]);
+  }
+}
+
+template <bool DGRAD, int S, bool ROWS3>
+__global__ void __launch_bounds__(kDwThreads, 4)
+dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, const uint16_t* __restrict__ src,
+               float* __restrict__ out) {
+  extern __shared__ __align__(16) unsigned char dw_smem[];
+  const int C = static_cast<int>(g.C), N = static_cast<int>(g.N);
+  const int Kh = static_cast<int>(g.Kh), Kw = static_cast<int>(g.Kw), p = static_cast<int>(g.pad);
+  const int s = S ? S : static_cast<int>(g.stride);
+  const int bw = blockIdx.x % t.tiles_w;
+  const int r = blockIdx.x / t.tiles_w;
+  const int bh = r % t.tiles_h, cgi = r / t.tiles_h;
+  const int oh0 = bh * t.th, ow0 = bw * t.tw, c0 = cgi * t.cg;
+  const int r0 = DGRAD ? dw_floordiv(oh0 + p - Kh + 1, s) : oh0 * s - p;
+  const int q0 = DGRAD ? dw_floordiv(ow0 + p - Kw + 1, s) : ow0 * s - p;
+  const int pix_elems = t.cg * N;                 // bf16 per staged pixel
+  float* wsh = reinterpret_cast<float*>(dw_smem);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(dw_smem + ((t.cg * Kh * Kw * 4 + 15) & ~15));
+  // the window: asynchronous copies, zero-filled outside the source
+  {
+    const int vb = t.vec16 ? 8 : 4;               // bf16 per copy
+    const int v_per_pix = pix_elems / vb;
+    const int ncopy = t.ih * t.iw * v_per_pix;
+    const uint32_t xs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+    for (int e = threadIdx.x; e < ncopy; e += kDwThreads) {
+      const int pix = e / v_per_pix, v = e - pix * v_per_pix;
+      const int y = pix / t.iw, x = pix - y * t.iw;
+      const int sh = r0 + y, sw = q0 + x;
+      const bool in = sh >= 0 && sh < t.src_h && sw >= 0 && sw < t.src_w;
+      const uint16_t* gp = in ? src + (static_cast<int64_t>(sh) * t.src_w + sw) * C * N +
+                                    static_cast<int64_t>(c0) * N + v * vb
+                              : src;
+      const uint32_t dst = xs_addr + static_cast<uint32_t>((pix * pix_elems + v * vb) * 2);
+      if (t.vec16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(gp), "r"(in ? 16 : 0)
+                     : "memory");
+      else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(gp), "r"(in ? 8 : 0)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  }
+  for (int e = threadIdx.x; e < t.cg * Kh * Kw; e += kDwThreads) wsh[e] = dw_bf16(w[c0 * Kh * Kw + e]);
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  __syncthreads();
+  if constexpr (ROWS3) {
+    dw_tile_rows3<DGRAD, S>(t, N, oh0, ow0, wsh, xs, out + static_cast<int64_t>(c0) * N, static_cast<int64_t>(C) * N,
+                            pix_elems);
+    return;
+  }
+  const int nq = N >> 2, lanes = t.cg * nq;       // lanes <= kDwThreads (host-checked)
+  const int pstep = kDwThreads / lanes;
+  if (threadIdx.x >= pstep * lanes) return;
+  const int lane = threadIdx.x % lanes, c = lane / nq, q = lane - c * nq;
+  const float* wc = wsh + c * Kh * Kw;
+  const uint16_t* xl = xs + c * N + 4 * q;
+  float* ol = out + static_cast<int64_t>(c0 + c) * N + 4 * q;
+  for (int pix = threadIdx.x / lanes; pix < t.th * t.tw; pix += pstep) {
+    const int oy = pix / t.tw, ox = pix - oy * t.tw;
+    const int oh = oh0 + oy, ow = ow0 + ox;
+    if (oh >= t.out_h || ow >= t.out_w) continue;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int kh = 0; kh < Kh; ++kh) {
+      int row;
+      if (DGRAD) {
+        const int rel = oh + p - kh - r0 * s;     // >= 0 inside the window
+        if (S != 1 && rel % s) continue;
+        row = rel / s;
+      } else {
+        row = oy * s + kh;
+      }
+      for (int kw = 0; kw < Kw; ++kw) {
+        int col;
+        if (DGRAD) {
+          const int rel = ow + p - kw - q0 * s;
+          if (S != 1 && rel % s) continue;
+          col = rel / s;
+        } else {
+          col = ox * s + kw;
+        }
+        const float wv = wc[kh * Kw + kw];
+        const uint2 v = *reinterpret_cast<const uint2*>(xl + (row * t.iw + col) * pix_elems);
+        acc[0] = __fmaf_rn(wv, __uint_as_float(v.x << 16), acc[0]);
+        acc[1] = __fmaf_rn(wv, __uint_as_float(v.x & 0xFFFF0000u), acc[1]);
+        acc[2] = __fmaf_rn(wv, __uint_as_float(v.y << 16), acc[2]);
+        acc[3] = __fmaf_rn(wv, __uint_as_float(v.y & 0xFFFF0000u), acc[3]);
+      }
+    }
+    *reinterpret_cast<float4*>(ol + (static_cast<int64_t>(oh) * t.out_w + ow) * C * N) =
+        make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+}
+
 }  // namespace mqv

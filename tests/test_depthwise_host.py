@@ -21,8 +21,10 @@ CSRC = os.path.join(ROOT, "microscaling_quantized_convolution_b200", "csrc")
 SHAPES = [(4, 3, 7, 9, 3, 3, 1, 1), (8, 5, 9, 7, 3, 3, 2, 1), (4, 6, 10, 10, 5, 5, 2, 2),
           (12, 4, 6, 6, 3, 1, 1, 0), (4, 7, 5, 5, 1, 1, 1, 0), (16, 2, 1, 8, 1, 3, 1, 0),
           (4, 3, 40, 36, 3, 3, 1, 1)]
-# larger layers the GPU test adds (a 80x80 and a strided 5x5 one)
-GPU_LARGE = [(16, 64, 80, 80, 3, 3, 1, 1), (16, 32, 40, 40, 5, 5, 2, 2)]
+# larger layers the GPU test adds: a 80x80 and a strided 5x5 one, one whose
+# 8x8 output tiles end ragged at stride 2, and one at stride 3
+GPU_LARGE = [(16, 64, 80, 80, 3, 3, 1, 1), (16, 32, 40, 40, 5, 5, 2, 2), (16, 64, 83, 77, 3, 3, 2, 1),
+             (8, 64, 50, 47, 5, 5, 3, 2)]
 
 
 @pytest.fixture(scope="module")
