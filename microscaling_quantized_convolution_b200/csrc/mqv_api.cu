@@ -1276,9 +1276,8 @@ unsigned dw_grid(int64_t total) { return static_cast<unsigned>((total + kDwThrea
 // 56 KB of shared memory (four CTAs per SM, as the kernel's register bound
 // allows); the first tile shape from 8 x 8 down, and the most channels per
 // tile (a divisor of C, at most 32), that give at least four CTAs per SM win;
-// if none does, the fitting choice with the most CTAs.  3x3 filters (forward
-// at stride 1 or 2, input gradient at stride 1) take the row path, whose
-// tiles are 8 wide.  N > 1024 (more than 256 batch quads per channel) has no
+// if none does, the fitting choice with the most CTAs.  3x3 filters at
+// stride 1 or 2 take the row path, whose tiles are 8 wide.  N > 1024 (more than 256 batch quads per channel) has no
 // tile.
 constexpr int kDwTileSmem = 56 * 1024;
 constexpr int64_t kDwTileMinCtas = 4 * 148;
@@ -1302,7 +1301,7 @@ int64_t dw_tile_smem(const DwGeom& g, int ih, int iw, int cg) {
 bool plan_dw_tile(const DwGeom& g, bool dgrad, DwTile* t) {
   static const int shapes[][2] = {{8, 8}, {4, 8}, {4, 4}, {2, 4}, {2, 2}, {1, 2}, {1, 1}};
   static const int rows3_shapes[][2] = {{8, 8}, {4, 8}, {2, 8}, {1, 8}};
-  t->rows3 = g.Kh == 3 && g.Kw == 3 && (dgrad ? g.stride == 1 : g.stride <= 2);
+  t->rows3 = g.Kh == 3 && g.Kw == 3 && g.stride <= 2;
   const int nq = (int)(g.N / 4);
   if (nq > kDwThreads) return false;
   const int out_h = (int)(dgrad ? g.H : g.Ho), out_w = (int)(dgrad ? g.W : g.Wo);
@@ -1359,7 +1358,7 @@ cudaError_t launch_dw_tile(const DwGeom& g, const DwTile& t, const uint16_t* w, 
                            cudaStream_t st) {
   if (t.rows3) {
     if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, true>(g, t, w, src, out, st);
-    if (!DGRAD) return launch_dw_tile_s<DGRAD, 2, !DGRAD>(g, t, w, src, out, st);
+    if (g.stride == 2) return launch_dw_tile_s<DGRAD, 2, true>(g, t, w, src, out, st);
   }
   if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, false>(g, t, w, src, out, st);
   if (g.stride == 2) return launch_dw_tile_s<DGRAD, 2, false>(g, t, w, src, out, st);

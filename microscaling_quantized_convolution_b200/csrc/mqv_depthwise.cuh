@@ -69,18 +69,42 @@ struct DwTile {
 
 __device__ __forceinline__ int dw_floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
 
-// 3x3 filters, the forward pass at stride S and the input gradient at stride
-// 1, tiles 8 pixels wide: a thread takes one output row of the tile for one
-// (channel, batch quad) lane, keeps its nine weights and the row's 8 x 4
+// One staged G_Y row of the stride-2 input gradient into the 8 sums of a
+// G_X row.  The tile starts at an even column, so G_X column ox takes tap kw
+// when ox + P + kw is even (P = p mod 2), from staged column
+// (ox + P + 2 - kw) / 2; the columns are walked right to left so that each
+// output sees kw in ascending order.
+template <int P>
+__device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_elems, const float* wk, float (&acc)[8][4]) {
+#pragma unroll
+  for (int jj = 0; jj < 6; ++jj) {
+    const int j = 5 - jj;
+    const uint2 v = *reinterpret_cast<const uint2*>(rp + j * pix_elems);
+    const float x[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                        __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u)};
+#pragma unroll
+    for (int kw = 0; kw < 3; ++kw) {
+      const int o = 2 * j + kw - P - 2;
+      if (o < 0 || o >= 8) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[o][e] = __fmaf_rn(wk[kw], x[e], acc[o][e]);
+    }
+  }
+}
+
+// 3x3 filters in tiles 8 pixels wide (the forward pass at stride S, the
+// input gradient at stride S): a thread takes one output row of the tile for
+// one (channel, batch quad) lane, keeps its nine weights and the row's 8 x 4
 // sums in registers, and streams the staged source columns of each kernel
-// row once (7·S + 3 of them), adding each into every output that reads it.
-// An output still sees its taps in (kh, kw) order: the forward pass walks
-// the columns left to right, the input gradient (a correlation with the
-// flipped filter) right to left.
+// row once, adding each into every output that reads it.  An output still
+// sees its taps in (kh, kw) order: the forward pass walks the columns left
+// to right, the input gradient right to left (at stride 1 a correlation
+// with the flipped filter; at stride 2 a G_X row takes kernel rows kh with
+// oh + p - kh even, from G_Y row (oh + p - kh) / 2).
 template <bool DGRAD, int S>
-__device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int oh0, int ow0, const float* wsh,
-                                              const uint16_t* xs, float* out, int64_t out_pix_stride,
-                                              int pix_elems) {
+__device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int p, int r0, int oh0, int ow0,
+                                              const float* wsh, const uint16_t* xs, float* out,
+                                              int64_t out_pix_stride, int pix_elems) {
   constexpr int TW = 8, NC = 7 * S + 3;
   const int nq = N >> 2, lanes = t.cg * nq;
   for (int u = threadIdx.x; u < t.th * lanes; u += kDwThreads) {
@@ -97,6 +121,17 @@ __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int oh0, i
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[o][j] = 0.0f;
     const uint16_t* xl = xs + c * N + 4 * q;
+    if constexpr (DGRAD && S == 2) {
+      for (int kh = 0; kh < 3; ++kh) {
+        const int tpos = oh + p - kh;
+        if (tpos & 1) continue;
+        const uint16_t* rp = xl + ((tpos - 2 * r0) >> 1) * t.iw * pix_elems;
+        if (p & 1)
+          dw_dgrad2_row<1>(rp, pix_elems, wr + 3 * kh, acc);
+        else
+          dw_dgrad2_row<0>(rp, pix_elems, wr + 3 * kh, acc);
+      }
+    } else {
 #pragma unroll
     for (int kh = 0; kh < 3; ++kh) {
       const int row = DGRAD ? oy + 2 - kh : oy * S + kh;
@@ -116,6 +151,7 @@ __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int oh0, i
           for (int e = 0; e < 4; ++e) acc[o][e] = __fmaf_rn(wr[kh * 3 + kw], x[e], acc[o][e]);
         }
       }
+    }
     }
     float* orow = out + (static_cast<int64_t>(oh) * t.out_w + ow0) * out_pix_stride + c * N + 4 * q;
 #pragma unroll
@@ -170,7 +206,7 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
   asm volatile("cp.async.wait_all;\n" ::: "memory");
   __syncthreads();
   if constexpr (ROWS3) {
-    dw_tile_rows3<DGRAD, S>(t, N, oh0, ow0, wsh, xs, out + static_cast<int64_t>(c0) * N, static_cast<int64_t>(C) * N,
+    dw_tile_rows3<DGRAD, S>(t, N, p, r0, oh0, ow0, wsh, xs, out + static_cast<int64_t>(c0) * N, static_cast<int64_t>(C) * N,
                             pix_elems);
     return;
   }
