@@ -375,13 +375,14 @@ mqv_status mqv_dw_fwd(const mqv_dw_desc* d, const void* w, const void* x, float*
  * whose output pixel exists of w[c][kh][kw]·gy[ho][wo][c][n]. */
 mqv_status mqv_dw_dgrad(const mqv_dw_desc* d, const void* w, const void* gy, float* gx, void* stream);
 
-/* Workspace bytes of mqv_dw_wgrad (the partial sums of its (ho, wo) parts).
- * Host-only. */
+/* Workspace bytes of mqv_dw_wgrad (the partial sums of its (ho, wo) parts:
+ * for 3x3 filters at stride 1 or 2 one per spatial tile of the output, 8
+ * pixels wide; otherwise one per range of output pixels).  Host-only. */
 mqv_status mqv_dw_wgrad_workspace_size(const mqv_dw_desc* d, size_t* bytes);
 
 /* gw[c][kh][kw] = sum_{ho,wo,n} gy[ho][wo][c][n]·x[ho·stride+kh-pad][wo·stride+kw-pad][c][n]:
- * partial sums over ranges of output pixels into ws, then added in range
- * order.  ws: at least mqv_dw_wgrad_workspace_size bytes. */
+ * partial sums over spatial tiles (or ranges) of output pixels into ws, then
+ * added in a fixed order.  ws: at least mqv_dw_wgrad_workspace_size bytes. */
 mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const void* x, float* gw, void* ws,
                         size_t ws_bytes, void* stream);
 

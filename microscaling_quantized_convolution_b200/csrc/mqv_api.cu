@@ -1341,6 +1341,60 @@ chosen:
   return (int64_t)t->tiles_w * t->tiles_h * (g.C / t->cg) < (int64_t{1} << 31);
 }
 
+// Tiles of dw_wgrad_tile_kernel (3x3 filters, stride 1 or 2): the staged x
+// window, G_Y tile and the CTA's 256 x 9 sums within 56 KB; channels per
+// tile such that lanes (channels x batch quads) divide 256.  Of the tile
+// shapes 8 wide and the channel counts, the one with the most working
+// threads (CTAs x the threads that get a row), capped at four full CTAs per
+// SM, wins; ties go to the larger tile and the more channels.
+int64_t dw_wgrad_tile_smem(const DwGeom& g, int th, int ih, int iw, int cg) {
+  return ((int64_t)(ih * iw + th * 8) * cg * g.N * 2 + 15) / 16 * 16 + (int64_t)kDwThreads * 9 * 4;
+}
+
+bool plan_dw_wgrad_tile(const DwGeom& g, DwTile* t) {
+  if (g.Kh != 3 || g.Kw != 3 || g.stride > 2) return false;
+  const int nq = (int)(g.N / 4);
+  if (nq > kDwThreads) return false;
+  const int s = (int)g.stride;
+  int64_t best = 0;
+  for (int th : {8, 4, 2, 1}) {
+    const int ih = (th - 1) * s + 3, iw = 7 * s + 3;
+    const int64_t tiles = (int64_t)((g.Ho + th - 1) / th) * ((g.Wo + 7) / 8);
+    for (int c = 32; c >= 1; --c) {
+      const int lanes = c * nq;
+      if (g.C % c || kDwThreads % lanes || dw_wgrad_tile_smem(g, th, ih, iw, c) > kDwTileSmem) continue;
+      const int64_t rows = std::min<int64_t>(kDwThreads / lanes, th);
+      const int64_t score = std::min<int64_t>(tiles * (g.C / c) * rows * lanes, kDwTileMinCtas * kDwThreads);
+      if (score > best) {
+        best = score;
+        t->th = th;
+        t->tw = 8;
+        t->cg = c;
+        t->ih = ih;
+        t->iw = iw;
+      }
+    }
+  }
+  if (best == 0) return false;
+  t->src_h = (int)g.H;
+  t->src_w = (int)g.W;
+  t->out_h = (int)g.Ho;
+  t->out_w = (int)g.Wo;
+  t->tiles_w = (t->out_w + 7) / 8;
+  t->tiles_h = (t->out_h + t->th - 1) / t->th;
+  t->vec16 = (g.C * g.N) % 8 == 0 && ((int64_t)t->cg * g.N) % 8 == 0;
+  t->rows3 = 1;
+  return (int64_t)t->tiles_w * t->tiles_h * (g.C / t->cg) < (int64_t{1} << 31);
+}
+
+// Workspace bytes of the weight gradient: the tiles' partial sums, or the
+// parts' of the gather kernel.
+int64_t dw_wgrad_ws_bytes(const DwGeom& g) {
+  DwTile t;
+  const int64_t n = plan_dw_wgrad_tile(g, &t) ? (int64_t)t.tiles_w * t.tiles_h * g.C * 9 : dw_wgrad_threads(g);
+  return n * (int64_t)sizeof(float);
+}
+
 template <bool DGRAD, int S, bool ROWS3>
 cudaError_t launch_dw_tile_s(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
                              cudaStream_t st) {
@@ -1372,7 +1426,7 @@ extern "C" mqv_status mqv_dw_wgrad_workspace_size(const mqv_dw_desc* d, size_t* 
   mqv_status st = plan_dw(d, &g);
   if (st) return st;
   if (!bytes) return fail(MQV_ERR_INVALID_ARG, "null output pointer");
-  *bytes = (size_t)((dw_wgrad_threads(g) * (int64_t)sizeof(float) + 255) / 256 * 256);
+  *bytes = (size_t)((dw_wgrad_ws_bytes(g) + 255) / 256 * 256);
   return ok();
 }
 
@@ -1426,17 +1480,39 @@ extern "C" mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const v
   if (st) return st;
   if (!gy || !x || !gw || !aligned16(gy) || !aligned16(x) || !aligned16(gw))
     return fail(MQV_ERR_INVALID_ARG, "gy, x and gw must be 16-byte aligned device pointers");
-  const int64_t total = dw_wgrad_threads(g);
-  const size_t need = (size_t)total * sizeof(float);
+  const size_t need = (size_t)dw_wgrad_ws_bytes(g);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return fail(MQV_ERR_WORKSPACE, "workspace of %zu bytes required", need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(ws);
-  dw_wgrad_kernel<<<dw_grid(total), kDwThreads, 0, s>>>(g, total, static_cast<const uint16_t*>(gy),
-                                                        static_cast<const uint16_t*>(x), part);
   const int64_t nw = g.C * g.Kh * g.Kw;
-  dw_wgrad_reduce_kernel<<<dw_grid(nw), kDwThreads, 0, s>>>(g, nw, part, gw);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  DwTile t;
+  if (plan_dw_wgrad_tile(g, &t)) {
+    const int64_t blocks = (int64_t)t.tiles_w * t.tiles_h * (g.C / t.cg);
+    const size_t smem = (size_t)dw_wgrad_tile_smem(g, t.th, t.ih, t.iw, t.cg);
+    static bool done1[kMaxDevices] = {}, done2[kMaxDevices] = {};
+    if (g.stride == 1) {
+      e = set_smem(dw_wgrad_tile_kernel<1>, kDwTileSmem, done1);
+      if (e == cudaSuccess)
+        dw_wgrad_tile_kernel<1><<<(unsigned)blocks, kDwThreads, smem, s>>>(
+            g, t, static_cast<const uint16_t*>(gy), static_cast<const uint16_t*>(x), part);
+    } else {
+      e = set_smem(dw_wgrad_tile_kernel<2>, kDwTileSmem, done2);
+      if (e == cudaSuccess)
+        dw_wgrad_tile_kernel<2><<<(unsigned)blocks, kDwThreads, smem, s>>>(
+            g, t, static_cast<const uint16_t*>(gy), static_cast<const uint16_t*>(x), part);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "depthwise wgrad launch");
+    const int64_t parts = (int64_t)t.tiles_w * t.tiles_h;
+    dw_wgrad_tile_reduce<<<dw_grid(nw * 32), kDwThreads, 0, s>>>(parts, nw, part, gw);
+  } else {
+    const int64_t total = dw_wgrad_threads(g);
+    dw_wgrad_kernel<<<dw_grid(total), kDwThreads, 0, s>>>(g, total, static_cast<const uint16_t*>(gy),
+                                                          static_cast<const uint16_t*>(x), part);
+    dw_wgrad_reduce_kernel<<<dw_grid(nw), kDwThreads, 0, s>>>(g, nw, part, gw);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "depthwise wgrad launch");
   return ok();
 }

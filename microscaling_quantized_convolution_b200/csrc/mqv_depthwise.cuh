@@ -69,6 +69,33 @@ struct DwTile {
 
 __device__ __forceinline__ int dw_floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
 
+// Stages rows x cols pixels of a [h][w][C][N] source, origin (r0, q0),
+// channels c0 .. c0 + pix_elems / N - 1, into shared memory at dst
+// ([row][col][pix_elems] bf16) with asynchronous 16- or 8-byte copies; pixels
+// outside the source are zero-filled (a copy of 0 source bytes).  The caller
+// commits and waits.
+__device__ __forceinline__ void dw_stage(uint16_t* dst, const uint16_t* __restrict__ src, int r0, int q0, int rows,
+                                         int cols, int src_h, int src_w, int C, int N, int c0, int pix_elems,
+                                         int vec16) {
+  const int vb = vec16 ? 8 : 4;                   // bf16 per copy
+  const int v_per_pix = pix_elems / vb;
+  const int ncopy = rows * cols * v_per_pix;
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  for (int e = threadIdx.x; e < ncopy; e += kDwThreads) {
+    const int pix = e / v_per_pix, v = e - pix * v_per_pix;
+    const int y = pix / cols, x = pix - y * cols;
+    const int sh = r0 + y, sw = q0 + x;
+    const bool in = sh >= 0 && sh < src_h && sw >= 0 && sw < src_w;
+    const uint16_t* gp =
+        in ? src + (static_cast<int64_t>(sh) * src_w + sw) * C * N + static_cast<int64_t>(c0) * N + v * vb : src;
+    const uint32_t da = base + static_cast<uint32_t>((pix * pix_elems + v * vb) * 2);
+    if (vec16)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(da), "l"(gp), "r"(in ? 16 : 0) : "memory");
+    else
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(da), "l"(gp), "r"(in ? 8 : 0) : "memory");
+  }
+}
+
 // One staged G_Y row of the stride-2 input gradient into the 8 sums of a
 // G_X row.  The tile starts at an even column, so G_X column ox takes tap kw
 // when ox + P + kw is even (P = p mod 2), from staged column
@@ -178,30 +205,8 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
   const int pix_elems = t.cg * N;                 // bf16 per staged pixel
   float* wsh = reinterpret_cast<float*>(dw_smem);
   uint16_t* xs = reinterpret_cast<uint16_t*>(dw_smem + ((t.cg * Kh * Kw * 4 + 15) & ~15));
-  // the window: asynchronous copies, zero-filled outside the source
-  {
-    const int vb = t.vec16 ? 8 : 4;               // bf16 per copy
-    const int v_per_pix = pix_elems / vb;
-    const int ncopy = t.ih * t.iw * v_per_pix;
-    const uint32_t xs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
-    for (int e = threadIdx.x; e < ncopy; e += kDwThreads) {
-      const int pix = e / v_per_pix, v = e - pix * v_per_pix;
-      const int y = pix / t.iw, x = pix - y * t.iw;
-      const int sh = r0 + y, sw = q0 + x;
-      const bool in = sh >= 0 && sh < t.src_h && sw >= 0 && sw < t.src_w;
-      const uint16_t* gp = in ? src + (static_cast<int64_t>(sh) * t.src_w + sw) * C * N +
-                                    static_cast<int64_t>(c0) * N + v * vb
-                              : src;
-      const uint32_t dst = xs_addr + static_cast<uint32_t>((pix * pix_elems + v * vb) * 2);
-      if (t.vec16)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(gp), "r"(in ? 16 : 0)
-                     : "memory");
-      else
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(dst), "l"(gp), "r"(in ? 8 : 0)
-                     : "memory");
-    }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-  }
+  dw_stage(xs, src, r0, q0, t.ih, t.iw, t.src_h, t.src_w, C, N, c0, pix_elems, t.vec16);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
   for (int e = threadIdx.x; e < t.cg * Kh * Kw; e += kDwThreads) wsh[e] = dw_bf16(w[c0 * Kh * Kw + e]);
   asm volatile("cp.async.wait_all;\n" ::: "memory");
   __syncthreads();
@@ -251,6 +256,99 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
     *reinterpret_cast<float4*>(ol + (static_cast<int64_t>(oh) * t.out_w + ow) * C * N) =
         make_float4(acc[0], acc[1], acc[2], acc[3]);
   }
+}
+
+// Weight gradient of 3x3 filters at stride S in the same tiles: a CTA stages
+// the G_Y tile (TH x 8 pixels of CG channels, zeros past the output) and the
+// x window it meets, and writes the tile's sums of G_Y·x for its CG x 9
+// weights to partial[tile][c][kh][kw] (tile = bh·tiles_w + bw).  A thread
+// has a fixed (channel, batch quad) lane and takes the tile's rows
+// r, r + 256 / lanes, ...: it keeps the row's 8 x 4 G_Y values and nine sums
+// in registers and streams each kernel row's x columns once (each product of
+// a G_Y pixel and an x pixel added over the four batch items in order).  The
+// CTA then adds the threads' sums of each weight in a fixed order (row group,
+// then batch quad), and dw_wgrad_tile_reduce adds the tiles' in order.
+template <int S>
+__global__ void __launch_bounds__(kDwThreads, 4)
+dw_wgrad_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ gy,
+                     const uint16_t* __restrict__ x, float* __restrict__ partial) {
+  extern __shared__ __align__(16) unsigned char dw_smem[];
+  constexpr int TW = 8, NC = 7 * S + 3;
+  const int C = static_cast<int>(g.C), N = static_cast<int>(g.N), p = static_cast<int>(g.pad);
+  const int bw = blockIdx.x % t.tiles_w;
+  const int r = blockIdx.x / t.tiles_w;
+  const int bh = r % t.tiles_h, cgi = r / t.tiles_h;
+  const int oh0 = bh * t.th, ow0 = bw * TW, c0 = cgi * t.cg;
+  const int pix_elems = t.cg * N;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(dw_smem);
+  uint16_t* gs = xs + t.ih * t.iw * pix_elems;
+  float* red = reinterpret_cast<float*>(dw_smem + ((t.ih * t.iw + t.th * TW) * pix_elems * 2 + 15) / 16 * 16);
+  dw_stage(xs, x, oh0 * S - p, ow0 * S - p, t.ih, t.iw, t.src_h, t.src_w, C, N, c0, pix_elems, t.vec16);
+  dw_stage(gs, gy, oh0, ow0, t.th, TW, t.out_h, t.out_w, C, N, c0, pix_elems, t.vec16);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  __syncthreads();
+  const int nq = N >> 2, lanes = t.cg * nq;       // lanes divides kDwThreads (host-checked)
+  const int pstep = kDwThreads / lanes;
+  const int lane = threadIdx.x % lanes, c = lane / nq, q = lane - c * nq;
+  float acc[9];
+#pragma unroll
+  for (int k = 0; k < 9; ++k) acc[k] = 0.0f;
+  for (int oy = threadIdx.x / lanes; oy < t.th && oh0 + oy < t.out_h; oy += pstep) {
+    float gv[TW][4];
+    const uint16_t* grow = gs + oy * TW * pix_elems + c * N + 4 * q;
+#pragma unroll
+    for (int o = 0; o < TW; ++o) {
+      const uint2 v = *reinterpret_cast<const uint2*>(grow + o * pix_elems);
+      gv[o][0] = __uint_as_float(v.x << 16);
+      gv[o][1] = __uint_as_float(v.x & 0xFFFF0000u);
+      gv[o][2] = __uint_as_float(v.y << 16);
+      gv[o][3] = __uint_as_float(v.y & 0xFFFF0000u);
+    }
+#pragma unroll
+    for (int kh = 0; kh < 3; ++kh) {
+      const uint16_t* rp = xs + (oy * S + kh) * t.iw * pix_elems + c * N + 4 * q;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) {
+        const uint2 v = *reinterpret_cast<const uint2*>(rp + j * pix_elems);
+        const float xv[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                             __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u)};
+#pragma unroll
+        for (int kw = 0; kw < 3; ++kw) {
+          const int o = (j - kw) / S;
+          if (j < kw || (j - kw) % S || o >= TW) continue;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[kh * 3 + kw] = __fmaf_rn(gv[o][e], xv[e], acc[kh * 3 + kw]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 9; ++k) red[threadIdx.x * 9 + k] = acc[k];
+  __syncthreads();
+  const int tile = bh * t.tiles_w + bw;
+  for (int e = threadIdx.x; e < t.cg * 9; e += kDwThreads) {
+    const int cc = e / 9, k = e - cc * 9;
+    float sum = 0.0f;
+    for (int rr = 0; rr < pstep; ++rr)
+      for (int qq = 0; qq < nq; ++qq) sum += red[(rr * lanes + cc * nq + qq) * 9 + k];
+    partial[(static_cast<int64_t>(tile) * C + c0 + cc) * 9 + k] = sum;
+  }
+}
+
+// gw[i] = the tiles' partial sums of weight i added in tile order: one warp
+// per weight, lane l adding tiles l, l + 32, ... in order, then the 32 lane
+// sums in a fixed tree.
+__global__ void __launch_bounds__(kDwThreads)
+dw_wgrad_tile_reduce(int64_t parts, int64_t per, const float* __restrict__ partial, float* __restrict__ gw) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * kDwThreads + threadIdx.x) / 32;
+  const int l = threadIdx.x & 31;
+  if (i >= per) return;                           // whole warps leave together
+  float s = 0.0f;
+  for (int64_t pt = l; pt < parts; pt += 32) s += partial[pt * per + i];
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) s += __shfl_down_sync(0xFFFFFFFFu, s, d);
+  if (l == 0) gw[i] = s;
 }
 
 }  // namespace mqv

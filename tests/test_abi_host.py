@@ -173,12 +173,15 @@ def test_cuda_path_has_no_cpu_fallback():
 
 def test_depthwise_entry_points_validate_before_launching(lib):
     """Workspace of the BF16 depthwise weight gradient (parts x C x Kh x Kw
-    floats, rounded up to 256 bytes) and descriptor or pointer errors
-    returned without a launch."""
-    d = mqv.dw_desc(16, 32, 20, 20, 3, 3, 1, 1)       # 400 pixels: 64 parts
-    assert mqv.dw_wgrad_workspace_bytes(d) == 64 * 32 * 9 * 4
-    d = mqv.dw_desc(32, 2, 56, 56, 3, 3, 1, 1)        # 3136 pixels x 8 lanes / 512 needs 49; 64 spread the threads
-    assert mqv.dw_wgrad_workspace_bytes(d) == 4608    # 64 x 18 x 4
+    floats, rounded up to 256 bytes: for 3x3 filters at stride 1 or 2 a part
+    per spatial tile, 8 output pixels wide, else a part per range of output
+    pixels) and descriptor or pointer errors returned without a launch."""
+    d = mqv.dw_desc(16, 32, 20, 20, 3, 3, 1, 1)       # 20x20 output in 8x8 tiles: 3 x 3 parts
+    assert mqv.dw_wgrad_workspace_bytes(d) == 10496   # 9 x 32 x 9 x 4 = 10368, rounded up
+    d = mqv.dw_desc(32, 2, 56, 56, 3, 3, 1, 1)        # 56x56 in 8x8 tiles: 49 parts
+    assert mqv.dw_wgrad_workspace_bytes(d) == 3584    # 49 x 18 x 4 = 3528, rounded up
+    d = mqv.dw_desc(16, 32, 40, 40, 5, 5, 2, 2)       # 5x5: 400 output pixels, 64 ranges
+    assert mqv.dw_wgrad_workspace_bytes(d) == 64 * 32 * 25 * 4
     for bad in (mqv.dw_desc(6, 2, 4, 4, 3, 3, 1, 1), mqv.dw_desc(4, 2, 4, 4, 3, 3, 0, 1),
                 mqv.dw_desc(4, 2, 4, 4, 3, 3, 1, 3), mqv.dw_desc(4, 0, 4, 4, 3, 3, 1, 1),
                 mqv.dw_desc(4, 2, 2, 2, 5, 5, 1, 1)):
