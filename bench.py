@@ -1189,6 +1189,32 @@ def run_probe(args):
         sys.exit(1)
 
 
+def run_probe_depthwise(args):
+    """The BF16 depthwise passes (fwd, dgrad, wgrad) of one layer of the
+    depthwise sweep, `args.probe_depthwise` times, for single-kernel ncu
+    captures.  Prints one line; no timing."""
+    import torch
+
+    import microscaling_quantized_convolution_b200 as mqv
+
+    C, H, stv = workloads.DEPTHWISE_SHAPES[args.depthwise_shape]
+    N = workloads.DEPTHWISE_N
+    dev = torch.device("cuda", 0)
+    x, w, gy = (t.to(torch.bfloat16).contiguous()
+                for t in workloads.make_depthwise_inputs(C, H, stv, N, seed=C + H, device=dev))
+    d = mqv.dw_desc(N, C, H, H, 3, 3, stv, 1)
+    for _ in range(args.probe_depthwise):
+        mqv.dw_fwd(d, w, x)
+        mqv.dw_dgrad(d, w, gy)
+        mqv.dw_wgrad(d, gy, x)
+    torch.cuda.synchronize()
+    flags = mqv.device_errors()
+    print(json.dumps({"probe": f"depthwise_c{C}_h{H}_s{stv}_n{N}", "iterations": args.probe_depthwise,
+                      "device_error_flags": flags}))
+    if flags:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1208,6 +1234,10 @@ def main():
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"))
     ap.add_argument("--probe", type=int, default=0,
                     help="run the layer's step this many times for a profiler capture and exit (no timing)")
+    ap.add_argument("--probe-depthwise", type=int, default=0,
+                    help="run one depthwise sweep layer's three passes this many times and exit (no timing)")
+    ap.add_argument("--depthwise-shape", type=int, default=0,
+                    help="index into the depthwise sweep shapes for --probe-depthwise")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.traffic = None
@@ -1216,6 +1246,8 @@ def main():
             args.traffic = json.load(f).get(args.workload)
     if args.probe > 0:
         run_probe(args)
+    elif args.probe_depthwise > 0:
+        run_probe_depthwise(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -898,9 +898,25 @@ mqv_status mqv_quantize_many(const mqv_quantize_job* jobs, int32_t count, void* 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* part = static_cast<float*>(ws);
   amax_many_kernel<<<a, kAmaxThreads, 0, s>>>(plan, part);
-  if (plan.job[0].qa.blocks == MQV_BLOCKS_4X4) quantize_many_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
-  else quantize_many_line_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (plan.job[0].qa.blocks == MQV_BLOCKS_4X4) {
+    // a programmatic dependent of the max pass: its CTAs become resident as
+    // the max pass runs and load their first blocks before they wait for it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(q));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, quantize_many_kernel, plan, static_cast<const float*>(part));
+    if (e != cudaSuccess) return cuda_fail(e, "quantize_many launch");
+  } else {
+    quantize_many_line_kernel<<<q, kQuantThreads, 0, s>>>(plan, part);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize_many launch");
   return ok();
 }

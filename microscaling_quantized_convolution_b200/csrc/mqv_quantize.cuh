@@ -352,6 +352,9 @@ __device__ __forceinline__ void quantize_body(const QuantArgs& qa, const float* 
       load_block(x[i], qa.src, cols, br, w - static_cast<int64_t>(br) * cb);
     }
   }
+  // launched as a programmatic dependent of the max pass (quantize_many),
+  // the amax partials are complete only after this wait; otherwise a no-op
+  pdl_wait_prerequisite();
   __shared__ float red[32];
   const TensorScale<FMT> ts(block_max_of(amax_src, amax_count, red));
   if (cta == 0 && threadIdx.x == 0) *qa.tscale = ts.T;
@@ -548,6 +551,9 @@ __device__ __forceinline__ int job_of(const QuantJobs& jobs, int cta, bool quant
 
 __global__ void __launch_bounds__(kAmaxThreads)
 amax_many_kernel(const __grid_constant__ QuantJobs jobs, float* __restrict__ partial) {
+  // the quantizer that follows may start now: it loads its first blocks and
+  // then waits for this grid (pdl_wait_prerequisite) before reading `partial`
+  pdl_launch_dependents();
   const QuantJob& jb = jobs.job[job_of(jobs, blockIdx.x, false)];
   amax_partial_body(reinterpret_cast<const float4*>(jb.qa.src), jb.qa.rows * jb.qa.cols / 4, partial + blockIdx.x,
                     blockIdx.x - jb.amax_cta0, jb.amax_ctas);
