@@ -81,18 +81,35 @@ __device__ __forceinline__ void dw_stage(uint16_t* dst, const uint16_t* __restri
   const int v_per_pix = pix_elems / vb;
   const int ncopy = rows * cols * v_per_pix;
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  // copy e = (y·cols + x)·v_per_pix + v; each thread steps e by kDwThreads,
+  // so (y, x, v) advance by fixed amounts with at most one carry each
+  // (every tensor has fewer than 2^31 elements, so 32-bit offsets suffice)
+  int pix = threadIdx.x / v_per_pix;
+  int v = threadIdx.x - pix * v_per_pix;
+  int y = pix / cols, x = pix - y * cols;
+  const int dp = kDwThreads / v_per_pix, dv = kDwThreads - dp * v_per_pix;
+  const int dy = dp / cols, dx = dp - dy * cols;
+  const int pix_stride = C * N;
   for (int e = threadIdx.x; e < ncopy; e += kDwThreads) {
-    const int pix = e / v_per_pix, v = e - pix * v_per_pix;
-    const int y = pix / cols, x = pix - y * cols;
     const int sh = r0 + y, sw = q0 + x;
     const bool in = sh >= 0 && sh < src_h && sw >= 0 && sw < src_w;
-    const uint16_t* gp =
-        in ? src + (static_cast<int64_t>(sh) * src_w + sw) * C * N + static_cast<int64_t>(c0) * N + v * vb : src;
-    const uint32_t da = base + static_cast<uint32_t>((pix * pix_elems + v * vb) * 2);
+    const uint16_t* gp = src + (in ? static_cast<uint32_t>((sh * src_w + sw) * pix_stride + c0 * N + v * vb) : 0u);
+    const uint32_t da = base + static_cast<uint32_t>(((y * cols + x) * pix_elems + v * vb) * 2);
     if (vec16)
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(da), "l"(gp), "r"(in ? 16 : 0) : "memory");
     else
       asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(da), "l"(gp), "r"(in ? 8 : 0) : "memory");
+    v += dv;
+    x += dx;
+    y += dy;
+    if (v >= v_per_pix) {
+      v -= v_per_pix;
+      ++x;
+    }
+    if (x >= cols) {
+      x -= cols;
+      ++y;
+    }
   }
 }
 
