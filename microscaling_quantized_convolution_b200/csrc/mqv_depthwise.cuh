@@ -118,6 +118,23 @@ __device__ __forceinline__ void dw_stage(uint16_t* dst, const uint16_t* __restri
 // when ox + P + kw is even (P = p mod 2), from staged column
 // (ox + P + 2 - kw) / 2; the columns are walked right to left so that each
 // output sees kw in ascending order.
+// a[e] = fma(w, x[e], a[e]) for e = 0..3, as two packed fp32 FMAs
+// (fma.rn.f32x2: each lane one IEEE fp32 FMA, the same result as fmaf).
+__device__ __forceinline__ void dw_fma4(float (&a)[4], float w, const float (&x)[4]) {
+  asm("{\n\t.reg .b64 p, q, r;\n\t"
+      "mov.b64 q, {%4, %4};\n\t"
+      "mov.b64 p, {%5, %6};\n\t"
+      "mov.b64 r, {%0, %1};\n\t"
+      "fma.rn.f32x2 r, p, q, r;\n\t"
+      "mov.b64 {%0, %1}, r;\n\t"
+      "mov.b64 p, {%7, %8};\n\t"
+      "mov.b64 r, {%2, %3};\n\t"
+      "fma.rn.f32x2 r, p, q, r;\n\t"
+      "mov.b64 {%2, %3}, r;\n\t}"
+      : "+f"(a[0]), "+f"(a[1]), "+f"(a[2]), "+f"(a[3])
+      : "f"(w), "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]));
+}
+
 template <int P>
 __device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_elems, const float* wk, float (&acc)[8][4]) {
 #pragma unroll
@@ -130,8 +147,7 @@ __device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_elems,
     for (int kw = 0; kw < 3; ++kw) {
       const int o = 2 * j + kw - P - 2;
       if (o < 0 || o >= 8) continue;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[o][e] = __fmaf_rn(wk[kw], x[e], acc[o][e]);
+      dw_fma4(acc[o], wk[kw], x);
     }
   }
 }
@@ -191,8 +207,7 @@ __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int p, int
           // the output that reads column j through tap kw
           const int o = DGRAD ? j + kw - 2 : (j - kw) / S;
           if (DGRAD ? (o < 0 || o >= TW) : (j < kw || (j - kw) % S || o >= TW)) continue;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[o][e] = __fmaf_rn(wr[kh * 3 + kw], x[e], acc[o][e]);
+          dw_fma4(acc[o], wr[kh * 3 + kw], x);
         }
       }
     }
