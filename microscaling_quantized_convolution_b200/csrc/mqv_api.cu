@@ -1403,6 +1403,31 @@ bool plan_dw_wgrad_tile(const DwGeom& g, DwTile* t) {
   return (int64_t)t->tiles_w * t->tiles_h * (g.C / t->cg) < (int64_t{1} << 31);
 }
 
+template <int S, int PIX>
+cudaError_t launch_dw_wgrad_tile_p(const DwGeom& g, const DwTile& t, int64_t blocks, size_t smem, const uint16_t* gy,
+                                   const uint16_t* x, float* part, cudaStream_t st) {
+  static bool done[kMaxDevices] = {};
+  cudaError_t e = set_smem(dw_wgrad_tile_kernel<S, PIX>, kDwTileSmem, done);
+  if (e != cudaSuccess) return e;
+  dw_wgrad_tile_kernel<S, PIX><<<(unsigned)blocks, kDwThreads, smem, st>>>(g, t, gy, x, part);
+  return cudaGetLastError();
+}
+
+// dw_wgrad_tile_kernel with the staged pixel's size as a constant for the
+// common sizes.
+template <int S>
+cudaError_t launch_dw_wgrad_tile(const DwGeom& g, const DwTile& t, int64_t blocks, size_t smem, const uint16_t* gy,
+                                 const uint16_t* x, float* part, cudaStream_t st) {
+  switch (t.cg * (int)g.N) {
+    case 32: return launch_dw_wgrad_tile_p<S, 32>(g, t, blocks, smem, gy, x, part, st);
+    case 64: return launch_dw_wgrad_tile_p<S, 64>(g, t, blocks, smem, gy, x, part, st);
+    case 128: return launch_dw_wgrad_tile_p<S, 128>(g, t, blocks, smem, gy, x, part, st);
+    case 256: return launch_dw_wgrad_tile_p<S, 256>(g, t, blocks, smem, gy, x, part, st);
+    case 512: return launch_dw_wgrad_tile_p<S, 512>(g, t, blocks, smem, gy, x, part, st);
+    default: return launch_dw_wgrad_tile_p<S, 0>(g, t, blocks, smem, gy, x, part, st);
+  }
+}
+
 // Workspace bytes of the weight gradient: the tiles' partial sums, or the
 // parts' of the gather kernel.
 int64_t dw_wgrad_ws_bytes(const DwGeom& g) {
@@ -1411,10 +1436,10 @@ int64_t dw_wgrad_ws_bytes(const DwGeom& g) {
   return n * (int64_t)sizeof(float);
 }
 
-template <bool DGRAD, int S, bool ROWS3>
+template <bool DGRAD, int S, bool ROWS3, int PIX = 0>
 cudaError_t launch_dw_tile_s(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
                              cudaStream_t st) {
-  auto kern = dw_tile_kernel<DGRAD, S, ROWS3>;
+  auto kern = dw_tile_kernel<DGRAD, S, ROWS3, PIX>;
   static bool done[kMaxDevices] = {};
   cudaError_t e = set_smem(kern, kDwTileSmem, done);
   if (e != cudaSuccess) return e;
@@ -1423,12 +1448,27 @@ cudaError_t launch_dw_tile_s(const DwGeom& g, const DwTile& t, const uint16_t* w
   return cudaGetLastError();
 }
 
+// The row path with the staged pixel's size (channels x batch, bf16) as a
+// constant for the common sizes.
+template <bool DGRAD, int S>
+cudaError_t launch_dw_rows3(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
+                            cudaStream_t st) {
+  switch (t.cg * (int)g.N) {
+    case 32: return launch_dw_tile_s<DGRAD, S, true, 32>(g, t, w, src, out, st);
+    case 64: return launch_dw_tile_s<DGRAD, S, true, 64>(g, t, w, src, out, st);
+    case 128: return launch_dw_tile_s<DGRAD, S, true, 128>(g, t, w, src, out, st);
+    case 256: return launch_dw_tile_s<DGRAD, S, true, 256>(g, t, w, src, out, st);
+    case 512: return launch_dw_tile_s<DGRAD, S, true, 512>(g, t, w, src, out, st);
+    default: return launch_dw_tile_s<DGRAD, S, true, 0>(g, t, w, src, out, st);
+  }
+}
+
 template <bool DGRAD>
 cudaError_t launch_dw_tile(const DwGeom& g, const DwTile& t, const uint16_t* w, const uint16_t* src, float* out,
                            cudaStream_t st) {
   if (t.rows3) {
-    if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, true>(g, t, w, src, out, st);
-    if (g.stride == 2) return launch_dw_tile_s<DGRAD, 2, true>(g, t, w, src, out, st);
+    if (g.stride == 1) return launch_dw_rows3<DGRAD, 1>(g, t, w, src, out, st);
+    if (g.stride == 2) return launch_dw_rows3<DGRAD, 2>(g, t, w, src, out, st);
   }
   if (g.stride == 1) return launch_dw_tile_s<DGRAD, 1, false>(g, t, w, src, out, st);
   if (g.stride == 2) return launch_dw_tile_s<DGRAD, 2, false>(g, t, w, src, out, st);
@@ -1507,18 +1547,10 @@ extern "C" mqv_status mqv_dw_wgrad(const mqv_dw_desc* d, const void* gy, const v
   if (plan_dw_wgrad_tile(g, &t)) {
     const int64_t blocks = (int64_t)t.tiles_w * t.tiles_h * (g.C / t.cg);
     const size_t smem = (size_t)dw_wgrad_tile_smem(g, t.th, t.ih, t.iw, t.cg);
-    static bool done1[kMaxDevices] = {}, done2[kMaxDevices] = {};
-    if (g.stride == 1) {
-      e = set_smem(dw_wgrad_tile_kernel<1>, kDwTileSmem, done1);
-      if (e == cudaSuccess)
-        dw_wgrad_tile_kernel<1><<<(unsigned)blocks, kDwThreads, smem, s>>>(
-            g, t, static_cast<const uint16_t*>(gy), static_cast<const uint16_t*>(x), part);
-    } else {
-      e = set_smem(dw_wgrad_tile_kernel<2>, kDwTileSmem, done2);
-      if (e == cudaSuccess)
-        dw_wgrad_tile_kernel<2><<<(unsigned)blocks, kDwThreads, smem, s>>>(
-            g, t, static_cast<const uint16_t*>(gy), static_cast<const uint16_t*>(x), part);
-    }
+    const uint16_t* gyp = static_cast<const uint16_t*>(gy);
+    const uint16_t* xp = static_cast<const uint16_t*>(x);
+    e = g.stride == 1 ? launch_dw_wgrad_tile<1>(g, t, blocks, smem, gyp, xp, part, s)
+                      : launch_dw_wgrad_tile<2>(g, t, blocks, smem, gyp, xp, part, s);
     if (e != cudaSuccess) return cuda_fail(e, "depthwise wgrad launch");
     const int64_t parts = (int64_t)t.tiles_w * t.tiles_h;
     dw_wgrad_tile_reduce<<<dw_grid(nw * 32), kDwThreads, 0, s>>>(parts, nw, part, gw);

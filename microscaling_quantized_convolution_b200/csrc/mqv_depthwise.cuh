@@ -135,8 +135,9 @@ __device__ __forceinline__ void dw_fma4(float (&a)[4], float w, const float (&x)
       : "f"(w), "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]));
 }
 
-template <int P>
-__device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_elems, const float* wk, float (&acc)[8][4]) {
+template <int P, int PIX>
+__device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_rt, const float* wk, float (&acc)[8][4]) {
+  const int pix_elems = PIX ? PIX : pix_rt;
 #pragma unroll
   for (int jj = 0; jj < 6; ++jj) {
     const int j = 5 - jj;
@@ -160,12 +161,16 @@ __device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_elems,
 // sees its taps in (kh, kw) order: the forward pass walks the columns left
 // to right, the input gradient right to left (at stride 1 a correlation
 // with the flipped filter; at stride 2 a G_X row takes kernel rows kh with
-// oh + p - kh even, from G_Y row (oh + p - kh) / 2).
-template <bool DGRAD, int S>
+// oh + p - kh even, from G_Y row (oh + p - kh) / 2).  PIX: the staged
+// pixel's bf16 count (channels x batch) when it is one of the common values,
+// so that every shared-memory offset is a constant; 0 for any other.
+template <bool DGRAD, int S, int PIX>
 __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int p, int r0, int oh0, int ow0,
                                               const float* wsh, const uint16_t* xs, float* out,
-                                              int64_t out_pix_stride, int pix_elems) {
+                                              int64_t out_pix_stride, int pix_rt) {
   constexpr int TW = 8, NC = 7 * S + 3;
+  constexpr int IW = DGRAD ? (S == 1 ? 10 : 6) : NC;   // staged columns (t.iw)
+  const int pix_elems = PIX ? PIX : pix_rt;
   const int nq = N >> 2, lanes = t.cg * nq;
   for (int u = threadIdx.x; u < t.th * lanes; u += kDwThreads) {
     const int oy = u / lanes, lane = u - oy * lanes;
@@ -185,17 +190,17 @@ __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int p, int
       for (int kh = 0; kh < 3; ++kh) {
         const int tpos = oh + p - kh;
         if (tpos & 1) continue;
-        const uint16_t* rp = xl + ((tpos - 2 * r0) >> 1) * t.iw * pix_elems;
+        const uint16_t* rp = xl + ((tpos - 2 * r0) >> 1) * IW * pix_elems;
         if (p & 1)
-          dw_dgrad2_row<1>(rp, pix_elems, wr + 3 * kh, acc);
+          dw_dgrad2_row<1, PIX>(rp, pix_elems, wr + 3 * kh, acc);
         else
-          dw_dgrad2_row<0>(rp, pix_elems, wr + 3 * kh, acc);
+          dw_dgrad2_row<0, PIX>(rp, pix_elems, wr + 3 * kh, acc);
       }
     } else {
 #pragma unroll
     for (int kh = 0; kh < 3; ++kh) {
       const int row = DGRAD ? oy + 2 - kh : oy * S + kh;
-      const uint16_t* rp = xl + row * t.iw * pix_elems;
+      const uint16_t* rp = xl + row * IW * pix_elems;
 #pragma unroll
       for (int jj = 0; jj < NC; ++jj) {
         const int j = DGRAD ? NC - 1 - jj : jj;
@@ -220,7 +225,7 @@ __device__ __forceinline__ void dw_tile_rows3(const DwTile& t, int N, int p, int
   }
 }
 
-template <bool DGRAD, int S, bool ROWS3>
+template <bool DGRAD, int S, bool ROWS3, int PIX = 0>
 __global__ void __launch_bounds__(kDwThreads, 4)
 dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, const uint16_t* __restrict__ src,
                float* __restrict__ out) {
@@ -234,7 +239,7 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
   const int oh0 = bh * t.th, ow0 = bw * t.tw, c0 = cgi * t.cg;
   const int r0 = DGRAD ? dw_floordiv(oh0 + p - Kh + 1, s) : oh0 * s - p;
   const int q0 = DGRAD ? dw_floordiv(ow0 + p - Kw + 1, s) : ow0 * s - p;
-  const int pix_elems = t.cg * N;                 // bf16 per staged pixel
+  const int pix_elems = PIX ? PIX : t.cg * N;     // bf16 per staged pixel
   float* wsh = reinterpret_cast<float*>(dw_smem);
   uint16_t* xs = reinterpret_cast<uint16_t*>(dw_smem + ((t.cg * Kh * Kw * 4 + 15) & ~15));
   dw_stage(xs, src, r0, q0, t.ih, t.iw, t.src_h, t.src_w, C, N, c0, pix_elems, t.vec16);
@@ -243,7 +248,7 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
   asm volatile("cp.async.wait_all;\n" ::: "memory");
   __syncthreads();
   if constexpr (ROWS3) {
-    dw_tile_rows3<DGRAD, S>(t, N, p, r0, oh0, ow0, wsh, xs, out + static_cast<int64_t>(c0) * N, static_cast<int64_t>(C) * N,
+    dw_tile_rows3<DGRAD, S, PIX>(t, N, p, r0, oh0, ow0, wsh, xs, out + static_cast<int64_t>(c0) * N, static_cast<int64_t>(C) * N,
                             pix_elems);
     return;
   }
@@ -300,18 +305,18 @@ dw_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ w, c
 // a G_Y pixel and an x pixel added over the four batch items in order).  The
 // CTA then adds the threads' sums of each weight in a fixed order (row group,
 // then batch quad), and dw_wgrad_tile_reduce adds the tiles' in order.
-template <int S>
+template <int S, int PIX = 0>
 __global__ void __launch_bounds__(kDwThreads, 4)
 dw_wgrad_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict__ gy,
                      const uint16_t* __restrict__ x, float* __restrict__ partial) {
   extern __shared__ __align__(16) unsigned char dw_smem[];
-  constexpr int TW = 8, NC = 7 * S + 3;
+  constexpr int TW = 8, NC = 7 * S + 3;          // NC = t.iw
   const int C = static_cast<int>(g.C), N = static_cast<int>(g.N), p = static_cast<int>(g.pad);
   const int bw = blockIdx.x % t.tiles_w;
   const int r = blockIdx.x / t.tiles_w;
   const int bh = r % t.tiles_h, cgi = r / t.tiles_h;
   const int oh0 = bh * t.th, ow0 = bw * TW, c0 = cgi * t.cg;
-  const int pix_elems = t.cg * N;
+  const int pix_elems = PIX ? PIX : t.cg * N;
   uint16_t* xs = reinterpret_cast<uint16_t*>(dw_smem);
   uint16_t* gs = xs + t.ih * t.iw * pix_elems;
   float* red = reinterpret_cast<float*>(dw_smem + ((t.ih * t.iw + t.th * TW) * pix_elems * 2 + 15) / 16 * 16);
@@ -339,7 +344,7 @@ dw_wgrad_tile_kernel(const DwGeom g, const DwTile t, const uint16_t* __restrict_
     }
 #pragma unroll
     for (int kh = 0; kh < 3; ++kh) {
-      const uint16_t* rp = xs + (oy * S + kh) * t.iw * pix_elems + c * N + 4 * q;
+      const uint16_t* rp = xs + (oy * S + kh) * NC * pix_elems + c * N + 4 * q;
 #pragma unroll
       for (int j = 0; j < NC; ++j) {
         const uint2 v = *reinterpret_cast<const uint2*>(rp + j * pix_elems);
