@@ -1,8 +1,12 @@
-// Kernels of the BF16 depthwise layers: one thread per unit of work of
-// mqv_depthwise_core.h.  Memory-bound (Kh·Kw multiply-adds per element), so
-// no tensor cores: consecutive threads take consecutive groups of four
-// batch items, then channels, so a warp's loads and stores are contiguous
-// runs of the [H][W][C][N] tensors.
+// Kernels of the BF16 depthwise layers.  Memory-bound (Kh·Kw multiply-adds
+// per element), so no tensor cores.
+//   - The gathers: one thread per unit of work of mqv_depthwise_core.h;
+//     consecutive threads take consecutive groups of four batch items, then
+//     channels, so a warp's loads and stores are contiguous runs of the
+//     [H][W][C][N] tensors.  They serve the layers the tiles do not take.
+//   - The spatial tiles (dw_tile_kernel, dw_wgrad_tile_kernel): a CTA
+//     stages the window its output tile reads once in shared memory and
+//     computes from there.
 #pragma once
 
 #include <cstdint>
@@ -57,6 +61,8 @@ dw_wgrad_reduce_kernel(const DwGeom g, int64_t total, const float* __restrict__ 
 // arithmetic), 0 for any other.  ROWS3: 3x3 filters in tiles 8 wide, one
 // output row per thread (dw_tile_rows3); otherwise a thread takes one output
 // pixel of one (channel, batch quad) lane at a time, taps in runtime loops.
+// PIX: the staged pixel's size in bf16 (CG·N) when it is one of 32 .. 512,
+// so that the row path's shared-memory offsets are constants; 0 otherwise.
 struct DwTile {
   int th, tw, cg;          // output pixels per tile (rows, columns), channels per tile
   int ih, iw;              // staged window, pixels (rows, columns)
@@ -113,11 +119,6 @@ __device__ __forceinline__ void dw_stage(uint16_t* dst, const uint16_t* __restri
   }
 }
 
-// One staged G_Y row of the stride-2 input gradient into the 8 sums of a
-// G_X row.  The tile starts at an even column, so G_X column ox takes tap kw
-// when ox + P + kw is even (P = p mod 2), from staged column
-// (ox + P + 2 - kw) / 2; the columns are walked right to left so that each
-// output sees kw in ascending order.
 // a[e] = fma(w, x[e], a[e]) for e = 0..3, as two packed fp32 FMAs
 // (fma.rn.f32x2: each lane one IEEE fp32 FMA, the same result as fmaf).
 __device__ __forceinline__ void dw_fma4(float (&a)[4], float w, const float (&x)[4]) {
@@ -135,6 +136,11 @@ __device__ __forceinline__ void dw_fma4(float (&a)[4], float w, const float (&x)
       : "f"(w), "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]));
 }
 
+// One staged G_Y row of the stride-2 input gradient into the 8 sums of a
+// G_X row.  The tile starts at an even column, so G_X column ox takes tap kw
+// when ox + P + kw is even (P = p mod 2), from staged column
+// (ox + P + 2 - kw) / 2; the columns are walked right to left so that each
+// output sees kw in ascending order.
 template <int P, int PIX>
 __device__ __forceinline__ void dw_dgrad2_row(const uint16_t* rp, int pix_rt, const float* wk, float (&acc)[8][4]) {
   const int pix_elems = PIX ? PIX : pix_rt;
